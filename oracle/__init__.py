@@ -1,0 +1,250 @@
+"""CPU oracle for the SPECTRA outlier-split INT4 decode matvec.
+
+TEST INFRASTRUCTURE ONLY: the test suite, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package; the library under
+``outlier_split_bit_b200`` never does, and this package never imports it.
+
+The arithmetic lives in ``spectra_ref.c`` (plain C99, IEEE double,
+``-O2 -ffp-contract=off``); this module compiles it with gcc and wraps it with
+ctypes on NumPy arrays.  Method source: "SPECTRA: Sparse-Precision Exact
+Channel Tensor Reconstruction Architecture" (aiwithghost.com re-post of the
+Dev.to abstract), abstract paragraph (kurtosis split with threshold 3.0,
+Group-32 4-bit codes with scale and bit-packed zero point, exact floating-point
+outlier channels).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "spectra_ref.c")
+_LIB = os.path.join(_HERE, "libspectra_ref.so")
+
+# Oracle status codes (its own numbering, see spectra_ref.c).
+OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_NONFINITE, ERR_RANGE = 0, 1, 2, 3, 4
+STATUS_NAMES = {OK: "ok", ERR_INVALID_ARG: "invalid_arg", ERR_SHAPE: "shape",
+                ERR_NONFINITE: "nonfinite", ERR_RANGE: "range"}
+
+
+class OracleError(RuntimeError):
+    def __init__(self, status: int):
+        super().__init__(f"oracle status {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into a shared library next to its source."""
+    if (not force and os.path.exists(_LIB)
+            and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
+        return _LIB
+    tmp = _LIB + f".tmp{os.getpid()}"
+    subprocess.check_call(["gcc", "-std=c99", "-O2", "-ffp-contract=off", "-fno-fast-math",
+                           "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        _declare(_lib)
+    return _lib
+
+
+def _declare(L):
+    P = ctypes.c_void_p
+    i32, i64, f64, u16 = ctypes.c_int32, ctypes.c_int64, ctypes.c_double, ctypes.c_uint16
+    L.spectra_ref_bf16_to_double.argtypes = [u16]
+    L.spectra_ref_bf16_to_double.restype = f64
+    L.spectra_ref_fp16_to_double.argtypes = [u16]
+    L.spectra_ref_fp16_to_double.restype = f64
+    L.spectra_ref_double_to_fp16.argtypes = [f64]
+    L.spectra_ref_double_to_fp16.restype = u16
+    L.spectra_ref_kurtosis.argtypes = [P, P, i32, i32, P]
+    L.spectra_ref_kurtosis.restype = ctypes.c_int
+    L.spectra_ref_split.argtypes = [P, i32, f64, P]
+    L.spectra_ref_split.restype = i32
+    L.spectra_ref_quantize.argtypes = [P, i32, i32, P, i32, P, P, P]
+    L.spectra_ref_quantize.restype = ctypes.c_int
+    L.spectra_ref_layout_sizes.argtypes = [i32, i32, i32, P]
+    L.spectra_ref_layout_sizes.restype = None
+    L.spectra_ref_pack_layout.argtypes = [i32, i32, P, P, P, P, P, i32, P, P, P, P]
+    L.spectra_ref_pack_layout.restype = None
+    L.spectra_ref_unpack_layout.argtypes = [i32, i32, P, P, P, P, P, P]
+    L.spectra_ref_unpack_layout.restype = None
+    L.spectra_ref_dequant.argtypes = [i32, i32, P, P, P, P]
+    L.spectra_ref_dequant.restype = None
+    L.spectra_ref_gemm.argtypes = [i32, i32, P, P, P, P, P, i32, P, i32, P, P]
+    L.spectra_ref_gemm.restype = None
+
+
+def _p(a: np.ndarray | None):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+# ------------------------------------------------------------------ numbers
+
+def bf16_to_double(bits) -> np.ndarray:
+    b = np.asarray(bits, dtype=np.uint16).ravel()
+    f = lib().spectra_ref_bf16_to_double
+    return np.array([f(int(v)) for v in b], dtype=np.float64).reshape(np.shape(bits))
+
+
+def fp16_to_double(bits) -> np.ndarray:
+    b = np.asarray(bits, dtype=np.uint16).ravel()
+    f = lib().spectra_ref_fp16_to_double
+    return np.array([f(int(v)) for v in b], dtype=np.float64).reshape(np.shape(bits))
+
+
+def double_to_fp16(values) -> np.ndarray:
+    v = np.asarray(values, dtype=np.float64).ravel()
+    f = lib().spectra_ref_double_to_fp16
+    return np.array([f(float(a)) for a in v], dtype=np.uint16).reshape(np.shape(values))
+
+
+# ------------------------------------------------------------------ pipeline
+
+def kurtosis(w_bits: np.ndarray, gain: np.ndarray | None) -> np.ndarray:
+    """Per-column Pearson kurtosis of W*g (FP64). w_bits: uint16 [n, k]."""
+    w = _c(w_bits, np.uint16)
+    n, k = w.shape
+    g = None if gain is None else _c(gain, np.float32)
+    kap = np.empty(k, dtype=np.float64)
+    st = lib().spectra_ref_kurtosis(_p(w), _p(g), n, k, _p(kap))
+    if st != OK:
+        raise OracleError(st)
+    return kap
+
+
+def split(kappa: np.ndarray, tau: float) -> np.ndarray:
+    """Ascending int32 indices of the columns with kappa > tau."""
+    kap = _c(kappa, np.float64)
+    idx = np.empty(max(1, kap.size), dtype=np.int32)
+    n_o = lib().spectra_ref_split(_p(kap), kap.size, float(tau), _p(idx))
+    return idx[:n_o].copy()
+
+
+@dataclass
+class Canonical:
+    """Row-major canonical quantised bulk: one code / zero per byte."""
+    codes: np.ndarray   # uint8 [n, k]
+    scales: np.ndarray  # uint16 (FP16 bits) [n, k/32]
+    zeros: np.ndarray   # uint8 [n, k/32]
+
+
+def quantize(w_bits: np.ndarray, idx: np.ndarray) -> Canonical:
+    w = _c(w_bits, np.uint16)
+    n, k = w.shape
+    ix = _c(idx, np.int32)
+    G = k // 32 if k % 32 == 0 else 1
+    codes = np.zeros((n, k), dtype=np.uint8)
+    scales = np.zeros((n, G), dtype=np.uint16)
+    zeros = np.zeros((n, G), dtype=np.uint8)
+    st = lib().spectra_ref_quantize(_p(w), n, k, _p(ix) if ix.size else None, ix.size,
+                                    _p(codes), _p(scales), _p(zeros))
+    if st != OK:
+        raise OracleError(st)
+    return Canonical(codes, scales, zeros)
+
+
+def layout_sizes(n: int, k: int, n_o: int) -> dict:
+    out = np.zeros(5, dtype=np.int64)
+    lib().spectra_ref_layout_sizes(n, k, n_o, _p(out))
+    return {"codes": int(out[0]), "scales": int(out[1]), "zeros": int(out[2]),
+            "outliers": int(out[3]), "n_pad": int(out[4])}
+
+
+@dataclass
+class Packed:
+    codes: np.ndarray     # uint8 [code bytes]
+    scales: np.ndarray    # uint16 FP16 bits
+    zeros: np.ndarray     # uint32 words
+    outliers: np.ndarray  # uint16 BF16 bits
+    idx: np.ndarray       # int32 [n_o]
+    n: int
+    k: int
+
+
+def pack_layout(can: Canonical, w_bits: np.ndarray, idx: np.ndarray) -> Packed:
+    w = _c(w_bits, np.uint16)
+    n, k = w.shape
+    ix = _c(idx, np.int32)
+    sz = layout_sizes(n, k, ix.size)
+    pc = np.zeros(sz["codes"], dtype=np.uint8)
+    ps = np.zeros(sz["scales"], dtype=np.uint16)
+    pz = np.zeros(sz["zeros"], dtype=np.uint32)
+    po = np.zeros(max(1, sz["outliers"]), dtype=np.uint16)
+    lib().spectra_ref_pack_layout(n, k, _p(_c(can.codes, np.uint8)), _p(_c(can.scales, np.uint16)),
+                                  _p(_c(can.zeros, np.uint8)), _p(w),
+                                  _p(ix) if ix.size else None, ix.size,
+                                  _p(pc), _p(ps), _p(pz), _p(po))
+    return Packed(pc, ps, pz, po[:sz["outliers"]], ix.copy(), n, k)
+
+
+def unpack_layout(p: Packed) -> Canonical:
+    n, k = p.n, p.k
+    G = k // 32
+    codes = np.zeros((n, k), dtype=np.uint8)
+    scales = np.zeros((n, G), dtype=np.uint16)
+    zeros = np.zeros((n, G), dtype=np.uint8)
+    lib().spectra_ref_unpack_layout(n, k, _p(_c(p.codes, np.uint8)), _p(_c(p.scales, np.uint16)),
+                                    _p(_c(p.zeros, np.uint32)), _p(codes), _p(scales), _p(zeros))
+    return Canonical(codes, scales, zeros)
+
+
+def dequant(can: Canonical) -> np.ndarray:
+    n, k = can.codes.shape
+    out = np.empty((n, k), dtype=np.float64)
+    lib().spectra_ref_dequant(n, k, _p(_c(can.codes, np.uint8)), _p(_c(can.scales, np.uint16)),
+                              _p(_c(can.zeros, np.uint8)), _p(out))
+    return out
+
+
+def gemm(can: Canonical, w_bits: np.ndarray, idx: np.ndarray, x_bits: np.ndarray):
+    """(y [m, n], bound [m, n]) in FP64; x_bits: uint16 BF16 [m, k] (or [k])."""
+    w = _c(w_bits, np.uint16)
+    n, k = w.shape
+    x = _c(x_bits, np.uint16).reshape(-1, k)
+    m = x.shape[0]
+    ix = _c(idx, np.int32)
+    y = np.empty((m, n), dtype=np.float64)
+    b = np.empty((m, n), dtype=np.float64)
+    lib().spectra_ref_gemm(n, k, _p(_c(can.codes, np.uint8)), _p(_c(can.scales, np.uint16)),
+                           _p(_c(can.zeros, np.uint8)), _p(w), _p(ix) if ix.size else None,
+                           ix.size, _p(x), m, _p(y), _p(b))
+    return y, b
+
+
+@dataclass
+class Layer:
+    """Everything the oracle derives from one weight matrix."""
+    kappa: np.ndarray
+    idx: np.ndarray
+    can: Canonical
+    packed: Packed
+
+
+def pack(w_bits: np.ndarray, gain: np.ndarray | None, tau: float) -> Layer:
+    """Saliency split, group quantiser and packed layout, in that order."""
+    kap = kurtosis(w_bits, gain)
+    idx = split(kap, tau)
+    can = quantize(w_bits, idx)
+    return Layer(kap, idx, can, pack_layout(can, w_bits, idx))
+
+
+def tolerance(bound: np.ndarray) -> np.ndarray:
+    """Acceptance bound of a GPU matvec result: 2e-3 * sum|w_hat||x| + 1e-5."""
+    return 2e-3 * bound + 1e-5

@@ -1,0 +1,99 @@
+"""Plant plausible mistakes in a copy of the CPU oracle and check that a pin fails.
+
+Each mutation edits the C source of a private copy (built under a temporary
+directory), loads it as a separate module and runs the closed-form, library
+and brute-force pins of ``test_oracle_pins`` against it.  A mutation that no
+pin notices would mean the pins leave that part of the oracle unchecked.
+Every mutation keeps its memory accesses in bounds.  Everything runs on the
+CPU.
+"""
+import importlib.util
+import os
+import shutil
+import sys
+
+import pytest
+
+import test_oracle_pins as pins
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+MUTATIONS = {
+    "kurtosis_dropped_square": ("m4 = m4 + q * q;", "m4 = m4 + q;"),
+    "kurtosis_biased_mean": ("double mu = s / (double)n;", "double mu = s / (double)(n + 1);"),
+    "kurtosis_m2_not_squared": ("m4 / (m2 * m2)", "m4 / m2"),
+    "split_not_strict": ("if (kappa[j] > tau)", "if (kappa[j] >= tau)"),
+    "zero_point_sign": ("double zq = rint(-lo / S);", "double zq = rint(lo / S);"),
+    "code_minus_zero": ("double c = rint(v[kk] / S) + z;", "double c = rint(v[kk] / S) - z;"),
+    "scale_divisor": ("diff / 15.0", "diff / 16.0"),
+    "fp16_truncates": ("double q = rint(ldexp(a, 10 - E));", "double q = floor(ldexp(a, 10 - E));"),
+    "layout_word_stride": ("* 16 + word * 4 + j / 2;\n            uint8_t c",
+                           "* 16 + word * 2 + j / 2;\n            uint8_t c"),
+    "layout_scale_slot_reversed": ("pscales[((t * S + g / 8) * 32 + r) * 8 + g % 8] = scales[i * G + g];",
+                                "pscales[((t * S + g / 8) * 32 + r) * 8 + 7 - g % 8] = scales[i * G + g];"),
+    "outlier_gather_reversed": ("poutl[((t * O8 + o / 8) * 32 + r) * 8 + o % 8] = w[i * k + idx[o]];",
+                                  "poutl[((t * O8 + o / 8) * 32 + r) * 8 + o % 8] = w[i * k + idx[n_o - 1 - o]];"),
+    "gemm_zero_index": ("(double)zeros[i * G + kk / 32]) * S;\n                double xv",
+                        "(double)zeros[i * G + kk % G]) * S;\n                double xv"),
+    "gemm_dequant_sign": ("double wd = ((double)codes[i * k + kk] - (double)zeros",
+                          "double wd = ((double)codes[i * k + kk] + (double)zeros"),
+    "gemm_outlier_x_index": ("double xv = spectra_ref_bf16_to_double(xr[idx[t]]);",
+                             "double xv = spectra_ref_bf16_to_double(xr[t]);"),
+}
+
+PIN_FUNCS = [
+    pins.test_fp16_golden_cases,
+    pins.test_fp16_random_doubles_match_numpy,
+    pins.test_kurtosis_closed_forms,
+    pins.test_kurtosis_matches_scipy_with_gain,
+    pins.test_split_strict_and_ascending,
+    pins.test_quantizer_exact_grid,
+    pins.test_quantizer_half_even_ties,
+    pins.test_quantizer_invariants_random,
+    pins.test_layout_golden_offsets,
+    pins.test_layout_roundtrip,
+    pins.test_gemm_brute_force_8x32,
+    pins.test_gemm_all_outliers_is_dense_product,
+    pins.test_gemm_unit_vectors_extract_columns,
+]
+_PARAMS = {
+    "test_quantizer_exact_grid": [{"S": 2.0 ** -7, "z": 5}],
+    "test_layout_roundtrip": [{"n": 40, "k": 96, "n_o": 9}],
+}
+
+
+def _load_variant(tmp_path, name, old, new):
+    d = tmp_path / f"oracle_{name}"
+    shutil.copytree(os.path.join(ROOT, "oracle"), d,
+                    ignore=shutil.ignore_patterns("*.so", "__pycache__"))
+    src = d / "spectra_ref.c"
+    text = src.read_text()
+    assert text.count(old) == 1, f"mutation anchor not unique: {name}"
+    src.write_text(text.replace(old, new))
+    spec = importlib.util.spec_from_file_location(f"oracle_{name}", d / "__init__.py")
+    mod = importlib.util.module_from_spec(spec)
+    sys.modules[spec.name] = mod
+    spec.loader.exec_module(mod)
+    mod.build(force=True)
+    return mod
+
+
+def _caught(mod, golden_dir) -> bool:
+    for f in PIN_FUNCS:
+        kwargs_list = _PARAMS.get(f.__name__, [{}])
+        for kw in kwargs_list:
+            args = {"ref": mod}
+            if "golden_dir" in f.__code__.co_varnames[:f.__code__.co_argcount]:
+                args["golden_dir"] = golden_dir
+            try:
+                f(**args, **kw)
+            except Exception:
+                return True
+    return False
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(tmp_path, golden_dir, name):
+    old, new = MUTATIONS[name]
+    mod = _load_variant(tmp_path, name, old, new)
+    assert _caught(mod, golden_dir), f"no pin fails for mutation {name}"
