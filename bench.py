@@ -1,0 +1,499 @@
+#!/usr/bin/env python
+"""Decode-step weight-stream benchmark of the SPECTRA outlier-split INT4 matvec.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one decode-step weight stream: 28 layers x 7 projections of a
+1.5B-class decoder (hidden 1536, intermediate 8960, KV width 256), one batch-1
+matvec per matrix with its own BF16 activation vector (196 launches, 1.31 G
+weights, 0.76 GB packed), captured once in a CUDA graph and replayed.  The
+packed weights exceed the 126 MB L2, so every step streams them from HBM.
+Rank 0 prints one JSON line.  For N > 1 every rank (one per GPU) runs its own
+replica of the stream: the problems are independent, there is no data-path
+collective, and the value is the bytes of all ranks over the slowest rank's
+time (weak scaling).
+
+--impl reference times the CPU oracle (oracle/, IEEE double, one core) on a
+bounded sample of the same workload: whole 32-row tiles of each matrix,
+unpacked from the oracle's own packed layout and multiplied.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from outlier_split_bit_b200 import workload as wl  # noqa: E402
+
+N_LAYERS = wl.N_LAYERS_1P5B
+METRIC = "achieved HBM GB/s (% of peak) of spectra_gemv at M=1; µs per decode-step weights"
+WORKLOAD = "decode-step weight stream, 28 layers x {q,k,v,o,gate,up,down} of the 1.5B-class shape, M=1"
+
+
+# ---------------------------------------------------------------- helpers
+
+def algorithmic_bytes(n: int, k: int, n_o: int, m: int = 1, y_bytes: int = 4) -> int:
+    """Bytes one matvec must move: 4.625 bits per bulk weight (codes, FP16
+    scales, 4-bit zero points), BF16 outlier columns, outlier indices, x, y."""
+    n_pad = -(-n // 32) * 32
+    return (n_pad * k // 2 + n_pad * k // 16 + n_pad * k // 64 + 2 * n * n_o + 4 * n_o
+            + 2 * m * k + y_bytes * m * n)
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        d["_source"] = "measured"
+        return d
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "_source": "fallback"}
+
+
+_REASONS = [(0x4, "sw_power_cap"), (0x8, "hw_slowdown"), (0x20, "sw_thermal_slowdown"),
+            (0x40, "hw_thermal_slowdown"), (0x80, "hw_power_brake_slowdown"),
+            (0x2, "applications_clocks_setting"), (0x10, "sync_boost")]
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            self._ok = False
+
+    def _run(self):
+        nv = self._nv
+        get_r = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = get_r(self._h)
+                for bit, name in _REASONS:
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- workload
+
+class Stream:
+    """The packed 28-layer weight stream with its activation and output buffers."""
+
+    def __init__(self, device, seed: int, tau: float):
+        import outlier_split_bit_b200 as sp
+        self.sp = sp
+        specs = [(layer, s) for layer in range(N_LAYERS) for s in wl.LAYER_1P5B]
+        xk = sum(s.k for _, s in specs)
+        yn = sum(s.n for _, s in specs)
+        self.x_all = torch.empty(xk, dtype=torch.bfloat16, device=device)
+        self.y_all = torch.empty(yn, dtype=torch.float32, device=device)
+        self.items = []
+        self.bytes = 0
+        self.n_outliers = 0
+        xo = yo = 0
+        for layer, spec in specs:
+            w = wl.weight(spec, seed, layer, device=device)
+            g = wl.gain(spec, seed, layer, device=device)
+            lay = sp.pack_layer(w, g, tau)
+            del w
+            x = self.x_all[xo:xo + spec.k]
+            x.copy_(wl.activations(spec.k, 1, seed, layer, slot=wl.PROJ.index(spec.name),
+                                   device=device)[0])
+            y = self.y_all[yo:yo + spec.n]
+            xo += spec.k
+            yo += spec.n
+            self.items.append((spec, lay, x, y, lay.view()))
+            self.bytes += algorithmic_bytes(spec.n, spec.k, lay.n_outliers)
+            self.n_outliers += lay.n_outliers
+        self.launches = len(self.items)
+
+    def run(self, stream):
+        for spec, lay, x, y, view in self.items:
+            self.sp.spectra_gemv(lay, x, y, view=view, stream=stream)
+
+    def capture(self, stream):
+        g = torch.cuda.CUDAGraph()
+        torch.cuda.synchronize()  # packing ran on the default stream
+        with torch.cuda.stream(stream):
+            self.run(stream)  # warm: sets kernel attributes outside capture
+            stream.synchronize()
+            with torch.cuda.graph(g, stream=stream):
+                self.run(stream)
+        return g
+
+
+def flush_l2(buf):
+    buf.add_(1)
+
+
+def time_single(fn, stream, reps, flush_buf):
+    """Median device time (µs) of fn() with L2 flushed before each rep."""
+    ts = []
+    for _ in range(reps):
+        flush_l2(flush_buf)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        ts.append(a.elapsed_time(b) * 1e3)
+    return float(statistics.median(ts)), float(np.percentile(ts, 10)), float(np.percentile(ts, 90))
+
+
+def extras(device, stream, peak_gbs, tau):
+    """Per-matrix, LM-head and batch-sweep measurements (single launches,
+    L2 flushed before each rep)."""
+    import outlier_split_bit_b200 as sp
+    out = {}
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+    with torch.cuda.stream(stream):
+        rows = []
+        for spec in wl.LAYER_1P5B:
+            w = wl.weight(spec, 0, 0, device=device)
+            g = wl.gain(spec, 0, 0, device=device)
+            n3 = int(sp.spectra_pack_plan(w, g, 3.0)[0].numel())
+            t0 = time.perf_counter()
+            lay = sp.pack_layer(w, g, tau)
+            pack_ms = (time.perf_counter() - t0) * 1e3
+            x = wl.activations(spec.k, 1, device=device)[0]
+            y = torch.empty(spec.n, device=device)
+            v = lay.view()
+            us, p10, p90 = time_single(lambda: sp.spectra_gemv(lay, x, y, view=v, stream=stream),
+                                       stream, 50, flush)
+            b = algorithmic_bytes(spec.n, spec.k, lay.n_outliers)
+            rows.append({"matrix": spec.name, "n": spec.n, "k": spec.k, "us": round(us, 2),
+                         "us_p10": round(p10, 2), "us_p90": round(p90, 2), "bytes": b,
+                         "gbs": round(b / us * 1e-3, 1), "frac": round(b / us * 1e-3 / peak_gbs, 3),
+                         "n_outliers_tau": lay.n_outliers, "n_outliers_tau3": n3,
+                         "pack_ms": round(pack_ms, 2)})
+            del w, lay
+        out["per_matrix_1p5b"] = rows
+        rows = []
+        for frac in wl.LM_HEAD_FRACTIONS:
+            spec = wl.lm_head_spec(frac)
+            w = wl.weight(spec, 0, 0, device=device)
+            g = wl.gain(spec, 0, 0, device=device)
+            lay = sp.pack_layer(w, g, tau)
+            x = wl.activations(spec.k, 1, device=device)[0]
+            y = torch.empty(spec.n, device=device)
+            v = lay.view()
+            us, p10, p90 = time_single(lambda: sp.spectra_gemv(lay, x, y, view=v, stream=stream),
+                                       stream, 20, flush)
+            dense = (w.float() @ x.float())
+            err = float(torch.linalg.vector_norm(y - dense) / torch.linalg.vector_norm(dense))
+            b = algorithmic_bytes(spec.n, spec.k, lay.n_outliers)
+            rows.append({"frac_t_columns": frac, "n_outliers": lay.n_outliers, "us": round(us, 2),
+                         "gbs": round(b / us * 1e-3, 1), "frac": round(b / us * 1e-3 / peak_gbs, 3),
+                         "rel_err_vs_bf16_dense": round(err, 5),
+                         "bits_per_weight": round(8 * lay.nbytes / (spec.n * spec.k), 3)})
+            del w, lay, dense
+        out["lm_head_131072x3072"] = rows
+        rows = []
+        spec = wl.LAYER_4B[4]
+        w = wl.weight(spec, 0, 0, device=device)
+        g = wl.gain(spec, 0, 0, device=device)
+        lay = sp.pack_layer(w, g, tau)
+        v = lay.view()
+        for m in wl.BATCH_SWEEP:
+            x = wl.activations(spec.k, m, device=device)
+            y = torch.empty((m, spec.n), device=device)
+            us, p10, p90 = time_single(
+                lambda: sp.spectra_gemm_small(lay, x, y, view=v, stream=stream), stream, 30, flush)
+            b = algorithmic_bytes(spec.n, spec.k, lay.n_outliers, m=m)
+            rows.append({"m": m, "us": round(us, 2), "gbs": round(b / us * 1e-3, 1),
+                         "frac": round(b / us * 1e-3 / peak_gbs, 3),
+                         "tflops": round(2 * m * spec.n * spec.k / us * 1e-6, 2)})
+        out["batch_sweep_4b_gate_9728x2560"] = rows
+        del w, lay
+    return out
+
+
+# ---------------------------------------------------------------- oracle leg
+
+def oracle_sample(seed: int, tau: float, tiles_per_matrix: int, reps: int = 1):
+    """Time the CPU oracle's matvec (unpack of the packed layout + FP64 product)
+    on whole 32-row tiles of each matrix of one layer.  Returns (bytes, seconds,
+    description)."""
+    import oracle
+    oracle.build()
+    prepared = []
+    for spec in wl.LAYER_1P5B:
+        w = wl.weight(spec, seed, 0, device="cpu")
+        g = wl.gain(spec, seed, 0, device="cpu")
+        wb = wl.bits(w)
+        lay = oracle.pack(wb, None if g is None else g.numpy(), tau)
+        x = wl.bits(wl.activations(spec.k, 1, seed, 0, slot=wl.PROJ.index(spec.name)))
+        T = -(-spec.n // 32)
+        tiles = np.linspace(0, T - 1, num=min(T, tiles_per_matrix)).astype(int)
+        prepared.append((spec, lay, wb, x, tiles))
+    return prepared
+
+
+def oracle_time(prepared):
+    import oracle
+    total_b, t0 = 0, time.perf_counter()
+    for spec, lay, wb, x, tiles in prepared:
+        p = lay.packed
+        G, S = spec.k // 32, -(-(spec.k // 32) // 8)
+        for t in tiles:
+            nr = min(spec.n, 32 * t + 32) - 32 * t
+            sub = oracle.Packed(p.codes[t * G * 512:(t + 1) * G * 512],
+                                p.scales[t * S * 256:(t + 1) * S * 256],
+                                p.zeros[t * S * 32:(t + 1) * S * 32], p.outliers, p.idx, nr, spec.k)
+            can = oracle.unpack_layout(sub)
+            oracle.gemm(can, wb[32 * t:32 * t + nr], lay.idx, x)
+            total_b += algorithmic_bytes(nr, spec.k, lay.idx.size)
+    return total_b, time.perf_counter() - t0
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    prepared = oracle_sample(0, args.tau, 1)
+    b1, t1 = oracle_time(prepared)
+    budget_s = 120.0
+    per_step = budget_s / max(1, args.steps + args.warmup)
+    tiles = int(max(1, min(64, per_step / max(t1, 1e-6))))
+    prepared = oracle_sample(0, args.tau, tiles)
+    for _ in range(args.warmup):
+        oracle_time(prepared)
+    tot_b, tot_t = 0, 0.0
+    for _ in range(args.steps):
+        b, t = oracle_time(prepared)
+        tot_b += b
+        tot_t += t
+    gbs = tot_b / tot_t * 1e-9
+    sample = (f"{tiles} row tile(s) of 32 rows from each of the 7 matrices of layer 0 per step "
+              f"({tot_b // max(1, args.steps)} algorithmic bytes per step)")
+    line = {"impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(tot_t / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "tau": args.tau, "m": 1},
+            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- our arm
+
+def kernel_source_digest() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "outlier_split_bit_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.startswith("gemv"):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(digest: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "gemv_decode_stream_traffic.md")
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    for line in open(p):
+        if ":" in line and line.startswith("- "):
+            k, v = line[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_sha256_16") != digest:
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def run_ours(args):
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    peaks = measured_peaks()
+    peak = float(peaks["hbm_gbs"])
+    stream = torch.cuda.Stream(device=device)
+    st = Stream(device, seed=rank, tau=args.tau)
+    graph = st.capture(stream)
+    for _ in range(args.warmup):
+        graph.replay()
+    stream.synchronize()
+
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.steps):
+                graph.replay()
+            e1.record(stream)
+        e1.synchronize()
+    torch.cuda.synchronize()
+    barrier()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    step_ms = ms / args.steps
+    total_bytes = st.bytes * args.steps * world
+    gbs = total_bytes / (ms * 1e-3) * 1e-9
+
+    # end to end: pinned host x in, y out, copies inside the timed region
+    x_host = torch.empty(st.x_all.shape, dtype=st.x_all.dtype, pin_memory=True)
+    x_host.copy_(st.x_all)
+    y_host = torch.empty(st.y_all.shape, dtype=st.y_all.dtype, pin_memory=True)
+    e2e_steps = max(1, min(args.steps, 200))
+    barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e2e_steps):
+            st.x_all.copy_(x_host, non_blocking=True)
+            graph.replay()
+            y_host.copy_(st.y_all, non_blocking=True)
+        b.record(stream)
+    b.synchronize()
+    barrier()
+    e2e_ms = a.elapsed_time(b)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_gbs = st.bytes * e2e_steps * world / (e2e_ms * 1e-3) * 1e-9
+
+    extra = {}
+    if rank == 0 and not args.quick:
+        extra = extras(device, stream, peak, args.tau)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        prepared = oracle_sample(0, args.tau, 8)
+        b_s, t_s = 0, 0.0
+        while t_s < 10.0:
+            bb, tt = oracle_time(prepared)
+            b_s += bb
+            t_s += tt
+        cpu = {"value": round(b_s / t_s * 1e-9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": "8 row tiles of 32 rows from each of the 7 matrices of one 1.5B-class "
+                         f"layer, repeated for {t_s:.1f} s (unpack + FP64 matvec, one thread)"}
+
+    digest = kernel_source_digest()
+    traffic = profiled_traffic(digest)
+    launch_bytes = st.bytes / st.launches
+    launch_us = step_ms * 1e3 / st.launches
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(gbs, 1), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
+            "us_per_step": round(step_ms * 1e3, 2),
+            "pct_of_peak": round(100.0 * gbs / world / peak, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4+bf16->f32",
+            "data": "synthetic (seeded N(0,0.02) weights with Student-t(3) columns, N(0,1) x)",
+            "config": {"workload": WORKLOAD, "matrices_per_step": st.launches,
+                       "bytes_per_step": st.bytes, "n_outliers_per_step": st.n_outliers,
+                       "tau": args.tau, "m": 1, "launch": "CUDA graph of 196 spectra_gemv, PDL",
+                       "l2": "inputs larger than L2 (0.76 GB of packed weights per step)",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "hbm", "achieved": round(launch_bytes / launch_us * 1e-3, 1),
+                         "peak": peak, "unit": "GB/s",
+                         "frac": round(launch_bytes / launch_us * 1e-3 / peak, 4),
+                         "traffic": traffic, "peak_source": peaks["_source"],
+                         "bytes_per_launch": round(launch_bytes), "us_per_launch": round(launch_us, 3)},
+            "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s",
+                    "h2d_bytes_per_step": st.x_all.numel() * 2,
+                    "d2h_bytes_per_step": st.y_all.numel() * 4},
+            "gpu_launches": st.launches * args.steps,
+            "clocks": clk.summary(),
+            "cpu_baseline": cpu,
+        }
+        if extra:
+            line["rows"] = extra
+        print(json.dumps(line), flush=True)
+    del graph
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--tau", type=float, default=3.0)
+    ap.add_argument("--quick", action="store_true", help="skip the per-matrix / LM-head / batch rows")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,210 @@
+/*
+ * spectra.h -- C ABI of the B200 (sm_100a) SPECTRA outlier-split INT4 library.
+ *
+ * The method ("SPECTRA: Sparse-Precision Exact Channel Tensor Reconstruction
+ * Architecture", Dev.to abstract, abstract paragraph): every input channel
+ * (column j of W[n][k]) whose fourth-moment kurtosis, taken on the column
+ * scaled by its upstream normalisation gain, exceeds a threshold (3.0 in the
+ * abstract) is kept bit-exact in BF16; the remaining bulk is stored as Group-32
+ * 4-bit codes with one FP16 scale and one bit-packed 4-bit zero point per
+ * group of 32 consecutive weights of a row.  Decoding happens in registers
+ * inside the matrix-vector kernel, which also runs the dense matvec of the
+ * BF16 outlier columns in the same pass (abstract: fused dequantisation
+ * "within register pipelines").
+ *
+ * Conventions shared by every entry point:
+ *   - All pointers named *_dev or documented as "device" are CUDA device
+ *     pointers (global memory of the current device) owned by the caller;
+ *     the library never allocates, frees or retains them.  Host pointers are
+ *     documented as such.
+ *   - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *     stream.  Work is enqueued on it.  Functions documented "synchronous"
+ *     wait for their own work on `stream` before returning.
+ *   - Argument checks run before any launch.  A failed check returns its
+ *     status and leaves every output untouched.  Launch failures return
+ *     SPECTRA_ERR_CUDA.  Faults of asynchronous work surface at the caller's
+ *     next synchronisation.
+ *   - Device pointers must be 16-byte aligned (SPECTRA_ERR_ALIGN otherwise).
+ *   - Results are bit-identical from run to run: every reduction has a fixed
+ *     order.
+ *   - No exception crosses the ABI.  The only library state is a per-device
+ *     cache of device properties, filled on first use under a lock.
+ *
+ * Shapes: n = out_features (rows of W), k = in_features (columns), m = batch
+ * rows of x.  k must be a positive multiple of 32; n >= 1.
+ *
+ * Packed layout ("RT32", this library's Blackwell layout; it replaces the
+ * Marlin interleave named in the abstract).  N_pad = ceil(n/32)*32,
+ * T = N_pad/32 row tiles, G = k/32 groups, S = ceil(G/8) super-groups,
+ * O8 = ceil(n_outliers/8):
+ *   codes   : 16-byte record per (tile t, group g, lane r) at byte offset
+ *             ((t*G + g)*32 + r)*16; the record's little-endian u32 word w
+ *             holds in nibble j (bits 4j..4j+3) the code of column
+ *             32g + 8w + j of row 32t + r.  A warp (lane r = row r of the
+ *             tile) reads one contiguous 512-byte segment per group.
+ *   scales  : FP16 bits, element ((t*S + g/8)*32 + r)*8 + g%8; one 16-byte
+ *             load gives a row its 8 scales of a super-group.
+ *   zeros   : u32 word (t*S + g/8)*32 + r, nibble g%8 holds the zero point.
+ *   outliers: BF16 bits, element ((t*O8 + j/8)*32 + r)*8 + j%8 holds
+ *             W[32t + r][idx[j]] for outlier slot j.
+ *   Padding rows, groups and outlier slots are zero.  Bulk storage is
+ *   4.625 bits per weight (0.578 bytes) plus 16 bits per outlier element.
+ */
+#ifndef SPECTRA_H
+#define SPECTRA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SPECTRA_API __attribute__((visibility("default")))
+#else
+#define SPECTRA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SPECTRA_OK = 0,
+    SPECTRA_ERR_INVALID_ARG = 1,      /* null pointer, negative count, bad enum value */
+    SPECTRA_ERR_SHAPE = 2,            /* k % 32 != 0, k < 32, n < 1, m outside [1, 32], too large */
+    SPECTRA_ERR_ALIGN = 3,            /* a device pointer is not 16-byte aligned */
+    SPECTRA_ERR_NONFINITE = 4,        /* NaN or infinity in W or in the gain */
+    SPECTRA_ERR_RANGE = 5,            /* a group's scale (max-min)/15 overflows FP16 */
+    SPECTRA_ERR_BUFFER_TOO_SMALL = 6, /* workspace smaller than the stated size */
+    SPECTRA_ERR_CUDA = 7,             /* a CUDA runtime call failed */
+    SPECTRA_ERR_UNSUPPORTED = 8,      /* the current device is not compute capability 10.0 */
+    SPECTRA_ERR_INTERNAL = 9          /* a kernel reported an inconsistent state */
+} spectra_status;
+
+typedef enum { SPECTRA_F32 = 0, SPECTRA_BF16 = 1 } spectra_dtype;
+
+/* A packed layer: a plain view of caller-owned device buffers. */
+typedef struct {
+    int32_t n;                   /* out_features */
+    int32_t k;                   /* in_features, multiple of 32 */
+    int32_t n_outliers;          /* number of BF16 outlier columns, 0..k */
+    const uint8_t *codes;        /* device, RT32 code records */
+    const uint16_t *scales;      /* device, FP16 bits */
+    const uint32_t *zeros;       /* device, 8 zero points per word */
+    const int32_t *outlier_idx;  /* device, ascending column indices [n_outliers] */
+    const uint16_t *outlier_w;   /* device, BF16 bits, RT32 outlier block */
+} spectra_layer;
+
+/* Byte sizes of the packed buffers of one layer. */
+typedef struct {
+    int64_t n_pad;
+    size_t codes_bytes;
+    size_t scales_bytes;
+    size_t zeros_bytes;
+    size_t outlier_idx_bytes;
+    size_t outlier_w_bytes;
+} spectra_sizes;
+
+/* Human-readable name of a status value (static string, never NULL). */
+SPECTRA_API const char *spectra_status_string(spectra_status s);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+SPECTRA_API int32_t spectra_version(void);
+
+/*
+ * Sizes of the packed buffers for an (n x k) layer with n_outliers outlier
+ * columns (layout above).  Host only, no CUDA call.
+ */
+SPECTRA_API spectra_status spectra_packed_sizes(int32_t n, int32_t k, int32_t n_outliers, spectra_sizes *out);
+
+/* Device workspace bytes that spectra_pack_plan needs for in_features k. */
+SPECTRA_API size_t spectra_pack_plan_workspace_size(int32_t k);
+
+/* Device workspace bytes that spectra_pack needs (a status word). */
+SPECTRA_API size_t spectra_pack_workspace_size(void);
+
+/*
+ * Saliency split (abstract: kurtosis of each channel from the upstream
+ * normalisation gain; channels above the threshold go to bit-exact storage).
+ *   w        device, BF16 bits, row-major [n][k]
+ *   gain     device, float [k], or NULL for g = 1
+ *   tau      threshold; column j is an outlier iff kappa_j > tau (strict)
+ *   kappa_out  device double [k] receiving kappa_j, or NULL
+ *   idx_out  device int32 [k]; receives the ascending outlier indices
+ *   n_outliers_out  HOST int32; receives |O|
+ *   workspace  device, >= spectra_pack_plan_workspace_size(k) bytes
+ * kappa_j is the Pearson kurtosis m4/m2^2 (population moments) of
+ * a_i = W[i][j]*g_j over rows i, computed in IEEE double in the fixed order
+ * sum -> mean -> (d, d^2, m2 += d^2, m4 += d^4) -> m2/n, m4/n -> m4/(m2*m2),
+ * with kappa := 0 when m2 == 0; the same order as the CPU oracle, so the
+ * values and the split are bit-identical to it.
+ * Synchronous: returns after the split is known.  Errors: SHAPE (n < 1 or
+ * k < 32 or k % 32), NONFINITE (NaN/inf in w or gain), BUFFER_TOO_SMALL.
+ */
+SPECTRA_API spectra_status spectra_pack_plan(const uint16_t *w, const float *gain, int32_t n, int32_t k,
+                                 double tau, double *kappa_out, int32_t *idx_out,
+                                 int32_t *n_outliers_out, void *workspace,
+                                 size_t workspace_bytes, void *stream);
+
+/*
+ * Group quantiser + packer (abstract: Group-32 4-bit microscaling with
+ * bit-packed zero points; outlier channels kept bit-exact).
+ *   w        device, BF16 bits [n][k]
+ *   idx      device int32 [n_outliers], ascending, from spectra_pack_plan
+ *   codes, scales, zeros, outlier_w   device outputs sized by
+ *            spectra_packed_sizes (outlier_w may be NULL when n_outliers == 0)
+ *   workspace  device, >= spectra_pack_workspace_size() bytes
+ *   layer_out  HOST; filled with a view of the outputs (may be NULL)
+ * Per row and group of 32 columns, over W with the outlier columns set to +0
+ * and -0 read as +0: lo = min, hi = max (double); s = FP16 of (hi-lo)/15 with
+ * one round-to-nearest-even step; S = (double)s; S == 0 -> zero point 0 and
+ * codes 0; else z = clamp(rint(-lo/S), 0, 15), c = clamp(rint(w/S) + z, 0, 15)
+ * (division in IEEE double, rint ties to even).  Bit-identical to the oracle.
+ * Synchronous.  Errors: SHAPE, NONFINITE, RANGE (a scale rounds to FP16
+ * infinity), INVALID_ARG (an index outside [0, k) or not ascending).
+ */
+SPECTRA_API spectra_status spectra_pack(const uint16_t *w, int32_t n, int32_t k, const int32_t *idx,
+                            int32_t n_outliers, uint8_t *codes, uint16_t *scales,
+                            uint32_t *zeros, uint16_t *outlier_w, void *workspace,
+                            size_t workspace_bytes, spectra_layer *layer_out, void *stream);
+
+/*
+ * Inverse of the layout step, for tests: packed layer -> canonical row-major
+ * arrays codes [n][k] (one code per byte), scales [n][k/32] (FP16 bits),
+ * zeros [n][k/32] (one zero point per byte), all device.  Asynchronous.
+ */
+SPECTRA_API spectra_status spectra_unpack(const spectra_layer *layer, uint8_t *codes, uint16_t *scales,
+                              uint8_t *zeros, void *stream);
+
+/*
+ * Batch-1 decode matvec, the hot path:
+ *   y[i] = sum_g s_ig * sum_{k in g} (c_ik - z_ig) * x[k]
+ *        + sum_t W[i][idx_t] * x[idx_t]
+ *   layer  HOST struct viewing device buffers
+ *   x      device, BF16 bits [k]
+ *   y      device, [n] of y_dtype (FP32 or BF16, round to nearest even)
+ * FP32 accumulation; accepted results satisfy |y - y_ref| <=
+ * 2e-3 * sum_j |w_hat_ij * x_j| + 1e-5 against the FP64 oracle.
+ * Asynchronous, allocates nothing, graph-capturable.  The kernel is launched
+ * with programmatic dependent launch: it may start streaming its (constant)
+ * packed weights while the previous kernel on the stream is finishing, and
+ * it reads x and writes y only after that kernel has completed.
+ * Errors: INVALID_ARG, SHAPE, ALIGN, UNSUPPORTED, CUDA.
+ */
+SPECTRA_API spectra_status spectra_gemv(const spectra_layer *layer, const uint16_t *x, void *y,
+                            spectra_dtype y_dtype, void *stream);
+
+/*
+ * Small-batch decode matmul, y[m][i] for m in [0, m_rows), 1 <= m_rows <= 32:
+ *   x  device, BF16 bits [m_rows][k] row-major;  y  device [m_rows][n].
+ * Same formula and tolerance as spectra_gemv per batch row.  m_rows <= 15 runs
+ * on CUDA cores (m_rows accumulators per lane); 16..32 runs the tensor-core
+ * path (weights dequantised in registers, then MMA with FP32 accumulation).
+ * Asynchronous, allocates nothing.
+ */
+SPECTRA_API spectra_status spectra_gemm_small(const spectra_layer *layer, const uint16_t *x, int32_t m_rows,
+                                  void *y, spectra_dtype y_dtype, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPECTRA_H */

@@ -1,0 +1,190 @@
+"""B200 (sm_100a) SPECTRA outlier-split INT4 decode matvec.
+
+Thin Python binding of the C ABI in ``include/spectra.h``: argument
+marshalling only.  Every step of the path (kurtosis, split, quantisation,
+packing, fused dequantise+matvec) runs in the library's CUDA kernels; PyTorch
+provides device memory and streams.  There is no CPU fallback: importing
+the binding loads ``libspectra.so`` on first use and raises ImportError when
+it is missing.
+
+Method: "SPECTRA: Sparse-Precision Exact Channel Tensor Reconstruction
+Architecture" (Dev.to abstract re-post), abstract paragraph.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+from ._lib import Layer, Sizes
+
+__all__ = ["SpectraError", "PackedLayer", "spectra_status_string", "spectra_version",
+           "spectra_packed_sizes", "spectra_pack_plan", "spectra_pack", "spectra_unpack",
+           "spectra_gemv", "spectra_gemm_small", "pack_layer", "library"]
+
+class _Lazy:
+    """Loads libspectra.so on first attribute access."""
+
+    def __getattr__(self, name):
+        return getattr(_lib.load(), name)
+
+
+_L = _Lazy()
+
+
+def library() -> ctypes.CDLL:
+    return _lib.load()
+
+
+class SpectraError(RuntimeError):
+    def __init__(self, status: int, where: str = ""):
+        msg = _L.spectra_status_string(status).decode()
+        super().__init__(f"{where}: {msg} (status {status})" if where else msg)
+        self.status = status
+
+
+def _check(status: int, where: str):
+    if status != _lib.OK:
+        raise SpectraError(status, where)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def spectra_status_string(status: int) -> str:
+    return _L.spectra_status_string(status).decode()
+
+
+def spectra_version() -> int:
+    return _L.spectra_version()
+
+
+def spectra_packed_sizes(n: int, k: int, n_outliers: int) -> dict:
+    s = Sizes()
+    _check(_L.spectra_packed_sizes(n, k, n_outliers, ctypes.byref(s)), "spectra_packed_sizes")
+    return {"n_pad": s.n_pad, "codes": s.codes_bytes, "scales": s.scales_bytes,
+            "zeros": s.zeros_bytes, "outlier_idx": s.outlier_idx_bytes,
+            "outlier_w": s.outlier_w_bytes}
+
+
+def spectra_pack_plan(w: torch.Tensor, gain: torch.Tensor | None, tau: float, *,
+                      want_kappa: bool = False, stream=None):
+    """Kurtosis split.  Returns (idx int32 [n_o], kappa float64 [k] or None)."""
+    n, k = w.shape
+    dev = w.device
+    kappa = torch.empty(k, dtype=torch.float64, device=dev) if want_kappa else None
+    idx = torch.empty(max(k, 1), dtype=torch.int32, device=dev)
+    ws_bytes = _L.spectra_pack_plan_workspace_size(k)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    n_o = ctypes.c_int32(0)
+    _check(_L.spectra_pack_plan(_ptr(w), _ptr(gain), n, k, float(tau), _ptr(kappa), _ptr(idx),
+                                ctypes.byref(n_o), _ptr(ws), ws_bytes, _stream(stream)),
+           "spectra_pack_plan")
+    return idx[: n_o.value], kappa
+
+
+@dataclass
+class PackedLayer:
+    """Device buffers of one packed layer plus the C view over them."""
+    n: int
+    k: int
+    n_outliers: int
+    codes: torch.Tensor        # uint8
+    scales: torch.Tensor       # int16 storage of FP16 bits
+    zeros: torch.Tensor        # int32 storage of u32 words
+    outlier_idx: torch.Tensor  # int32
+    outlier_w: torch.Tensor    # int16 storage of BF16 bits
+
+    def view(self) -> Layer:
+        return Layer(self.n, self.k, self.n_outliers, _ptr(self.codes), _ptr(self.scales),
+                     _ptr(self.zeros), _ptr(self.outlier_idx) if self.n_outliers else None,
+                     _ptr(self.outlier_w) if self.n_outliers else None)
+
+    @property
+    def nbytes(self) -> int:
+        """Bytes a matvec streams from these buffers (codes, scales, zeros,
+        outlier weights and indices)."""
+        return (self.codes.numel() + 2 * self.scales.numel() + 4 * self.zeros.numel()
+                + 4 * self.n_outliers + 2 * self.outlier_w.numel())
+
+
+def _alloc(nbytes: int, dtype, dev):
+    item = torch.empty((), dtype=dtype).element_size()
+    return torch.zeros(max(nbytes // item, 1), dtype=dtype, device=dev)
+
+
+def spectra_pack(w: torch.Tensor, idx: torch.Tensor, *, stream=None) -> PackedLayer:
+    """Quantise and pack W given the outlier indices from spectra_pack_plan."""
+    n, k = w.shape
+    n_o = int(idx.numel())
+    dev = w.device
+    sz = spectra_packed_sizes(n, k, n_o)
+    codes = _alloc(sz["codes"], torch.uint8, dev)
+    scales = _alloc(sz["scales"], torch.int16, dev)
+    zeros = _alloc(sz["zeros"], torch.int32, dev)
+    outw = _alloc(sz["outlier_w"], torch.int16, dev)
+    idx_c = idx.contiguous() if n_o else torch.zeros(1, dtype=torch.int32, device=dev)
+    ws_bytes = _L.spectra_pack_workspace_size()
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    view = Layer()
+    _check(_L.spectra_pack(_ptr(w), n, k, _ptr(idx_c) if n_o else None, n_o, _ptr(codes),
+                           _ptr(scales), _ptr(zeros), _ptr(outw) if n_o else None, _ptr(ws),
+                           ws_bytes, ctypes.byref(view), _stream(stream)), "spectra_pack")
+    return PackedLayer(n, k, n_o, codes, scales, zeros, idx_c, outw)
+
+
+def pack_layer(w: torch.Tensor, gain: torch.Tensor | None, tau: float, *, stream=None):
+    """spectra_pack_plan followed by spectra_pack."""
+    idx, _ = spectra_pack_plan(w, gain, tau, stream=stream)
+    return spectra_pack(w, idx, stream=stream)
+
+
+def spectra_unpack(layer: PackedLayer, *, stream=None):
+    """Canonical (codes u8 [n,k], scales int16-bits [n,k/32], zeros u8 [n,k/32])."""
+    dev = layer.codes.device
+    G = layer.k // 32
+    codes = torch.empty((layer.n, layer.k), dtype=torch.uint8, device=dev)
+    scales = torch.empty((layer.n, G), dtype=torch.int16, device=dev)
+    zeros = torch.empty((layer.n, G), dtype=torch.uint8, device=dev)
+    v = layer.view()
+    _check(_L.spectra_unpack(ctypes.byref(v), _ptr(codes), _ptr(scales), _ptr(zeros),
+                             _stream(stream)), "spectra_unpack")
+    return codes, scales, zeros
+
+
+_DT = {torch.float32: _lib.F32, torch.bfloat16: _lib.BF16}
+
+
+def spectra_gemv(layer: PackedLayer, x: torch.Tensor, y: torch.Tensor | None = None, *,
+                 y_dtype=torch.float32, view: Layer | None = None, stream=None) -> torch.Tensor:
+    """y = W_hat x for one BF16 vector x [k]."""
+    if y is None:
+        y = torch.empty(layer.n, dtype=y_dtype, device=x.device)
+    v = layer.view() if view is None else view
+    _check(_L.spectra_gemv(ctypes.byref(v), _ptr(x), _ptr(y), _DT[y.dtype], _stream(stream)),
+           "spectra_gemv")
+    return y
+
+
+def spectra_gemm_small(layer: PackedLayer, x: torch.Tensor, y: torch.Tensor | None = None, *,
+                       y_dtype=torch.float32, view: Layer | None = None,
+                       stream=None) -> torch.Tensor:
+    """y [m, n] = x [m, k] W_hat^T for 1 <= m <= 32."""
+    m = x.shape[0]
+    if y is None:
+        y = torch.empty((m, layer.n), dtype=y_dtype, device=x.device)
+    v = layer.view() if view is None else view
+    _check(_L.spectra_gemm_small(ctypes.byref(v), _ptr(x), m, _ptr(y), _DT[y.dtype],
+                                 _stream(stream)), "spectra_gemm_small")
+    return y

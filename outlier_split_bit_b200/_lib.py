@@ -1,0 +1,73 @@
+"""ctypes declarations of the C ABI in include/spectra.h (no logic here)."""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libspectra.so")
+
+# spectra_status values
+OK = 0
+ERR_INVALID_ARG = 1
+ERR_SHAPE = 2
+ERR_ALIGN = 3
+ERR_NONFINITE = 4
+ERR_RANGE = 5
+ERR_BUFFER_TOO_SMALL = 6
+ERR_CUDA = 7
+ERR_UNSUPPORTED = 8
+ERR_INTERNAL = 9
+
+F32 = 0
+BF16 = 1
+
+
+class Layer(ctypes.Structure):
+    """spectra_layer: a view of caller-owned device buffers."""
+    _fields_ = [("n", ctypes.c_int32), ("k", ctypes.c_int32), ("n_outliers", ctypes.c_int32),
+                ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("zeros", ctypes.c_void_p),
+                ("outlier_idx", ctypes.c_void_p), ("outlier_w", ctypes.c_void_p)]
+
+
+class Sizes(ctypes.Structure):
+    _fields_ = [("n_pad", ctypes.c_int64), ("codes_bytes", ctypes.c_size_t),
+                ("scales_bytes", ctypes.c_size_t), ("zeros_bytes", ctypes.c_size_t),
+                ("outlier_idx_bytes", ctypes.c_size_t), ("outlier_w_bytes", ctypes.c_size_t)]
+
+
+# name -> (restype, argtypes), mirroring spectra.h
+P = ctypes.c_void_p
+i32, f64, sz = ctypes.c_int32, ctypes.c_double, ctypes.c_size_t
+LP = ctypes.POINTER(Layer)
+SIGNATURES = {
+    "spectra_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "spectra_version": (i32, []),
+    "spectra_packed_sizes": (ctypes.c_int, [i32, i32, i32, ctypes.POINTER(Sizes)]),
+    "spectra_pack_plan_workspace_size": (sz, [i32]),
+    "spectra_pack_workspace_size": (sz, []),
+    "spectra_pack_plan": (ctypes.c_int, [P, P, i32, i32, f64, P, P, ctypes.POINTER(i32), P, sz, P]),
+    "spectra_pack": (ctypes.c_int, [P, i32, i32, P, i32, P, P, P, P, P, sz, LP, P]),
+    "spectra_unpack": (ctypes.c_int, [LP, P, P, P, P]),
+    "spectra_gemv": (ctypes.c_int, [LP, P, P, ctypes.c_int, P]),
+    "spectra_gemm_small": (ctypes.c_int, [LP, P, i32, P, ctypes.c_int, P]),
+}
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libspectra.so from the package directory; raise if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with `python -m outlier_split_bit_b200.build` "
+                "(there is no fallback implementation)")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib

@@ -1,0 +1,233 @@
+// api.cu -- extern "C" entry points declared in spectra.h.
+//
+// Every entry point validates its arguments on the host before it touches
+// CUDA, so argument errors return without launching anything and can be
+// tested on a machine without a GPU.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "internal.cuh"
+#include "spectra.h"
+
+namespace spectra {
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_dev_mutex;
+bool g_dev_valid[kMaxDevices];
+DeviceInfo g_dev_info[kMaxDevices];
+spectra_status g_dev_status[kMaxDevices];
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+spectra_status check_shape(int32_t n, int32_t k) {
+    if (n < 1 || k < 32 || (k % 32) != 0) return SPECTRA_ERR_SHAPE;
+    // keep every element index below 2^31 per matrix dimension product
+    if ((int64_t)n * (int64_t)k > ((int64_t)1 << 40)) return SPECTRA_ERR_SHAPE;
+    return SPECTRA_OK;
+}
+
+spectra_status check_layer(const spectra_layer *l) {
+    if (!l) return SPECTRA_ERR_INVALID_ARG;
+    spectra_status st = check_shape(l->n, l->k);
+    if (st != SPECTRA_OK) return st;
+    if (l->n_outliers < 0 || l->n_outliers > l->k) return SPECTRA_ERR_INVALID_ARG;
+    if (!l->codes || !l->scales || !l->zeros) return SPECTRA_ERR_INVALID_ARG;
+    if (l->n_outliers > 0 && (!l->outlier_idx || !l->outlier_w)) return SPECTRA_ERR_INVALID_ARG;
+    if (!aligned16(l->codes) || !aligned16(l->scales) || !aligned16(l->zeros))
+        return SPECTRA_ERR_ALIGN;
+    if (l->n_outliers > 0 && (!aligned16(l->outlier_w) || !aligned4(l->outlier_idx)))
+        return SPECTRA_ERR_ALIGN;
+    return SPECTRA_OK;
+}
+}  // namespace
+
+spectra_status current_device(DeviceInfo *out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SPECTRA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return SPECTRA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!g_dev_valid[dev]) {
+        DeviceInfo d = {};
+        d.device = dev;
+        int optin = 0;
+        if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+            return SPECTRA_ERR_CUDA;
+        d.smem_optin = (size_t)optin;
+        g_dev_info[dev] = d;
+        g_dev_status[dev] =
+            (d.cc_major == 10 && d.cc_minor == 0) ? SPECTRA_OK : SPECTRA_ERR_UNSUPPORTED;
+        g_dev_valid[dev] = true;
+    }
+    *out = g_dev_info[dev];
+    return g_dev_status[dev];
+}
+
+}  // namespace spectra
+
+using namespace spectra;
+
+extern "C" {
+
+const char *spectra_status_string(spectra_status s) {
+    switch (s) {
+        case SPECTRA_OK: return "ok";
+        case SPECTRA_ERR_INVALID_ARG: return "invalid argument";
+        case SPECTRA_ERR_SHAPE: return "unsupported shape";
+        case SPECTRA_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case SPECTRA_ERR_NONFINITE: return "non-finite value in weights or gain";
+        case SPECTRA_ERR_RANGE: return "group scale overflows FP16";
+        case SPECTRA_ERR_BUFFER_TOO_SMALL: return "workspace too small";
+        case SPECTRA_ERR_CUDA: return "CUDA runtime error";
+        case SPECTRA_ERR_UNSUPPORTED: return "device is not compute capability 10.0";
+        case SPECTRA_ERR_INTERNAL: return "internal error";
+    }
+    return "unknown status";
+}
+
+int32_t spectra_version(void) { return 100; }
+
+spectra_status spectra_packed_sizes(int32_t n, int32_t k, int32_t n_outliers, spectra_sizes *out) {
+    if (!out) return SPECTRA_ERR_INVALID_ARG;
+    spectra_status st = check_shape(n, k);
+    if (st != SPECTRA_OK) return st;
+    if (n_outliers < 0 || n_outliers > k) return SPECTRA_ERR_INVALID_ARG;
+    const Geometry g = Geometry::of(n, k, n_outliers);
+    const int64_t np = (int64_t)g.T * 32;
+    out->n_pad = np;
+    out->codes_bytes = (size_t)(np * k / 2);
+    out->scales_bytes = (size_t)(np * g.S * 8 * 2);
+    out->zeros_bytes = (size_t)(np * g.S * 4);
+    out->outlier_idx_bytes = (size_t)n_outliers * 4;
+    out->outlier_w_bytes = (size_t)(np * g.O8 * 8 * 2);
+    return SPECTRA_OK;
+}
+
+size_t spectra_pack_plan_workspace_size(int32_t k) {
+    if (k < 0) return 0;
+    return ((size_t)k * sizeof(double) + 255u) / 256u * 256u + 256u;
+}
+
+size_t spectra_pack_workspace_size(void) { return 256u; }
+
+spectra_status spectra_pack_plan(const uint16_t *w, const float *gain, int32_t n, int32_t k,
+                                 double tau, double *kappa_out, int32_t *idx_out,
+                                 int32_t *n_outliers_out, void *workspace,
+                                 size_t workspace_bytes, void *stream) {
+    if (!w || !idx_out || !n_outliers_out || !workspace) return SPECTRA_ERR_INVALID_ARG;
+    spectra_status st = check_shape(n, k);
+    if (st != SPECTRA_OK) return st;
+    if (tau != tau) return SPECTRA_ERR_INVALID_ARG;
+    if (!aligned16(w) || !aligned16(workspace) || !aligned4(idx_out) ||
+        (gain && !aligned4(gain)) || (kappa_out && ((uintptr_t)kappa_out & 7u)))
+        return SPECTRA_ERR_ALIGN;
+    if (workspace_bytes < spectra_pack_plan_workspace_size(k)) return SPECTRA_ERR_BUFFER_TOO_SMALL;
+    DeviceInfo dev;
+    st = current_device(&dev);
+    if (st != SPECTRA_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    char *ws = (char *)workspace;
+    const size_t kap_bytes = ((size_t)k * sizeof(double) + 255u) / 256u * 256u;
+    double *kappa = kappa_out ? kappa_out : (double *)ws;
+    int *words = (int *)(ws + kap_bytes);  // [0] error bits, [1] outlier count
+    if (cudaMemsetAsync(words, 0, 2 * sizeof(int), s) != cudaSuccess) return SPECTRA_ERR_CUDA;
+    if (launch_kurtosis(w, gain, n, k, kappa, words, s) != cudaSuccess) return SPECTRA_ERR_CUDA;
+    if (launch_split(kappa, k, tau, idx_out, words + 1, s) != cudaSuccess) return SPECTRA_ERR_CUDA;
+    int host[2] = {0, 0};
+    if (cudaMemcpyAsync(host, words, sizeof host, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return SPECTRA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SPECTRA_ERR_CUDA;
+    if (host[0] & kErrNonfinite) return SPECTRA_ERR_NONFINITE;
+    if (host[1] < 0 || host[1] > k) return SPECTRA_ERR_INTERNAL;
+    *n_outliers_out = host[1];
+    return SPECTRA_OK;
+}
+
+spectra_status spectra_pack(const uint16_t *w, int32_t n, int32_t k, const int32_t *idx,
+                            int32_t n_outliers, uint8_t *codes, uint16_t *scales,
+                            uint32_t *zeros, uint16_t *outlier_w, void *workspace,
+                            size_t workspace_bytes, spectra_layer *layer_out, void *stream) {
+    if (!w || !codes || !scales || !zeros || !workspace) return SPECTRA_ERR_INVALID_ARG;
+    spectra_status st = check_shape(n, k);
+    if (st != SPECTRA_OK) return st;
+    if (n_outliers < 0 || n_outliers > k) return SPECTRA_ERR_INVALID_ARG;
+    if (n_outliers > 0 && (!idx || !outlier_w)) return SPECTRA_ERR_INVALID_ARG;
+    if (!aligned16(w) || !aligned16(codes) || !aligned16(scales) || !aligned16(zeros) ||
+        !aligned16(workspace) || (n_outliers > 0 && (!aligned16(outlier_w) || !aligned4(idx))))
+        return SPECTRA_ERR_ALIGN;
+    if (workspace_bytes < spectra_pack_workspace_size()) return SPECTRA_ERR_BUFFER_TOO_SMALL;
+    DeviceInfo dev;
+    st = current_device(&dev);
+    if (st != SPECTRA_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    const Geometry g = Geometry::of(n, k, n_outliers);
+    int *err = (int *)workspace;
+    if (cudaMemsetAsync(err, 0, sizeof(int), s) != cudaSuccess) return SPECTRA_ERR_CUDA;
+    if (launch_quantize_pack(w, g, n_outliers > 0 ? idx : nullptr, codes, scales, zeros, err, s) !=
+        cudaSuccess)
+        return SPECTRA_ERR_CUDA;
+    if (launch_outlier_gather(w, g, idx, outlier_w, s) != cudaSuccess) return SPECTRA_ERR_CUDA;
+    int host = 0;
+    if (cudaMemcpyAsync(&host, err, sizeof host, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return SPECTRA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SPECTRA_ERR_CUDA;
+    if (host & kErrBadIndex) return SPECTRA_ERR_INVALID_ARG;
+    if (host & kErrNonfinite) return SPECTRA_ERR_NONFINITE;
+    if (host & kErrRange) return SPECTRA_ERR_RANGE;
+    if (layer_out) {
+        layer_out->n = n;
+        layer_out->k = k;
+        layer_out->n_outliers = n_outliers;
+        layer_out->codes = codes;
+        layer_out->scales = scales;
+        layer_out->zeros = zeros;
+        layer_out->outlier_idx = idx;
+        layer_out->outlier_w = outlier_w;
+    }
+    return SPECTRA_OK;
+}
+
+spectra_status spectra_unpack(const spectra_layer *layer, uint8_t *codes, uint16_t *scales,
+                              uint8_t *zeros, void *stream) {
+    spectra_status st = check_layer(layer);
+    if (st != SPECTRA_OK) return st;
+    if (!codes || !scales || !zeros) return SPECTRA_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    st = current_device(&dev);
+    if (st != SPECTRA_OK) return st;
+    if (launch_unpack(*layer, codes, scales, zeros, (cudaStream_t)stream) != cudaSuccess)
+        return SPECTRA_ERR_CUDA;
+    return SPECTRA_OK;
+}
+
+static spectra_status matvec(const spectra_layer *layer, const uint16_t *x, int32_t m, void *y,
+                             spectra_dtype y_dtype, void *stream) {
+    spectra_status st = check_layer(layer);
+    if (st != SPECTRA_OK) return st;
+    if (!x || !y) return SPECTRA_ERR_INVALID_ARG;
+    if (y_dtype != SPECTRA_F32 && y_dtype != SPECTRA_BF16) return SPECTRA_ERR_INVALID_ARG;
+    if (m < 1 || m > 32) return SPECTRA_ERR_SHAPE;
+    if (!aligned16(x)) return SPECTRA_ERR_ALIGN;
+    if (y_dtype == SPECTRA_F32 ? !aligned4(y) : ((uintptr_t)y & 1u)) return SPECTRA_ERR_ALIGN;
+    DeviceInfo dev;
+    st = current_device(&dev);
+    if (st != SPECTRA_OK) return st;
+    return launch_gemv(*layer, x, m, y, (int)y_dtype, (cudaStream_t)stream, dev);
+}
+
+spectra_status spectra_gemv(const spectra_layer *layer, const uint16_t *x, void *y,
+                            spectra_dtype y_dtype, void *stream) {
+    return matvec(layer, x, 1, y, y_dtype, stream);
+}
+
+spectra_status spectra_gemm_small(const spectra_layer *layer, const uint16_t *x, int32_t m_rows,
+                                  void *y, spectra_dtype y_dtype, void *stream) {
+    return matvec(layer, x, m_rows, y, y_dtype, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,68 @@
+// internal.cuh -- declarations shared by the library's translation units.
+// Device-side helpers and host launchers of the sm_100a kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "spectra.h"
+
+namespace spectra {
+
+// Bits of the device status word written by the packing kernels.
+enum : int {
+    kErrNonfinite = 1,   // NaN / infinity in W or gain
+    kErrRange = 2,       // a group's FP16 scale is infinite
+    kErrBadIndex = 4,    // outlier index outside [0, k) or not ascending
+};
+
+struct DeviceInfo {
+    int device;
+    int sm_count;
+    int cc_major, cc_minor;
+    size_t smem_optin;   // max dynamic shared memory per block (opt-in)
+};
+
+// Cached per-device properties of the current device.  Returns
+// SPECTRA_ERR_UNSUPPORTED unless the device is compute capability 10.0.
+spectra_status current_device(DeviceInfo *out);
+
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Geometry of the RT32 layout.
+struct Geometry {
+    int n, k, n_o;
+    int T;      // row tiles of 32
+    int G;      // groups of 32 columns
+    int S;      // super-groups of 8 groups
+    int O8;     // outlier octets
+    static Geometry of(int n, int k, int n_o) {
+        Geometry g;
+        g.n = n; g.k = k; g.n_o = n_o;
+        g.T = (int)cdiv(n, 32);
+        g.G = k / 32;
+        g.S = (int)cdiv(g.G, 8);
+        g.O8 = (int)cdiv(n_o, 8);
+        return g;
+    }
+};
+
+// ---- packing (pack.cu) ----
+cudaError_t launch_kurtosis(const uint16_t *w, const float *gain, int n, int k, double *kappa,
+                            int *err, cudaStream_t s);
+cudaError_t launch_split(const double *kappa, int k, double tau, int32_t *idx, int *count,
+                         cudaStream_t s);
+cudaError_t launch_quantize_pack(const uint16_t *w, const Geometry &g, const int32_t *idx,
+                                 uint8_t *codes, uint16_t *scales, uint32_t *zeros, int *err,
+                                 cudaStream_t s);
+cudaError_t launch_outlier_gather(const uint16_t *w, const Geometry &g, const int32_t *idx,
+                                  uint16_t *outlier_w, cudaStream_t s);
+cudaError_t launch_unpack(const spectra_layer &l, uint8_t *codes, uint16_t *scales, uint8_t *zeros,
+                          cudaStream_t s);
+
+// ---- matvec (gemv.cu) ----
+// CUDA-core decode matvec for 1 <= m <= 15 batch rows.
+spectra_status launch_gemv(const spectra_layer &l, const uint16_t *x, int m, void *y, int ytype,
+                           cudaStream_t s, const DeviceInfo &dev);
+
+}  // namespace spectra

@@ -1,0 +1,141 @@
+"""The C-ABI library loads and exports every symbol that include/spectra.h
+declares; host-side argument checks return their status without a GPU.
+
+No test here launches work: every call below fails validation before the
+library touches CUDA, so these run on machines without a GPU as well.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from outlier_split_bit_b200 import _lib
+from outlier_split_bit_b200 import build as libbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "spectra.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    libbuild.build()
+    return _lib.load()
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"SPECTRA_API\s+[^;(]*?\b(spectra_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for must in ["spectra_pack_plan", "spectra_pack", "spectra_unpack", "spectra_gemv",
+                 "spectra_gemm_small", "spectra_packed_sizes", "spectra_status_string"]:
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    names = _declared()
+    assert names
+    for name in names:
+        assert hasattr(L, name), name
+    assert set(names) <= set(_lib.SIGNATURES)
+
+
+def test_status_strings(L):
+    for s in range(10):
+        assert L.spectra_status_string(s)
+    assert L.spectra_status_string(99) == b"unknown status"
+    assert L.spectra_version() >= 100
+
+
+def test_packed_sizes(L):
+    s = _lib.Sizes()
+    assert L.spectra_packed_sizes(512, 512, 10, ctypes.byref(s)) == _lib.OK
+    assert s.n_pad == 512 and s.codes_bytes == 512 * 256 and s.scales_bytes == 512 * 2 * 2 * 8
+    assert s.zeros_bytes == 512 * 2 * 4 and s.outlier_w_bytes == 512 * 16 * 2
+    assert s.outlier_idx_bytes == 40
+    assert L.spectra_packed_sizes(40, 96, 0, ctypes.byref(s)) == _lib.OK
+    assert s.n_pad == 64 and s.scales_bytes == 64 * 8 * 2 and s.outlier_w_bytes == 0
+    assert L.spectra_packed_sizes(0, 512, 0, ctypes.byref(s)) == _lib.ERR_SHAPE
+    assert L.spectra_packed_sizes(8, 48, 0, ctypes.byref(s)) == _lib.ERR_SHAPE
+    assert L.spectra_packed_sizes(8, 64, 65, ctypes.byref(s)) == _lib.ERR_INVALID_ARG
+    assert L.spectra_packed_sizes(8, 64, 1, None) == _lib.ERR_INVALID_ARG
+
+
+def test_workspace_sizes(L):
+    assert L.spectra_pack_plan_workspace_size(3072) >= 3072 * 8 + 8
+    assert L.spectra_pack_workspace_size() >= 4
+
+
+FAKE = 0x10000  # never dereferenced: every call below fails its checks first
+
+
+def _layer(n=64, k=128, n_o=0, off=0):
+    return _lib.Layer(n, k, n_o, FAKE + off, FAKE, FAKE, FAKE if n_o else None,
+                      FAKE if n_o else None)
+
+
+def test_gemv_argument_checks(L):
+    y = FAKE
+    assert L.spectra_gemv(None, FAKE, y, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.spectra_gemv(ctypes.byref(_layer(k=100)), FAKE, y, 0, None) == _lib.ERR_SHAPE
+    assert L.spectra_gemv(ctypes.byref(_layer(n=0)), FAKE, y, 0, None) == _lib.ERR_SHAPE
+    assert L.spectra_gemv(ctypes.byref(_layer(off=8)), FAKE, y, 0, None) == _lib.ERR_ALIGN
+    assert L.spectra_gemv(ctypes.byref(_layer()), FAKE + 2, y, 0, None) == _lib.ERR_ALIGN
+    assert L.spectra_gemv(ctypes.byref(_layer()), FAKE, FAKE + 2, 0, None) == _lib.ERR_ALIGN
+    assert L.spectra_gemv(ctypes.byref(_layer()), None, y, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.spectra_gemv(ctypes.byref(_layer()), FAKE, y, 7, None) == _lib.ERR_INVALID_ARG
+    bad = _lib.Layer(64, 128, 3, FAKE, FAKE, FAKE, None, None)
+    assert L.spectra_gemv(ctypes.byref(bad), FAKE, y, 0, None) == _lib.ERR_INVALID_ARG
+    bad = _lib.Layer(64, 128, 200, FAKE, FAKE, FAKE, FAKE, FAKE)
+    assert L.spectra_gemv(ctypes.byref(bad), FAKE, y, 0, None) == _lib.ERR_INVALID_ARG
+
+
+def test_gemm_small_argument_checks(L):
+    lay = ctypes.byref(_layer())
+    assert L.spectra_gemm_small(lay, FAKE, 0, FAKE, 0, None) == _lib.ERR_SHAPE
+    assert L.spectra_gemm_small(lay, FAKE, 33, FAKE, 0, None) == _lib.ERR_SHAPE
+    assert L.spectra_gemm_small(lay, FAKE + 4, 4, FAKE, 0, None) == _lib.ERR_ALIGN
+
+
+def test_pack_argument_checks(L):
+    n_o = ctypes.c_int32(-1)
+    ws = L.spectra_pack_plan_workspace_size(128)
+    assert L.spectra_pack_plan(None, None, 8, 128, 3.0, None, FAKE, ctypes.byref(n_o), FAKE, ws,
+                               None) == _lib.ERR_INVALID_ARG
+    assert L.spectra_pack_plan(FAKE, None, 8, 120, 3.0, None, FAKE, ctypes.byref(n_o), FAKE, ws,
+                               None) == _lib.ERR_SHAPE
+    assert L.spectra_pack_plan(FAKE, None, 8, 128, float("nan"), None, FAKE, ctypes.byref(n_o),
+                               FAKE, ws, None) == _lib.ERR_INVALID_ARG
+    assert L.spectra_pack_plan(FAKE + 2, None, 8, 128, 3.0, None, FAKE, ctypes.byref(n_o), FAKE,
+                               ws, None) == _lib.ERR_ALIGN
+    assert L.spectra_pack_plan(FAKE, None, 8, 128, 3.0, None, FAKE, ctypes.byref(n_o), FAKE,
+                               ws - 1, None) == _lib.ERR_BUFFER_TOO_SMALL
+    assert n_o.value == -1  # outputs untouched
+    wsb = L.spectra_pack_workspace_size()
+    assert L.spectra_pack(FAKE, 8, 128, None, 2, FAKE, FAKE, FAKE, FAKE, FAKE, wsb, None,
+                          None) == _lib.ERR_INVALID_ARG
+    assert L.spectra_pack(FAKE, 8, 128, None, 0, FAKE, FAKE + 4, FAKE, None, FAKE, wsb, None,
+                          None) == _lib.ERR_ALIGN
+    assert L.spectra_pack(FAKE, 8, 128, None, 0, FAKE, FAKE, FAKE, None, FAKE, 0, None,
+                          None) == _lib.ERR_BUFFER_TOO_SMALL
+    assert L.spectra_unpack(None, FAKE, FAKE, FAKE, None) == _lib.ERR_INVALID_ARG
+
+
+def test_binding_mirrors_the_abi_names():
+    import outlier_split_bit_b200 as sp
+    for name in ["spectra_pack_plan", "spectra_pack", "spectra_unpack", "spectra_gemv",
+                 "spectra_gemm_small", "spectra_packed_sizes", "spectra_status_string"]:
+        assert callable(getattr(sp, name))
+
+
+def test_product_path_does_not_reference_the_oracle():
+    pkg = os.path.join(ROOT, "outlier_split_bit_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "spectra_ref" not in text, f

@@ -1,0 +1,280 @@
+"""CUDA path vs the CPU oracle: packing bit-exact, matvec within tolerance.
+
+Method: "SPECTRA: Sparse-Precision Exact Channel Tensor Reconstruction
+Architecture" (Dev.to abstract), abstract paragraph.  The tolerance of the
+matvec, |y - y_ref| <= 2e-3 * sum_j |w_hat_ij x_j| + 1e-5, is the acceptance
+rule of the build; packing outputs (kurtosis, outlier indices, codes,
+scales, zero points, outlier block) must be identical bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import outlier_split_bit_b200 as sp
+from outlier_split_bit_b200 import workload as wl
+
+from gpu_helpers import (DEV, check_gemv, draw, np_gain, oracle_rows, tile_slices, u8, u16, u32)
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    (wl.SINGLE_512, 3.0, True),
+    (wl.SINGLE_512, 6.0, True),
+    (wl.MatrixSpec("single", 40, 96, 3), 1.2, False),
+    (wl.MatrixSpec("single", 7, 352, 17), 3.0, True),
+    (wl.MatrixSpec("single", 1, 32, 0), 3.0, False),
+    (wl.MatrixSpec("single", 33, 64, 2), -np.inf, True),
+    (wl.MatrixSpec("single", 100, 2080, 31), 6.0, True),
+    (wl.MatrixSpec("single", 96, 256, 4), np.inf, True),
+]
+SMALL_IDS = [f"{s.n}x{s.k}-tau{t}" for s, t, _ in SMALL]
+
+
+def _full_pack(spec, tau, with_gain, seed=0, layer=0, m=1):
+    w, g, x = draw(spec, seed, layer, m, with_gain)
+    idx, kappa = sp.spectra_pack_plan(w, g, tau, want_kappa=True)
+    lay = sp.spectra_pack(w, idx)
+    wb = wl.bits(w)
+    ref = oracle.pack(wb, np_gain(g), tau)
+    return w, g, x, idx, kappa, lay, wb, ref
+
+
+@pytest.mark.parametrize("spec,tau,with_gain", SMALL, ids=SMALL_IDS)
+def test_pack_bit_exact_small(spec, tau, with_gain):
+    w, g, x, idx, kappa, lay, wb, ref = _full_pack(spec, tau, with_gain)
+    assert np.array_equal(kappa.cpu().numpy().view(np.uint64), ref.kappa.view(np.uint64))
+    assert np.array_equal(idx.cpu().numpy(), ref.idx)
+    p = ref.packed
+    assert np.array_equal(u8(lay.codes)[: p.codes.size], p.codes)
+    assert np.array_equal(u16(lay.scales)[: p.scales.size], p.scales)
+    assert np.array_equal(u32(lay.zeros)[: p.zeros.size], p.zeros)
+    if ref.idx.size:
+        assert np.array_equal(u16(lay.outlier_w)[: p.outliers.size], p.outliers)
+    codes, scales, zeros = sp.spectra_unpack(lay)
+    assert np.array_equal(codes.cpu().numpy(), ref.can.codes)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint16), ref.can.scales)
+    assert np.array_equal(zeros.cpu().numpy(), ref.can.zeros)
+
+
+@pytest.mark.parametrize("spec,tau,with_gain", SMALL, ids=SMALL_IDS)
+@pytest.mark.parametrize("ydt", [torch.float32, torch.bfloat16])
+def test_gemv_small(spec, tau, with_gain, ydt):
+    w, g, x, idx, kappa, lay, wb, ref = _full_pack(spec, tau, with_gain)
+    y = sp.spectra_gemv(lay, x[0], y_dtype=ydt)
+    torch.cuda.synchronize()
+    y_ref, bound = oracle.gemm(ref.can, wb, ref.idx, wl.bits(x))
+    check_gemv(y, y_ref[0], bound[0], bf16=(ydt == torch.bfloat16))
+
+
+@pytest.mark.parametrize("spec", wl.LAYER_1P5B, ids=[s.name for s in wl.LAYER_1P5B])
+@pytest.mark.parametrize("tau", [3.0, 6.0])
+def test_decoder_layer_1p5b(spec, tau):
+    """All 7 projections of a 1.5B-class layer: packing bit-exact, matvec in tolerance."""
+    w, g, x, idx, kappa, lay, wb, ref = _full_pack(spec, tau, True, seed=0, layer=0)
+    assert np.array_equal(idx.cpu().numpy(), ref.idx)
+    assert np.array_equal(kappa.cpu().numpy().view(np.uint64), ref.kappa.view(np.uint64))
+    p = ref.packed
+    assert np.array_equal(u8(lay.codes), p.codes)
+    assert np.array_equal(u16(lay.scales), p.scales)
+    assert np.array_equal(u32(lay.zeros), p.zeros)
+    if ref.idx.size:
+        assert np.array_equal(u16(lay.outlier_w), p.outliers)
+    y = sp.spectra_gemv(lay, x[0])
+    torch.cuda.synchronize()
+    y_ref, bound = oracle.gemm(ref.can, wb, ref.idx, wl.bits(x))
+    check_gemv(y, y_ref[0], bound[0])
+
+
+def test_unit_vectors_extract_columns_exactly():
+    spec = wl.MatrixSpec("single", 200, 1024, 16)
+    w, g, x, idx, kappa, lay, wb, ref = _full_pack(spec, 6.0, True)
+    what = oracle.dequant(ref.can)
+    wv = wl.bits(w).view(np.uint16)
+    wvals = torch.from_numpy(wv.view(np.int16)).view(torch.bfloat16).double().numpy()
+    cols = [0, 1, 31, 32, 255, 256, 511, 1000, 1023] + ref.idx[:4].tolist()
+    for j in cols:
+        e = torch.zeros(1024, dtype=torch.bfloat16, device=DEV)
+        e[j] = 1.0
+        y = sp.spectra_gemv(lay, e).cpu().numpy().astype(np.float64)
+        expect = what[:, j] + (wvals[:, j] if j in ref.idx else 0.0)
+        assert np.array_equal(y, expect), j
+
+
+def test_zero_input_gives_zero():
+    spec = wl.MatrixSpec("single", 300, 512, 5)
+    w, g, x, idx, kappa, lay, wb, ref = _full_pack(spec, 6.0, True)
+    y = sp.spectra_gemv(lay, torch.zeros(512, dtype=torch.bfloat16, device=DEV))
+    assert torch.count_nonzero(y).item() == 0
+
+
+def test_deterministic_bitwise():
+    spec = wl.LAYER_1P5B[6]  # down: the cluster split-K path
+    w, g, x = draw(spec)
+    lay = sp.pack_layer(w, g, 6.0)
+    y1 = sp.spectra_gemv(lay, x[0]).clone()
+    for _ in range(5):
+        y2 = sp.spectra_gemv(lay, x[0])
+        assert torch.equal(y1.view(torch.int32), y2.view(torch.int32))
+
+
+@pytest.mark.parametrize("m", list(range(1, 16)))
+def test_gemm_small_cuda_core(m):
+    spec = wl.MatrixSpec("single", 512, 512, 10)
+    w, g, x, idx, kappa, lay, wb, ref = _full_pack(spec, 6.0, True, m=m)
+    y = sp.spectra_gemm_small(lay, x)
+    torch.cuda.synchronize()
+    y_ref, bound = oracle.gemm(ref.can, wb, ref.idx, wl.bits(x))
+    check_gemv(y, y_ref, bound)
+
+
+@pytest.mark.parametrize("spec", wl.LAYER_4B, ids=[s.name for s in wl.LAYER_4B])
+@pytest.mark.parametrize("m", [1, 2, 4, 8])
+def test_decoder_layer_4b_batch(spec, m):
+    """4B-class shapes: packing on sampled tiles, batched matvec on those rows."""
+    w, g, x = draw(spec, m=m)
+    idx, kappa = sp.spectra_pack_plan(w, g, 6.0, want_kappa=True)
+    lay = sp.spectra_pack(w, idx)
+    y = sp.spectra_gemm_small(lay, x)
+    torch.cuda.synchronize()
+    wb = wl.bits(w)
+    ref_idx = oracle.split(oracle.kurtosis(wb, np_gain(g)), 6.0)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+    T = lay.codes.numel() // ((spec.k // 32) * 512)
+    tiles = sorted({0, 1, T // 2, T - 1})
+    rows, can, packed = oracle_rows(wb, ref_idx, tiles)
+    got = tile_slices(lay, tiles)
+    for key in ("codes", "scales", "zeros", "outliers"):
+        assert np.array_equal(got[key], packed[key]), key
+    y_ref, bound = oracle.gemm(can, np.ascontiguousarray(wb[rows]), ref_idx, wl.bits(x))
+    check_gemv(y[:, rows], y_ref, bound)
+
+
+@pytest.mark.parametrize("frac", wl.LM_HEAD_FRACTIONS)
+def test_lm_head_full_size_sampled(frac):
+    """131072 x 3072 LM head: kurtosis on sampled columns, packing and matvec on
+    sampled tiles (the first two, a middle one and the last), in the launch
+    configuration of the benchmark."""
+    spec = wl.lm_head_spec(frac)
+    w, g, x = draw(spec)
+    idx, kappa = sp.spectra_pack_plan(w, g, 6.0, want_kappa=True)
+    lay = sp.spectra_pack(w, idx)
+    y = sp.spectra_gemv(lay, x[0])
+    torch.cuda.synchronize()
+    wb = wl.bits(w)
+    idx_np = idx.cpu().numpy()
+    kap = kappa.cpu().numpy()
+    assert np.array_equal(idx_np, np.flatnonzero(kap > 6.0))
+    rng = np.random.default_rng(0)
+    cols = np.unique(np.concatenate([rng.choice(spec.k, 48, replace=False), idx_np[:16]]))
+    gn = np_gain(g)
+    kref = oracle.kurtosis(np.ascontiguousarray(wb[:, cols]), None if gn is None else gn[cols])
+    assert np.array_equal(kap[cols].view(np.uint64), kref.view(np.uint64))
+    # heavy columns are found: at 131072 rows every Student-t(3) column passes
+    assert idx_np.size >= spec.n_t
+    T = spec.n // 32
+    tiles = [0, 1, T // 2, T - 1]
+    rows, can, packed = oracle_rows(wb, idx_np, tiles)
+    got = tile_slices(lay, tiles)
+    for key in ("codes", "scales", "zeros", "outliers"):
+        assert np.array_equal(got[key], packed[key]), key
+    y_ref, bound = oracle.gemm(can, np.ascontiguousarray(wb[rows]), idx_np, wl.bits(x))
+    check_gemv(y[rows], y_ref[0], bound[0])
+
+
+@pytest.mark.parametrize("n,k,m", [(64, 32768, 1), (64, 32768, 8), (32, 65536, 1), (96, 14336, 3)])
+def test_long_rows_use_cluster_split(n, k, m):
+    spec = wl.MatrixSpec("single", n, k, 40)
+    w, g, x, idx, kappa, lay, wb, ref = _full_pack(spec, 6.0, True, m=m)
+    y = sp.spectra_gemm_small(lay, x)
+    torch.cuda.synchronize()
+    y_ref, bound = oracle.gemm(ref.can, wb, ref.idx, wl.bits(x))
+    check_gemv(y, y_ref, bound)
+
+
+def test_graph_capture_and_replay():
+    spec = wl.LAYER_1P5B[4]
+    w, g, x = draw(spec)
+    lay = sp.pack_layer(w, g, 6.0)
+    y_eager = sp.spectra_gemv(lay, x[0]).clone()
+    y = torch.empty_like(y_eager)
+    view = lay.view()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(graph, stream=s):
+            sp.spectra_gemv(lay, x[0], y, view=view, stream=s)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_eager)
+
+
+def test_dependent_chain_reads_previous_output():
+    """y of one matvec is x of the next on the same stream: the programmatic
+    dependent launch must not let the second kernel read x early."""
+    spec = wl.MatrixSpec("q", 1536, 1536, 23)
+    layers = []
+    for i in range(6):
+        w, g, _ = draw(spec, seed=i)
+        layers.append(sp.pack_layer(w, g, 6.0))
+    x0 = wl.activations(1536, 1, seed=9, device=DEV)[0]
+    bufs = [torch.empty(1536, dtype=torch.bfloat16, device=DEV) for _ in range(7)]
+    bufs[0].copy_(x0)
+    for _ in range(3):
+        for i, lay in enumerate(layers):
+            sp.spectra_gemv(lay, bufs[i], bufs[i + 1])
+        torch.cuda.synchronize()
+        chained = bufs[-1].clone()
+        # the same steps with a full synchronisation between them
+        cur = x0.clone()
+        for lay in layers:
+            nxt = sp.spectra_gemv(lay, cur, y_dtype=torch.bfloat16)
+            torch.cuda.synchronize()
+            cur = nxt
+        assert torch.equal(chained, cur)
+
+
+def test_error_status_on_gpu():
+    w = torch.randn(64, 128, device=DEV).to(torch.bfloat16)
+    w[3, 5] = float("nan")
+    with pytest.raises(sp.SpectraError) as e:
+        sp.spectra_pack_plan(w, None, 3.0)
+    assert e.value.status == 4
+    with pytest.raises(sp.SpectraError) as e:
+        sp.spectra_pack(w, torch.empty(0, dtype=torch.int32, device=DEV))
+    assert e.value.status == 4
+    big = torch.zeros(32, 64, device=DEV, dtype=torch.bfloat16)
+    big[0, 0], big[0, 1] = 2.0 ** 20, -2.0 ** 20
+    with pytest.raises(sp.SpectraError) as e:
+        sp.spectra_pack(big, torch.empty(0, dtype=torch.int32, device=DEV))
+    assert e.value.status == 5
+    lay = sp.spectra_pack(big, torch.tensor([0, 1], dtype=torch.int32, device=DEV))
+    assert lay.n_outliers == 2
+    ok = torch.zeros(32, 64, device=DEV, dtype=torch.bfloat16)
+    for bad in ([5, 3], [64], [-1]):
+        with pytest.raises(sp.SpectraError) as e:
+            sp.spectra_pack(ok, torch.tensor(bad, dtype=torch.int32, device=DEV))
+        assert e.value.status == 1
+    g = torch.ones(128, device=DEV)
+    g[7] = float("inf")
+    with pytest.raises(sp.SpectraError) as e:
+        sp.spectra_pack_plan(torch.zeros(8, 128, device=DEV, dtype=torch.bfloat16), g, 3.0)
+    assert e.value.status == 4
+
+
+def test_matvec_allocates_nothing():
+    spec = wl.LAYER_1P5B[0]
+    w, g, x = draw(spec)
+    lay = sp.pack_layer(w, g, 6.0)
+    y = torch.empty(spec.n, device=DEV)
+    view = lay.view()
+    sp.spectra_gemv(lay, x[0], y, view=view)
+    torch.cuda.synchronize()
+    a0 = torch.cuda.memory_allocated()
+    r0 = torch.cuda.memory_reserved()
+    for _ in range(1000):
+        sp.spectra_gemv(lay, x[0], y, view=view)
+    torch.cuda.synchronize()
+    assert torch.cuda.memory_allocated() == a0
+    assert torch.cuda.memory_reserved() == r0
