@@ -5,9 +5,15 @@
 
 A step is one decode-step weight stream: 28 layers x 7 projections of a
 1.5B-class decoder (hidden 1536, intermediate 8960, KV width 256), one batch-1
-matvec per matrix with its own BF16 activation vector (196 launches, 1.31 G
-weights, 0.76 GB packed), captured once in a CUDA graph and replayed.  The
-packed weights exceed the 126 MB L2, so every step streams them from HBM.
+matvec per matrix with its own BF16 activation vector (196 matvecs, 1.31 G
+weights, 0.76 GB of packed bulk plus the BF16 outlier columns).  The
+activations of the synthetic stream are independent inputs, so the step is
+ONE spectra_gemv_batched launch that streams all 196 matrices in order
+(captured in a CUDA graph and replayed).  The same stream as a dependent
+chain -- 196 spectra_gemv launches where each may consume the previous
+output (programmatic dependent launch) -- is timed too and reported under
+"rows".  The packed weights exceed the 126 MB L2, so every step streams them
+from HBM.
 Rank 0 prints one JSON line.  For N > 1 every rank (one per GPU) runs its own
 replica of the stream: the problems are independent, there is no data-path
 collective, and the value is the bytes of all ranks over the slowest rank's
@@ -153,19 +159,26 @@ class Stream:
             self.n_outliers += lay.n_outliers
         self.launches = len(self.items)
 
-    def run(self, stream):
+        self.batch = sp.BatchViews([it[1] for it in self.items], [it[2] for it in self.items],
+                                   [it[3] for it in self.items])
+
+    def run(self, stream, mode):
+        if mode == "batched":
+            self.sp.spectra_gemv_batched(views=self.batch, stream=stream)
+            return 1
         for spec, lay, x, y, view in self.items:
             self.sp.spectra_gemv(lay, x, y, view=view, stream=stream)
+        return len(self.items)
 
-    def capture(self, stream):
+    def capture(self, stream, mode):
         g = torch.cuda.CUDAGraph()
         torch.cuda.synchronize()  # packing ran on the default stream
         with torch.cuda.stream(stream):
-            self.run(stream)  # warm: sets kernel attributes outside capture
+            self.run(stream, mode)  # warm: sets kernel attributes outside capture
             stream.synchronize()
             with torch.cuda.graph(g, stream=stream):
-                self.run(stream)
-        return g
+                launches = self.run(stream, mode)
+        return g, launches
 
 
 def flush_l2(buf):
@@ -374,7 +387,7 @@ def run_ours(args):
     peak = float(peaks["hbm_gbs"])
     stream = torch.cuda.Stream(device=device)
     st = Stream(device, seed=rank, tau=args.tau)
-    graph = st.capture(stream)
+    graph, launches_per_step = st.capture(stream, "batched")
     for _ in range(args.warmup):
         graph.replay()
     stream.synchronize()
@@ -424,9 +437,30 @@ def run_ours(args):
         e2e_ms = float(t.item())
     e2e_gbs = st.bytes * e2e_steps * world / (e2e_ms * 1e-3) * 1e-9
 
-    extra = {}
+    # the same stream as a dependent chain of 196 launches (graph + PDL)
+    chain_graph, chain_launches = st.capture(stream, "chain")
+    for _ in range(args.warmup):
+        chain_graph.replay()
+    stream.synchronize()
+    barrier()
+    chain_steps = max(1, args.steps // 2)
+    with torch.cuda.stream(stream):
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        for _ in range(chain_steps):
+            chain_graph.replay()
+        c1.record(stream)
+    c1.synchronize()
+    chain_ms = c0.elapsed_time(c1) / chain_steps
+    del chain_graph
+
+    extra = {"decode_stream_dependent_chain": {
+        "launches_per_step": chain_launches, "us_per_step": round(chain_ms * 1e3, 2),
+        "gbs": round(st.bytes / (chain_ms * 1e-3) * 1e-9, 1),
+        "frac": round(st.bytes / (chain_ms * 1e-3) * 1e-9 / peak, 4),
+        "us_per_launch": round(chain_ms * 1e3 / chain_launches, 3)}}
     if rank == 0 and not args.quick:
-        extra = extras(device, stream, peak, args.tau)
+        extra.update(extras(device, stream, peak, args.tau))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -442,8 +476,8 @@ def run_ours(args):
 
     digest = kernel_source_digest()
     traffic = profiled_traffic(digest)
-    launch_bytes = st.bytes / st.launches
-    launch_us = step_ms * 1e3 / st.launches
+    launch_bytes = st.bytes / launches_per_step
+    launch_us = step_ms * 1e3 / launches_per_step
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(gbs, 1), "unit": "GB/s", "n_gpus": world,
@@ -454,7 +488,8 @@ def run_ours(args):
             "data": "synthetic (seeded N(0,0.02) weights with Student-t(3) columns, N(0,1) x)",
             "config": {"workload": WORKLOAD, "matrices_per_step": st.launches,
                        "bytes_per_step": st.bytes, "n_outliers_per_step": st.n_outliers,
-                       "tau": args.tau, "m": 1, "launch": "CUDA graph of 196 spectra_gemv, PDL",
+                       "tau": args.tau, "m": 1,
+                       "launch": "one spectra_gemv_batched launch per step (CUDA graph replay)",
                        "l2": "inputs larger than L2 (0.76 GB of packed weights per step)",
                        "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "hbm", "achieved": round(launch_bytes / launch_us * 1e-3, 1),
@@ -465,7 +500,7 @@ def run_ours(args):
             "e2e": {"value": round(e2e_gbs, 1), "unit": "GB/s",
                     "h2d_bytes_per_step": st.x_all.numel() * 2,
                     "d2h_bytes_per_step": st.y_all.numel() * 4},
-            "gpu_launches": st.launches * args.steps,
+            "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
         }
@@ -478,6 +513,38 @@ def run_ours(args):
     return 0
 
 
+def run_single(args):
+    """One matrix (n x k, n_t Student-t columns), m batch rows, timed alone with
+    L2 flushed before every launch; prints one JSON line.  Used for per-matrix
+    numbers and as the small case of profiler captures."""
+    import outlier_split_bit_b200 as sp
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    peak = float(measured_peaks()["hbm_gbs"])
+    spec = wl.MatrixSpec("lm_head", args.n, args.k, args.nt)
+    w = wl.weight(spec, 0, 0, device=device)
+    g = wl.gain(spec, 0, 0, device=device)
+    lay = sp.pack_layer(w, g, args.tau)
+    del w
+    x = wl.activations(spec.k, args.m, device=device)
+    y = torch.empty((args.m, spec.n), device=device)
+    v = lay.view()
+    stream = torch.cuda.Stream(device=device)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+    fn = (lambda: sp.spectra_gemv(lay, x[0], y[0], view=v, stream=stream)) if args.m == 1 else \
+        (lambda: sp.spectra_gemm_small(lay, x, y, view=v, stream=stream))
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            fn()
+        us, p10, p90 = time_single(fn, stream, args.steps, flush)
+    b = algorithmic_bytes(spec.n, spec.k, lay.n_outliers, m=args.m)
+    print(json.dumps({"case": "single", "n": spec.n, "k": spec.k, "m": args.m, "tau": args.tau,
+                      "n_outliers": lay.n_outliers, "us": round(us, 2), "us_p10": round(p10, 2),
+                      "us_p90": round(p90, 2), "bytes": b, "gbs": round(b / us * 1e-3, 1),
+                      "frac": round(b / us * 1e-3 / peak, 4)}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -487,11 +554,19 @@ def main():
     ap.add_argument("--tau", type=float, default=3.0)
     ap.add_argument("--quick", action="store_true", help="skip the per-matrix / LM-head / batch rows")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", choices=["stream", "single"], default="stream",
+                    help="stream: the decode-step weight stream (the benchmark); single: one matrix")
+    ap.add_argument("--n", type=int, default=wl.LM_HEAD_N)
+    ap.add_argument("--k", type=int, default=wl.LM_HEAD_K)
+    ap.add_argument("--nt", type=int, default=0, help="Student-t columns of the single matrix")
+    ap.add_argument("--m", type=int, default=1)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.case == "single":
+        return run_single(args)
     return run_ours(args)
 
 

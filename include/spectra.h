@@ -81,6 +81,9 @@ typedef enum {
 
 typedef enum { SPECTRA_F32 = 0, SPECTRA_BF16 = 1 } spectra_dtype;
 
+/* Largest number of matvecs one spectra_gemv_batched call accepts. */
+#define SPECTRA_MAX_BATCH 224
+
 /* A packed layer: a plain view of caller-owned device buffers. */
 typedef struct {
     int32_t n;                   /* out_features */
@@ -202,6 +205,36 @@ SPECTRA_API spectra_status spectra_gemv(const spectra_layer *layer, const uint16
  */
 SPECTRA_API spectra_status spectra_gemm_small(const spectra_layer *layer, const uint16_t *x, int32_t m_rows,
                                   void *y, spectra_dtype y_dtype, void *stream);
+
+/*
+ * Many independent batch-1 matvecs in ONE launch: y[i] = W_i x[i] for
+ * i in [0, count), 1 <= count <= SPECTRA_MAX_BATCH, each with the formula,
+ * tolerance and output type of spectra_gemv.
+ *   layers  HOST array [count] of layer views (device buffers)
+ *   x       HOST array [count] of device pointers, BF16 bits [layers[i].k]
+ *   y       HOST array [count] of device pointers, [layers[i].n] of y_dtype
+ * The matvecs run concurrently: no y[i] may overlap any x[j] or another
+ * y[j].  This is the decode-step weight stream when the inputs of the
+ * matrices are all available (e.g. q/k/v of one layer sharing x, or the
+ * stream of a whole step whose activations are given); CTAs are issued in
+ * problem order, so the weights are streamed in that order.  The host arrays
+ * are read during the call only.  Asynchronous, allocates nothing,
+ * graph-capturable, programmatic dependent launch as spectra_gemv.
+ * Errors: INVALID_ARG, SHAPE, ALIGN, UNSUPPORTED, CUDA.
+ */
+SPECTRA_API spectra_status spectra_gemv_batched(const spectra_layer *layers,
+                                                const uint16_t *const *x, void *const *y,
+                                                int32_t count, spectra_dtype y_dtype,
+                                                void *stream);
+
+/*
+ * Health of the matvec kernels on the current device.  Their waits for the
+ * asynchronous weight copies are bounded: a wait that gives up raises a
+ * per-device flag instead of hanging, and the outputs of that launch are
+ * invalid.  Returns SPECTRA_ERR_INTERNAL if the flag was raised since the
+ * last call (and clears it), SPECTRA_OK otherwise.  Synchronous on `stream`.
+ */
+SPECTRA_API spectra_status spectra_device_status(void *stream);
 
 #ifdef __cplusplus
 }

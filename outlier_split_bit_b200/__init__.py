@@ -22,7 +22,8 @@ from ._lib import Layer, Sizes
 
 __all__ = ["SpectraError", "PackedLayer", "spectra_status_string", "spectra_version",
            "spectra_packed_sizes", "spectra_pack_plan", "spectra_pack", "spectra_unpack",
-           "spectra_gemv", "spectra_gemm_small", "pack_layer", "library"]
+           "spectra_gemv", "spectra_gemm_small", "spectra_gemv_batched", "spectra_device_status",
+           "pack_layer", "library"]
 
 class _Lazy:
     """Loads libspectra.so on first attribute access."""
@@ -68,6 +69,11 @@ def spectra_status_string(status: int) -> str:
 
 def spectra_version() -> int:
     return _L.spectra_version()
+
+
+def spectra_device_status(*, stream=None) -> None:
+    """Raise SpectraError if a bounded wait in a matvec kernel gave up."""
+    _check(_L.spectra_device_status(_stream(stream)), "spectra_device_status")
 
 
 def spectra_packed_sizes(n: int, k: int, n_outliers: int) -> dict:
@@ -188,3 +194,29 @@ def spectra_gemm_small(layer: PackedLayer, x: torch.Tensor, y: torch.Tensor | No
     _check(_L.spectra_gemm_small(ctypes.byref(v), _ptr(x), m, _ptr(y), _DT[y.dtype],
                                  _stream(stream)), "spectra_gemm_small")
     return y
+
+
+class BatchViews:
+    """Host arrays of layer views and device pointers for spectra_gemv_batched,
+    built once and reused (e.g. for graph capture)."""
+
+    def __init__(self, layers, xs, ys):
+        n = len(layers)
+        self.count = n
+        self.layers = (Layer * n)(*[l.view() for l in layers])
+        self.xs = (ctypes.c_void_p * n)(*[x.data_ptr() for x in xs])
+        self.ys = (ctypes.c_void_p * n)(*[y.data_ptr() for y in ys])
+        dts = {y.dtype for y in ys}
+        if len(dts) != 1:
+            raise ValueError("all outputs of one batched call share one dtype")
+        self.y_dtype = _DT[dts.pop()]
+        self._keep = (list(layers), list(xs), list(ys))
+
+
+def spectra_gemv_batched(layers=None, xs=None, ys=None, *, views: BatchViews | None = None,
+                         stream=None) -> BatchViews:
+    """Independent batch-1 matvecs ys[i] = W_i xs[i] in one launch."""
+    v = views if views is not None else BatchViews(layers, xs, ys)
+    _check(_L.spectra_gemv_batched(v.layers, v.xs, v.ys, v.count, v.y_dtype, _stream(stream)),
+           "spectra_gemv_batched")
+    return v

@@ -51,7 +51,11 @@ SIGNATURES = {
     "spectra_unpack": (ctypes.c_int, [LP, P, P, P, P]),
     "spectra_gemv": (ctypes.c_int, [LP, P, P, ctypes.c_int, P]),
     "spectra_gemm_small": (ctypes.c_int, [LP, P, i32, P, ctypes.c_int, P]),
+    "spectra_gemv_batched": (ctypes.c_int, [LP, P, P, i32, ctypes.c_int, P]),
+    "spectra_device_status": (ctypes.c_int, [P]),
 }
+
+MAX_BATCH = 224
 
 _lib = None
 

@@ -230,4 +230,34 @@ spectra_status spectra_gemm_small(const spectra_layer *layer, const uint16_t *x,
     return matvec(layer, x, m_rows, y, y_dtype, stream);
 }
 
+spectra_status spectra_gemv_batched(const spectra_layer *layers, const uint16_t *const *x,
+                                    void *const *y, int32_t count, spectra_dtype y_dtype,
+                                    void *stream) {
+    if (!layers || !x || !y) return SPECTRA_ERR_INVALID_ARG;
+    if (count < 1 || count > SPECTRA_MAX_BATCH) return SPECTRA_ERR_SHAPE;
+    if (y_dtype != SPECTRA_F32 && y_dtype != SPECTRA_BF16) return SPECTRA_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < count; ++i) {
+        spectra_status st = check_layer(&layers[i]);
+        if (st != SPECTRA_OK) return st;
+        if (!x[i] || !y[i]) return SPECTRA_ERR_INVALID_ARG;
+        if (!aligned16(x[i])) return SPECTRA_ERR_ALIGN;
+        if (y_dtype == SPECTRA_F32 ? !aligned4(y[i]) : ((uintptr_t)y[i] & 1u))
+            return SPECTRA_ERR_ALIGN;
+    }
+    DeviceInfo dev;
+    spectra_status st = current_device(&dev);
+    if (st != SPECTRA_OK) return st;
+    return launch_gemv_batched(layers, x, y, count, (int)y_dtype, (cudaStream_t)stream, dev);
+}
+
+spectra_status spectra_device_status(void *stream) {
+    DeviceInfo dev;
+    spectra_status st = current_device(&dev);
+    if (st != SPECTRA_OK) return st;
+    bool raised = false;
+    st = device_error(&raised, (cudaStream_t)stream);
+    if (st != SPECTRA_OK) return st;
+    return raised ? SPECTRA_ERR_INTERNAL : SPECTRA_OK;
+}
+
 }  // extern "C"

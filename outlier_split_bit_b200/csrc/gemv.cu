@@ -6,26 +6,49 @@
 // and the BF16 outlier channels are multiplied in the same pass.
 //
 // Work decomposition.  Lane r of a warp owns row r of a 32-row tile, so every
-// x value a lane needs is a shared-memory broadcast and one warp-wide 16-byte
-// load per group streams one contiguous 512-byte segment of codes.  The
-// super-groups (8 groups = 256 columns) of a tile are split over P slices:
-// `ppc` warps of a CTA times `cl` CTAs of a thread-block cluster; slice sums
-// are reduced in a fixed order through shared memory and, across the
-// cluster, distributed shared memory.  No workspace, no atomics.
+// x value a lane needs is a shared-memory broadcast, and one 16-byte record
+// per lane per group makes the codes of a warp one contiguous 512-byte
+// segment.  The work of a tile is a list of U units: its S super-groups (8
+// groups = 256 columns: 4096 bytes of codes, 512 of scales, 128 of zero
+// points) followed by its outlier batches (up to 8 octets of outlier columns,
+// 4096 bytes).  The units of a tile are split evenly over P slices, each
+// slice run by one warp; slice sums are reduced in a fixed order (shared
+// memory, and distributed shared memory across a cluster), so results are
+// bit-identical from run to run, with no workspace and no atomics.
 //
-// Inner loop per group (32 codes, one 16-byte record per lane):
-//   A = (word & 0x0F0F0F0F) | 0x80808080, B = ((word >> 4) & ...) | ...;
-//   one byte permute per code builds the FP32 value f = 1 + c/128
-//   (exponent 127, code in mantissa bits 16..19); packed FP32x2 FMAs
-//   accumulate sum_k f_k x_k.  With X_g = sum_k x_k,
-//   sum_k (c_k - z) x_k = 128 * sum_k f_k x_k - (128 + z) * X_g,
-//   so the zero point and the scale are applied once per group:
-//   y += s * (128 * A_g - (128 + z) * X_g).
+// Inner loop per group (32 codes, one 16-byte record per lane): for each
+// 32-bit word (8 codes, code j in nibble j) and s = 0..3, ONE logic op
+//   p_s = ((word >> 4s) & 0x000F000F) | 0x43004300
+// yields the BF16 pair (128 + c_s, 128 + c_{s+4}) -- BF16 has 7 mantissa
+// bits, so 128 + c (c < 16) is exact -- and the mixed-precision FMA
+// (fma.rn.f32.bf16: BF16 x BF16 products, FP32 accumulation) multiplies the
+// pair by the matching BF16 pair of x straight from shared memory.  With
+// X_g = sum_k x_k (FP32),
+//   sum_k (c_k - z) x_k = sum_k (128 + c_k) x_k - (128 + z) X_g,
+// so the zero point and the scale are applied once per group:
+//   y += s * (A_g - (128 + z) X_g),  A_g = sum_k (128 + c_k) x_k.
+// This keeps the integer pipe (half rate on sm_100) at ~0.9 operations per
+// weight and puts the multiply-adds on the FMA pipe.
 //
-// Programmatic dependent launch: the kernel lets the next kernel on the
-// stream launch as soon as all of its CTAs run, issues the loads of its first
-// super-group of (constant) weights, then waits for the previous grid before
-// it reads x or writes y.
+// Weight streaming: every warp owns a ring of D shared-memory stages, one
+// unit per stage, filled by cp.async.bulk copies that complete on the
+// stage's mbarrier.  Lane 0 keeps D units in flight; the warp waits on a
+// stage (a bounded wait), decodes it from shared memory and refills it with
+// the unit D ahead.
+//
+// Two launch shapes share this machinery:
+//  - cluster kernel (one matrix, few tiles): a CTA runs `tpc` tiles x `ppc`
+//    slices, a cluster of `cl` CTAs splits the units of the same tiles, and
+//    rank 0 reduces the cluster through distributed shared memory;
+//  - persistent kernel (one large matrix, or many independent matrices): one
+//    16-warp CTA per SM, each walking a byte-balanced contiguous range of
+//    work items (tpc tiles x ppc slices of one matrix); the rings keep
+//    prefetching across item boundaries and x is restaged only when the
+//    matrix changes.
+// Programmatic dependent launch: a kernel lets the next kernel on the stream
+// launch once all of its CTAs run, issues its first D units of (constant)
+// weights, and only then waits for the previous grid before it reads x or
+// writes y.
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -39,15 +62,21 @@ namespace cg = cooperative_groups;
 namespace spectra {
 namespace {
 
-// CTA size limit per batch width: more accumulators need more registers.
-template <int MB>
-struct MaxWarps {
-    static constexpr int value = 8;
-};
+constexpr int kClusterWarps = 8;               // warps per CTA of the cluster kernel
+constexpr int kPersistWarps = 16;              // warps per CTA of the persistent kernel
+constexpr int kOB = 8;                         // outlier octets per unit
 constexpr int kSgBytes = 8 * 512 + 512 + 128;  // codes + scales + zeros of a warp per super-group
 constexpr int kOctBytes = 512;                 // outlier bytes of a warp per octet
+constexpr int kStageBytes = kSgBytes;          // one ring stage (16-byte multiple)
+constexpr uint32_t kSpinLimit = 1u << 22;      // try_wait rounds before a wait gives up
+constexpr int kMaxCtas = 320;                  // persistent grid bound (2 x SMs of a B200 + margin)
 
-struct GemvArgs {
+// Set (bit 0) when a bounded wait in a kernel gave up; read and cleared by
+// spectra_device_status().
+__device__ unsigned int g_device_error;
+
+// One matvec problem as the kernels see it.
+struct Prob {
     const uint4 *codes;
     const uint4 *scales;
     const uint32_t *zeros;
@@ -56,260 +85,479 @@ struct GemvArgs {
     const uint16_t *x;
     void *y;
     int n, k, m, G, S, O8, n_o, T;
-    int ppc, tpc, cl;
+    int U;         // units per tile
+    int ppc, tpc;  // slices per tile, tiles per CTA item
+    int cl;        // CTAs per cluster (cluster kernel)
     int ytype;
-    int smem_sg, smem_oc;  // capacity of the x stage (super-groups, octets)
+    int items;     // ceil(T / tpc)
 };
 
-__device__ __forceinline__ uint4 ld_stream(const uint4 *p) {
-    uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
-}
+// Launch-wide shared-memory geometry.
+struct Smem {
+    int depth;  // ring stages per warp
+    int xg;     // x-stage capacity in groups
+    int xo;     // x-stage capacity in outlier slots
+    int tpc;    // partial-sum rows (tiles) for the cluster reduction
+};
 
-__device__ __forceinline__ uint32_t ld_stream32(const uint32_t *p) {
-    uint32_t r;
-    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r) : "l"(p));
-    return r;
-}
+struct ClusterArgs {
+    Prob p;
+    Smem sm;
+};
+
+// Parameters of the persistent kernel, passed by value (kernel parameter space).
+struct PersistArgs {
+    Smem sm;
+    int count;                      // problems
+    int item_start[kMaxBatch + 1];  // first item of each problem
+    int cta_first[kMaxCtas + 1];    // first item of each CTA
+    Prob probs[kMaxBatch];
+};
+static_assert(sizeof(PersistArgs) <= 32760, "kernel parameter space");
 
 __device__ __forceinline__ void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// f = 1 + c/128 from byte b of a pre-masked register (byte = 0x80 | c).
-template <int b>
-__device__ __forceinline__ float code_f(uint32_t a) {
-    return __uint_as_float(__byte_perm(a, 0x3F000000u, 0x7054u | (b << 8)));
+// Barrier among the `threads` threads (a multiple of 32) that use barrier `id`.
+__device__ __forceinline__ void named_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-__device__ __forceinline__ int slice_begin(int total, int s, int P) {
+__device__ __forceinline__ int split_at(int total, int s, int P) {
     return (int)(((int64_t)total * s) / P);
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
-// Shared-memory x stage.  Bulk x is stored per group in the lane-broadcast
-// order: position 8w + 4*(j & 1) + (j >> 1) holds column 8w + j, and the
-// MB batch rows of one position are contiguous.
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes,
+                                         uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(dst), "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+// Wait for phase `parity` of an mbarrier; gives up after kSpinLimit rounds.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (ok) return true;
+    }
+    return false;
+}
+
+// ---------------------------------------------------------------- shared memory
+
+// Shared-memory layout of one CTA.  Bulk x is stored per group as 16 BF16
+// pairs in the order the decoder pairs the codes: pair 4w + s holds
+// (x_{8w+s}, x_{8w+s+4}); the MB batch rows of one pair are contiguous.
 template <int MB>
 struct Stage {
-    float *xs;    // [smem_sg*8][32][MB]
-    float *xsum;  // [smem_sg*8][MB]
-    float *xo;    // [smem_oc*8][MB]
-    float *red;   // [NW][32][MB]
-    float *part;  // [tpc][32][MB]
+    uint8_t *ring;  // [nw][depth][kStageBytes]
+    uint64_t *bar;  // [nw][depth]
+    uint32_t *xs;   // [xg][16 pairs][MB]: BF16 pairs (x_{8w+s}, x_{8w+s+4}), pair 4w+s
+    float *xsum;    // [xg][MB]
+    uint32_t *xo;   // [xo/2][MB]: BF16 pairs of outlier slots (2i, 2i+1)
+    float *red;     // [2][nw][32][MB]
+    float *part;    // [tpc][32][MB]
 };
 
+__host__ __device__ inline size_t ring_bytes(int nw, int depth) {
+    return (size_t)nw * depth * kStageBytes + (size_t)((nw * depth + 1) & ~1) * 8;
+}
+
+__host__ __device__ inline size_t stage_bytes(int MB, int nw, const Smem &s) {
+    return ring_bytes(nw, s.depth) +
+           sizeof(float) * ((size_t)s.xg * 16 * MB + (size_t)s.xg * MB + (size_t)s.xo / 2 * MB +
+                            (size_t)2 * nw * 32 * MB + (size_t)s.tpc * 32 * MB);
+}
+
 template <int MB>
-__device__ __forceinline__ Stage<MB> carve(float *sm, const GemvArgs &a, int nw) {
+__device__ __forceinline__ Stage<MB> carve(float *sm, const Smem &s, int nw) {
     Stage<MB> st;
-    st.xs = sm;
-    st.xsum = st.xs + (size_t)a.smem_sg * 8 * 32 * MB;
-    st.xo = st.xsum + (size_t)a.smem_sg * 8 * MB;
-    st.red = st.xo + (size_t)a.smem_oc * 8 * MB;
-    st.part = st.red + (size_t)nw * 32 * MB;
+    st.ring = reinterpret_cast<uint8_t *>(sm);
+    st.bar = reinterpret_cast<uint64_t *>(st.ring + (size_t)nw * s.depth * kStageBytes);
+    st.xs = reinterpret_cast<uint32_t *>(st.bar + ((nw * s.depth + 1) & ~1));
+    st.xsum = reinterpret_cast<float *>(st.xs + (size_t)s.xg * 16 * MB);
+    st.xo = reinterpret_cast<uint32_t *>(st.xsum + (size_t)s.xg * MB);
+    st.red = reinterpret_cast<float *>(st.xo + (size_t)s.xo / 2 * MB);
+    st.part = st.red + (size_t)2 * nw * 32 * MB;
     return st;
 }
 
-template <int MB>
-__device__ void stage_x(const GemvArgs &a, const Stage<MB> &st, int csg0, int csg1, int coc0,
-                        int coc1) {
-    const int ng = 8 * (csg1 - csg0);
-    const int chunks = MB * ng * 4;  // 8 columns per chunk
-    for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
-        const int m = c / (ng * 4);
-        const int kc = c - m * ng * 4;
-        const int gl = kc >> 2, w = kc & 3;
-        const int g = 8 * csg0 + gl;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (g < a.G && m < a.m)
-            v = *reinterpret_cast<const uint4 *>(a.x + (size_t)m * a.k + 32 * g + 8 * w);
-        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-        float *dst = st.xs + (size_t)gl * 32 * MB;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float f = (j & 1) ? bf16_hi(u[j >> 1]) : bf16_lo(u[j >> 1]);
-            const int pos = 8 * w + 4 * (j & 1) + (j >> 1);
-            dst[pos * MB + m] = f;
-        }
-    }
-    const int no = 8 * (coc1 - coc0);
-    for (int c = threadIdx.x; c < no * MB; c += blockDim.x) {
-        const int jl = c / MB, m = c - (c / MB) * MB;
-        const int j = 8 * coc0 + jl;
-        float f = 0.f;
-        if (j < a.n_o && m < a.m) f = bf16_lo(a.x[(size_t)m * a.k + a.oidx[j]]);
-        st.xo[jl * MB + m] = f;
-    }
-    __syncthreads();
-    for (int c = threadIdx.x; c < ng * MB; c += blockDim.x) {
-        const int gl = c / MB, m = c - (c / MB) * MB;
-        const float *src = st.xs + (size_t)gl * 32 * MB + m;
-        float s = 0.f;
-#pragma unroll 8
-        for (int p = 0; p < 32; ++p) s += src[p * MB];
-        st.xsum[c] = s;
-    }
-}
-
-struct SgRegs {
-    uint4 q[8];
-    uint4 sc;
-    uint32_t zw;
+// A slice of a tile: its super-groups and its outlier batches, each split
+// evenly over the P slices so that every slice has the same mix of work.
+struct Slice {
+    int sg0, nsg;  // super-groups [sg0, sg0 + nsg)
+    int ob0, nob;  // outlier batches [ob0, ob0 + nob)
 };
 
-__device__ __forceinline__ void load_sg(SgRegs &r, const GemvArgs &a, int t, int sg, int lane) {
-    const uint4 *cp = a.codes + ((size_t)t * a.G + 8 * sg) * 32 + lane;
-    const int ng = min(8, a.G - 8 * sg);
-    if (ng == 8) {
+__device__ __forceinline__ Slice slice_of(const Prob &a, int s, int P) {
+    const int OB = a.U - a.S;
+    Slice r;
+    r.sg0 = split_at(a.S, s, P);
+    r.nsg = split_at(a.S, s + 1, P) - r.sg0;
+    r.ob0 = split_at(OB, s, P);
+    r.nob = split_at(OB, s + 1, P) - r.ob0;
+    return r;
+}
+
+// Local unit u of a slice -> unit id (super-group id, or S + batch id).
+__device__ __forceinline__ int unit_id(const Prob &a, const Slice &sl, int u) {
+    return u < sl.nsg ? sl.sg0 + u : a.S + sl.ob0 + (u - sl.nsg);
+}
+
+// x staged for slices [s0, s1) of P: groups and outlier slots.
+struct XRange {
+    int g0, g1;  // groups [g0, g1) (g1 may pass G: padding groups)
+    int j0, j1;  // outlier slots [j0, j1) (j1 may pass n_o: padding slots)
+};
+
+__device__ __forceinline__ XRange x_range(const Prob &a, int s0, int s1, int P) {
+    const int OB = a.U - a.S;
+    XRange r;
+    r.g0 = 8 * split_at(a.S, s0, P);
+    r.g1 = 8 * split_at(a.S, s1, P);
+    r.j0 = 8 * kOB * split_at(OB, s0, P);
+    r.j1 = 8 * kOB * split_at(OB, s1, P);
+    return r;
+}
+
+// Stage x for a unit range: bulk groups as BF16 pairs in the decoder's order
+// with their FP32 sums X_g (column order), and the BF16 pairs of the outlier
+// slots, gathered through the index list.
+template <int MB>
+__device__ void stage_x(const Prob &a, const Stage<MB> &st, const XRange &xr) {
+    const int nth = blockDim.x;
+    const int ng = xr.g1 - xr.g0;
+    for (int c = threadIdx.x; c < ng * MB; c += nth) {
+        const int gl = c / MB, m = c - gl * MB;
+        const int g = xr.g0 + gl;
+        uint32_t *dst = st.xs + (size_t)gl * 16 * MB + m;
+        float sum = 0.f;
+        if (g < a.G && m < a.m) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)m * a.k + 32 * g);
+            uint4 v[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) r.q[i] = ld_stream(cp + i * 32);
+            for (int w = 0; w < 4; ++w) v[w] = src[w];
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const uint32_t u[4] = {v[w].x, v[w].y, v[w].z, v[w].w};
+                // u[i] holds columns 8w + 2i (low half) and 8w + 2i + 1 (high half)
+                uint32_t h[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) h[j] = (j & 1) ? (u[j >> 1] >> 16) : (u[j >> 1] & 0xFFFFu);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) sum += __uint_as_float(h[j] << 16);
+#pragma unroll
+                for (int sp = 0; sp < 4; ++sp) dst[(4 * w + sp) * MB] = h[sp] | (h[sp + 4] << 16);
+            }
+        } else {
+#pragma unroll
+            for (int p = 0; p < 16; ++p) dst[p * MB] = 0u;
+        }
+        st.xsum[c] = sum;
+    }
+    // outlier slots as BF16 pairs: 8 pairs per thread in flight
+    const int np = (xr.j1 - xr.j0) / 2;
+    for (int base = 0; base < np * MB; base += 8 * nth) {
+        int i0[8], i1[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int c = base + threadIdx.x + i * nth;
+            const int j = xr.j0 + 2 * (c / MB);
+            const bool ok = c < np * MB;
+            i0[i] = (ok && j < a.n_o) ? a.oidx[j] : -1;
+            i1[i] = (ok && j + 1 < a.n_o) ? a.oidx[j + 1] : -1;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int c = base + threadIdx.x + i * nth;
+            if (c < np * MB) {
+                const int m = c % MB;
+                const bool mv = m < a.m;
+                const uint32_t lo = (i0[i] >= 0 && mv) ? a.x[(size_t)m * a.k + i0[i]] : 0u;
+                const uint32_t hi = (i1[i] >= 0 && mv) ? a.x[(size_t)m * a.k + i1[i]] : 0u;
+                st.xo[c] = lo | (hi << 16);
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------- units
+
+// Copies of unit u of tile t into ring stage `dst`.  Called by one lane.
+__device__ __forceinline__ void issue_unit(const Prob &a, int t, int u, uint32_t dst,
+                                           uint32_t bar) {
+    if (u < a.S) {
+        const int ng = min(8, a.G - 8 * u);
+        const uint32_t cb = (uint32_t)ng * 512u;
+        mbar_expect_tx(bar, cb + 512u + 128u);
+        bulk_g2s(dst, a.codes + ((size_t)t * a.G + 8 * u) * 32, cb, bar);
+        bulk_g2s(dst + 4096u, a.scales + ((size_t)t * a.S + u) * 32, 512u, bar);
+        bulk_g2s(dst + 4608u, a.zeros + ((size_t)t * a.S + u) * 32, 128u, bar);
+    } else {
+        const int oc = (u - a.S) * kOB;
+        const uint32_t b = (uint32_t)min(kOB, a.O8 - oc) * 512u;
+        mbar_expect_tx(bar, b);
+        bulk_g2s(dst, a.outw + ((size_t)t * a.O8 + oc) * 32, b, bar);
+    }
+}
+
+// lo += c.lo * x.lo, hi += c.hi * x.hi: BF16 products, FP32 accumulation.
+__device__ __forceinline__ void mfma2(float &lo, float &hi, uint32_t c, uint32_t x) {
+    asm("{\n\t.reg .b16 cl, ch, xl, xh;\n\t"
+        "mov.b32 {cl, ch}, %2;\n\t"
+        "mov.b32 {xl, xh}, %3;\n\t"
+        "fma.rn.f32.bf16 %0, cl, xl, %0;\n\t"
+        "fma.rn.f32.bf16 %1, ch, xh, %1;\n\t}"
+        : "+f"(lo), "+f"(hi)
+        : "r"(c), "r"(x));
+}
+
+// BF16 pair (128 + c_s, 128 + c_{s+4}) of nibbles s and s + 4 of a word.
+template <int sh>
+__device__ __forceinline__ uint32_t code_pair(uint32_t w) {
+    return ((w >> (4 * sh)) & 0x000F000Fu) | 0x43004300u;
+}
+
+// A_g[m] = sum_k (128 + c_k) x[m][k] for one group.
+template <int MB>
+__device__ __forceinline__ void group_dot(const uint4 &q, const uint32_t *xg, float *out) {
+    float acc[MB][4];
+#pragma unroll
+    for (int m = 0; m < MB; ++m) acc[m][0] = acc[m][1] = acc[m][2] = acc[m][3] = 0.f;
+    const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const uint32_t cp[4] = {code_pair<0>(wv[w]), code_pair<1>(wv[w]), code_pair<2>(wv[w]),
+                                code_pair<3>(wv[w])};
+        if constexpr (MB == 1) {
+            const uint4 xw = *reinterpret_cast<const uint4 *>(xg + 4 * w);
+            mfma2(acc[0][0], acc[0][1], cp[0], xw.x);
+            mfma2(acc[0][2], acc[0][3], cp[1], xw.y);
+            mfma2(acc[0][0], acc[0][1], cp[2], xw.z);
+            mfma2(acc[0][2], acc[0][3], cp[3], xw.w);
+        } else {
+#pragma unroll
+            for (int sp = 0; sp < 4; ++sp) {
+                const uint32_t *xp = xg + (4 * w + sp) * MB;
+#pragma unroll
+                for (int m = 0; m < MB; m += 2) {
+                    const uint2 x2 = *reinterpret_cast<const uint2 *>(xp + m);
+                    mfma2(acc[m][sp & 1], acc[m][2 + (sp & 1)], cp[sp], x2.x);
+                    mfma2(acc[m + 1][sp & 1], acc[m + 1][2 + (sp & 1)], cp[sp], x2.y);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < MB; ++m) out[m] = (acc[m][0] + acc[m][1]) + (acc[m][2] + acc[m][3]);
+}
+
+template <int MB>
+__device__ __forceinline__ void compute_group(const uint8_t *stage, int gg, int lane,
+                                              const uint32_t *scw, uint32_t zw,
+                                              const uint32_t *xs_sg, const float *xsum_sg,
+                                              float *yacc) {
+    const uint4 q = *reinterpret_cast<const uint4 *>(stage + gg * 512 + lane * 16);
+    const float s = __half2float(__ushort_as_half(
+        (unsigned short)((gg & 1) ? (scw[gg >> 1] >> 16) : (scw[gg >> 1] & 0xFFFFu))));
+    // 128 + z as a float: exponent of 128, z in mantissa bits 16..19
+    const uint32_t zsh = (gg <= 4) ? (zw << (16 - 4 * gg)) : (zw >> (4 * gg - 16));
+    const float zf = __uint_as_float((zsh & 0x000F0000u) | 0x43000000u);
+    float Ag[MB];
+    group_dot<MB>(q, xs_sg + gg * 16 * MB, Ag);
+#pragma unroll
+    for (int m = 0; m < MB; ++m) yacc[m] = fmaf(s, fmaf(-zf, xsum_sg[gg * MB + m], Ag[m]), yacc[m]);
+}
+
+template <int MB>
+__device__ __forceinline__ void compute_sg(const uint8_t *stage, int ng, int lane,
+                                           const uint32_t *xs_sg, const float *xsum_sg,
+                                           float *yacc) {
+    const uint4 sc = *reinterpret_cast<const uint4 *>(stage + 4096 + lane * 16);
+    const uint32_t zw = *reinterpret_cast<const uint32_t *>(stage + 4608 + lane * 4);
+    const uint32_t scw[4] = {sc.x, sc.y, sc.z, sc.w};
+    if (ng == 8) {
+        // full super-group: straight-line code, the 8 groups overlap
+#pragma unroll
+        for (int gg = 0; gg < 8; ++gg) compute_group<MB>(stage, gg, lane, scw, zw, xs_sg, xsum_sg, yacc);
     } else {
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            r.q[i] = (i < ng) ? ld_stream(cp + i * 32) : make_uint4(0u, 0u, 0u, 0u);
+        for (int gg = 0; gg < 8; ++gg)
+            if (gg < ng) compute_group<MB>(stage, gg, lane, scw, zw, xs_sg, xsum_sg, yacc);
     }
-    r.sc = ld_stream(a.scales + ((size_t)t * a.S + sg) * 32 + lane);
-    r.zw = ld_stream32(a.zeros + ((size_t)t * a.S + sg) * 32 + lane);
 }
 
-// sum_k f_k x_k for one group, MB == 1.
-__device__ __forceinline__ float group_dot1(const uint4 &q, const float *xg) {
-    const float4 *x4 = reinterpret_cast<const float4 *>(xg);
-    float2 a0 = make_float2(0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
-    const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-        const uint32_t A = (wv[w] & 0x0F0F0F0Fu) | 0x80808080u;
-        const uint32_t B = ((wv[w] >> 4) & 0x0F0F0F0Fu) | 0x80808080u;
-        const float4 xa = x4[2 * w], xb = x4[2 * w + 1];
-        a0 = __ffma2_rn(make_float2(code_f<0>(A), code_f<1>(A)), make_float2(xa.x, xa.y), a0);
-        a1 = __ffma2_rn(make_float2(code_f<2>(A), code_f<3>(A)), make_float2(xa.z, xa.w), a1);
-        a2 = __ffma2_rn(make_float2(code_f<0>(B), code_f<1>(B)), make_float2(xb.x, xb.y), a2);
-        a3 = __ffma2_rn(make_float2(code_f<2>(B), code_f<3>(B)), make_float2(xb.z, xb.w), a3);
-    }
-    const float2 s = __fadd2_rn(__fadd2_rn(a0, a1), __fadd2_rn(a2, a3));
-    return s.x + s.y;
-}
-
-// sum_k f_k x[m][k] for one group, MB > 1 (MB even): acc[m] for all rows.
+// Outlier octets: BF16 weight pairs times BF16 x pairs, FP32 accumulation.
 template <int MB>
-__device__ __forceinline__ void group_dotm(const uint4 &q, const float *xg, float *out) {
-    float2 ea[MB / 2], eb[MB / 2];
+__device__ __forceinline__ void compute_ob(const uint8_t *stage, int lane, const uint32_t *xo,
+                                           int n_valid, float *yacc) {
+    float lo[MB], hi[MB];
 #pragma unroll
-    for (int i = 0; i < MB / 2; ++i) ea[i] = eb[i] = make_float2(0.f, 0.f);
-    const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
+    for (int m = 0; m < MB; ++m) lo[m] = hi[m] = 0.f;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-        const uint32_t A = (wv[w] & 0x0F0F0F0Fu) | 0x80808080u;
-        const uint32_t B = ((wv[w] >> 4) & 0x0F0F0F0Fu) | 0x80808080u;
-        float fa[4] = {code_f<0>(A), code_f<1>(A), code_f<2>(A), code_f<3>(A)};
-        float fb[4] = {code_f<0>(B), code_f<1>(B), code_f<2>(B), code_f<3>(B)};
+    for (int i = 0; i < kOB; ++i) {
+        if (i >= n_valid) break;
+        const uint4 w4 = *reinterpret_cast<const uint4 *>(stage + i * 512 + lane * 16);
+        const uint32_t wp[4] = {w4.x, w4.y, w4.z, w4.w};
+        const uint32_t *xi = xo + i * 4 * MB;
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            const float2 *xa = reinterpret_cast<const float2 *>(xg + (8 * w + b) * MB);
-            const float2 *xb = reinterpret_cast<const float2 *>(xg + (8 * w + 4 + b) * MB);
-            const float2 fa2 = make_float2(fa[b], fa[b]);
-            const float2 fb2 = make_float2(fb[b], fb[b]);
+        for (int e = 0; e < 4; ++e) {
 #pragma unroll
-            for (int i = 0; i < MB / 2; ++i) {
-                ea[i] = __ffma2_rn(fa2, xa[i], ea[i]);
-                eb[i] = __ffma2_rn(fb2, xb[i], eb[i]);
-            }
+            for (int m = 0; m < MB; ++m) mfma2(lo[m], hi[m], wp[e], xi[e * MB + m]);
         }
     }
 #pragma unroll
-    for (int i = 0; i < MB / 2; ++i) {
-        const float2 s = __fadd2_rn(ea[i], eb[i]);
-        out[2 * i] = s.x;
-        out[2 * i + 1] = s.y;
+    for (int m = 0; m < MB; ++m) yacc[m] += lo[m] + hi[m];
+}
+
+// Decode unit u from a ring stage against the staged x of range xr.
+template <int MB>
+__device__ __forceinline__ void compute_unit(const Prob &a, const uint8_t *stage, int lane,
+                                             const Stage<MB> &st, const XRange &xr, int u,
+                                             float *yacc) {
+    if (u < a.S) {
+        const int l = 8 * u - xr.g0;  // local index of the super-group's first group
+        compute_sg<MB>(stage, min(8, a.G - 8 * u), lane, st.xs + (size_t)l * 16 * MB,
+                       st.xsum + l * MB, yacc);
+    } else {
+        const int b = u - a.S;
+        compute_ob<MB>(stage, lane, st.xo + (size_t)((8 * kOB * b - xr.j0) / 2) * MB,
+                       min(kOB, a.O8 - kOB * b), yacc);
     }
 }
 
-template <int MB>
-__device__ __forceinline__ void compute_sg(const SgRegs &r, const float *xs_sg,
-                                           const float *xsum_sg, float *yacc) {
-    const uint32_t scw[4] = {r.sc.x, r.sc.y, r.sc.z, r.sc.w};
-#pragma unroll
-    for (int gg = 0; gg < 8; ++gg) {
-        const float s = __half2float(__ushort_as_half(
-            (unsigned short)((gg & 1) ? (scw[gg >> 1] >> 16) : (scw[gg >> 1] & 0xFFFFu))));
-        // 128 + z as a float: exponent of 128, z in mantissa bits 16..19
-        const uint32_t zsh = (gg <= 4) ? (r.zw << (16 - 4 * gg)) : (r.zw >> (4 * gg - 16));
-        const float zf = __uint_as_float((zsh & 0x000F0000u) | 0x43000000u);
-        const float *xg = xs_sg + gg * 32 * MB;
-        if constexpr (MB == 1) {
-            const float Ag = group_dot1(r.q[gg], xg);
-            const float tg = fmaf(128.f, Ag, -zf * xsum_sg[gg]);
-            yacc[0] = fmaf(s, tg, yacc[0]);
-        } else {
-            float Ag[MB];
-            group_dotm<MB>(r.q[gg], xg, Ag);
-#pragma unroll
-            for (int m = 0; m < MB; ++m) {
-                const float tg = fmaf(128.f, Ag[m], -zf * xsum_sg[gg * MB + m]);
-                yacc[m] = fmaf(s, tg, yacc[m]);
-            }
-        }
+__device__ __forceinline__ void store_y(const Prob &a, int t, int lane, int m, float v) {
+    const int row = 32 * t + lane;
+    if (row < a.n && m < a.m) {
+        if (a.ytype == SPECTRA_F32)
+            reinterpret_cast<float *>(a.y)[(size_t)m * a.n + row] = v;
+        else
+            reinterpret_cast<__nv_bfloat16 *>(a.y)[(size_t)m * a.n + row] = __float2bfloat16_rn(v);
     }
 }
 
+// Per-warp ring of D stages: units are consumed in the order they were issued.
+struct Ring {
+    uint8_t *base;
+    uint32_t base_s, bar_s;
+    int D;
+    int consumed, issued;
+    bool ok;
+    int failed_at;
+};
+
+__device__ __forceinline__ void ring_init(Ring &r, uint8_t *base, uint64_t *bars, int D, int lane) {
+    r.base = base;
+    r.base_s = smem_u32(base);
+    r.bar_s = smem_u32(bars);
+    r.D = D;
+    r.consumed = r.issued = 0;
+    r.ok = true;
+    r.failed_at = 0;
+    if (lane == 0) {
+        for (int d = 0; d < D; ++d) mbar_init(r.bar_s + 8u * d, 1u);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+}
+
+__device__ __forceinline__ void ring_issue(Ring &r, const Prob &a, int t, int u, int lane) {
+    const int d = r.issued % r.D;
+    if (r.ok && lane == 0)
+        issue_unit(a, t, u, r.base_s + (uint32_t)d * kStageBytes, r.bar_s + 8u * d);
+    if (r.ok) ++r.issued;
+}
+
+// Wait for the next stage to fill; returns its address (nullptr after a failure).
+__device__ __forceinline__ const uint8_t *ring_acquire(Ring &r, int lane) {
+    const int d = r.consumed % r.D;
+    if (r.ok && !mbar_wait(r.bar_s + 8u * d, (uint32_t)(r.consumed / r.D) & 1u)) {
+        r.ok = false;
+        r.failed_at = r.consumed;
+        if (lane == 0) atomicOr(&g_device_error, 1u);
+    }
+    return r.ok ? r.base + (size_t)d * kStageBytes : nullptr;
+}
+
+__device__ __forceinline__ void ring_release(Ring &r) {
+    __syncwarp();
+    if (r.ok) ++r.consumed;
+}
+
+// After a failed wait, let the copies already in flight land before the CTA
+// releases its shared memory (bounded as well).
+__device__ __forceinline__ void ring_drain(const Ring &r) {
+    if (r.ok) return;
+    for (int n = r.failed_at; n < r.issued; ++n)
+        mbar_wait(r.bar_s + 8u * (n % r.D), (uint32_t)(n / r.D) & 1u);
+}
+
+// ---------------------------------------------------------------- cluster kernel
+
+// One matrix: CTA = tpc tiles x ppc slices, cluster of cl CTAs along the units.
 template <int MB>
-__global__ void __launch_bounds__(MaxWarps<MB>::value * 32, 1) gemv_kernel(const GemvArgs a) {
+__global__ void __launch_bounds__(kClusterWarps * 32, MB == 1 ? 2 : 1)
+    gemv_cluster_kernel(const ClusterArgs args) {
     extern __shared__ __align__(16) float smem[];
-    const int nw = blockDim.x >> 5;
+    const Prob &a = args.p;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cr = (a.cl > 1) ? (int)cg::this_cluster().block_rank() : 0;
     const int cid = blockIdx.x / a.cl;
     const int P = a.ppc * a.cl;
-    const int tl = warp / a.ppc, sl = warp - (warp / a.ppc) * a.ppc;
+    const int tl = warp / a.ppc, sl = warp - tl * a.ppc;
     const int t = cid * a.tpc + tl;
-    const bool active = t < a.T;
-    const int slice = cr * a.ppc + sl;
-    const int sg0 = slice_begin(a.S, slice, P), sg1 = slice_begin(a.S, slice + 1, P);
-    const int oc0 = slice_begin(a.O8, slice, P), oc1 = slice_begin(a.O8, slice + 1, P);
-    const int csg0 = slice_begin(a.S, cr * a.ppc, P), csg1 = slice_begin(a.S, (cr + 1) * a.ppc, P);
-    const int coc0 = slice_begin(a.O8, cr * a.ppc, P),
-              coc1 = slice_begin(a.O8, (cr + 1) * a.ppc, P);
-    const Stage<MB> st = carve<MB>(smem, a, nw);
+    const bool active = tl < a.tpc && t < a.T;
+    const Slice slc = slice_of(a, cr * a.ppc + sl, P);
+    const int nunits = active ? slc.nsg + slc.nob : 0;
+    const XRange xr = x_range(a, cr * a.ppc, (cr + 1) * a.ppc, P);
+    const Stage<MB> st = carve<MB>(smem, args.sm, kClusterWarps);
 
+    Ring ring;
+    ring_init(ring, st.ring + (size_t)warp * args.sm.depth * kStageBytes,
+              st.bar + warp * args.sm.depth, args.sm.depth, lane);
     pdl_launch_dependents();
-    SgRegs ra, rb;
-    if (active && sg0 < sg1) load_sg(ra, a, t, sg0, lane);
+    int next = 0;
+    for (; next < nunits && next < ring.D; ++next) ring_issue(ring, a, t, unit_id(a, slc, next), lane);
     pdl_wait();
-    stage_x<MB>(a, st, csg0, csg1, coc0, coc1);
+    stage_x<MB>(a, st, xr);
     __syncthreads();
 
     float yacc[MB];
 #pragma unroll
     for (int m = 0; m < MB; ++m) yacc[m] = 0.f;
-    if (active) {
-        for (int sg = sg0; sg < sg1; sg += 2) {
-            if (sg + 1 < sg1) load_sg(rb, a, t, sg + 1, lane);
-            const int la = sg - csg0;
-            compute_sg<MB>(ra, st.xs + (size_t)la * 8 * 32 * MB, st.xsum + la * 8 * MB, yacc);
-            if (sg + 1 >= sg1) break;
-            if (sg + 2 < sg1) load_sg(ra, a, t, sg + 2, lane);
-            compute_sg<MB>(rb, st.xs + (size_t)(la + 1) * 8 * 32 * MB,
-                           st.xsum + (la + 1) * 8 * MB, yacc);
-        }
-        for (int oc = oc0; oc < oc1; ++oc) {
-            const uint4 ow = ld_stream(a.outw + ((size_t)t * a.O8 + oc) * 32 + lane);
-            const uint32_t ov[4] = {ow.x, ow.y, ow.z, ow.w};
-            const float *xo = st.xo + (size_t)(oc - coc0) * 8 * MB;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float wv = (e & 1) ? bf16_hi(ov[e >> 1]) : bf16_lo(ov[e >> 1]);
-#pragma unroll
-                for (int m = 0; m < MB; ++m) yacc[m] = fmaf(wv, xo[e * MB + m], yacc[m]);
-            }
-        }
+    for (int u = 0; u < nunits; ++u) {
+        const uint8_t *stage = ring_acquire(ring, lane);
+        if (stage) compute_unit<MB>(a, stage, lane, st, xr, unit_id(a, slc, u), yacc);
+        ring_release(ring);
+        if (next < nunits) ring_issue(ring, a, t, unit_id(a, slc, next++), lane);
     }
+    ring_drain(ring);
 
     // fixed-order reduction: slices of the CTA, then CTAs of the cluster
 #pragma unroll
@@ -337,7 +585,8 @@ __global__ void __launch_bounds__(MaxWarps<MB>::value * 32, 1) gemv_kernel(const
 #pragma unroll
             for (int m = 0; m < MB; ++m) tot[m] = 0.f;
             for (int rk = 0; rk < a.cl; ++rk) {
-                const float *rp = cluster.map_shared_rank(st.part, rk) + ((size_t)tl * 32 + lane) * MB;
+                const float *rp =
+                    cluster.map_shared_rank(st.part, rk) + ((size_t)tl * 32 + lane) * MB;
 #pragma unroll
                 for (int m = 0; m < MB; ++m) tot[m] += rp[m];
             }
@@ -345,36 +594,153 @@ __global__ void __launch_bounds__(MaxWarps<MB>::value * 32, 1) gemv_kernel(const
         cluster.sync();
     }
     if (leader && cr == 0) {
-        const int row = 32 * t + lane;
-        if (row < a.n) {
 #pragma unroll
-            for (int m = 0; m < MB; ++m) {
-                if (m < a.m) {
-                    if (a.ytype == SPECTRA_F32)
-                        reinterpret_cast<float *>(a.y)[(size_t)m * a.n + row] = tot[m];
-                    else
-                        reinterpret_cast<__nv_bfloat16 *>(a.y)[(size_t)m * a.n + row] =
-                            __float2bfloat16_rn(tot[m]);
-                }
-            }
-        }
+        for (int m = 0; m < MB; ++m) store_y(a, t, lane, m, tot[m]);
     }
 }
 
-struct Plan {
-    int ppc, tpc, cl, nw;
-    int smem_sg, smem_oc;
-    size_t smem;
-    unsigned grid;
+// ---------------------------------------------------------------- persistent kernel
+
+__device__ __forceinline__ int prob_of(const PersistArgs &args, int item) {
+    int lo = 0, hi = args.count - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (args.item_start[mid] <= item)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo;
+}
+
+// Where one warp's issue pointer stands: item, its problem, tile, slice and
+// local unit.
+struct Cursor {
+    int item, p, t, u;
+    Slice sl;
 };
 
-size_t smem_bytes(int MB, int smem_sg, int smem_oc, int nw, int tpc) {
-    return sizeof(float) * ((size_t)smem_sg * 8 * 32 * MB + (size_t)smem_sg * 8 * MB +
-                            (size_t)smem_oc * 8 * MB + (size_t)nw * 32 * MB + (size_t)tpc * 32 * MB);
+// Move the cursor to the first unit of `c.item` or of a later item of this warp.
+__device__ __forceinline__ void cursor_load(const PersistArgs &args, int it1, int warp, Cursor &c) {
+    while (c.item < it1) {
+        c.p = prob_of(args, c.item);
+        const Prob &a = args.probs[c.p];
+        const int blk = c.item - args.item_start[c.p];
+        const int tl = warp / a.ppc;
+        c.t = blk * a.tpc + tl;
+        if (c.t < a.T) {
+            c.sl = slice_of(a, warp - tl * a.ppc, a.ppc);
+            c.u = 0;
+            if (c.sl.nsg + c.sl.nob > 0) return;
+        }
+        ++c.item;
+    }
+}
+
+__device__ __forceinline__ void cursor_next(const PersistArgs &args, int it1, int warp, Cursor &c) {
+    if (++c.u < c.sl.nsg + c.sl.nob) return;
+    ++c.item;
+    cursor_load(args, it1, warp, c);
+}
+
+__device__ __forceinline__ void cursor_issue(const PersistArgs &args, Ring &ring, const Cursor &c,
+                                             int lane) {
+    const Prob &a = args.probs[c.p];
+    ring_issue(ring, a, c.t, unit_id(a, c.sl, c.u), lane);
+}
+
+template <int MB>
+__global__ void __launch_bounds__(kPersistWarps * 32, 1)
+    gemv_persistent_kernel(const PersistArgs args) {
+    extern __shared__ __align__(16) float smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int it0 = args.cta_first[blockIdx.x], it1 = args.cta_first[blockIdx.x + 1];
+    const Stage<MB> st = carve<MB>(smem, args.sm, kPersistWarps);
+
+    Ring ring;
+    ring_init(ring, st.ring + (size_t)warp * args.sm.depth * kStageBytes,
+              st.bar + warp * args.sm.depth, args.sm.depth, lane);
+    pdl_launch_dependents();
+    Cursor ic;
+    ic.item = it0;
+    cursor_load(args, it1, warp, ic);
+    for (int d = 0; d < ring.D && ic.item < it1; ++d) {
+        cursor_issue(args, ring, ic, lane);
+        cursor_next(args, it1, warp, ic);
+    }
+    pdl_wait();
+
+    int cur_p = -1;
+    int rbuf = 0;
+    XRange xr = {0, 0, 0, 0};
+    for (int item = it0; item < it1; ++item) {
+        const int p = prob_of(args, item);
+        const Prob &a = args.probs[p];
+        if (p != cur_p) {
+            // every warp is done with the previous x (the branch is CTA-uniform)
+            __syncthreads();
+            xr = x_range(a, 0, 1, 1);
+            stage_x<MB>(a, st, xr);
+            __syncthreads();
+            cur_p = p;
+        }
+        const int blk = item - args.item_start[p];
+        const int tl = warp / a.ppc, sl = warp - tl * a.ppc;
+        const int t = blk * a.tpc + tl;
+        const bool active = t < a.T;
+        const Slice slc = slice_of(a, sl, a.ppc);
+        const int nunits = active ? slc.nsg + slc.nob : 0;
+        float yacc[MB];
+#pragma unroll
+        for (int m = 0; m < MB; ++m) yacc[m] = 0.f;
+        for (int u = 0; u < nunits; ++u) {
+            const uint8_t *stage = ring_acquire(ring, lane);
+            if (stage) compute_unit<MB>(a, stage, lane, st, xr, unit_id(a, slc, u), yacc);
+            ring_release(ring);
+            if (ic.item < it1) {
+                cursor_issue(args, ring, ic, lane);
+                cursor_next(args, it1, warp, ic);
+            }
+        }
+        if (a.ppc == 1) {
+            if (active) {
+#pragma unroll
+                for (int m = 0; m < MB; ++m) store_y(a, t, lane, m, yacc[m]);
+            }
+        } else {
+            // the ppc warps of one tile meet on their own barrier (ids 1..tpc)
+            float *red = st.red + (size_t)rbuf * kPersistWarps * 32 * MB;
+#pragma unroll
+            for (int m = 0; m < MB; ++m) red[((size_t)warp * 32 + lane) * MB + m] = yacc[m];
+            named_sync(1 + tl, 32 * a.ppc);
+            if (active && sl == 0) {
+#pragma unroll
+                for (int m = 0; m < MB; ++m) {
+                    float tot = 0.f;
+                    for (int s = 0; s < a.ppc; ++s)
+                        tot += red[((size_t)(tl * a.ppc + s) * 32 + lane) * MB + m];
+                    store_y(a, t, lane, m, tot);
+                }
+            }
+            rbuf ^= 1;
+        }
+    }
+    ring_drain(ring);
+}
+
+// ---------------------------------------------------------------- host planning
+
+constexpr size_t kSmPerSm = 228 * 1024;  // shared memory of one SM
+constexpr size_t kCtaReserve = 1024;     // per-CTA shared memory the system reserves
+constexpr int kMaxDepth = 4;
+
+int units_of(const Geometry &g) { return g.S + (int)cdiv(g.O8, kOB); }
+
+int64_t tile_bytes(const Geometry &g) {
+    return (int64_t)g.S * kSgBytes + (int64_t)g.O8 * kOctBytes;
 }
 
 int max_share(int total, int parts_per, int cl, int P) {
-    // the largest CTA share of `total` units when P slices are grouped by `parts_per`
     int mx = 0;
     for (int c = 0; c < cl; ++c) {
         const int b = (int)(((int64_t)total * c * parts_per) / P);
@@ -384,86 +750,268 @@ int max_share(int total, int parts_per, int cl, int P) {
     return mx;
 }
 
-// Pick slices per tile (P = ppc * cl) and tiles per CTA from a simple model:
-// time ~ waves(T*P warps) * bytes of the largest slice, plus a small cost per
-// reduction level.  Shared memory must hold the CTA's slice of x.
-bool make_plan(const Geometry &g, int MB, int max_warps, const DeviceInfo &dev, Plan *out) {
-    const int64_t warp_cap = (int64_t)dev.sm_count * 24;
-    double best = 1e300;
+// Deepest ring that fits `budget` with the x stage of `sm` (0 if none fits).
+int fit_depth(int MB, int nw, Smem sm, size_t budget) {
+    for (int d = kMaxDepth; d >= 1; --d) {
+        sm.depth = d;
+        if (stage_bytes(MB, nw, sm) <= budget) return d;
+    }
+    return 0;
+}
+
+// Cluster kernel: depth for two CTAs per SM if that leaves >= 2 stages per
+// warp, else the deepest ring of one CTA.
+int choose_depth(int MB, const Smem &sm, const DeviceInfo &dev) {
+    const int d2 = fit_depth(MB, kClusterWarps, sm, kSmPerSm / 2 - kCtaReserve);
+    if (d2 >= 2 || (d2 >= 1 && MB == 1 && fit_depth(MB, kClusterWarps, sm, dev.smem_optin) < 2))
+        return d2;
+    return fit_depth(MB, kClusterWarps, sm, dev.smem_optin);
+}
+
+int ctas_per_sm(int MB, const Smem &sm) {
+    const int per = (int)(kSmPerSm / (stage_bytes(MB, kClusterWarps, sm) + kCtaReserve));
+    const int reg_cap = MB == 1 ? 2 : 1;
+    return per < 1 ? 1 : (per > reg_cap ? reg_cap : per);
+}
+
+struct ClusterPlan {
+    int ppc, tpc, cl;
+    Smem sm;
+    unsigned grid;
+    double cost;
+};
+
+// Cluster kernel: slices per tile P = ppc * cl and tiles per CTA from a simple
+// model -- waves of CTAs times the bytes of the largest slice, plus a cost per
+// CTA start and per reduction level.
+bool plan_cluster(const Geometry &g, int MB, const DeviceInfo &dev, ClusterPlan *out) {
+    const int U = units_of(g);
+    const int OB = U - g.S;
     bool found = false;
+    out->cost = 1e300;
     for (int cl = 1; cl <= 8; ++cl) {
-        for (int ppc = 1; ppc <= max_warps; ++ppc) {
+        for (int ppc = 1; ppc <= kClusterWarps; ++ppc) {
             const int P = ppc * cl;
-            if (P > 1 && P > g.S) continue;
-            const int tpc = (ppc >= 8) ? 1 : (g.T >= 2 * warp_cap / ppc ? 8 / ppc : 1);
-            const int nw = tpc * ppc;
-            if (nw > max_warps) continue;
-            const int64_t warps = (int64_t)g.T * P;
-            const int64_t waves = (warps + warp_cap - 1) / warp_cap;
-            const int64_t slice_bytes = cdiv(g.S, P) * kSgBytes + cdiv(g.O8, P) * kOctBytes;
-            const double cost = (double)waves * (double)slice_bytes + (ppc > 1 ? 1024.0 : 0.0) +
-                                (cl > 1 ? 4096.0 + 512.0 * cl : 0.0);
-            const int ssg = max_share(g.S, ppc, cl, P);
-            const int soc = max_share(g.O8, ppc, cl, P);
-            const size_t smem = smem_bytes(MB, ssg, soc, nw, tpc);
-            if (smem > dev.smem_optin) continue;
-            if (cost < best) {
-                best = cost;
+            if (P > 1 && P > U) continue;
+            const int tpc = kClusterWarps / ppc;
+            Smem sm;
+            sm.xg = 8 * max_share(g.S, ppc, cl, P);
+            sm.xo = 8 * kOB * max_share(OB, ppc, cl, P);
+            sm.tpc = tpc;
+            sm.depth = choose_depth(MB, sm, dev);
+            if (sm.depth == 0) continue;
+            const int64_t ctas = cdiv(g.T, tpc) * cl;
+            const int64_t waves = cdiv(ctas, (int64_t)dev.sm_count * ctas_per_sm(MB, sm));
+            const int64_t slice = cdiv(g.S, P) * kSgBytes + cdiv(OB, P) * kOB * kOctBytes;
+            const double cost = (double)waves * (double)(slice + 8192) +
+                                (ppc > 1 ? 256.0 * ppc : 0.0) + (cl > 1 ? 4096.0 + 512.0 * cl : 0.0);
+            if (cost < out->cost) {
                 found = true;
+                out->cost = cost;
                 out->ppc = ppc;
                 out->tpc = tpc;
                 out->cl = cl;
-                out->nw = nw;
-                out->smem_sg = ssg;
-                out->smem_oc = soc;
-                out->smem = smem;
-                out->grid = (unsigned)(cdiv(g.T, tpc) * cl);
+                out->sm = sm;
+                out->grid = (unsigned)ctas;
             }
         }
     }
     return found;
 }
 
-// Raise the dynamic shared-memory limit of one kernel instance, once per device.
-template <int MB>
-cudaError_t prepare_kernel(const DeviceInfo &dev) {
-    static std::mutex mu;
-    static bool done[64];
-    std::lock_guard<std::mutex> lock(mu);
+// Persistent kernel: item = tpc tiles x ppc slices.  ppc is the smallest power
+// of two (<= 16, <= units per tile) that keeps an item at or below
+// `target` bytes, so each CTA walks several items (balance) while as many
+// warps as possible own whole tiles (no reduction, no barrier).
+void item_shape(const Geometry &g, int64_t target, int *ppc, int *tpc) {
+    const int U = units_of(g);
+    int p = 1;
+    while (p < kPersistWarps && 2 * p <= U && (int64_t)(kPersistWarps / p) * tile_bytes(g) > target)
+        p *= 2;
+    *ppc = p;
+    *tpc = kPersistWarps / p;
+}
+
+// Item byte target: about 8 items per CTA, at least 64 KB.
+int64_t item_target(int64_t total, int ncta) {
+    const int64_t t = total / ((int64_t)ncta * 8);
+    return t < 65536 ? 65536 : t;
+}
+
+void fill_prob(Prob &a, const spectra_layer &l, const Geometry &g, const uint16_t *x, int mc,
+               void *y, int ytype) {
+    a.codes = reinterpret_cast<const uint4 *>(l.codes);
+    a.scales = reinterpret_cast<const uint4 *>(l.scales);
+    a.zeros = l.zeros;
+    a.outw = reinterpret_cast<const uint4 *>(l.outlier_w);
+    a.oidx = l.outlier_idx;
+    a.x = x;
+    a.y = y;
+    a.n = l.n;
+    a.k = l.k;
+    a.m = mc;
+    a.G = g.G;
+    a.S = g.S;
+    a.O8 = g.O8;
+    a.n_o = g.n_o;
+    a.T = g.T;
+    a.U = units_of(g);
+    a.ppc = 1;
+    a.tpc = 1;
+    a.cl = 1;
+    a.ytype = ytype;
+    a.items = 0;
+}
+
+std::mutex g_attr_mu;
+
+// Raise the dynamic shared-memory limit of one kernel, once per device.
+template <typename K>
+cudaError_t prepare_kernel(K kernel, bool *done, const DeviceInfo &dev) {
+    std::lock_guard<std::mutex> lock(g_attr_mu);
     if (dev.device >= 0 && dev.device < 64 && done[dev.device]) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<MB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)dev.smem_optin);
     if (e == cudaSuccess && dev.device >= 0 && dev.device < 64) done[dev.device] = true;
     return e;
 }
 
-template <int MB>
-cudaError_t launch_mb(const GemvArgs &a, const Plan &p, const DeviceInfo &dev, cudaStream_t s) {
-    cudaError_t pe = prepare_kernel<MB>(dev);
-    if (pe != cudaSuccess) return pe;
+template <typename K, typename A>
+cudaError_t launch_kernel(K kernel, const A &args, unsigned grid, size_t smem, int nw, int cl,
+                          cudaStream_t s) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.grid, 1, 1);
-    cfg.blockDim = dim3(p.nw * 32, 1, 1);
-    cfg.dynamicSmemBytes = p.smem;
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(nw * 32, 1, 1);
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attrs[2];
     int na = 0;
     attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attrs[na].val.programmaticStreamSerializationAllowed = 1;
     ++na;
-    if (p.cl > 1) {
+    if (cl > 1) {
         attrs[na].id = cudaLaunchAttributeClusterDimension;
-        attrs[na].val.clusterDim.x = p.cl;
+        attrs[na].val.clusterDim.x = cl;
         attrs[na].val.clusterDim.y = 1;
         attrs[na].val.clusterDim.z = 1;
         ++na;
     }
     cfg.attrs = attrs;
     cfg.numAttrs = na;
-    return cudaLaunchKernelEx(&cfg, gemv_kernel<MB>, a);
+    return cudaLaunchKernelEx(&cfg, kernel, args);
+}
+
+// The persistent launch over the `count` problems filled in args.probs.
+template <int MB>
+spectra_status run_persistent(PersistArgs &args, int count, const DeviceInfo &dev, cudaStream_t s) {
+    static bool done[64];
+    Smem sm = {1, 0, 0, 0};
+    int items = 0;
+    int64_t total = 0;
+    for (int i = 0; i < count; ++i) {
+        const Prob &a = args.probs[i];
+        total += (int64_t)a.T * tile_bytes(Geometry::of(a.n, a.k, a.n_o));
+    }
+    const int64_t target = item_target(total, dev.sm_count);
+    total = 0;
+    for (int i = 0; i < count; ++i) {
+        Prob &a = args.probs[i];
+        const Geometry g = Geometry::of(a.n, a.k, a.n_o);
+        item_shape(g, target, &a.ppc, &a.tpc);
+        a.items = (int)cdiv(a.T, a.tpc);
+        args.item_start[i] = items;
+        items += a.items;
+        total += (int64_t)a.T * tile_bytes(g);
+        sm.xg = max(sm.xg, 8 * a.S);
+        sm.xo = max(sm.xo, 8 * kOB * (a.U - a.S));
+    }
+    args.item_start[count] = items;
+    args.count = count;
+    sm.depth = fit_depth(MB, kPersistWarps, sm, dev.smem_optin);
+    if (sm.depth > 2) sm.depth = 2;  // 16 warps x 2 stages keep ~150 KB in flight per SM
+    if (sm.depth == 0) return SPECTRA_ERR_SHAPE;
+    args.sm = sm;
+    int ncta = dev.sm_count;
+    if (ncta > kMaxCtas) ncta = kMaxCtas;
+    if (ncta > items) ncta = items;
+    // contiguous item ranges of about equal bytes
+    int64_t acc = 0;
+    int c = 1;
+    args.cta_first[0] = 0;
+    for (int i = 0; i < count && c < ncta; ++i) {
+        const Prob &a = args.probs[i];
+        const Geometry g = Geometry::of(a.n, a.k, a.n_o);
+        for (int it = 0; it < a.items && c < ncta; ++it) {
+            const int tiles = min(a.tpc, a.T - it * a.tpc);
+            acc += (int64_t)tiles * tile_bytes(g);
+            while (c < ncta && acc * ncta >= total * (int64_t)c)
+                args.cta_first[c++] = args.item_start[i] + it + 1;
+        }
+    }
+    while (c <= ncta) args.cta_first[c++] = items;
+    cudaError_t e = prepare_kernel(gemv_persistent_kernel<MB>, done, dev);
+    if (e != cudaSuccess) return SPECTRA_ERR_CUDA;
+    e = launch_kernel(gemv_persistent_kernel<MB>, args, (unsigned)ncta,
+                      stage_bytes(MB, kPersistWarps, sm), kPersistWarps, 1, s);
+    return e == cudaSuccess ? SPECTRA_OK : SPECTRA_ERR_CUDA;
+}
+
+template <int MB>
+spectra_status run_cluster(const Prob &a0, const ClusterPlan &p, const DeviceInfo &dev,
+                           cudaStream_t s) {
+    static bool done[64];
+    ClusterArgs args;
+    args.p = a0;
+    args.p.ppc = p.ppc;
+    args.p.tpc = p.tpc;
+    args.p.cl = p.cl;
+    args.sm = p.sm;
+    cudaError_t e = prepare_kernel(gemv_cluster_kernel<MB>, done, dev);
+    if (e != cudaSuccess) return SPECTRA_ERR_CUDA;
+    e = launch_kernel(gemv_cluster_kernel<MB>, args, p.grid, stage_bytes(MB, kClusterWarps, p.sm),
+                      kClusterWarps, p.cl, s);
+    return e == cudaSuccess ? SPECTRA_OK : SPECTRA_ERR_CUDA;
+}
+
+// One matrix, MB batch rows: the persistent kernel when the matrix gives every
+// SM several balanced items (large matrices), else the cluster kernel.
+template <int MB>
+spectra_status run_one(const Prob &a, const DeviceInfo &dev, cudaStream_t s) {
+    const Geometry g = Geometry::of(a.n, a.k, a.n_o);
+    const int64_t total = (int64_t)g.T * tile_bytes(g);
+    int ppc, tpc;
+    item_shape(g, item_target(total, dev.sm_count), &ppc, &tpc);
+    const int64_t items = cdiv(g.T, tpc);
+    if (items >= 4LL * dev.sm_count && total >= (int64_t)dev.sm_count * 512 * 1024) {
+        static std::mutex mu;
+        static PersistArgs args;  // large: kept off the stack, guarded by the mutex
+        std::lock_guard<std::mutex> lock(mu);
+        args.probs[0] = a;
+        return run_persistent<MB>(args, 1, dev, s);
+    }
+    ClusterPlan p;
+    if (!plan_cluster(g, MB, dev, &p)) return SPECTRA_ERR_SHAPE;
+    return run_cluster<MB>(a, p, dev, s);
 }
 
 }  // namespace
+
+spectra_status device_error(bool *raised, cudaStream_t s) {
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbolAsync(&v, g_device_error, sizeof v, 0, cudaMemcpyDeviceToHost, s) !=
+        cudaSuccess)
+        return SPECTRA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SPECTRA_ERR_CUDA;
+    *raised = v != 0;
+    if (v != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof zero, 0, cudaMemcpyHostToDevice,
+                                    s) != cudaSuccess ||
+            cudaStreamSynchronize(s) != cudaSuccess)
+            return SPECTRA_ERR_CUDA;
+    }
+    return SPECTRA_OK;
+}
 
 spectra_status launch_gemv(const spectra_layer &l, const uint16_t *x, int m, void *y, int ytype,
                            cudaStream_t s, const DeviceInfo &dev) {
@@ -472,35 +1020,35 @@ spectra_status launch_gemv(const spectra_layer &l, const uint16_t *x, int m, voi
     while (done < m) {
         const int mc = (m - done) > 8 ? 8 : (m - done);
         const int MB = mc == 1 ? 1 : (mc == 2 ? 2 : (mc <= 4 ? 4 : 8));
-        Plan p;
-        const int max_warps = MB <= 2 ? MaxWarps<1>::value : MaxWarps<8>::value;
-        if (!make_plan(g, MB, max_warps, dev, &p)) return SPECTRA_ERR_SHAPE;
-        GemvArgs a;
-        a.codes = reinterpret_cast<const uint4 *>(l.codes);
-        a.scales = reinterpret_cast<const uint4 *>(l.scales);
-        a.zeros = l.zeros;
-        a.outw = reinterpret_cast<const uint4 *>(l.outlier_w);
-        a.oidx = l.outlier_idx;
-        a.x = x + (size_t)done * l.k;
-        a.y = (ytype == SPECTRA_F32)
-                  ? (void *)(reinterpret_cast<float *>(y) + (size_t)done * l.n)
-                  : (void *)(reinterpret_cast<uint16_t *>(y) + (size_t)done * l.n);
-        a.n = l.n; a.k = l.k; a.m = mc;
-        a.G = g.G; a.S = g.S; a.O8 = g.O8; a.n_o = g.n_o; a.T = g.T;
-        a.ppc = p.ppc; a.tpc = p.tpc; a.cl = p.cl;
-        a.ytype = ytype;
-        a.smem_sg = p.smem_sg; a.smem_oc = p.smem_oc;
-        cudaError_t e;
+        Prob a;
+        void *yc = (ytype == SPECTRA_F32)
+                       ? (void *)(reinterpret_cast<float *>(y) + (size_t)done * l.n)
+                       : (void *)(reinterpret_cast<uint16_t *>(y) + (size_t)done * l.n);
+        fill_prob(a, l, g, x + (size_t)done * l.k, mc, yc, ytype);
+        spectra_status st;
         switch (MB) {
-            case 1: e = launch_mb<1>(a, p, dev, s); break;
-            case 2: e = launch_mb<2>(a, p, dev, s); break;
-            case 4: e = launch_mb<4>(a, p, dev, s); break;
-            default: e = launch_mb<8>(a, p, dev, s); break;
+            case 1: st = run_one<1>(a, dev, s); break;
+            case 2: st = run_one<2>(a, dev, s); break;
+            case 4: st = run_one<4>(a, dev, s); break;
+            default: st = run_one<8>(a, dev, s); break;
         }
-        if (e != cudaSuccess) return SPECTRA_ERR_CUDA;
+        if (st != SPECTRA_OK) return st;
         done += mc;
     }
     return SPECTRA_OK;
+}
+
+spectra_status launch_gemv_batched(const spectra_layer *layers, const uint16_t *const *xs,
+                                   void *const *ys, int count, int ytype, cudaStream_t s,
+                                   const DeviceInfo &dev) {
+    static std::mutex mu;
+    static PersistArgs args;  // large: kept off the stack, guarded by the mutex
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < count; ++i) {
+        const Geometry g = Geometry::of(layers[i].n, layers[i].k, layers[i].n_outliers);
+        fill_prob(args.probs[i], layers[i], g, xs[i], 1, ys[i], ytype);
+    }
+    return run_persistent<1>(args, count, dev, s);
 }
 
 }  // namespace spectra

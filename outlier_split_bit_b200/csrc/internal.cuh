@@ -61,8 +61,16 @@ cudaError_t launch_unpack(const spectra_layer &l, uint8_t *codes, uint16_t *scal
                           cudaStream_t s);
 
 // ---- matvec (gemv.cu) ----
+constexpr int kMaxBatch = SPECTRA_MAX_BATCH;
 // CUDA-core decode matvec for 1 <= m <= 15 batch rows.
 spectra_status launch_gemv(const spectra_layer &l, const uint16_t *x, int m, void *y, int ytype,
                            cudaStream_t s, const DeviceInfo &dev);
+// Reads (and clears) the flag the matvec kernels raise when a bounded wait
+// for a weight copy gives up.
+spectra_status device_error(bool *raised, cudaStream_t s);
+// Independent batch-1 matvecs in one launch (count <= kMaxBatch).
+spectra_status launch_gemv_batched(const spectra_layer *layers, const uint16_t *const *xs,
+                                   void *const *ys, int count, int ytype, cudaStream_t s,
+                                   const DeviceInfo &dev);
 
 }  // namespace spectra
