@@ -84,6 +84,9 @@ typedef enum { SPECTRA_F32 = 0, SPECTRA_BF16 = 1 } spectra_dtype;
 /* Largest number of matvecs one spectra_gemv_batched call accepts. */
 #define SPECTRA_MAX_BATCH 224
 
+/* Largest in_features k that spectra_pack_plan_noalloc accepts. */
+#define SPECTRA_NOALLOC_MAX_K 65536
+
 /* A packed layer: a plain view of caller-owned device buffers. */
 typedef struct {
     int32_t n;                   /* out_features */
@@ -146,6 +149,32 @@ SPECTRA_API spectra_status spectra_pack_plan(const uint16_t *w, const float *gai
                                  double tau, double *kappa_out, int32_t *idx_out,
                                  int32_t *n_outliers_out, void *workspace,
                                  size_t workspace_bytes, void *stream);
+
+/*
+ * spectra_pack_plan for callers that cannot allocate device memory.  The
+ * paper has no counterpart to this entry point; it exists for callers that
+ * must not call cudaMalloc while they plan a layer (code running under a
+ * foreign allocator or a pre-carved memory pool, tools that must leave a
+ * process's allocations untouched).  Same arguments, results and errors as
+ * spectra_pack_plan, minus the workspace: the scratch it needs (kurtosis
+ * values when kappa_out is NULL, the outlier count, an error word) lives in
+ * one fixed library-owned device array of 512 KiB + 256 bytes that every GPU
+ * which loads the library holds until the process exits.
+ *   - k must not exceed SPECTRA_NOALLOC_MAX_K (SPECTRA_ERR_SHAPE otherwise).
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   - All calls on a device share the array and it keeps the last call's
+ *     contents.  Calls that overlap on the GPU (issued on two streams or from
+ *     two host threads for the same device) race on it: serialise them.
+ *     Each call clears the words that must start at zero.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before capturing a stream into a graph.
+ * Synchronous, like spectra_pack_plan.
+ */
+SPECTRA_API spectra_status spectra_pack_plan_noalloc(const uint16_t *w, const float *gain,
+                                                     int32_t n, int32_t k, double tau,
+                                                     double *kappa_out, int32_t *idx_out,
+                                                     int32_t *n_outliers_out, void *stream);
 
 /*
  * Group quantiser + packer (abstract: Group-32 4-bit microscaling with
