@@ -68,7 +68,8 @@ constexpr int kOB = 8;                         // outlier octets per unit
 constexpr int kSgBytes = 8 * 512 + 512 + 128;  // codes + scales + zeros of a warp per super-group
 constexpr int kOctBytes = 512;                 // outlier bytes of a warp per octet
 constexpr int kStageBytes = kSgBytes;          // one ring stage (16-byte multiple)
-constexpr uint32_t kSpinLimit = 1u << 22;      // try_wait rounds before a wait gives up
+constexpr uint32_t kSpinLimit = 1u << 12;      // try_wait rounds before a wait gives up
+constexpr uint32_t kSuspendNs = 500000;        // per-round suspend hint: the limit is ~2 s
 constexpr int kMaxCtas = 320;                  // persistent grid bound (2 x SMs of a B200 + margin)
 
 // Set (bit 0) when a bounded wait in a kernel gave up; read and cleared by
@@ -125,8 +126,10 @@ __device__ __forceinline__ void named_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// floor(total * s / P); total * s stays far below 2^31 (total <= a few
+// thousand units, s <= 16), so 32-bit arithmetic is exact.
 __device__ __forceinline__ int split_at(int total, int s, int P) {
-    return (int)(((int64_t)total * s) / P);
+    return (int)((unsigned)(total * s) / (unsigned)P);
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
@@ -157,12 +160,14 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     for (uint32_t i = 0; i < kSpinLimit; ++i) {
         uint32_t ok;
+        // the thread sleeps until the phase completes or the hint expires,
+        // so waiting warps leave the issue slots to the computing ones
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
             "selp.u32 %0, 1, 0, p;\n\t}"
             : "=r"(ok)
-            : "r"(bar), "r"(parity)
+            : "r"(bar), "r"(parity), "r"(kSuspendNs)
             : "memory");
         if (ok) return true;
     }
@@ -397,8 +402,23 @@ __device__ __forceinline__ void compute_group(const uint8_t *stage, int gg, int 
 
 template <int MB>
 __device__ __forceinline__ void compute_sg(const uint8_t *stage, int ng, int lane,
-                                           const uint32_t *xs_sg, const float *xsum_sg,
+                                           const uint32_t *xs_sg, const float *xsum_in,
                                            float *yacc) {
+    // the group sums of the super-group: for MB <= 2 vector loads into
+    // registers, for wider batches straight from shared memory
+    constexpr int kRegSums = MB <= 2 ? 8 * MB : 1;
+    float xsum_reg[kRegSums];
+    if constexpr (MB <= 2) {
+#pragma unroll
+        for (int i = 0; i < 2 * MB; ++i) {
+            const float4 v = reinterpret_cast<const float4 *>(xsum_in)[i];
+            xsum_reg[4 * i] = v.x;
+            xsum_reg[4 * i + 1] = v.y;
+            xsum_reg[4 * i + 2] = v.z;
+            xsum_reg[4 * i + 3] = v.w;
+        }
+    }
+    const float *xsum_sg = MB <= 2 ? xsum_reg : xsum_in;
     const uint4 sc = *reinterpret_cast<const uint4 *>(stage + 4096 + lane * 16);
     const uint32_t zw = *reinterpret_cast<const uint32_t *>(stage + 4608 + lane * 4);
     const uint32_t scw[4] = {sc.x, sc.y, sc.z, sc.w};
@@ -819,17 +839,32 @@ bool plan_cluster(const Geometry &g, int MB, const DeviceInfo &dev, ClusterPlan 
     return found;
 }
 
-// Persistent kernel: item = tpc tiles x ppc slices.  ppc is the smallest power
-// of two (<= 16, <= units per tile) that keeps an item at or below
-// `target` bytes, so each CTA walks several items (balance) while as many
-// warps as possible own whole tiles (no reduction, no barrier).
+// Persistent kernel: item = tpc tiles x ppc slices, ppc a power of two <= 16.
+// Among the shapes whose item stays within twice `target` bytes (so that each
+// CTA walks several items), take the one whose slices are most even -- the
+// warps of a tile meet on a barrier at the end of an item -- and, on a tie,
+// the fewest slices (more warps own whole tiles: no reduction at all).
 void item_shape(const Geometry &g, int64_t target, int *ppc, int *tpc) {
-    const int U = units_of(g);
-    int p = 1;
-    while (p < kPersistWarps && 2 * p <= U && (int64_t)(kPersistWarps / p) * tile_bytes(g) > target)
-        p *= 2;
-    *ppc = p;
-    *tpc = kPersistWarps / p;
+    const int OB = (int)cdiv(g.O8, kOB);
+    const int U = g.S + OB;
+    const double tb = (double)tile_bytes(g);
+    int best_p = 0;
+    double best_eff = -1.0;
+    for (int p = 1; p <= kPersistWarps; p *= 2) {
+        if (p > 1 && p > U) break;
+        if ((double)(kPersistWarps / p) * tb > 2.0 * (double)target && p < kPersistWarps) continue;
+        // slowest slice vs mean slice, in bytes
+        const double mean = tb / p;
+        const double mx = (double)cdiv(g.S, p) * kSgBytes + (double)cdiv(OB, p) * kOB * kOctBytes;
+        const double eff = mean / mx;
+        if (eff > best_eff + 1e-9) {
+            best_eff = eff;
+            best_p = p;
+        }
+    }
+    if (best_p == 0) best_p = kPersistWarps;
+    *ppc = best_p;
+    *tpc = kPersistWarps / best_p;
 }
 
 // Item byte target: about 8 items per CTA, at least 64 KB.
