@@ -174,6 +174,23 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     return false;
 }
 
+// Bounded wait without a suspend hint (for phases completed by the tensor
+// cores, which the suspended form does not wake up for promptly).
+__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity) {
+    for (uint32_t i = 0; i < (1u << 26); ++i) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (ok) return true;
+    }
+    return false;
+}
+
 // ---------------------------------------------------------------- shared memory
 
 // Shared-memory layout of one CTA.  Bulk x is stored per group as 16 BF16
@@ -1029,6 +1046,401 @@ spectra_status run_one(const Prob &a, const DeviceInfo &dev, cudaStream_t s) {
     return run_cluster<MB>(a, p, dev, s);
 }
 
+// ---------------------------------------------------------------- tensor-core path (M = 16..32)
+//
+// y[m][n] for 16 < m_rows <= 32 (MB = 16 or 32 batch rows) with the fifth-
+// generation tensor cores.  A CTA owns 128 rows (4 tiles, one per warp: TMEM
+// lane = row = thread, as in the decoder above) and a cluster of `cl` CTAs
+// splits the units (super-groups, outlier batches) of those rows.  Per
+// K-slice of 64 columns each thread dequantises its row exactly in FP32,
+// s * (c - z) = fma(s, 128 + c, -s * (128 + z)) (every term exact in FP32),
+// or converts its 64 BF16 outlier weights, and stores them into a double-
+// buffered TMEM A operand (tcgen05.st).  x is staged once per unit in shared
+// memory as TF32 in the K-major canonical layout (B operand, no swizzle:
+// 8-row x 16-byte core matrices, k-halves 128 B apart, 8-row groups 256 B
+// apart).  One thread issues tcgen05.mma kind::tf32 (M = 128, N = MB,
+// K = 8) with the FP32 accumulator in TMEM and commits to an mbarrier per A
+// buffer.  TF32 keeps FP32's range; its 11-bit significand rounds the
+// dequantised weights by at most 2^-10 relative (BF16 x and the BF16
+// outlier weights are exact in TF32).
+constexpr int kTcWarps = 4;       // 128 rows per CTA
+constexpr int kTcSub = 64;        // K columns per A buffer
+constexpr int kTcNA = 4;          // TMEM A buffers (MMA pipeline depth in K-slices)
+constexpr int kTcNX = 4;          // x buffers in shared memory (>= kTcNA, see below)
+constexpr int kTcTmemCols = 512;  // A buffers [0, 256), D at 256
+
+struct TcArgs {
+    Prob p;        // problem (MB batch rows in p.m <= MB)
+    int depth;     // ring stages per warp
+    int xbuf;      // bytes of one x buffer (256 columns x MB rows x 4 B)
+};
+
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    // start address, leading and stride byte offsets (all >> 4), version 1,
+    // base offset 0, no swizzle
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
+template <int MB>
+__device__ __forceinline__ uint32_t tf32_idesc() {
+    // D = F32 (bits 4-5 = 1), A = B = TF32 (format 2 at bits 7 and 10),
+    // both K-major, N = MB (>> 3 at bit 17), M = 128 (>> 4 at bit 24)
+    return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(MB >> 3) << 17) | (8u << 24);
+}
+
+// x of one unit, prefetched into registers one unit ahead and then written
+// to shared memory as TF32 in the K-major canonical layout: column-step j
+// (8 columns) at j * MB * 32 bytes; inside it, (m / 8) * 256 + (kk / 4) *
+// 128 + (m % 8) * 16 + (kk % 4) * 4.  A super-group is MB rows x 256
+// consecutive columns (16-byte loads of 8 columns); an outlier batch is
+// MB rows x 64 gathered columns (padding slots read as 0).
+template <int MB>
+struct XPre {
+    uint4 v[MB / 4];
+};
+
+template <int MB>
+__device__ __forceinline__ void tc_load_x(const Prob &a, bool is_sg, int idx, XPre<MB> &r) {
+    if (is_sg) {
+#pragma unroll
+        for (int i = 0; i < MB / 4; ++i) {
+            const int c = threadIdx.x + kTcWarps * 32 * i;
+            const int m = c >> 5, col = 256 * idx + 8 * (c & 31);
+            r.v[i] = (m < a.m && col < a.k)
+                         ? *reinterpret_cast<const uint4 *>(a.x + (size_t)m * a.k + col)
+                         : make_uint4(0u, 0u, 0u, 0u);
+        }
+    } else {
+        const int slot = threadIdx.x & 63;
+        const int j = 8 * kOB * idx + slot;
+        const int src = j < a.n_o ? a.oidx[j] : -1;
+        uint32_t *u = reinterpret_cast<uint32_t *>(r.v);
+#pragma unroll
+        for (int i = 0; i < MB / 2; ++i) {
+            const int m = (threadIdx.x >> 6) + 2 * i;
+            u[i] = (src >= 0 && m < a.m) ? (uint32_t)a.x[(size_t)m * a.k + src] : 0u;
+        }
+    }
+}
+
+template <int MB>
+__device__ __forceinline__ void tc_store_x(bool is_sg, const XPre<MB> &r, uint8_t *xb) {
+    if (is_sg) {
+#pragma unroll
+        for (int i = 0; i < MB / 4; ++i) {
+            const int c = threadIdx.x + kTcWarps * 32 * i;
+            const int m = c >> 5, j = c & 31;
+            uint8_t *dst = xb + (size_t)j * MB * 32 + (m >> 3) * 256 + (m & 7) * 16;
+            const uint4 v = r.v[i];
+            *reinterpret_cast<float4 *>(dst) = make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
+            *reinterpret_cast<float4 *>(dst + 128) = make_float4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w));
+        }
+    } else {
+        const int slot = threadIdx.x & 63;
+        const int j = slot >> 3, kk = slot & 7;
+        const uint32_t *u = reinterpret_cast<const uint32_t *>(r.v);
+#pragma unroll
+        for (int i = 0; i < MB / 2; ++i) {
+            const int m = (threadIdx.x >> 6) + 2 * i;
+            *reinterpret_cast<float *>(xb + (size_t)j * MB * 32 + (m >> 3) * 256 + (kk >> 2) * 128 +
+                                       (m & 7) * 16 + (kk & 3) * 4) = bf16_lo(u[i]);
+        }
+    }
+}
+
+// 32 dequantised weights of one group (exact FP32), in column order.
+__device__ __forceinline__ void tc_dequant_group(const uint4 &q, float s, uint32_t z, float *out) {
+    const float off = -s * (float)(128 + z);  // exact: 11 x 8 significant bits
+    const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+#pragma unroll
+        for (int sp = 0; sp < 4; ++sp) {
+            const uint32_t p = ((wv[w] >> (4 * sp)) & 0x000F000Fu) | 0x43004300u;
+            const float2 c2 = make_float2(__uint_as_float(p << 16), __uint_as_float(p & 0xFFFF0000u));
+            const float2 r = __ffma2_rn(c2, make_float2(s, s), make_float2(off, off));
+            out[8 * w + sp] = r.x;
+            out[8 * w + sp + 4] = r.y;
+        }
+    }
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_st(uint32_t taddr, const float *v) {
+    static_assert(N == 32, "32 columns per store");
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+        "%29, %30, %31, %32};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+        "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+        "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+        "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+        "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+        "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+template <int MB>
+__global__ void __launch_bounds__(kTcWarps * 32, 1) gemm_tc_kernel(const TcArgs args) {
+    extern __shared__ __align__(1024) uint8_t tsm[];
+    const Prob &a = args.p;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int cr = (a.cl > 1) ? (int)cg::this_cluster().block_rank() : 0;
+    const int blk = blockIdx.x / a.cl;
+    const int t = blk * kTcWarps + warp;  // this warp's tile
+    const bool active = t < a.T;
+    const int D = args.depth;
+    // shared memory: [ring kTcWarps x D x kStageBytes][x kTcNX x xbuf][bars][mma bars kTcNA]
+    // [tmem slot][part]
+    uint8_t *ring_base = tsm;
+    uint8_t *xbufs = ring_base + (size_t)kTcWarps * D * kStageBytes;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(xbufs + kTcNX * (size_t)args.xbuf);
+    uint64_t *mma_bar = bars + kTcWarps * D;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_bar + kTcNA);
+    float *part = reinterpret_cast<float *>(tmem_slot + 4);  // [128][MB]
+
+    // units of this CTA (same for every warp): super-groups, then outlier batches
+    const int OB = a.U - a.S;
+    const int sg0 = split_at(a.S, cr, a.cl), sg1 = split_at(a.S, cr + 1, a.cl);
+    const int ob0 = split_at(OB, cr, a.cl), ob1 = split_at(OB, cr + 1, a.cl);
+    const int nsg = sg1 - sg0, nunits = nsg + (ob1 - ob0);
+
+    // TMEM: one warp allocates, everyone reads the base after the barrier
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(kTcTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    if (threadIdx.x == 0) {
+        for (int b = 0; b < kTcNA; ++b) mbar_init(smem_u32(&mma_bar[b]), 1u);
+    }
+    Ring ring;
+    ring_init(ring, ring_base + (size_t)warp * D * kStageBytes, bars + warp * D, D, lane);
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem_warp = tmem + ((uint32_t)(32 * warp) << 16);
+
+    pdl_launch_dependents();
+    int next = 0;
+    if (active)
+        for (; next < nunits && next < D; ++next) {
+            const int gu = next < nsg ? sg0 + next : a.S + ob0 + (next - nsg);
+            ring_issue(ring, a, t, gu, lane);
+        }
+    pdl_wait();
+
+    const uint32_t idesc = tf32_idesc<MB>();
+    XPre<MB> xpre;
+    if (nunits > 0) tc_load_x<MB>(a, nsg > 0, nsg > 0 ? sg0 : ob0, xpre);
+    bool ok = true;
+    int q = 0;  // K-slice counter
+    uint4 sc = make_uint4(0u, 0u, 0u, 0u);
+    uint32_t zw = 0u;
+    for (int u = 0; u < nunits; ++u) {
+        const bool is_sg = u < nsg;
+        const int idx = is_sg ? sg0 + u : ob0 + (u - nsg);
+        const int nsub = is_sg ? 4 : 1;
+        // x buffer u % kTcNX was last read by the MMAs of unit u - kTcNX, whose
+        // last slice is at most q - kTcNX <= q - kTcNA: the A-buffer wait below
+        // (MMAs complete in issue order) covers it
+        uint8_t *xb = xbufs + (size_t)(u % kTcNX) * args.xbuf;
+        const uint8_t *stage = nullptr;
+        if (active) stage = ring_acquire(ring, lane);
+        if (active && !stage) ok = false;
+        for (int c = 0; c < nsub; ++c, ++q) {
+            const int qb = q % kTcNA;
+            if (q >= kTcNA &&
+                !mbar_wait_spin(smem_u32(&mma_bar[qb]), (uint32_t)((q - kTcNA) / kTcNA) & 1u)) {
+                ok = false;
+                if (threadIdx.x == 0) atomicOr(&g_device_error, 1u);
+            }
+            if (c == 0) {
+                tc_store_x<MB>(is_sg, xpre, xb);
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                if (u + 1 < nunits) {
+                    const bool nsgu = u + 1 < nsg;
+                    tc_load_x<MB>(a, nsgu, nsgu ? sg0 + u + 1 : ob0 + (u + 1 - nsg), xpre);
+                }
+            }
+            if (active) {
+                float v[kTcSub];
+                if (stage) {
+                    if (is_sg) {
+                        if (c == 0) {
+                            sc = *reinterpret_cast<const uint4 *>(stage + 4096 + lane * 16);
+                            zw = *reinterpret_cast<const uint32_t *>(stage + 4608 + lane * 4);
+                        }
+                        const uint32_t scw[4] = {sc.x, sc.y, sc.z, sc.w};
+                        const int ng = min(8, a.G - 8 * idx);
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int gg = 2 * c + h;
+                            if (gg < ng) {
+                                const uint4 qq = *reinterpret_cast<const uint4 *>(stage + gg * 512 + lane * 16);
+                                const uint32_t sw = scw[gg >> 1];
+                                const float s = __half2float(__ushort_as_half(
+                                    (unsigned short)((gg & 1) ? (sw >> 16) : (sw & 0xFFFFu))));
+                                tc_dequant_group(qq, s, (zw >> (4 * gg)) & 0xFu, v + 32 * h);
+                            } else {
+#pragma unroll
+                                for (int i = 0; i < 32; ++i) v[32 * h + i] = 0.f;
+                            }
+                        }
+                    } else {
+                        const int nv = min(kOB, a.O8 - kOB * idx);
+#pragma unroll
+                        for (int o = 0; o < kOB; ++o) {
+                            uint4 w4 = make_uint4(0u, 0u, 0u, 0u);
+                            if (o < nv) w4 = *reinterpret_cast<const uint4 *>(stage + o * 512 + lane * 16);
+                            const uint32_t wp[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                v[8 * o + 2 * e] = bf16_lo(wp[e]);
+                                v[8 * o + 2 * e + 1] = bf16_hi(wp[e]);
+                            }
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < kTcSub; ++i) v[i] = 0.f;
+                }
+                tmem_st<32>(tmem_warp + (uint32_t)(qb * kTcSub), v);
+                tmem_st<32>(tmem_warp + (uint32_t)(qb * kTcSub + 32), v + 32);
+                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+            }
+            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                const uint32_t xs = smem_u32(xb) + (uint32_t)(c * 8 * MB * 32);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint64_t bdesc = umma_desc(xs + (uint32_t)(j * MB * 32), 128u, 256u);
+                    const uint32_t acc = (q > 0 || j > 0) ? 1u : 0u;
+                    asm volatile(
+                        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %3, 0;\n\t"
+                        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %4, p;\n\t}" ::"r"(
+                            tmem + (uint32_t)(kTcNA * kTcSub)),
+                        "r"(tmem + (uint32_t)(qb * kTcSub + 8 * j)), "l"(bdesc), "r"(acc),
+                        "r"(idesc)
+                        : "memory");
+                }
+                asm volatile(
+                    "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                        smem_u32(&mma_bar[qb]))
+                    : "memory");
+            }
+        }
+        if (active) {
+            ring_release(ring);
+            if (next < nunits) {
+                const int gu = next < nsg ? sg0 + next : a.S + ob0 + (next - nsg);
+                ring_issue(ring, a, t, gu, lane);
+                ++next;
+            }
+        }
+    }
+    // the last commit covers every MMA of this CTA
+    if (q > 0 && !mbar_wait_spin(smem_u32(&mma_bar[(q - 1) % kTcNA]), (uint32_t)((q - 1) / kTcNA) & 1u)) {
+        ok = false;
+        if (threadIdx.x == 0) atomicOr(&g_device_error, 1u);
+    }
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    float yv[MB];
+#pragma unroll
+    for (int m = 0; m < MB; ++m) yv[m] = 0.f;
+    if (q > 0) {
+#pragma unroll
+        for (int h = 0; h < MB / 16; ++h)
+            tmem_ld16(tmem_warp + (uint32_t)(kTcNA * kTcSub) + 16u * h, yv + 16 * h);
+    }
+    ring_drain(ring);
+    (void)ok;
+    // cluster split: rank 0 adds the partial sums of all ranks in rank order
+    if (a.cl > 1) {
+        cg::cluster_group cluster = cg::this_cluster();
+#pragma unroll
+        for (int m = 0; m < MB; ++m) part[threadIdx.x * MB + m] = yv[m];
+        cluster.sync();
+        if (cr == 0) {
+#pragma unroll
+            for (int m = 0; m < MB; ++m) yv[m] = 0.f;
+            for (int rk = 0; rk < a.cl; ++rk) {
+                const float *rp = cluster.map_shared_rank(part, rk) + threadIdx.x * MB;
+#pragma unroll
+                for (int m = 0; m < MB; ++m) yv[m] += rp[m];
+            }
+        }
+        cluster.sync();
+    }
+    if (cr == 0 && active) {
+#pragma unroll
+        for (int m = 0; m < MB; ++m) store_y(a, t, lane, m, yv[m]);
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (warp == 0) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(kTcTmemCols));
+    }
+}
+
+size_t tc_smem_bytes(int MB, int depth) {
+    return (size_t)kTcWarps * depth * kStageBytes + kTcNX * (size_t)256 * MB * 4 +
+           (size_t)(kTcWarps * depth + kTcNA) * 8 + 16 + (size_t)kTcWarps * 32 * MB * 4;
+}
+
+template <int MB>
+spectra_status run_tc(const Prob &a0, const DeviceInfo &dev, cudaStream_t s) {
+    static bool done[64];
+    TcArgs args;
+    args.p = a0;
+    const Geometry g = Geometry::of(a0.n, a0.k, a0.n_o);
+    const int64_t blocks = cdiv(g.T, kTcWarps);
+    int cl = (int)cdiv(dev.sm_count, blocks);
+    const int units = units_of(g);
+    if (cl > 8) cl = 8;
+    if (cl > units) cl = units;
+    if (cl < 1) cl = 1;
+    args.p.cl = cl;
+    args.xbuf = 256 * MB * 4;
+    int depth = 4;
+    while (depth > 1 && tc_smem_bytes(MB, depth) > dev.smem_optin) --depth;
+    args.depth = depth;
+    const size_t smem = tc_smem_bytes(MB, depth);
+    if (smem > dev.smem_optin) return SPECTRA_ERR_SHAPE;
+    cudaError_t e = prepare_kernel(gemm_tc_kernel<MB>, done, dev);
+    if (e != cudaSuccess) return SPECTRA_ERR_CUDA;
+    e = launch_kernel(gemm_tc_kernel<MB>, args, (unsigned)(blocks * cl), smem, kTcWarps, cl, s);
+    return e == cudaSuccess ? SPECTRA_OK : SPECTRA_ERR_CUDA;
+}
+
 }  // namespace
 
 spectra_status device_error(bool *raised, cudaStream_t s) {
@@ -1051,6 +1463,12 @@ spectra_status device_error(bool *raised, cudaStream_t s) {
 spectra_status launch_gemv(const spectra_layer &l, const uint16_t *x, int m, void *y, int ytype,
                            cudaStream_t s, const DeviceInfo &dev) {
     const Geometry g = Geometry::of(l.n, l.k, l.n_outliers);
+    if (m >= 16) {
+        // a real dense contraction: the tensor-core path
+        Prob a;
+        fill_prob(a, l, g, x, m, y, ytype);
+        return m <= 16 ? run_tc<16>(a, dev, s) : run_tc<32>(a, dev, s);
+    }
     int done = 0;
     while (done < m) {
         const int mc = (m - done) > 8 ? 8 : (m - done);

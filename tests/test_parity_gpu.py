@@ -322,3 +322,36 @@ def test_batched_against_oracle(spec):
 def test_device_status_clear_after_all_launches():
     """No bounded wait in any matvec above gave up."""
     sp.spectra_device_status()
+
+
+@pytest.mark.parametrize("m", [16, 17, 24, 32])
+@pytest.mark.parametrize("spec,tau", [(wl.SINGLE_512, 3.0), (wl.MatrixSpec("single", 40, 96, 3), 1.2),
+                                      (wl.MatrixSpec("single", 300, 2080, 31), 6.0),
+                                      (wl.MatrixSpec("single", 130, 512, 0), np.inf)],
+                         ids=["512", "40x96", "300x2080", "130x512-noout"])
+def test_gemm_small_tensor_cores(spec, tau, m):
+    """M = 16..32 runs on tcgen05 (TF32 operands, FP32 accumulation in TMEM)."""
+    w, g, x, idx, kappa, lay, wb, ref = _full_pack(spec, tau, True, m=m)
+    y = sp.spectra_gemm_small(lay, x)
+    torch.cuda.synchronize()
+    sp.spectra_device_status()
+    y_ref, bound = oracle.gemm(ref.can, wb, ref.idx, wl.bits(x))
+    check_gemv(y, y_ref, bound)
+
+
+@pytest.mark.parametrize("spec", [wl.LAYER_4B[4], wl.LAYER_4B[6], wl.LAYER_4B[1]], ids=["gate", "down", "k"])
+@pytest.mark.parametrize("m", [16, 32])
+def test_decoder_layer_4b_tensor_cores(spec, m):
+    """4B-class shapes at M = 16 and 32 (batch sweep rows): sampled tiles against the oracle."""
+    w, g, x = draw(spec, m=m)
+    lay = sp.pack_layer(w, g, 6.0)
+    y = sp.spectra_gemm_small(lay, x)
+    torch.cuda.synchronize()
+    sp.spectra_device_status()
+    wb = wl.bits(w)
+    idx_np = lay.outlier_idx[: lay.n_outliers].cpu().numpy() if lay.n_outliers else np.zeros(0, np.int32)
+    T = -(-spec.n // 32)
+    tiles = sorted({0, 1, T // 2, T - 1})
+    rows, can, packed = oracle_rows(wb, idx_np, tiles)
+    y_ref, bound = oracle.gemm(can, np.ascontiguousarray(wb[rows]), idx_np, wl.bits(x))
+    check_gemv(y[:, rows], y_ref, bound)
