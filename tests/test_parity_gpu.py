@@ -330,7 +330,8 @@ def test_device_status_clear_after_all_launches():
                                       (wl.MatrixSpec("single", 130, 512, 0), np.inf)],
                          ids=["512", "40x96", "300x2080", "130x512-noout"])
 def test_gemm_small_tensor_cores(spec, tau, m):
-    """M = 16..32 runs on tcgen05 (TF32 operands, FP32 accumulation in TMEM)."""
+    """M = 16..32 runs on tcgen05 (exact BF16 c - z and x operands, FP32 per-group
+    products in TMEM, scales applied in FP32)."""
     w, g, x, idx, kappa, lay, wb, ref = _full_pack(spec, tau, True, m=m)
     y = sp.spectra_gemm_small(lay, x)
     torch.cuda.synchronize()
@@ -355,3 +356,54 @@ def test_decoder_layer_4b_tensor_cores(spec, m):
     rows, can, packed = oracle_rows(wb, idx_np, tiles)
     y_ref, bound = oracle.gemm(can, np.ascontiguousarray(wb[rows]), idx_np, wl.bits(x))
     check_gemv(y[:, rows], y_ref, bound)
+
+
+@pytest.mark.parametrize("m", [16, 32])
+def test_tensor_cores_unit_vectors_exact(m):
+    """x row r = e_{j_r}: every product is exact on the tensor cores, so row r of y
+    is column j_r of the dequantised matrix (plus its BF16 outlier column) bit for bit."""
+    spec = wl.MatrixSpec("single", 200, 1024, 16)
+    w, g, x, idx, kappa, lay, wb, ref = _full_pack(spec, 6.0, True)
+    what = oracle.dequant(ref.can)
+    wv = wl.bits(w).view(np.uint16)
+    wvals = torch.from_numpy(wv.view(np.int16)).view(torch.bfloat16).double().numpy()
+    base = [0, 1, 3, 4, 7, 8, 31, 32, 255, 256, 511, 1000, 1023] + ref.idx[:8].tolist()
+    rng = np.random.default_rng(1)
+    extra = rng.choice(1024, m, replace=False).tolist()
+    cols = (base + extra)[:m]
+    e = torch.zeros((m, 1024), dtype=torch.bfloat16, device=DEV)
+    for r, j in enumerate(cols):
+        e[r, j] = 1.0
+    y = sp.spectra_gemm_small(lay, e).cpu().numpy().astype(np.float64)
+    for r, j in enumerate(cols):
+        expect = what[:, j] + (wvals[:, j] if j in ref.idx else 0.0)
+        assert np.array_equal(y[r], expect), (r, j)
+
+
+@pytest.mark.parametrize("m,tau", [(32, 3.0), (16, 6.0), (20, 3.0)])
+def test_tensor_cores_persistent_blocks(m, tau):
+    """More 128-row blocks than SMs: each CTA walks several blocks; sampled tiles
+    (first, middle, and the ragged last block) against the oracle."""
+    spec = wl.MatrixSpec("single", 20000, 512, 8)
+    w, g, x = draw(spec, m=m)
+    lay = sp.pack_layer(w, g, tau)
+    y = sp.spectra_gemm_small(lay, x)
+    torch.cuda.synchronize()
+    sp.spectra_device_status()
+    wb = wl.bits(w)
+    idx_np = lay.outlier_idx[: lay.n_outliers].cpu().numpy() if lay.n_outliers else np.zeros(0, np.int32)
+    T = -(-spec.n // 32)
+    tiles = sorted({0, 1, 2, 3, 4, 300, 301, T - 2, T - 1})
+    rows, can, packed = oracle_rows(wb, idx_np, tiles)
+    y_ref, bound = oracle.gemm(can, np.ascontiguousarray(wb[rows]), idx_np, wl.bits(x))
+    check_gemv(y[:, rows], y_ref, bound)
+
+
+def test_tensor_cores_deterministic():
+    spec = wl.LAYER_4B[6]  # down: cluster split across CTAs
+    w, g, x = draw(spec, m=32)
+    lay = sp.pack_layer(w, g, 3.0)
+    y0 = sp.spectra_gemm_small(lay, x)
+    y1 = sp.spectra_gemm_small(lay, x)
+    torch.cuda.synchronize()
+    assert torch.equal(y0, y1)
