@@ -264,6 +264,24 @@ def extras(device, stream, peak_gbs, tau):
                          "tflops": round(2 * m * spec.n * spec.k / us * 1e-6, 2)})
         out["batch_sweep_4b_gate_9728x2560"] = rows
         del w, lay
+        # the tensor-core path on the large matrix (1 % Student-t columns)
+        rows = []
+        spec = wl.lm_head_spec(0.01)
+        w = wl.weight(spec, 0, 0, device=device)
+        g = wl.gain(spec, 0, 0, device=device)
+        lay = sp.pack_layer(w, g, tau)
+        v = lay.view()
+        for m in (1, 16, 32):
+            x = wl.activations(spec.k, m, device=device)
+            y = torch.empty((m, spec.n), device=device)
+            us, p10, p90 = time_single(
+                lambda: sp.spectra_gemm_small(lay, x, y, view=v, stream=stream), stream, 20, flush)
+            b = algorithmic_bytes(spec.n, spec.k, lay.n_outliers, m=m)
+            rows.append({"m": m, "n_outliers": lay.n_outliers, "us": round(us, 2),
+                         "gbs": round(b / us * 1e-3, 1), "frac": round(b / us * 1e-3 / peak_gbs, 3),
+                         "tflops": round(2 * m * spec.n * spec.k / us * 1e-6, 2)})
+        out["lm_head_batch_131072x3072"] = rows
+        del w, lay
     return out
 
 
@@ -341,10 +359,12 @@ def run_reference(args):
 # ---------------------------------------------------------------- our arm
 
 def kernel_source_digest() -> str:
+    """Digest of the source the matvec kernels are compiled from (gemv.cu and
+    the streaming machinery it includes); the tensor-core kernel lives apart."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "outlier_split_bit_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
-        if f.startswith("gemv"):
+        if f.startswith("gemv") or f == "stream.cuh":
             h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 

@@ -62,7 +62,8 @@ cudaError_t launch_unpack(const spectra_layer &l, uint8_t *codes, uint16_t *scal
 
 // ---- matvec (gemv.cu) ----
 constexpr int kMaxBatch = SPECTRA_MAX_BATCH;
-// CUDA-core decode matvec for 1 <= m <= 15 batch rows.
+// Decode matvec for 1 <= m <= 32 batch rows (CUDA cores below 16 rows, the
+// tensor cores from 16).
 spectra_status launch_gemv(const spectra_layer &l, const uint16_t *x, int m, void *y, int ytype,
                            cudaStream_t s, const DeviceInfo &dev);
 // Reads (and clears) the flag the matvec kernels raise when a bounded wait
@@ -72,5 +73,12 @@ spectra_status device_error(bool *raised, cudaStream_t s);
 spectra_status launch_gemv_batched(const spectra_layer *layers, const uint16_t *const *xs,
                                    void *const *ys, int count, int ytype, cudaStream_t s,
                                    const DeviceInfo &dev);
+
+// ---- tensor-core matmul (gemm_tc.cu) ----
+// y[m][n] for 16 <= m <= 32 batch rows on the tensor cores.
+spectra_status launch_tc(const spectra_layer &l, const uint16_t *x, int m, void *y, int ytype,
+                         cudaStream_t s, const DeviceInfo &dev);
+// Reads (and clears) the tensor-core kernel's bounded-wait error flag.
+spectra_status tc_device_error(bool *raised, cudaStream_t s);
 
 }  // namespace spectra
