@@ -158,23 +158,69 @@ __device__ __forceinline__ XRange x_range(const Prob &a, int s0, int s1, int P) 
     return r;
 }
 
+// Column indices of the first round of outlier slots a thread gathers (8
+// pairs per thread in flight).  They are part of the packed layer, not an
+// output of the previous kernel, so they may be loaded before the wait on it.
+struct XIdx {
+    int i0[8], i1[8];
+};
+
+__device__ __forceinline__ void load_x_idx(const Prob &a, const XRange &xr, int MB, XIdx &xi) {
+    const int np = (xr.j1 - xr.j0) / 2;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int c = threadIdx.x + i * blockDim.x;
+        const int j = xr.j0 + 2 * (c / MB);
+        const bool ok = c < np * MB;
+        xi.i0[i] = (ok && j < a.n_o) ? a.oidx[j] : -1;
+        xi.i1[i] = (ok && j + 1 < a.n_o) ? a.oidx[j + 1] : -1;
+    }
+}
+
 // Stage x for a unit range: bulk groups as BF16 pairs in the decoder's order
 // with their FP32 sums X_g (column order), and the BF16 pairs of the outlier
-// slots, gathered through the index list.
+// slots, gathered through the index list (first round: indices `xi`).  The
+// first bulk round and the first gather round are in flight together.
 template <int MB>
-__device__ void stage_x(const Prob &a, const Stage<MB> &st, const XRange &xr) {
+__device__ void stage_x(const Prob &a, const Stage<MB> &st, const XRange &xr, const XIdx &xi) {
     const int nth = blockDim.x;
     const int ng = xr.g1 - xr.g0;
+    const int np = (xr.j1 - xr.j0) / 2;
+    // first bulk round: this thread's 4 x 16 bytes
+    uint4 v0[4];
+    {
+        const int c = threadIdx.x, gl = c / MB, m = c - gl * MB, g = xr.g0 + gl;
+        if (c < ng * MB && g < a.G && m < a.m) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)m * a.k + 32 * g);
+#pragma unroll
+            for (int w = 0; w < 4; ++w) v0[w] = src[w];
+        }
+    }
+    // first gather round
+    uint32_t lo[8], hi[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int c = threadIdx.x + i * nth;
+        const int m = c % MB;
+        const bool mv = c < np * MB && m < a.m;
+        lo[i] = (mv && xi.i0[i] >= 0) ? a.x[(size_t)m * a.k + xi.i0[i]] : 0u;
+        hi[i] = (mv && xi.i1[i] >= 0) ? a.x[(size_t)m * a.k + xi.i1[i]] : 0u;
+    }
     for (int c = threadIdx.x; c < ng * MB; c += nth) {
         const int gl = c / MB, m = c - gl * MB;
         const int g = xr.g0 + gl;
         uint32_t *dst = st.xs + (size_t)gl * 16 * MB + m;
         float sum = 0.f;
         if (g < a.G && m < a.m) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)m * a.k + 32 * g);
             uint4 v[4];
+            if (c == (int)threadIdx.x) {
 #pragma unroll
-            for (int w = 0; w < 4; ++w) v[w] = src[w];
+                for (int w = 0; w < 4; ++w) v[w] = v0[w];
+            } else {
+                const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)m * a.k + 32 * g);
+#pragma unroll
+                for (int w = 0; w < 4; ++w) v[w] = src[w];
+            }
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
                 const uint32_t u[4] = {v[w].x, v[w].y, v[w].z, v[w].w};
@@ -193,9 +239,13 @@ __device__ void stage_x(const Prob &a, const Stage<MB> &st, const XRange &xr) {
         }
         st.xsum[c] = sum;
     }
-    // outlier slots as BF16 pairs: 8 pairs per thread in flight
-    const int np = (xr.j1 - xr.j0) / 2;
-    for (int base = 0; base < np * MB; base += 8 * nth) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int c = threadIdx.x + i * nth;
+        if (c < np * MB) st.xo[c] = lo[i] | (hi[i] << 16);
+    }
+    // further gather rounds: 8 pairs per thread in flight
+    for (int base = 8 * nth; base < np * MB; base += 8 * nth) {
         int i0[8], i1[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -211,9 +261,9 @@ __device__ void stage_x(const Prob &a, const Stage<MB> &st, const XRange &xr) {
             if (c < np * MB) {
                 const int m = c % MB;
                 const bool mv = m < a.m;
-                const uint32_t lo = (i0[i] >= 0 && mv) ? a.x[(size_t)m * a.k + i0[i]] : 0u;
-                const uint32_t hi = (i1[i] >= 0 && mv) ? a.x[(size_t)m * a.k + i1[i]] : 0u;
-                st.xo[c] = lo | (hi << 16);
+                const uint32_t l = (i0[i] >= 0 && mv) ? a.x[(size_t)m * a.k + i0[i]] : 0u;
+                const uint32_t h = (i1[i] >= 0 && mv) ? a.x[(size_t)m * a.k + i1[i]] : 0u;
+                st.xo[c] = l | (h << 16);
             }
         }
     }
@@ -381,8 +431,10 @@ __global__ void __launch_bounds__(kClusterWarps * 32, MB == 1 ? 2 : 1)
     pdl_launch_dependents();
     int next = 0;
     for (; next < nunits && next < ring.D; ++next) ring_issue(ring, a, t, unit_id(a, slc, next), lane);
+    XIdx xi;
+    load_x_idx(a, xr, MB, xi);
     pdl_wait();
-    stage_x<MB>(a, st, xr);
+    stage_x<MB>(a, st, xr, xi);
     __syncthreads();
 
     float yacc[MB];
@@ -517,7 +569,9 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1)
             // every warp is done with the previous x (the branch is CTA-uniform)
             __syncthreads();
             xr = x_range(a, 0, 1, 1);
-            stage_x<MB>(a, st, xr);
+            XIdx xi;
+            load_x_idx(a, xr, MB, xi);
+            stage_x<MB>(a, st, xr, xi);
             __syncthreads();
             cur_p = p;
         }
@@ -617,10 +671,52 @@ struct ClusterPlan {
     double cost;
 };
 
+// Clusters of `cl` CTAs of `smem` bytes each that the device runs at once.
+// Clusters are placed within one GPC, so this can be well below
+// sm_count * CTAs per SM / cl; a launch with more clusters runs a second
+// wave.  Cached per device and shape (0: the shape cannot run).
+template <int MB>
+int cluster_capacity(int cl, size_t smem, const DeviceInfo &dev) {
+    struct Entry {
+        int device, cl;
+        size_t smem;
+        int cap;
+    };
+    static std::mutex mu;
+    static Entry cache[256];
+    static int n = 0;
+    static bool done[64];
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n; ++i)
+        if (cache[i].device == dev.device && cache[i].cl == cl && cache[i].smem == smem) return cache[i].cap;
+    int cap = 0;
+    if (prepare_kernel(gemv_cluster_kernel<MB>, done, dev) == cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(cl * dev.sm_count), 1, 1);
+        cfg.blockDim = dim3(kClusterWarps * 32, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = (unsigned)cl;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&cap, gemv_cluster_kernel<MB>, &cfg) != cudaSuccess) {
+            cap = 0;
+            (void)cudaGetLastError();
+        }
+    }
+    if (n < 256) cache[n++] = Entry{dev.device, cl, smem, cap};
+    return cap;
+}
+
 // Cluster kernel: slices per tile P = ppc * cl and tiles per CTA from a simple
-// model -- waves of CTAs times the bytes of the largest slice, plus a cost per
-// CTA start and per reduction level.
-bool plan_cluster(const Geometry &g, int MB, const DeviceInfo &dev, ClusterPlan *out) {
+// model -- waves of CTAs (of clusters, by the device's cluster capacity)
+// times the bytes of the largest slice, plus a cost per CTA start and per
+// reduction level.
+template <int MB>
+bool plan_cluster(const Geometry &g, const DeviceInfo &dev, ClusterPlan *out) {
     const int U = units_of(g);
     const int OB = U - g.S;
     bool found = false;
@@ -637,7 +733,12 @@ bool plan_cluster(const Geometry &g, int MB, const DeviceInfo &dev, ClusterPlan 
             sm.depth = choose_depth(MB, sm, dev);
             if (sm.depth == 0) continue;
             const int64_t ctas = cdiv(g.T, tpc) * cl;
-            const int64_t waves = cdiv(ctas, (int64_t)dev.sm_count * ctas_per_sm(MB, sm));
+            int64_t waves = cdiv(ctas, (int64_t)dev.sm_count * ctas_per_sm(MB, sm));
+            if (cl > 1) {
+                const int cap = cluster_capacity<MB>(cl, stage_bytes(MB, kClusterWarps, sm), dev);
+                if (cap <= 0) continue;
+                waves = cdiv(ctas / cl, cap);
+            }
             const int64_t slice = cdiv(g.S, P) * kSgBytes + cdiv(OB, P) * kOB * kOctBytes;
             const double cost = (double)waves * (double)(slice + 8192) +
                                 (ppc > 1 ? 256.0 * ppc : 0.0) + (cl > 1 ? 4096.0 + 512.0 * cl : 0.0);
@@ -778,7 +879,7 @@ spectra_status run_one(const Prob &a, const DeviceInfo &dev, cudaStream_t s) {
         return run_persistent<MB>(args, 1, dev, s);
     }
     ClusterPlan p;
-    if (!plan_cluster(g, MB, dev, &p)) return SPECTRA_ERR_SHAPE;
+    if (!plan_cluster<MB>(g, dev, &p)) return SPECTRA_ERR_SHAPE;
     return run_cluster<MB>(a, p, dev, s);
 }
 
