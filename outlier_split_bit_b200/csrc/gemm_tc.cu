@@ -25,9 +25,11 @@ namespace {
 //    32 columns) into a TMEM buffer, and later reads back that group's FP32
 //    product D = (c - z) x from TMEM and adds s * D to its rows' sums.  The
 //    outlier columns enter the same way with their BF16 weights and s = 1.
-//  * one MMA warp whose elected lane issues two tcgen05.mma kind::f16
-//    (M = 128, N = MB, K = 16) per group and commits them to the group's
-//    mbarrier.
+//  * one MMA warp per set, whose elected lane issues two tcgen05.mma
+//    kind::f16 (M = 128, N = MB, K = 16) per group of its set and commits
+//    them to the group's mbarrier (each mbarrier operation costs the issuing
+//    thread on the order of a hundred cycles, so one issuer for both sets
+//    would pace the whole CTA).
 //
 // The products are exact: c - z is an integer in [-15, 15] and x is BF16, so
 // each product has at most 12 significant bits; D holds FP32 sums of 32 of
@@ -46,7 +48,7 @@ namespace {
 // device error bit and turns the remaining waits into no-ops.
 constexpr int kTcSets = 2;
 constexpr int kTcComputeWarps = 4 * kTcSets;
-constexpr int kTcWarps = kTcComputeWarps + 1;  // + the MMA warp
+constexpr int kTcWarps = kTcComputeWarps + kTcSets;  // + one MMA warp per set
 constexpr int kTcTmemCols = 512;
 
 template <int MB>
@@ -307,8 +309,8 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) gemm_tc_kernel(const TcArgs 
     uint64_t *bars = reinterpret_cast<uint64_t *>(red + 128 * MB);
     uint64_t *full = bars + kTcComputeWarps * D;  // [kTcSets][P]
     uint64_t *done = full + kTcSets * C::P;        // [kTcSets][P]
-    uint64_t *fin = done + kTcSets * C::P;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(fin + 1);
+    uint64_t *fin = done + kTcSets * C::P;                          // [kTcSets]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(fin + kTcSets);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     // this CTA's share of the units of every block it visits
@@ -329,7 +331,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) gemm_tc_kernel(const TcArgs 
             mbar_init(smem_u32(&full[b]), 4u);  // one arrival per compute warp of the set
             mbar_init(smem_u32(&done[b]), 1u);
         }
-        mbar_init(smem_u32(fin), 1u);
+        for (int j = 0; j < kTcSets; ++j) mbar_init(smem_u32(&fin[j]), 1u);
         *abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -460,61 +462,49 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) gemm_tc_kernel(const TcArgs 
         }
         ring_drain(ring);
     } else if (lane == 0) {
-        // ------------------------------------------------ MMA issuer (one lane)
+        // ------------------------------------------------ MMA issuer of set j (one lane)
+        const int j = warp - kTcComputeWarps;
         pdl_wait();
         const uint32_t idesc = bf16_idesc<MB>();
-        int gis[kTcSets] = {}, xls[kTcSets] = {};
+        int q = 0, xl = 0;
         bool any = false;
         for (int blk = blockIdx.x / a.cl; blk < args.nblk; blk += bstride) {
-            for (int lub = 0; lub < nunits; lub += kTcSets) {
-                int ngr[kTcSets], gmax = 0;
+            for (int lu = j; lu < nunits; lu += kTcSets, ++xl) {
+                const int ngr = tc_groups(a, tc_unit(a, sg0, nsg, ob0, lu));
+                const uint32_t xs0 = smem_u32(ximg + (size_t)(j * 2 + (xl & 1)) * C::XBYTES);
+                for (int g = 0; g < ngr; ++g, ++q) {
+                    const int b = q % C::P;
+                    const bool ok = tc_wait(smem_u32(&full[j * C::P + b]), (uint32_t)(q / C::P) & 1u, abort);
+                    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                    if (ok) {
+                        const uint32_t xs = xs0 + (uint32_t)(2 * g * C::KSTEP);
+                        const uint32_t ta = tmem + (uint32_t)((j * C::P + b) * 16);
+                        const uint32_t td = tmem + (uint32_t)(C::DCOL + (j * C::P + b) * MB);
 #pragma unroll
-                for (int s = 0; s < kTcSets; ++s) {
-                    ngr[s] = lub + s < nunits ? tc_groups(a, tc_unit(a, sg0, nsg, ob0, lub + s)) : 0;
-                    gmax = max(gmax, ngr[s]);
-                }
-                for (int g = 0; g < gmax; ++g) {
-#pragma unroll
-                    for (int s = 0; s < kTcSets; ++s) {
-                        if (g >= ngr[s]) continue;
-                        const int b = gis[s] % C::P;
-                        const bool ok = tc_wait(smem_u32(&full[s * C::P + b]), (uint32_t)(gis[s] / C::P) & 1u, abort);
-                        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-                        if (ok) {
-                            const uint32_t xs = smem_u32(ximg + (size_t)(s * 2 + (xls[s] & 1)) * C::XBYTES) +
-                                                (uint32_t)(2 * g * C::KSTEP);
-                            const uint32_t ta = tmem + (uint32_t)((s * C::P + b) * 16);
-                            const uint32_t td = tmem + (uint32_t)(C::DCOL + (s * C::P + b) * MB);
-#pragma unroll
-                            for (int h = 0; h < 2; ++h) {
-                                const uint64_t bdesc = umma_desc(xs + (uint32_t)(h * C::KSTEP), 128u, 256u);
-                                asm volatile(
-                                    "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %3, 0;\n\t"
-                                    "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p;\n\t}" ::"r"(td),
-                                    "r"(ta + 8u * h), "l"(bdesc), "r"((uint32_t)h), "r"(idesc)
-                                    : "memory");
-                            }
-                            any = true;
+                        for (int h = 0; h < 2; ++h) {
+                            const uint64_t bdesc = umma_desc(xs + (uint32_t)(h * C::KSTEP), 128u, 256u);
+                            asm volatile(
+                                "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %3, 0;\n\t"
+                                "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p;\n\t}" ::"r"(td),
+                                "r"(ta + 8u * h), "l"(bdesc), "r"((uint32_t)h), "r"(idesc)
+                                : "memory");
                         }
-                        asm volatile(
-                            "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                                smem_u32(&done[s * C::P + b]))
-                            : "memory");
-                        ++gis[s];
+                        any = true;
                     }
+                    asm volatile(
+                        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                            smem_u32(&done[j * C::P + b]))
+                        : "memory");
                 }
-#pragma unroll
-                for (int s = 0; s < kTcSets; ++s)
-                    if (lub + s < nunits) ++xls[s];
             }
         }
-        // every MMA of this CTA has completed before TMEM is released
+        // every MMA this lane issued has completed before TMEM is released
         if (any) {
             asm volatile(
                 "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                    smem_u32(fin))
+                    smem_u32(&fin[j]))
                 : "memory");
-            tc_wait(smem_u32(fin), 0u, abort);
+            tc_wait(smem_u32(&fin[j]), 0u, abort);
         }
     }
     __syncwarp();
@@ -554,7 +544,7 @@ size_t tc_smem_bytes(int MB, int depth) {
     const int P = MB == 32 ? TcCfg<32>::P : TcCfg<16>::P;
     return (size_t)kTcSets * 2 * 256 * MB * 2 + (size_t)kTcComputeWarps * depth * kStageBytes +
            (size_t)kTcComputeWarps * P * 32 * 4 + (size_t)128 * MB * 4 +
-           (size_t)(kTcComputeWarps * depth + 2 * kTcSets * P + 1) * 8 + 16;
+           (size_t)(kTcComputeWarps * depth + 2 * kTcSets * P + kTcSets) * 8 + 16;
 }
 
 template <int MB>
