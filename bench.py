@@ -402,6 +402,23 @@ def run_reference(args):
     return 0
 
 
+# ---------------------------------------------------------------- ranks
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The slowest rank's value (all ranks call it, in the same order)."""
+    if world <= 1:
+        return float(value)
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(bytes_per_rank_step: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job GB/s: the bytes every rank streamed over the slowest rank's time."""
+    return bytes_per_rank_step * steps * world / (max_ms * 1e-3) * 1e-9
+
+
 # ---------------------------------------------------------------- our arm
 
 def kernel_source_digest() -> str:
@@ -470,14 +487,9 @@ def run_ours(args):
         e1.synchronize()
     torch.cuda.synchronize()
     barrier()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), world, device)
     step_ms = ms / args.steps
-    total_bytes = st.bytes * args.steps * world
-    gbs = total_bytes / (ms * 1e-3) * 1e-9
+    gbs = job_gbs(st.bytes, args.steps, world, ms)
 
     # end to end: pinned host x in, y out, copies inside the timed region
     x_host = torch.empty(st.x_all.shape, dtype=st.x_all.dtype, pin_memory=True)
@@ -496,12 +508,8 @@ def run_ours(args):
         b.record(stream)
     b.synchronize()
     barrier()
-    e2e_ms = a.elapsed_time(b)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_gbs = st.bytes * e2e_steps * world / (e2e_ms * 1e-3) * 1e-9
+    e2e_ms = max_over_ranks(a.elapsed_time(b), world, device)
+    e2e_gbs = job_gbs(st.bytes, e2e_steps, world, e2e_ms)
 
     # the same stream as a dependent chain of 196 launches (graph + PDL)
     chain_graph, chain_launches = st.capture(stream, "chain")
@@ -517,7 +525,7 @@ def run_ours(args):
             chain_graph.replay()
         c1.record(stream)
     c1.synchronize()
-    chain_ms = c0.elapsed_time(c1) / chain_steps
+    chain_ms = max_over_ranks(c0.elapsed_time(c1), world, device) / chain_steps
     del chain_graph
 
     extra = {"decode_stream_dependent_chain": {
