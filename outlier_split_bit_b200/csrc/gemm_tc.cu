@@ -18,8 +18,8 @@ namespace {
 // lane = row) and streams their units (super-groups, outlier batches) with
 // three kinds of warps:
 //
-//  * two sets of four compute warps.  Set j takes every second unit of the
-//    block; warp 4j + r owns tile r (rows 32r..32r+31) and keeps its own
+//  * SETS sets of four compute warps (three for 16 batch rows, two for 32).
+//    Set j takes every SETS-th unit of the block; warp 4j + r owns tile r (rows 32r..32r+31) and keeps its own
 //    cp.async.bulk ring of that tile's units.  Per group of 32 columns it
 //    writes the exact integer weights c - z as a BF16 A operand (128 rows x
 //    32 columns) into a TMEM buffer, and later reads back that group's FP32
@@ -46,19 +46,21 @@ namespace {
 // A buffer is rewritten only after its previous D was read, so the MMA that
 // read its A has completed.  Every wait is bounded; a timeout raises the
 // device error bit and turns the remaining waits into no-ops.
-constexpr int kTcSets = 2;
-constexpr int kTcComputeWarps = 4 * kTcSets;
-constexpr int kTcWarps = kTcComputeWarps + kTcSets;  // + one MMA warp per set
 constexpr int kTcTmemCols = 512;
 
 template <int MB>
 struct TcCfg {
-    static constexpr int P = MB == 32 ? 5 : 8;       // TMEM buffers per set
+    // warp sets: three for 16 batch rows (127 registers: four warps per
+    // sub-partition fit), two for 32 (165 registers: three per sub-partition)
+    static constexpr int SETS = MB == 16 ? 3 : 2;
+    static constexpr int CW = 4 * SETS;              // compute warps
+    static constexpr int WARPS = CW + SETS;          // + one MMA warp per set
+    static constexpr int P = 5;                      // TMEM buffers per set
     static constexpr int L = P - 1;                  // groups produced ahead of the one read back
-    static constexpr int DCOL = kTcSets * P * 16;    // A buffers at [0, DCOL), D after
+    static constexpr int DCOL = (SETS * P * 16 + 31) / 32 * 32;  // A buffers below, D from here
     static constexpr int XBYTES = 256 * MB * 2;      // x image of one super-group
     static constexpr int KSTEP = MB * 32;            // bytes of one 16-column K step of x
-    static_assert(DCOL + kTcSets * P * MB <= kTcTmemCols, "TMEM budget");
+    static_assert(DCOL + SETS * P * MB <= kTcTmemCols, "TMEM budget");
     static_assert(DCOL % 32 == 0, "D alignment");
 };
 
@@ -293,24 +295,24 @@ __device__ __forceinline__ float tc_build_a(const Prob &a, int u, int g, const u
 }
 
 template <int MB>
-__global__ void __launch_bounds__(kTcWarps * 32, 1) gemm_tc_kernel(const TcArgs args) {
+__global__ void __launch_bounds__(TcCfg<MB>::WARPS * 32, 1) gemm_tc_kernel(const TcArgs args) {
     using C = TcCfg<MB>;
     extern __shared__ __align__(1024) uint8_t tsm[];
     const Prob &a = args.p;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cr = (a.cl > 1) ? (int)cg::this_cluster().block_rank() : 0;
     const int D = args.depth;
-    // shared memory: [x images kTcSets x 2][ring kTcComputeWarps x D][scales
-    // kTcComputeWarps x P x 32][red 128 x MB][bars][tmem slot, abort]
+    // shared memory: [x images SETS x 2][ring CW x D][scales CW x P x 32]
+    // [red (SETS - 1) x 128 x MB][bars][tmem slot, abort]
     uint8_t *ximg = tsm;
-    uint8_t *ring_base = ximg + (size_t)kTcSets * 2 * C::XBYTES;
-    float *sbuf = reinterpret_cast<float *>(ring_base + (size_t)kTcComputeWarps * D * kStageBytes);
-    float *red = sbuf + kTcComputeWarps * C::P * 32;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(red + 128 * MB);
-    uint64_t *full = bars + kTcComputeWarps * D;  // [kTcSets][P]
-    uint64_t *done = full + kTcSets * C::P;        // [kTcSets][P]
-    uint64_t *fin = done + kTcSets * C::P;                          // [kTcSets]
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(fin + kTcSets);
+    uint8_t *ring_base = ximg + (size_t)C::SETS * 2 * C::XBYTES;
+    float *sbuf = reinterpret_cast<float *>(ring_base + (size_t)C::CW * D * kStageBytes);
+    float *red = sbuf + C::CW * C::P * 32;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(red + (C::SETS - 1) * 128 * MB);
+    uint64_t *full = bars + C::CW * D;      // [SETS][P]
+    uint64_t *done = full + C::SETS * C::P;  // [SETS][P]
+    uint64_t *fin = done + C::SETS * C::P;   // [SETS]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(fin + C::SETS);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     // this CTA's share of the units of every block it visits
@@ -327,16 +329,16 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) gemm_tc_kernel(const TcArgs 
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     if (threadIdx.x == 32) {
-        for (int b = 0; b < kTcSets * C::P; ++b) {
+        for (int b = 0; b < C::SETS * C::P; ++b) {
             mbar_init(smem_u32(&full[b]), 4u);  // one arrival per compute warp of the set
             mbar_init(smem_u32(&done[b]), 1u);
         }
-        for (int j = 0; j < kTcSets; ++j) mbar_init(smem_u32(&fin[j]), 1u);
+        for (int j = 0; j < C::SETS; ++j) mbar_init(smem_u32(&fin[j]), 1u);
         *abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     Ring ring;
-    if (warp < kTcComputeWarps)
+    if (warp < C::CW)
         ring_init(ring, ring_base + (size_t)warp * D * kStageBytes, bars + warp * D, D, lane);
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
@@ -344,7 +346,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) gemm_tc_kernel(const TcArgs 
     const uint32_t tmem = *tmem_slot;
     pdl_launch_dependents();
 
-    if (warp < kTcComputeWarps) {
+    if (warp < C::CW) {
         // ------------------------------------------------ compute warps
         const int j = warp >> 2, r = warp & 3, tid = threadIdx.x - 128 * j;
         const uint32_t tl = tmem + ((uint32_t)(32 * r) << 16);
@@ -353,7 +355,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) gemm_tc_kernel(const TcArgs 
         // issue iterator (ring) and x iterator run ahead of the work iterator
         int iblk = blockIdx.x / a.cl, ilu = j;
         auto advance = [&](int &blk, int &lu) {
-            lu += kTcSets;
+            lu += C::SETS;
             if (lu >= nunits) {
                 blk += bstride;
                 lu = j;
@@ -399,7 +401,7 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) gemm_tc_kernel(const TcArgs 
         for (int blk = blockIdx.x / a.cl; blk < args.nblk; blk += bstride) {
             const int t = 4 * blk + r;
             const bool active = t < a.T;
-            for (int lu = j; lu < nunits; lu += kTcSets, ++xl) {
+            for (int lu = j; lu < nunits; lu += C::SETS, ++xl) {
                 const int u = tc_unit(a, sg0, nsg, ob0, lu);
                 uint8_t *xb = ximg + (size_t)(j * 2 + (xl & 1)) * C::XBYTES;
                 // the MMAs of unit xl - 2 read this x buffer: wait for them
@@ -438,16 +440,19 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) gemm_tc_kernel(const TcArgs 
                 }
             }
             while (gc < gi) consume();
-            // block end: set 1 hands its sums to set 0, which stores the rows
-            // (or, in a cluster, leaves them for the rank-ordered reduction)
-            if (j == 1) {
+            // block end: sets 1.. hand their sums to set 0, which adds them in set
+            // order and stores the rows (or, in a cluster, leaves them for the
+            // rank-ordered reduction)
+            if (j > 0) {
 #pragma unroll
-                for (int m = 0; m < MB; ++m) red[(32 * r + lane) * MB + m] = y[m];
+                for (int m = 0; m < MB; ++m) red[((j - 1) * 128 + 32 * r + lane) * MB + m] = y[m];
             }
-            named_sync(1, 32 * kTcComputeWarps);
+            named_sync(1, 32 * C::CW);
             if (j == 0) {
+                for (int o = 0; o < C::SETS - 1; ++o) {
 #pragma unroll
-                for (int m = 0; m < MB; ++m) y[m] += red[(32 * r + lane) * MB + m];
+                    for (int m = 0; m < MB; ++m) y[m] += red[(o * 128 + 32 * r + lane) * MB + m];
+                }
                 if (a.cl > 1) {
 #pragma unroll
                     for (int m = 0; m < MB; ++m) red[(32 * r + lane) * MB + m] = y[m];
@@ -456,20 +461,20 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) gemm_tc_kernel(const TcArgs 
                     for (int m = 0; m < MB; ++m) store_y(a, t, lane, m, y[m]);
                 }
             }
-            named_sync(1, 32 * kTcComputeWarps);
+            named_sync(1, 32 * C::CW);
 #pragma unroll
             for (int m = 0; m < MB; ++m) y[m] = 0.f;
         }
         ring_drain(ring);
     } else if (lane == 0) {
         // ------------------------------------------------ MMA issuer of set j (one lane)
-        const int j = warp - kTcComputeWarps;
+        const int j = warp - C::CW;
         pdl_wait();
         const uint32_t idesc = bf16_idesc<MB>();
         int q = 0, xl = 0;
         bool any = false;
         for (int blk = blockIdx.x / a.cl; blk < args.nblk; blk += bstride) {
-            for (int lu = j; lu < nunits; lu += kTcSets, ++xl) {
+            for (int lu = j; lu < nunits; lu += C::SETS, ++xl) {
                 const int ngr = tc_groups(a, tc_unit(a, sg0, nsg, ob0, lu));
                 const uint32_t xs0 = smem_u32(ximg + (size_t)(j * 2 + (xl & 1)) * C::XBYTES);
                 for (int g = 0; g < ngr; ++g, ++q) {
@@ -540,11 +545,12 @@ __global__ void __launch_bounds__(kTcWarps * 32, 1) gemm_tc_kernel(const TcArgs 
     }
 }
 
-size_t tc_smem_bytes(int MB, int depth) {
-    const int P = MB == 32 ? TcCfg<32>::P : TcCfg<16>::P;
-    return (size_t)kTcSets * 2 * 256 * MB * 2 + (size_t)kTcComputeWarps * depth * kStageBytes +
-           (size_t)kTcComputeWarps * P * 32 * 4 + (size_t)128 * MB * 4 +
-           (size_t)(kTcComputeWarps * depth + 2 * kTcSets * P + kTcSets) * 8 + 16;
+template <int MB>
+size_t tc_smem_bytes(int depth) {
+    using C = TcCfg<MB>;
+    return (size_t)C::SETS * 2 * C::XBYTES + (size_t)C::CW * depth * kStageBytes +
+           (size_t)C::CW * C::P * 32 * 4 + (size_t)(C::SETS - 1) * 128 * MB * 4 +
+           (size_t)(C::CW * depth + 2 * C::SETS * C::P + C::SETS) * 8 + 16;
 }
 
 template <int MB>
@@ -570,13 +576,13 @@ spectra_status run_tc(const Prob &a0, const DeviceInfo &dev, cudaStream_t s) {
     args.p.cl = cl;
     args.nblk = (int)nblk;
     int depth = 4;
-    while (depth > 1 && tc_smem_bytes(MB, depth) > dev.smem_optin) --depth;
+    while (depth > 1 && tc_smem_bytes<MB>(depth) > dev.smem_optin) --depth;
     args.depth = depth;
-    const size_t smem = tc_smem_bytes(MB, depth);
+    const size_t smem = tc_smem_bytes<MB>(depth);
     if (smem > dev.smem_optin) return SPECTRA_ERR_SHAPE;
     cudaError_t e = prepare_kernel(gemm_tc_kernel<MB>, done, dev);
     if (e != cudaSuccess) return SPECTRA_ERR_CUDA;
-    e = launch_kernel(gemm_tc_kernel<MB>, args, (unsigned)grid, smem, kTcWarps, cl, s);
+    e = launch_kernel(gemm_tc_kernel<MB>, args, (unsigned)grid, smem, TcCfg<MB>::WARPS, cl, s);
     return e == cudaSuccess ? SPECTRA_OK : SPECTRA_ERR_CUDA;
 }
 
