@@ -227,9 +227,10 @@ SPECTRA_API spectra_status spectra_gemv(const spectra_layer *layer, const uint16
 /*
  * Small-batch decode matmul, y[m][i] for m in [0, m_rows), 1 <= m_rows <= 32:
  *   x  device, BF16 bits [m_rows][k] row-major;  y  device [m_rows][n].
- * Same formula and tolerance as spectra_gemv per batch row.  m_rows <= 15 runs
- * on CUDA cores (m_rows accumulators per lane); 16..32 runs the tensor-core
- * path (weights dequantised in registers, then MMA with FP32 accumulation).
+ * Same formula and tolerance as spectra_gemv per batch row.  m_rows <= 7 runs
+ * on CUDA cores (m_rows accumulators per lane); 8..32 runs the tensor-core
+ * path (weights dequantised in registers to exact integer BF16 operands, MMA
+ * with FP32 accumulation per group of 32 columns, scale applied in FP32).
  * Asynchronous, allocates nothing.
  */
 SPECTRA_API spectra_status spectra_gemm_small(const spectra_layer *layer, const uint16_t *x, int32_t m_rows,

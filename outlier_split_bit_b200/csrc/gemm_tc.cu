@@ -1,11 +1,12 @@
-// gemm_tc.cu -- y = x W_hat^T for 16 <= m <= 32 batch rows on the fifth-
+// gemm_tc.cu -- y = x W_hat^T for 8 <= m <= 32 batch rows on the fifth-
 // generation tensor cores (tcgen05, sm_100a).
 //
 // Method: "SPECTRA: Sparse-Precision Exact Channel Tensor Reconstruction
 // Architecture" (Dev.to abstract), abstract paragraph: the Group-32 4-bit
 // weights are dequantised in registers and the BF16 outlier channels enter
-// the same product.  For a batch of 16 or more rows the product is a real
-// dense contraction, so the decoded operand goes to the tensor cores.
+// the same product.  For a batch of 8 or more rows the product is a real
+// dense contraction, so the decoded operand goes to the tensor cores (8..16
+// rows run the 16-row variant; its surplus rows are computed and dropped).
 #include "stream.cuh"
 
 namespace spectra {
@@ -13,7 +14,7 @@ namespace {
 
 // ---------------------------------------------------------------- tensor-core path (M = 16..32)
 //
-// y[m][n] for 16 <= m_rows <= 32 (MB = 16 or 32 batch rows) on the fifth-
+// y[m][n] for 8 <= m_rows <= 32 (MB = 16 or 32 batch rows) on the fifth-
 // generation tensor cores.  A CTA owns blocks of 128 rows (4 tiles; TMEM
 // lane = row) and streams their units (super-groups, outlier batches) with
 // three kinds of warps:

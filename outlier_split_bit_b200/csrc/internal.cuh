@@ -62,8 +62,8 @@ cudaError_t launch_unpack(const spectra_layer &l, uint8_t *codes, uint16_t *scal
 
 // ---- matvec (gemv.cu) ----
 constexpr int kMaxBatch = SPECTRA_MAX_BATCH;
-// Decode matvec for 1 <= m <= 32 batch rows (CUDA cores below 16 rows, the
-// tensor cores from 16).
+// Decode matvec for 1 <= m <= 32 batch rows (CUDA cores below 8 rows, the
+// tensor cores from 8).
 spectra_status launch_gemv(const spectra_layer &l, const uint16_t *x, int m, void *y, int ytype,
                            cudaStream_t s, const DeviceInfo &dev);
 // Reads (and clears) the flag the matvec kernels raise when a bounded wait
@@ -75,7 +75,7 @@ spectra_status launch_gemv_batched(const spectra_layer *layers, const uint16_t *
                                    const DeviceInfo &dev);
 
 // ---- tensor-core matmul (gemm_tc.cu) ----
-// y[m][n] for 16 <= m <= 32 batch rows on the tensor cores.
+// y[m][n] for 8 <= m <= 32 batch rows on the tensor cores.
 spectra_status launch_tc(const spectra_layer &l, const uint16_t *x, int m, void *y, int ytype,
                          cudaStream_t s, const DeviceInfo &dev);
 // Reads (and clears) the tensor-core kernel's bounded-wait error flag.

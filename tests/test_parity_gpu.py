@@ -119,7 +119,9 @@ def test_deterministic_bitwise():
 
 
 @pytest.mark.parametrize("m", list(range(1, 16)))
-def test_gemm_small_cuda_core(m):
+def test_gemm_small_every_m_below_16(m):
+    """m = 1..7 on the CUDA-core decode (1, 2, 4 or 8 accumulators per lane),
+    8..15 on the tensor cores' 16-row variant."""
     spec = wl.MatrixSpec("single", 512, 512, 10)
     w, g, x, idx, kappa, lay, wb, ref = _full_pack(spec, 6.0, True, m=m)
     y = sp.spectra_gemm_small(lay, x)
@@ -324,13 +326,13 @@ def test_device_status_clear_after_all_launches():
     sp.spectra_device_status()
 
 
-@pytest.mark.parametrize("m", [16, 17, 24, 32])
+@pytest.mark.parametrize("m", [8, 11, 16, 17, 24, 32])
 @pytest.mark.parametrize("spec,tau", [(wl.SINGLE_512, 3.0), (wl.MatrixSpec("single", 40, 96, 3), 1.2),
                                       (wl.MatrixSpec("single", 300, 2080, 31), 6.0),
                                       (wl.MatrixSpec("single", 130, 512, 0), np.inf)],
                          ids=["512", "40x96", "300x2080", "130x512-noout"])
 def test_gemm_small_tensor_cores(spec, tau, m):
-    """M = 16..32 runs on tcgen05 (exact BF16 c - z and x operands, FP32 per-group
+    """M = 8..32 runs on tcgen05 (exact BF16 c - z and x operands, FP32 per-group
     products in TMEM, scales applied in FP32)."""
     w, g, x, idx, kappa, lay, wb, ref = _full_pack(spec, tau, True, m=m)
     y = sp.spectra_gemm_small(lay, x)
@@ -358,7 +360,7 @@ def test_decoder_layer_4b_tensor_cores(spec, m):
     check_gemv(y[:, rows], y_ref, bound)
 
 
-@pytest.mark.parametrize("m", [16, 32])
+@pytest.mark.parametrize("m", [8, 16, 32])
 def test_tensor_cores_unit_vectors_exact(m):
     """x row r = e_{j_r}: every product is exact on the tensor cores, so row r of y
     is column j_r of the dequantised matrix (plus its BF16 outlier column) bit for bit."""
