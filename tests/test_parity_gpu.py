@@ -409,3 +409,62 @@ def test_tensor_cores_deterministic():
     y1 = sp.spectra_gemm_small(lay, x)
     torch.cuda.synchronize()
     assert torch.equal(y0, y1)
+
+
+@pytest.mark.parametrize("m", [8, 16, 32])
+def test_tensor_cores_bf16_output(m):
+    """BF16 y on the tensor-core path: the FP32 result rounded once."""
+    spec = wl.MatrixSpec("single", 300, 2080, 31)
+    w, g, x, idx, kappa, lay, wb, ref = _full_pack(spec, 3.0, True, m=m)
+    y = sp.spectra_gemm_small(lay, x, y_dtype=torch.bfloat16)
+    y32 = sp.spectra_gemm_small(lay, x)
+    torch.cuda.synchronize()
+    y_ref, bound = oracle.gemm(ref.can, wb, ref.idx, wl.bits(x))
+    check_gemv(y, y_ref, bound, bf16=True)
+    assert torch.equal(y, y32.to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("m", [16, 32])
+def test_tensor_cores_graph_capture_and_replay(m):
+    spec = wl.LAYER_4B[4]
+    w, g, x = draw(spec, m=m)
+    lay = sp.pack_layer(w, g, 3.0)
+    y_eager = sp.spectra_gemm_small(lay, x).clone()
+    y = torch.empty_like(y_eager)
+    view = lay.view()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(graph, stream=s):
+            sp.spectra_gemm_small(lay, x, y, view=view, stream=s)
+    for _ in range(3):
+        y.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(y, y_eager)
+    sp.spectra_device_status()
+
+
+def test_tensor_cores_dependent_chain_reads_previous_output():
+    """The output of one 16-row product is the input of the next on the same
+    stream: the programmatic dependent launch must not let the second kernel
+    read x early."""
+    spec = wl.MatrixSpec("q", 2048, 2048, 30)
+    layers = []
+    for i in range(4):
+        w, g, _ = draw(spec, seed=i)
+        layers.append(sp.pack_layer(w, g, 6.0))
+    x0 = wl.activations(2048, 16, seed=9, device=DEV)
+    bufs = [torch.empty((16, 2048), dtype=torch.bfloat16, device=DEV) for _ in range(5)]
+    bufs[0].copy_(x0)
+    for i, lay in enumerate(layers):
+        sp.spectra_gemm_small(lay, bufs[i], bufs[i + 1])
+    torch.cuda.synchronize()
+    cur = x0.clone()
+    for lay in layers:
+        nxt = sp.spectra_gemm_small(lay, cur, y_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        cur = nxt
+    assert torch.equal(bufs[-1], cur)
+    sp.spectra_device_status()
