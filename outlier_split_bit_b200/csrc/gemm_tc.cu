@@ -19,8 +19,8 @@ namespace {
 // lane = row) and streams their units (super-groups, outlier batches) with
 // three kinds of warps:
 //
-//  * SETS sets of four compute warps (three for 16 batch rows, two for 32).
-//    Set j takes every SETS-th unit of the block; warp 4j + r owns tile r (rows 32r..32r+31) and keeps its own
+//  * three sets of four compute warps.  Set j takes every third unit of the
+//    block; warp 4j + r owns tile r (rows 32r..32r+31) and keeps its own
 //    cp.async.bulk ring of that tile's units.  Per group of 32 columns it
 //    writes the exact integer weights c - z as a BF16 A operand (128 rows x
 //    32 columns) into a TMEM buffer, and later reads back that group's FP32
@@ -51,12 +51,13 @@ constexpr int kTcTmemCols = 512;
 
 template <int MB>
 struct TcCfg {
-    // warp sets: three for 16 batch rows (127 registers: four warps per
-    // sub-partition fit), two for 32 (165 registers: three per sub-partition)
-    static constexpr int SETS = MB == 16 ? 3 : 2;
+    // three warp sets: four warps per sub-partition, so at most 128 registers
+    // (16 rows: 121; 32 rows: 128, with the accumulators read back 16 columns
+    // at a time); TMEM holds 5 buffers per set at 16 rows, 3 at 32
+    static constexpr int SETS = 3;
     static constexpr int CW = 4 * SETS;              // compute warps
     static constexpr int WARPS = CW + SETS;          // + one MMA warp per set
-    static constexpr int P = 5;                      // TMEM buffers per set
+    static constexpr int P = MB == 16 ? 5 : 3;       // TMEM buffers per set
     static constexpr int L = P - 1;                  // groups produced ahead of the one read back
     static constexpr int DCOL = (SETS * P * 16 + 31) / 32 * 32;  // A buffers below, D from here
     static constexpr int XBYTES = 256 * MB * 2;      // x image of one super-group
@@ -304,12 +305,14 @@ __global__ void __launch_bounds__(TcCfg<MB>::WARPS * 32, 1) gemm_tc_kernel(const
     const int cr = (a.cl > 1) ? (int)cg::this_cluster().block_rank() : 0;
     const int D = args.depth;
     // shared memory: [x images SETS x 2][ring CW x D][scales CW x P x 32]
-    // [red (SETS - 1) x 128 x MB][bars][tmem slot, abort]
+    // [bars][tmem slot, abort].  At a block end, once every group of the block
+    // has been read back, set j's first x image holds its 128 x MB partial
+    // sums (the same 256 x MB x 2 bytes).
     uint8_t *ximg = tsm;
     uint8_t *ring_base = ximg + (size_t)C::SETS * 2 * C::XBYTES;
     float *sbuf = reinterpret_cast<float *>(ring_base + (size_t)C::CW * D * kStageBytes);
-    float *red = sbuf + C::CW * C::P * 32;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(red + (C::SETS - 1) * 128 * MB);
+    auto red_of = [&](int set) { return reinterpret_cast<float *>(ximg + (size_t)set * 2 * C::XBYTES); };
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sbuf + C::CW * C::P * 32);
     uint64_t *full = bars + C::CW * D;      // [SETS][P]
     uint64_t *done = full + C::SETS * C::P;  // [SETS][P]
     uint64_t *fin = done + C::SETS * C::P;   // [SETS]
@@ -386,15 +389,19 @@ __global__ void __launch_bounds__(TcCfg<MB>::WARPS * 32, 1) gemm_tc_kernel(const
             if (lane == 0) tc_wait(smem_u32(&donej[b]), (uint32_t)(gc / C::P) & 1u, abort);
             __syncwarp();
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            float dv[MB];
-            tmem_ld_d<MB>(tl + (uint32_t)(C::DCOL + (j * C::P + b) * MB), dv);
             const float s = sb[b * 32];
             const float2 s2 = make_float2(s, s);
 #pragma unroll
-            for (int m = 0; m < MB; m += 2) {
-                const float2 r2 = __ffma2_rn(s2, make_float2(dv[m], dv[m + 1]), make_float2(y[m], y[m + 1]));
-                y[m] = r2.x;
-                y[m + 1] = r2.y;
+            for (int h = 0; h < MB / 16; ++h) {
+                float dv[16];
+                tmem_ld_d<16>(tl + (uint32_t)(C::DCOL + (j * C::P + b) * MB + 16 * h), dv);
+#pragma unroll
+                for (int m = 0; m < 16; m += 2) {
+                    const float2 r2 = __ffma2_rn(s2, make_float2(dv[m], dv[m + 1]),
+                                                 make_float2(y[16 * h + m], y[16 * h + m + 1]));
+                    y[16 * h + m] = r2.x;
+                    y[16 * h + m + 1] = r2.y;
+                }
             }
             ++gc;
         };
@@ -441,20 +448,24 @@ __global__ void __launch_bounds__(TcCfg<MB>::WARPS * 32, 1) gemm_tc_kernel(const
                 }
             }
             while (gc < gi) consume();
-            // block end: sets 1.. hand their sums to set 0, which adds them in set
-            // order and stores the rows (or, in a cluster, leaves them for the
-            // rank-ordered reduction)
+            // block end: sets 1.. hand their sums to set 0 (each set's own x
+            // image is free: its groups are all read back), which adds them in
+            // set order and stores the rows (or, in a cluster, leaves them for
+            // the rank-ordered reduction)
             if (j > 0) {
+                float *red = red_of(j);
 #pragma unroll
-                for (int m = 0; m < MB; ++m) red[((j - 1) * 128 + 32 * r + lane) * MB + m] = y[m];
+                for (int m = 0; m < MB; ++m) red[(32 * r + lane) * MB + m] = y[m];
             }
             named_sync(1, 32 * C::CW);
             if (j == 0) {
-                for (int o = 0; o < C::SETS - 1; ++o) {
+                for (int o = 1; o < C::SETS; ++o) {
+                    const float *red = red_of(o);
 #pragma unroll
-                    for (int m = 0; m < MB; ++m) y[m] += red[(o * 128 + 32 * r + lane) * MB + m];
+                    for (int m = 0; m < MB; ++m) y[m] += red[(32 * r + lane) * MB + m];
                 }
                 if (a.cl > 1) {
+                    float *red = red_of(0);
 #pragma unroll
                     for (int m = 0; m < MB; ++m) red[(32 * r + lane) * MB + m] = y[m];
                 } else if (active) {
@@ -526,7 +537,7 @@ __global__ void __launch_bounds__(TcCfg<MB>::WARPS * 32, 1) gemm_tc_kernel(const
 #pragma unroll
             for (int m = 0; m < MB; ++m) yv[m] = 0.f;
             for (int rk = 0; rk < a.cl; ++rk) {
-                const float *rp = cluster.map_shared_rank(red, rk) + (32 * warp + lane) * MB;
+                const float *rp = cluster.map_shared_rank(red_of(0), rk) + (32 * warp + lane) * MB;
 #pragma unroll
                 for (int m = 0; m < MB; ++m) yv[m] += rp[m];
             }
@@ -550,7 +561,7 @@ template <int MB>
 size_t tc_smem_bytes(int depth) {
     using C = TcCfg<MB>;
     return (size_t)C::SETS * 2 * C::XBYTES + (size_t)C::CW * depth * kStageBytes +
-           (size_t)C::CW * C::P * 32 * 4 + (size_t)(C::SETS - 1) * 128 * MB * 4 +
+           (size_t)C::CW * C::P * 32 * 4 +
            (size_t)(C::CW * depth + 2 * C::SETS * C::P + C::SETS) * 8 + 16;
 }
 
