@@ -587,7 +587,7 @@ spectra_status run_tc(const Prob &a0, const DeviceInfo &dev, cudaStream_t s) {
     }
     args.p.cl = cl;
     args.nblk = (int)nblk;
-    int depth = 4;
+    int depth = 2;  // two units in flight per warp; a third measured slower (shared memory left to L1)
     while (depth > 1 && tc_smem_bytes<MB>(depth) > dev.smem_optin) --depth;
     args.depth = depth;
     const size_t smem = tc_smem_bytes<MB>(depth);
