@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(TcCfg<MB>::WARPS * 32, 1) gemm_tc_kernel(const
         for (int d = 0; d < D && iblk < args.nblk; ++d) {
             const int t = 4 * iblk + r;
             if (t < a.T) ring_issue(ring, a, t, tc_unit(a, sg0, nsg, ob0, ilu), lane);
-            else ring.issued += ring.ok ? 1 : 0;  // keeps issue and acquire counts aligned
+            else ring_advance_issue(ring);  // keeps issue and acquire counts aligned
             advance(iblk, ilu);
         }
         pdl_wait();
@@ -421,7 +421,7 @@ __global__ void __launch_bounds__(TcCfg<MB>::WARPS * 32, 1) gemm_tc_kernel(const
                 }
                 const uint8_t *stage = nullptr;
                 if (active) stage = ring_acquire(ring, lane);
-                else if (ring.ok) ++ring.consumed;
+                else ring_advance_consume(ring);
                 __syncwarp();
                 const int ngr = tc_groups(a, u);
                 for (int g = 0; g < ngr; ++g) {
@@ -443,7 +443,7 @@ __global__ void __launch_bounds__(TcCfg<MB>::WARPS * 32, 1) gemm_tc_kernel(const
                 if (iblk < args.nblk) {
                     const int ti = 4 * iblk + r;
                     if (ti < a.T) ring_issue(ring, a, ti, tc_unit(a, sg0, nsg, ob0, ilu), lane);
-                    else ring.issued += ring.ok ? 1 : 0;
+                    else ring_advance_issue(ring);
                     advance(iblk, ilu);
                 }
             }

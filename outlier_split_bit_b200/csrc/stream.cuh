@@ -147,6 +147,8 @@ struct Ring {
     uint32_t base_s, bar_s;
     int D;
     int consumed, issued;
+    int cslot, islot;  // consumed % D and issued % D, kept incrementally
+    uint32_t cphase;   // (consumed / D) & 1
     bool ok;
     int failed_at;
 };
@@ -157,6 +159,8 @@ __device__ __forceinline__ void ring_init(Ring &r, uint8_t *base, uint64_t *bars
     r.bar_s = smem_u32(bars);
     r.D = D;
     r.consumed = r.issued = 0;
+    r.cslot = r.islot = 0;
+    r.cphase = 0u;
     r.ok = true;
     r.failed_at = 0;
     if (lane == 0) {
@@ -166,17 +170,25 @@ __device__ __forceinline__ void ring_init(Ring &r, uint8_t *base, uint64_t *bars
     __syncwarp();
 }
 
+// Advance the issue side by one stage (after a copy, or for a unit that is
+// skipped on both sides).
+__device__ __forceinline__ void ring_advance_issue(Ring &r) {
+    if (!r.ok) return;
+    ++r.issued;
+    if (++r.islot == r.D) r.islot = 0;
+}
+
 __device__ __forceinline__ void ring_issue(Ring &r, const Prob &a, int t, int u, int lane) {
-    const int d = r.issued % r.D;
+    const int d = r.islot;
     if (r.ok && lane == 0)
         issue_unit(a, t, u, r.base_s + (uint32_t)d * kStageBytes, r.bar_s + 8u * d);
-    if (r.ok) ++r.issued;
+    ring_advance_issue(r);
 }
 
 // Wait for the next stage to fill; returns its address (nullptr after a failure).
 __device__ __forceinline__ const uint8_t *ring_acquire(Ring &r, int lane) {
-    const int d = r.consumed % r.D;
-    if (r.ok && !mbar_wait(r.bar_s + 8u * d, (uint32_t)(r.consumed / r.D) & 1u)) {
+    const int d = r.cslot;
+    if (r.ok && !mbar_wait(r.bar_s + 8u * d, r.cphase)) {
         r.ok = false;
         r.failed_at = r.consumed;
         if (lane == 0) atomicOr(&g_device_error, 1u);
@@ -184,9 +196,19 @@ __device__ __forceinline__ const uint8_t *ring_acquire(Ring &r, int lane) {
     return r.ok ? r.base + (size_t)d * kStageBytes : nullptr;
 }
 
+// Advance the consume side by one stage.
+__device__ __forceinline__ void ring_advance_consume(Ring &r) {
+    if (!r.ok) return;
+    ++r.consumed;
+    if (++r.cslot == r.D) {
+        r.cslot = 0;
+        r.cphase ^= 1u;
+    }
+}
+
 __device__ __forceinline__ void ring_release(Ring &r) {
     __syncwarp();
-    if (r.ok) ++r.consumed;
+    ring_advance_consume(r);
 }
 
 // After a failed wait, let the copies already in flight land before the CTA
