@@ -137,6 +137,17 @@ __device__ __forceinline__ Slice slice_of(const Prob &a, int s, int P) {
     return r;
 }
 
+// slice_of for P = 2^lg slices (shifts instead of divisions).
+__device__ __forceinline__ Slice slice_of_pow2(const Prob &a, int s, int lg) {
+    const int OB = a.U - a.S;
+    Slice r;
+    r.sg0 = (a.S * s) >> lg;
+    r.nsg = ((a.S * (s + 1)) >> lg) - r.sg0;
+    r.ob0 = (OB * s) >> lg;
+    r.nob = ((OB * (s + 1)) >> lg) - r.ob0;
+    return r;
+}
+
 // Local unit u of a slice -> unit id (super-group id, or S + batch id).
 __device__ __forceinline__ int unit_id(const Prob &a, const Slice &sl, int u) {
     return u < sl.nsg ? sl.sg0 + u : a.S + sl.ob0 + (u - sl.nsg);
@@ -509,16 +520,22 @@ struct Cursor {
     Slice sl;
 };
 
+// Problem of `item`, searched forward from `p` (items only increase).
+__device__ __forceinline__ int prob_from(const PersistArgs &args, int item, int p) {
+    while (p + 1 < args.count && args.item_start[p + 1] <= item) ++p;
+    return p;
+}
+
 // Move the cursor to the first unit of `c.item` or of a later item of this warp.
 __device__ __forceinline__ void cursor_load(const PersistArgs &args, int it1, int warp, Cursor &c) {
     while (c.item < it1) {
-        c.p = prob_of(args, c.item);
+        c.p = prob_from(args, c.item, c.p);
         const Prob &a = args.probs[c.p];
         const int blk = c.item - args.item_start[c.p];
-        const int tl = warp / a.ppc;
+        const int tl = warp >> a.lgp;
         c.t = blk * a.tpc + tl;
         if (c.t < a.T) {
-            c.sl = slice_of(a, warp - tl * a.ppc, a.ppc);
+            c.sl = slice_of_pow2(a, warp & (a.ppc - 1), a.lgp);
             c.u = 0;
             if (c.sl.nsg + c.sl.nob > 0) return;
         }
@@ -552,6 +569,7 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1)
     pdl_launch_dependents();
     Cursor ic;
     ic.item = it0;
+    ic.p = it0 < it1 ? prob_of(args, it0) : 0;
     cursor_load(args, it1, warp, ic);
     for (int d = 0; d < ring.D && ic.item < it1; ++d) {
         cursor_issue(args, ring, ic, lane);
@@ -562,8 +580,9 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1)
     int cur_p = -1;
     int rbuf = 0;
     XRange xr = {0, 0, 0, 0};
+    int p = it0 < it1 ? prob_of(args, it0) : 0;
     for (int item = it0; item < it1; ++item) {
-        const int p = prob_of(args, item);
+        p = prob_from(args, item, p);
         const Prob &a = args.probs[p];
         if (p != cur_p) {
             // every warp is done with the previous x (the branch is CTA-uniform)
@@ -576,10 +595,10 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1)
             cur_p = p;
         }
         const int blk = item - args.item_start[p];
-        const int tl = warp / a.ppc, sl = warp - tl * a.ppc;
+        const int tl = warp >> a.lgp, sl = warp & (a.ppc - 1);
         const int t = blk * a.tpc + tl;
         const bool active = t < a.T;
-        const Slice slc = slice_of(a, sl, a.ppc);
+        const Slice slc = slice_of_pow2(a, sl, a.lgp);
         const int nunits = active ? slc.nsg + slc.nob : 0;
         float yacc[MB];
 #pragma unroll
@@ -807,6 +826,8 @@ spectra_status run_persistent(PersistArgs &args, int count, const DeviceInfo &de
         Prob &a = args.probs[i];
         const Geometry g = Geometry::of(a.n, a.k, a.n_o);
         item_shape(g, target, &a.ppc, &a.tpc);
+        a.lgp = 0;
+        while ((1 << a.lgp) < a.ppc) ++a.lgp;
         a.items = (int)cdiv(a.T, a.tpc);
         args.item_start[i] = items;
         items += a.items;

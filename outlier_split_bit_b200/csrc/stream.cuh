@@ -43,6 +43,7 @@ struct Prob {
     int n, k, m, G, S, O8, n_o, T;
     int U;         // units per tile
     int ppc, tpc;  // slices per tile, tiles per CTA item
+    int lgp;       // log2(ppc) where ppc is a power of two (persistent kernel)
     int cl;        // CTAs per cluster (cluster kernel)
     int ytype;
     int items;     // ceil(T / tpc)
@@ -243,6 +244,7 @@ void fill_prob(Prob &a, const spectra_layer &l, const Geometry &g, const uint16_
     a.U = units_of(g);
     a.ppc = 1;
     a.tpc = 1;
+    a.lgp = 0;
     a.cl = 1;
     a.ytype = ytype;
     a.items = 0;
