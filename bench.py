@@ -432,9 +432,10 @@ def kernel_source_digest() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(digest: str):
+def profiled_traffic(digest: str, algorithmic_bytes=None):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel source."""
+    the current kernel source and (when given) on a launch with the same
+    algorithmic bytes, i.e. the same workload and threshold."""
     p = os.path.join(ROOT, "profiles", "gemv_decode_stream_traffic.md")
     if not os.path.exists(p):
         return None
@@ -446,6 +447,9 @@ def profiled_traffic(digest: str):
     if vals.get("kernel_source_sha256_16") != digest:
         return None
     try:
+        if algorithmic_bytes is not None and \
+                int(vals["algorithmic_bytes_per_launch"]) != int(algorithmic_bytes):
+            return None
         return float(vals["dram_bytes_per_launch"])
     except (KeyError, ValueError):
         return None
@@ -549,8 +553,8 @@ def run_ours(args):
                          f"layer, repeated for {t_s:.1f} s (unpack + FP64 matvec, one thread)"}
 
     digest = kernel_source_digest()
-    traffic = profiled_traffic(digest)
     launch_bytes = st.bytes / launches_per_step
+    traffic = profiled_traffic(digest, launch_bytes)
     launch_us = step_ms * 1e3 / launches_per_step
     if rank == 0:
         line = {
