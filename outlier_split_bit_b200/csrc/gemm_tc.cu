@@ -17,20 +17,26 @@ namespace {
 // y[m][n] for 8 <= m_rows <= 32 (MB = 16 or 32 batch rows) on the fifth-
 // generation tensor cores.  A CTA owns blocks of 128 rows (4 tiles; TMEM
 // lane = row) and streams their units (super-groups, outlier batches) with
-// three kinds of warps:
+// two kinds of warps:
 //
-//  * three sets of four compute warps.  Set j takes every third unit of the
-//    block; warp 4j + r owns tile r (rows 32r..32r+31) and keeps its own
-//    cp.async.bulk ring of that tile's units.  Per group of 32 columns it
-//    writes the exact integer weights c - z as a BF16 A operand (128 rows x
-//    32 columns) into a TMEM buffer, and later reads back that group's FP32
-//    product D = (c - z) x from TMEM and adds s * D to its rows' sums.  The
-//    outlier columns enter the same way with their BF16 weights and s = 1.
+//  * SETS sets of four compute warps (three at 16 rows, two at 32).  Set j
+//    takes every SETS-th unit of the block; warp 4j + r owns tile r (rows
+//    32r..32r+31) and keeps its own cp.async.bulk ring of that tile's units.
+//    Per group of 32 columns it writes the exact integer weights c - z as a
+//    BF16 A operand (128 rows x 32 columns) into a TMEM buffer, and later
+//    reads back that group's FP32 product D = (c - z) x from TMEM and adds
+//    s * D to its rows' sums.  The outlier columns enter the same way with
+//    their BF16 weights and s = 1.
 //  * one MMA warp per set, whose elected lane issues two tcgen05.mma
-//    kind::f16 (M = 128, N = MB, K = 16) per group of its set and commits
-//    them to the group's mbarrier (each mbarrier operation costs the issuing
-//    thread on the order of a hundred cycles, so one issuer for both sets
-//    would pace the whole CTA).
+//    kind::f16 (M = 128, N = MB, K = 16) per group into the group's own D
+//    buffer.
+//
+// Groups travel in chunks of H: the compute warps store H groups' A operands
+// and arrive once, the MMA lane waits once, issues 2H MMAs and commits once,
+// and the compute warps wait once before reading the H D buffers back.  Each
+// mbarrier operation costs the issuing thread on the order of a hundred
+// cycles, more than one group's two MMAs, so handshakes per group would pace
+// the kernel.
 //
 // The products are exact: c - z is an integer in [-15, 15] and x is BF16, so
 // each product has at most 12 significant bits; D holds FP32 sums of 32 of
@@ -41,30 +47,36 @@ namespace {
 // the decoder pairs the codes: the two BF16 halves of TMEM column 4w + s are
 // columns 8w + s and 8w + s + 4 of the group.
 //
-// Handshakes, per set and TMEM buffer b (P buffers, used round robin):
-// full[b] (one arrival per compute warp, after its TMEM stores and x writes)
-// -> MMA issue -> done[b] (tcgen05.commit) -> compute threads read D[b].
-// A buffer is rewritten only after its previous D was read, so the MMA that
-// read its A has completed.  Every wait is bounded; a timeout raises the
+// Handshakes, per set and chunk slot q (Q slots of H TMEM buffers, used
+// round robin): full[q] (one arrival per compute warp, after its TMEM stores
+// and x writes) -> MMA issue -> done[q] (tcgen05.commit) -> compute threads
+// read the chunk's D buffers.  A slot is rebuilt only after its previous
+// chunk was read back, so the MMAs that read its A operands have completed.  Every wait is bounded; a timeout raises the
 // device error bit and turns the remaining waits into no-ops.
 constexpr int kTcTmemCols = 512;
 
-template <int MB>
+template <int MB_, int SETS_, int H_, int Q_>
 struct TcCfg {
-    // three warp sets: four warps per sub-partition, so at most 128 registers
-    // (16 rows: 121; 32 rows: 128, with the accumulators read back 16 columns
-    // at a time); TMEM holds 5 buffers per set at 16 rows, 3 at 32
-    static constexpr int SETS = 3;
+    static constexpr int MB = MB_;
+    static constexpr int SETS = SETS_;               // warp sets
+    static constexpr int H = H_;                     // groups per handshake (a chunk)
+    static constexpr int Q = Q_;                     // chunk slots per set
+    static constexpr int P = H * Q;                  // TMEM group buffers per set
     static constexpr int CW = 4 * SETS;              // compute warps
     static constexpr int WARPS = CW + SETS;          // + one MMA warp per set
-    static constexpr int P = MB == 16 ? 5 : 3;       // TMEM buffers per set
-    static constexpr int L = P - 1;                  // groups produced ahead of the one read back
     static constexpr int DCOL = (SETS * P * 16 + 31) / 32 * 32;  // A buffers below, D from here
     static constexpr int XBYTES = 256 * MB * 2;      // x image of one super-group
     static constexpr int KSTEP = MB * 32;            // bytes of one 16-column K step of x
     static_assert(DCOL + SETS * P * MB <= kTcTmemCols, "TMEM budget");
     static_assert(DCOL % 32 == 0, "D alignment");
+    static_assert(H >= 1 && H <= 8 && Q >= 2 && Q <= 8, "chunk shape");
 };
+
+// 16 rows: three sets of four compute warps (four warps per sub-partition
+// keep each thread within 128 registers), chunks of two groups, two chunk
+// slots per set.  32 rows: the D buffers are twice as wide, so two sets.
+using TcCfg16 = TcCfg<16, 3, 2, 2>;
+using TcCfg32 = TcCfg<32, 2, 2, 2>;
 
 struct TcArgs {
     Prob p;
@@ -191,7 +203,7 @@ __device__ __forceinline__ void tc_store_x(const Prob &a, int u, int tid, const 
             const uint4 v = xp.v[i];
             const uint4 p = make_uint4(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632),
                                        __byte_perm(v.y, v.w, 0x5410), __byte_perm(v.y, v.w, 0x7632));
-            *reinterpret_cast<uint4 *>(xb + (W >> 1) * TcCfg<MB>::KSTEP + (m >> 3) * 256 +
+            *reinterpret_cast<uint4 *>(xb + (W >> 1) * (MB * 32) + (m >> 3) * 256 +
                                        (W & 1) * 128 + (m & 7) * 16) = p;
         }
     } else {
@@ -205,7 +217,7 @@ __device__ __forceinline__ void tc_store_x(const Prob &a, int u, int tid, const 
             const uint32_t k1 = nv >= 4 ? 0xFFFFFFFFu : (nv == 3 ? 0x0000FFFFu : 0u);
             const uint32_t k2 = nv >= 6 ? 0xFFFFFFFFu : (nv == 5 ? 0x0000FFFFu : 0u);
             const uint32_t k3 = nv >= 8 ? 0xFFFFFFFFu : (nv == 7 ? 0x0000FFFFu : 0u);
-            *reinterpret_cast<uint4 *>(xb + (o >> 1) * TcCfg<MB>::KSTEP + (m >> 3) * 256 +
+            *reinterpret_cast<uint4 *>(xb + (o >> 1) * (MB * 32) + (m >> 3) * 256 +
                                        (o & 1) * 128 + (m & 7) * 16) =
                 make_uint4(v.x & k0, v.y & k1, v.z & k2, v.w & k3);
         }
@@ -296,9 +308,9 @@ __device__ __forceinline__ float tc_build_a(const Prob &a, int u, int g, const u
     return 1.f;
 }
 
-template <int MB>
-__global__ void __launch_bounds__(TcCfg<MB>::WARPS * 32, 1) gemm_tc_kernel(const TcArgs args) {
-    using C = TcCfg<MB>;
+template <typename C>
+__global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs args) {
+    constexpr int MB = C::MB;
     extern __shared__ __align__(1024) uint8_t tsm[];
     const Prob &a = args.p;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -313,9 +325,9 @@ __global__ void __launch_bounds__(TcCfg<MB>::WARPS * 32, 1) gemm_tc_kernel(const
     float *sbuf = reinterpret_cast<float *>(ring_base + (size_t)C::CW * D * kStageBytes);
     auto red_of = [&](int set) { return reinterpret_cast<float *>(ximg + (size_t)set * 2 * C::XBYTES); };
     uint64_t *bars = reinterpret_cast<uint64_t *>(sbuf + C::CW * C::P * 32);
-    uint64_t *full = bars + C::CW * D;      // [SETS][P]
-    uint64_t *done = full + C::SETS * C::P;  // [SETS][P]
-    uint64_t *fin = done + C::SETS * C::P;   // [SETS]
+    uint64_t *full = bars + C::CW * D;      // [SETS][Q]
+    uint64_t *done = full + C::SETS * C::Q;  // [SETS][Q]
+    uint64_t *fin = done + C::SETS * C::Q;   // [SETS]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(fin + C::SETS);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -333,7 +345,7 @@ __global__ void __launch_bounds__(TcCfg<MB>::WARPS * 32, 1) gemm_tc_kernel(const
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     if (threadIdx.x == 32) {
-        for (int b = 0; b < C::SETS * C::P; ++b) {
+        for (int b = 0; b < C::SETS * C::Q; ++b) {
             mbar_init(smem_u32(&full[b]), 4u);  // one arrival per compute warp of the set
             mbar_init(smem_u32(&done[b]), 1u);
         }
@@ -354,7 +366,7 @@ __global__ void __launch_bounds__(TcCfg<MB>::WARPS * 32, 1) gemm_tc_kernel(const
         // ------------------------------------------------ compute warps
         const int j = warp >> 2, r = warp & 3, tid = threadIdx.x - 128 * j;
         const uint32_t tl = tmem + ((uint32_t)(32 * r) << 16);
-        uint64_t *fullj = full + j * C::P, *donej = done + j * C::P;
+        uint64_t *fullj = full + j * C::Q, *donej = done + j * C::Q;
         float *sb = sbuf + (warp * C::P) * 32 + lane;
         // issue iterator (ring) and x iterator run ahead of the work iterator
         int iblk = blockIdx.x / a.cl, ilu = j;
@@ -379,31 +391,41 @@ __global__ void __launch_bounds__(TcCfg<MB>::WARPS * 32, 1) gemm_tc_kernel(const
         if (xblk < args.nblk) tc_load_x<MB>(a, tc_unit(a, sg0, nsg, ob0, xlu), tid, xp);
         advance(xblk, xlu);
 
-        int gi = 0, gc = 0, xl = 0;
-        int lastg[2] = {-1, -1};
+        // chunks built (ci) and read back (cc); groups of each slot's chunk,
+        // four bits per slot
+        int ci = 0, cc = 0, xl = 0;
+        uint32_t nhs = 0;
+        int lastc0 = -1, lastc1 = -1;  // last chunk of the units in x image 0 / 1
         float y[MB];
 #pragma unroll
         for (int m = 0; m < MB; ++m) y[m] = 0.f;
         auto consume = [&]() {
-            const int b = gc % C::P;
-            if (lane == 0) tc_wait(smem_u32(&donej[b]), (uint32_t)(gc / C::P) & 1u, abort);
+            const int q = cc % C::Q;
+            if (lane == 0) tc_wait(smem_u32(&donej[q]), (uint32_t)(cc / C::Q) & 1u, abort);
             __syncwarp();
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            const float s = sb[b * 32];
-            const float2 s2 = make_float2(s, s);
+            const int nh = (int)((nhs >> (4 * q)) & 0xFu);
 #pragma unroll
-            for (int h = 0; h < MB / 16; ++h) {
-                float dv[16];
-                tmem_ld_d<16>(tl + (uint32_t)(C::DCOL + (j * C::P + b) * MB + 16 * h), dv);
+            for (int h = 0; h < C::H; ++h) {
+                if (h < nh) {  // warp-uniform
+                    const int b = q * C::H + h;
+                    const float s = sb[b * 32];
+                    const float2 s2 = make_float2(s, s);
 #pragma unroll
-                for (int m = 0; m < 16; m += 2) {
-                    const float2 r2 = __ffma2_rn(s2, make_float2(dv[m], dv[m + 1]),
-                                                 make_float2(y[16 * h + m], y[16 * h + m + 1]));
-                    y[16 * h + m] = r2.x;
-                    y[16 * h + m + 1] = r2.y;
+                    for (int hh = 0; hh < MB / 16; ++hh) {
+                        float dv[16];
+                        tmem_ld_d<16>(tl + (uint32_t)(C::DCOL + (j * C::P + b) * MB + 16 * hh), dv);
+#pragma unroll
+                        for (int m = 0; m < 16; m += 2) {
+                            const float2 r2 = __ffma2_rn(s2, make_float2(dv[m], dv[m + 1]),
+                                                         make_float2(y[16 * hh + m], y[16 * hh + m + 1]));
+                            y[16 * hh + m] = r2.x;
+                            y[16 * hh + m + 1] = r2.y;
+                        }
+                    }
                 }
             }
-            ++gc;
+            ++cc;
         };
 
         for (int blk = blockIdx.x / a.cl; blk < args.nblk; blk += bstride) {
@@ -413,7 +435,7 @@ __global__ void __launch_bounds__(TcCfg<MB>::WARPS * 32, 1) gemm_tc_kernel(const
                 const int u = tc_unit(a, sg0, nsg, ob0, lu);
                 uint8_t *xb = ximg + (size_t)(j * 2 + (xl & 1)) * C::XBYTES;
                 // the MMAs of unit xl - 2 read this x buffer: wait for them
-                while (gc <= lastg[xl & 1]) consume();
+                while (cc <= ((xl & 1) ? lastc1 : lastc0)) consume();
                 tc_store_x<MB>(a, u, tid, xp, xb);
                 if (xblk < args.nblk) {
                     tc_load_x<MB>(a, tc_unit(a, sg0, nsg, ob0, xlu), tid, xp);
@@ -424,21 +446,34 @@ __global__ void __launch_bounds__(TcCfg<MB>::WARPS * 32, 1) gemm_tc_kernel(const
                 else ring_advance_consume(ring);
                 __syncwarp();
                 const int ngr = tc_groups(a, u);
-                for (int g = 0; g < ngr; ++g) {
-                    const int b = gi % C::P;
-                    uint32_t av[16];
-                    const float s = tc_build_a(a, u, g, stage, lane, av);
-                    tmem_st16(tl + (uint32_t)((j * C::P + b) * 16), av);
-                    sb[b * 32] = s;
+                for (int g0 = 0; g0 < ngr; g0 += C::H) {
+                    // one chunk: up to H groups' A operands, then one arrival
+                    const int q = ci % C::Q;
+                    const int nh = min(C::H, ngr - g0);
+#pragma unroll
+                    for (int h = 0; h < C::H; ++h) {
+                        if (h < nh) {  // warp-uniform
+                            const int b = q * C::H + h;
+                            uint32_t av[16];
+                            const float s = tc_build_a(a, u, g0 + h, stage, lane, av);
+                            tmem_st16(tl + (uint32_t)((j * C::P + b) * 16), av);
+                            sb[b * 32] = s;
+                        }
+                    }
                     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_u32(&fullj[b]));
-                    ++gi;
-                    if (gi - gc > C::L) consume();
+                    if (lane == 0) mbar_arrive(smem_u32(&fullj[q]));
+                    nhs = (nhs & ~(0xFu << (4 * q))) | ((uint32_t)nh << (4 * q));
+                    ++ci;
+                    // a slot is rebuilt only after its chunk was read back
+                    if (ci - cc > C::Q - 1) consume();
                 }
-                lastg[xl & 1] = gi - 1;
+                if (xl & 1)
+                    lastc1 = ci - 1;
+                else
+                    lastc0 = ci - 1;
                 if (active) ring_release(ring);
                 if (iblk < args.nblk) {
                     const int ti = 4 * iblk + r;
@@ -447,7 +482,7 @@ __global__ void __launch_bounds__(TcCfg<MB>::WARPS * 32, 1) gemm_tc_kernel(const
                     advance(iblk, ilu);
                 }
             }
-            while (gc < gi) consume();
+            while (cc < ci) consume();
             // block end: sets 1.. hand their sums to set 0 (each set's own x
             // image is free: its groups are all read back), which adds them in
             // set order and stores the rows (or, in a cluster, leaves them for
@@ -489,28 +524,33 @@ __global__ void __launch_bounds__(TcCfg<MB>::WARPS * 32, 1) gemm_tc_kernel(const
             for (int lu = j; lu < nunits; lu += C::SETS, ++xl) {
                 const int ngr = tc_groups(a, tc_unit(a, sg0, nsg, ob0, lu));
                 const uint32_t xs0 = smem_u32(ximg + (size_t)(j * 2 + (xl & 1)) * C::XBYTES);
-                for (int g = 0; g < ngr; ++g, ++q) {
-                    const int b = q % C::P;
-                    const bool ok = tc_wait(smem_u32(&full[j * C::P + b]), (uint32_t)(q / C::P) & 1u, abort);
+                for (int g0 = 0; g0 < ngr; g0 += C::H, ++q) {
+                    const int sl = q % C::Q;
+                    const int nh = min(C::H, ngr - g0);
+                    const bool ok = tc_wait(smem_u32(&full[j * C::Q + sl]), (uint32_t)(q / C::Q) & 1u, abort);
                     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                     if (ok) {
-                        const uint32_t xs = xs0 + (uint32_t)(2 * g * C::KSTEP);
-                        const uint32_t ta = tmem + (uint32_t)((j * C::P + b) * 16);
-                        const uint32_t td = tmem + (uint32_t)(C::DCOL + (j * C::P + b) * MB);
+                        for (int h = 0; h < nh; ++h) {
+                            const int b = sl * C::H + h;
+                            const uint32_t xs = xs0 + (uint32_t)(2 * (g0 + h) * C::KSTEP);
+                            const uint32_t ta = tmem + (uint32_t)((j * C::P + b) * 16);
+                            const uint32_t td = tmem + (uint32_t)(C::DCOL + (j * C::P + b) * MB);
 #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const uint64_t bdesc = umma_desc(xs + (uint32_t)(h * C::KSTEP), 128u, 256u);
-                            asm volatile(
-                                "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %3, 0;\n\t"
-                                "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p;\n\t}" ::"r"(td),
-                                "r"(ta + 8u * h), "l"(bdesc), "r"((uint32_t)h), "r"(idesc)
-                                : "memory");
+                            for (int k = 0; k < 2; ++k) {
+                                const uint64_t bdesc = umma_desc(xs + (uint32_t)(k * C::KSTEP), 128u, 256u);
+                                asm volatile(
+                                    "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %3, 0;\n\t"
+                                    "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p;\n\t}" ::"r"(td),
+                                    "r"(ta + 8u * k), "l"(bdesc), "r"((uint32_t)k), "r"(idesc)
+                                    : "memory");
+                            }
                         }
                         any = true;
                     }
+                    // one commit per chunk: done[sl] fires when all its MMAs completed
                     asm volatile(
                         "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                            smem_u32(&done[j * C::P + b]))
+                            smem_u32(&done[j * C::Q + sl]))
                         : "memory");
                 }
             }
@@ -557,15 +597,14 @@ __global__ void __launch_bounds__(TcCfg<MB>::WARPS * 32, 1) gemm_tc_kernel(const
     }
 }
 
-template <int MB>
+template <typename C>
 size_t tc_smem_bytes(int depth) {
-    using C = TcCfg<MB>;
     return (size_t)C::SETS * 2 * C::XBYTES + (size_t)C::CW * depth * kStageBytes +
            (size_t)C::CW * C::P * 32 * 4 +
-           (size_t)(C::CW * depth + 2 * C::SETS * C::P + C::SETS) * 8 + 16;
+           (size_t)(C::CW * depth + 2 * C::SETS * C::Q + C::SETS) * 8 + 16;
 }
 
-template <int MB>
+template <typename C>
 spectra_status run_tc(const Prob &a0, const DeviceInfo &dev, cudaStream_t s) {
     static bool done[64];
     TcArgs args;
@@ -588,13 +627,13 @@ spectra_status run_tc(const Prob &a0, const DeviceInfo &dev, cudaStream_t s) {
     args.p.cl = cl;
     args.nblk = (int)nblk;
     int depth = 2;  // two units in flight per warp; a third measured slower (shared memory left to L1)
-    while (depth > 1 && tc_smem_bytes<MB>(depth) > dev.smem_optin) --depth;
+    while (depth > 1 && tc_smem_bytes<C>(depth) > dev.smem_optin) --depth;
     args.depth = depth;
-    const size_t smem = tc_smem_bytes<MB>(depth);
+    const size_t smem = tc_smem_bytes<C>(depth);
     if (smem > dev.smem_optin) return SPECTRA_ERR_SHAPE;
-    cudaError_t e = prepare_kernel(gemm_tc_kernel<MB>, done, dev);
+    cudaError_t e = prepare_kernel(gemm_tc_kernel<C>, done, dev);
     if (e != cudaSuccess) return SPECTRA_ERR_CUDA;
-    e = launch_kernel(gemm_tc_kernel<MB>, args, (unsigned)grid, smem, TcCfg<MB>::WARPS, cl, s);
+    e = launch_kernel(gemm_tc_kernel<C>, args, (unsigned)grid, smem, C::WARPS, cl, s);
     return e == cudaSuccess ? SPECTRA_OK : SPECTRA_ERR_CUDA;
 }
 
@@ -605,7 +644,7 @@ spectra_status launch_tc(const spectra_layer &l, const uint16_t *x, int m, void 
     const Geometry g = Geometry::of(l.n, l.k, l.n_outliers);
     Prob a;
     fill_prob(a, l, g, x, m, y, ytype);
-    return m <= 16 ? run_tc<16>(a, dev, s) : run_tc<32>(a, dev, s);
+    return m <= 16 ? run_tc<TcCfg16>(a, dev, s) : run_tc<TcCfg32>(a, dev, s);
 }
 
 spectra_status tc_device_error(bool *raised, cudaStream_t s) {

@@ -46,9 +46,9 @@
 //    prefetching across item boundaries and x is restaged only when the
 //    matrix changes.
 // Programmatic dependent launch: a kernel lets the next kernel on the stream
-// launch once all of its CTAs run, issues its first D units of (constant)
+// launch once all of its CTAs run, issues its first units of (constant)
 // weights, and only then waits for the previous grid before it reads x or
-// writes y.
+// writes y; x's first loads go out before the rest of the ring is filled.
 #include "stream.cuh"
 
 namespace spectra {
@@ -69,11 +69,13 @@ struct Smem {
 struct ClusterArgs {
     Prob p;
     Smem sm;
+    int pre;  // ring stages a warp issues before waiting on the previous grid
 };
 
 // Parameters of the persistent kernel, passed by value (kernel parameter space).
 struct PersistArgs {
     Smem sm;
+    int pre;                        // ring stages a warp issues before the wait
     int count;                      // problems
     int item_start[kMaxBatch + 1];  // first item of each problem
     int cta_first[kMaxCtas + 1];    // first item of each CTA
@@ -188,35 +190,48 @@ __device__ __forceinline__ void load_x_idx(const Prob &a, const XRange &xr, int 
     }
 }
 
-// Stage x for a unit range: bulk groups as BF16 pairs in the decoder's order
-// with their FP32 sums X_g (column order), and the BF16 pairs of the outlier
-// slots, gathered through the index list (first round: indices `xi`).  The
-// first bulk round and the first gather round are in flight together.
+// The first round of a thread's x loads, held in registers: the first bulk
+// round (4 x 16 bytes of one group) and the first gather round (8 outlier
+// pairs).  Loading them before the kernel issues its remaining weight stages
+// puts them ahead of those stages in the memory system's queues.
+struct XFirst {
+    uint4 v0[4];
+    uint32_t lo[8], hi[8];
+};
+
 template <int MB>
-__device__ void stage_x(const Prob &a, const Stage<MB> &st, const XRange &xr, const XIdx &xi) {
+__device__ __forceinline__ void stage_x_load(const Prob &a, const XRange &xr, const XIdx &xi,
+                                             XFirst &f) {
     const int nth = blockDim.x;
     const int ng = xr.g1 - xr.g0;
     const int np = (xr.j1 - xr.j0) / 2;
-    // first bulk round: this thread's 4 x 16 bytes
-    uint4 v0[4];
     {
         const int c = threadIdx.x, gl = c / MB, m = c - gl * MB, g = xr.g0 + gl;
         if (c < ng * MB && g < a.G && m < a.m) {
             const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)m * a.k + 32 * g);
 #pragma unroll
-            for (int w = 0; w < 4; ++w) v0[w] = src[w];
+            for (int w = 0; w < 4; ++w) f.v0[w] = src[w];
         }
     }
-    // first gather round
-    uint32_t lo[8], hi[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int c = threadIdx.x + i * nth;
         const int m = c % MB;
         const bool mv = c < np * MB && m < a.m;
-        lo[i] = (mv && xi.i0[i] >= 0) ? a.x[(size_t)m * a.k + xi.i0[i]] : 0u;
-        hi[i] = (mv && xi.i1[i] >= 0) ? a.x[(size_t)m * a.k + xi.i1[i]] : 0u;
+        f.lo[i] = (mv && xi.i0[i] >= 0) ? a.x[(size_t)m * a.k + xi.i0[i]] : 0u;
+        f.hi[i] = (mv && xi.i1[i] >= 0) ? a.x[(size_t)m * a.k + xi.i1[i]] : 0u;
     }
+}
+
+// Stage x for a unit range: bulk groups as BF16 pairs in the decoder's order
+// with their FP32 sums X_g (column order), and the BF16 pairs of the outlier
+// slots, gathered through the index list; the first round comes from `f`.
+template <int MB>
+__device__ void stage_x_store(const Prob &a, const Stage<MB> &st, const XRange &xr,
+                              const XFirst &f) {
+    const int nth = blockDim.x;
+    const int ng = xr.g1 - xr.g0;
+    const int np = (xr.j1 - xr.j0) / 2;
     for (int c = threadIdx.x; c < ng * MB; c += nth) {
         const int gl = c / MB, m = c - gl * MB;
         const int g = xr.g0 + gl;
@@ -226,7 +241,7 @@ __device__ void stage_x(const Prob &a, const Stage<MB> &st, const XRange &xr, co
             uint4 v[4];
             if (c == (int)threadIdx.x) {
 #pragma unroll
-                for (int w = 0; w < 4; ++w) v[w] = v0[w];
+                for (int w = 0; w < 4; ++w) v[w] = f.v0[w];
             } else {
                 const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)m * a.k + 32 * g);
 #pragma unroll
@@ -253,7 +268,7 @@ __device__ void stage_x(const Prob &a, const Stage<MB> &st, const XRange &xr, co
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int c = threadIdx.x + i * nth;
-        if (c < np * MB) st.xo[c] = lo[i] | (hi[i] << 16);
+        if (c < np * MB) st.xo[c] = f.lo[i] | (f.hi[i] << 16);
     }
     // further gather rounds: 8 pairs per thread in flight
     for (int base = 8 * nth; base < np * MB; base += 8 * nth) {
@@ -278,6 +293,14 @@ __device__ void stage_x(const Prob &a, const Stage<MB> &st, const XRange &xr, co
             }
         }
     }
+}
+
+template <int MB>
+__device__ __forceinline__ void stage_x(const Prob &a, const Stage<MB> &st, const XRange &xr,
+                                        const XIdx &xi) {
+    XFirst f;
+    stage_x_load<MB>(a, xr, xi, f);
+    stage_x_store<MB>(a, st, xr, f);
 }
 
 // ---------------------------------------------------------------- units
@@ -440,12 +463,17 @@ __global__ void __launch_bounds__(kClusterWarps * 32, MB == 1 ? 2 : 1)
     ring_init(ring, st.ring + (size_t)warp * args.sm.depth * kStageBytes,
               st.bar + warp * args.sm.depth, args.sm.depth, lane);
     pdl_launch_dependents();
+    // `pre` stages cover the wait; the rest are issued behind x's first loads
+    const int pre = min(args.pre, ring.D);
     int next = 0;
-    for (; next < nunits && next < ring.D; ++next) ring_issue(ring, a, t, unit_id(a, slc, next), lane);
+    for (; next < nunits && next < pre; ++next) ring_issue(ring, a, t, unit_id(a, slc, next), lane);
     XIdx xi;
     load_x_idx(a, xr, MB, xi);
     pdl_wait();
-    stage_x<MB>(a, st, xr, xi);
+    XFirst xf;
+    stage_x_load<MB>(a, xr, xi, xf);
+    for (; next < nunits && next < ring.D; ++next) ring_issue(ring, a, t, unit_id(a, slc, next), lane);
+    stage_x_store<MB>(a, st, xr, xf);
     __syncthreads();
 
     float yacc[MB];
@@ -571,16 +599,35 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1)
     ic.item = it0;
     ic.p = it0 < it1 ? prob_of(args, it0) : 0;
     cursor_load(args, it1, warp, ic);
-    for (int d = 0; d < ring.D && ic.item < it1; ++d) {
+    // `pre` stages cover the wait; the rest are issued behind x's first loads
+    const int pre = min(args.pre, ring.D);
+    int d = 0;
+    for (; d < pre && ic.item < it1; ++d) {
         cursor_issue(args, ring, ic, lane);
         cursor_next(args, it1, warp, ic);
     }
-    pdl_wait();
-
-    int cur_p = -1;
-    int rbuf = 0;
-    XRange xr = {0, 0, 0, 0};
     int p = it0 < it1 ? prob_of(args, it0) : 0;
+    int cur_p = -1;
+    XRange xr = {0, 0, 0, 0};
+    XIdx xi;
+    if (it0 < it1) {
+        xr = x_range(args.probs[p], 0, 1, 1);
+        load_x_idx(args.probs[p], xr, MB, xi);
+    }
+    pdl_wait();
+    if (it0 < it1) {
+        XFirst xf;
+        stage_x_load<MB>(args.probs[p], xr, xi, xf);
+        for (; d < ring.D && ic.item < it1; ++d) {
+            cursor_issue(args, ring, ic, lane);
+            cursor_next(args, it1, warp, ic);
+        }
+        stage_x_store<MB>(args.probs[p], st, xr, xf);
+        __syncthreads();
+        cur_p = p;
+    }
+
+    int rbuf = 0;
     for (int item = it0; item < it1; ++item) {
         p = prob_from(args, item, p);
         const Prob &a = args.probs[p];
@@ -643,6 +690,11 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1)
 constexpr size_t kSmPerSm = 228 * 1024;  // shared memory of one SM
 constexpr size_t kCtaReserve = 1024;     // per-CTA shared memory the system reserves
 constexpr int kMaxDepth = 4;
+// Ring stages a warp issues before it waits on the previous grid.  All of
+// them would queue x's loads behind the whole of this SM's weights (x can
+// only be read after the wait), so the decode could not start before the
+// stream had landed; one stage per warp (about 75 KB per SM) covers the wait.
+constexpr int kPreStages = 1;
 
 
 int64_t tile_bytes(const Geometry &g) {
@@ -841,6 +893,7 @@ spectra_status run_persistent(PersistArgs &args, int count, const DeviceInfo &de
     if (sm.depth > 2) sm.depth = 2;  // 16 warps x 2 stages keep ~150 KB in flight per SM
     if (sm.depth == 0) return SPECTRA_ERR_SHAPE;
     args.sm = sm;
+    args.pre = kPreStages;
     int ncta = dev.sm_count;
     if (ncta > kMaxCtas) ncta = kMaxCtas;
     if (ncta > items) ncta = items;
@@ -876,6 +929,7 @@ spectra_status run_cluster(const Prob &a0, const ClusterPlan &p, const DeviceInf
     args.p.tpc = p.tpc;
     args.p.cl = p.cl;
     args.sm = p.sm;
+    args.pre = kPreStages;
     cudaError_t e = prepare_kernel(gemv_cluster_kernel<MB>, done, dev);
     if (e != cudaSuccess) return SPECTRA_ERR_CUDA;
     e = launch_kernel(gemv_cluster_kernel<MB>, args, p.grid, stage_bytes(MB, kClusterWarps, p.sm),

@@ -6,6 +6,8 @@ matvec, |y - y_ref| <= 2e-3 * sum_j |w_hat_ij x_j| + 1e-5, is the acceptance
 rule of the build; packing outputs (kurtosis, outlier indices, codes,
 scales, zero points, outlier block) must be identical bit for bit.
 """
+import gc
+
 import numpy as np
 import pytest
 import torch
@@ -273,13 +275,20 @@ def test_matvec_allocates_nothing():
     view = lay.view()
     sp.spectra_gemv(lay, x[0], y, view=view)
     torch.cuda.synchronize()
-    a0 = torch.cuda.memory_allocated()
-    r0 = torch.cuda.memory_reserved()
-    for _ in range(1000):
-        sp.spectra_gemv(lay, x[0], y, view=view)
-    torch.cuda.synchronize()
-    assert torch.cuda.memory_allocated() == a0
-    assert torch.cuda.memory_reserved() == r0
+    # tensors of earlier tests that a garbage-collection pass frees inside the
+    # loop would change the count without any allocation by the matvec
+    gc.collect()
+    gc.disable()
+    try:
+        a0 = torch.cuda.memory_allocated()
+        r0 = torch.cuda.memory_reserved()
+        for _ in range(1000):
+            sp.spectra_gemv(lay, x[0], y, view=view)
+        torch.cuda.synchronize()
+        assert torch.cuda.memory_allocated() == a0
+        assert torch.cuda.memory_reserved() == r0
+    finally:
+        gc.enable()
 
 
 def test_batched_equals_single_launches():

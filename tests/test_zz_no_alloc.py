@@ -8,6 +8,7 @@ This file is collected last on purpose, so that a run stopping at the first
 failure has already run every other test.
 """
 import ctypes
+import gc
 
 import numpy as np
 import pytest
@@ -28,11 +29,16 @@ def _noalloc(L, w, g, tau, kappa_out):
     n_o = ctypes.c_int32(-1)
     stream = torch.cuda.current_stream().cuda_stream
     torch.cuda.synchronize()
-    before = torch.cuda.memory_allocated()
-    st = L.spectra_pack_plan_noalloc(w.data_ptr(), None if g is None else g.data_ptr(), n, k,
-                                     float(tau), None if kappa_out is None else kappa_out.data_ptr(),
-                                     idx.data_ptr(), ctypes.byref(n_o), stream)
-    assert torch.cuda.memory_allocated() == before
+    gc.collect()  # no collection of earlier tests' tensors inside the measured call
+    gc.disable()
+    try:
+        before = torch.cuda.memory_allocated()
+        st = L.spectra_pack_plan_noalloc(w.data_ptr(), None if g is None else g.data_ptr(), n, k,
+                                         float(tau), None if kappa_out is None else kappa_out.data_ptr(),
+                                         idx.data_ptr(), ctypes.byref(n_o), stream)
+        assert torch.cuda.memory_allocated() == before
+    finally:
+        gc.enable()
     assert st == _lib.OK, sp.spectra_status_string(st)
     return idx[: n_o.value].clone()
 
