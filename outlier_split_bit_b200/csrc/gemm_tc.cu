@@ -125,20 +125,22 @@ __device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile 
     uint64_t t0 = 0;
     for (uint32_t i = 0;; ++i) {
         uint32_t ok;
+        // the thread sleeps until the phase completes or the hint expires, so
+        // a waiting lane leaves the issue slots to the warps that build operands
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
             "selp.u32 %0, 1, 0, p;\n\t}"
             : "=r"(ok)
-            : "r"(bar), "r"(parity)
+            : "r"(bar), "r"(parity), "r"(kSuspendNs)
             : "memory");
         if (ok) return true;
-        if ((i & 255u) == 0u) {
-            if (*abort) return false;
-            const uint64_t now = global_ns();
-            if (i == 0) t0 = now;
-            else if (now - t0 > kTcWaitNs) break;
-        }
+        if (*abort) return false;
+        const uint64_t now = global_ns();
+        if (i == 0)
+            t0 = now;
+        else if (now - t0 > kTcWaitNs)
+            break;
     }
     *abort = 1;
     atomicOr(&g_device_error, 1u);
@@ -230,6 +232,21 @@ __device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
     return d;
 }
 
+// Shared-memory loads by 32-bit address (the ring stages are shared memory).
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *v) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
@@ -280,9 +297,10 @@ __device__ __forceinline__ float tc_build_a(const Prob &a, int u, int g, const u
         return 0.f;
     }
     if (u < a.S) {
-        const uint4 q = *reinterpret_cast<const uint4 *>(stage + g * 512 + lane * 16);
-        const uint32_t sw = *reinterpret_cast<const uint32_t *>(stage + 4096 + lane * 16 + (g >> 1) * 4);
-        const uint32_t zw = *reinterpret_cast<const uint32_t *>(stage + 4608 + lane * 4);
+        const uint32_t sa = smem_u32(stage);
+        const uint4 q = lds128(sa + g * 512 + lane * 16);
+        const uint32_t sw = lds32(sa + 4096 + lane * 16 + (g >> 1) * 4);
+        const uint32_t zw = lds32(sa + 4608 + lane * 4);
         const uint32_t z = (zw >> (4 * g)) & 0xFu;
         const uint32_t zz = (0x4300u | z) * 0x00010001u;  // BF16 pair (128 + z, 128 + z)
         const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
@@ -316,15 +334,14 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cr = (a.cl > 1) ? (int)cg::this_cluster().block_rank() : 0;
     const int D = args.depth;
-    // shared memory: [x images SETS x 2][ring CW x D][scales CW x P x 32]
+    // shared memory: [x images SETS x 2][ring CW x D]
     // [bars][tmem slot, abort].  At a block end, once every group of the block
     // has been read back, set j's first x image holds its 128 x MB partial
     // sums (the same 256 x MB x 2 bytes).
     uint8_t *ximg = tsm;
     uint8_t *ring_base = ximg + (size_t)C::SETS * 2 * C::XBYTES;
-    float *sbuf = reinterpret_cast<float *>(ring_base + (size_t)C::CW * D * kStageBytes);
     auto red_of = [&](int set) { return reinterpret_cast<float *>(ximg + (size_t)set * 2 * C::XBYTES); };
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sbuf + C::CW * C::P * 32);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(ring_base + (size_t)C::CW * D * kStageBytes);
     uint64_t *full = bars + C::CW * D;      // [SETS][Q]
     uint64_t *done = full + C::SETS * C::Q;  // [SETS][Q]
     uint64_t *fin = done + C::SETS * C::Q;   // [SETS]
@@ -367,7 +384,6 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
         const int j = warp >> 2, r = warp & 3, tid = threadIdx.x - 128 * j;
         const uint32_t tl = tmem + ((uint32_t)(32 * r) << 16);
         uint64_t *fullj = full + j * C::Q, *donej = done + j * C::Q;
-        float *sb = sbuf + (warp * C::P) * 32 + lane;
         // issue iterator (ring) and x iterator run ahead of the work iterator
         int iblk = blockIdx.x / a.cl, ilu = j;
         auto advance = [&](int &blk, int &lu) {
@@ -391,30 +407,35 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
         if (xblk < args.nblk) tc_load_x<MB>(a, tc_unit(a, sg0, nsg, ob0, xlu), tid, xp);
         advance(xblk, xlu);
 
-        // chunks built (ci) and read back (cc); groups of each slot's chunk,
-        // four bits per slot
-        int ci = 0, cc = 0, xl = 0;
-        uint32_t nhs = 0;
-        int lastc0 = -1, lastc1 = -1;  // last chunk of the units in x image 0 / 1
+        // Two chunk slots: the chunk built last is read back right after the
+        // next one is built, so one chunk is in the MMA while the warp builds
+        // the next.  When a unit starts, every chunk of the unit before the
+        // previous one has been read back, so the MMAs that read the x image
+        // about to be rewritten have completed.
+        static_assert(C::Q == 2, "two chunk slots");
+        int ci = 0, xl = 0;
+        int pnh = 0;       // groups of the pending chunk (0: none)
+        float ps[C::H];    // their scales
         float y[MB];
 #pragma unroll
         for (int m = 0; m < MB; ++m) y[m] = 0.f;
-        auto consume = [&]() {
-            const int q = cc % C::Q;
-            if (lane == 0) tc_wait(smem_u32(&donej[q]), (uint32_t)(cc / C::Q) & 1u, abort);
-            __syncwarp();
+#pragma unroll
+        for (int h = 0; h < C::H; ++h) ps[h] = 0.f;
+        // read back the pending chunk (built as chunk ci - 1, slot (ci - 1) & 1)
+        auto read_back = [&]() {
+            const int q = (ci - 1) & 1;
+            // every lane waits: no divergent branch around the wait
+            tc_wait(smem_u32(&donej[q]), (uint32_t)((ci - 1) >> 1) & 1u, abort);
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            const int nh = (int)((nhs >> (4 * q)) & 0xFu);
 #pragma unroll
             for (int h = 0; h < C::H; ++h) {
-                if (h < nh) {  // warp-uniform
-                    const int b = q * C::H + h;
-                    const float s = sb[b * 32];
-                    const float2 s2 = make_float2(s, s);
+                if (h < pnh) {  // warp-uniform
+                    const uint32_t td = tl + (uint32_t)(C::DCOL + (j * C::P + q * C::H + h) * MB);
+                    const float2 s2 = make_float2(ps[h], ps[h]);
 #pragma unroll
                     for (int hh = 0; hh < MB / 16; ++hh) {
                         float dv[16];
-                        tmem_ld_d<16>(tl + (uint32_t)(C::DCOL + (j * C::P + b) * MB + 16 * hh), dv);
+                        tmem_ld_d<16>(td + 16 * hh, dv);
 #pragma unroll
                         for (int m = 0; m < 16; m += 2) {
                             const float2 r2 = __ffma2_rn(s2, make_float2(dv[m], dv[m + 1]),
@@ -425,7 +446,7 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
                     }
                 }
             }
-            ++cc;
+            pnh = 0;
         };
 
         for (int blk = blockIdx.x / a.cl; blk < args.nblk; blk += bstride) {
@@ -434,8 +455,6 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
             for (int lu = j; lu < nunits; lu += C::SETS, ++xl) {
                 const int u = tc_unit(a, sg0, nsg, ob0, lu);
                 uint8_t *xb = ximg + (size_t)(j * 2 + (xl & 1)) * C::XBYTES;
-                // the MMAs of unit xl - 2 read this x buffer: wait for them
-                while (cc <= ((xl & 1) ? lastc1 : lastc0)) consume();
                 tc_store_x<MB>(a, u, tid, xp, xb);
                 if (xblk < args.nblk) {
                     tc_load_x<MB>(a, tc_unit(a, sg0, nsg, ob0, xlu), tid, xp);
@@ -448,16 +467,16 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
                 const int ngr = tc_groups(a, u);
                 for (int g0 = 0; g0 < ngr; g0 += C::H) {
                     // one chunk: up to H groups' A operands, then one arrival
-                    const int q = ci % C::Q;
+                    const int q = ci & 1;
                     const int nh = min(C::H, ngr - g0);
+                    float sc[C::H];
 #pragma unroll
                     for (int h = 0; h < C::H; ++h) {
+                        sc[h] = 0.f;
                         if (h < nh) {  // warp-uniform
-                            const int b = q * C::H + h;
                             uint32_t av[16];
-                            const float s = tc_build_a(a, u, g0 + h, stage, lane, av);
-                            tmem_st16(tl + (uint32_t)((j * C::P + b) * 16), av);
-                            sb[b * 32] = s;
+                            sc[h] = tc_build_a(a, u, g0 + h, stage, lane, av);
+                            tmem_st16(tl + (uint32_t)((j * C::P + q * C::H + h) * 16), av);
                         }
                     }
                     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
@@ -465,15 +484,12 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
                     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
                     __syncwarp();
                     if (lane == 0) mbar_arrive(smem_u32(&fullj[q]));
-                    nhs = (nhs & ~(0xFu << (4 * q))) | ((uint32_t)nh << (4 * q));
+                    if (pnh) read_back();
                     ++ci;
-                    // a slot is rebuilt only after its chunk was read back
-                    if (ci - cc > C::Q - 1) consume();
+                    pnh = nh;
+#pragma unroll
+                    for (int h = 0; h < C::H; ++h) ps[h] = sc[h];
                 }
-                if (xl & 1)
-                    lastc1 = ci - 1;
-                else
-                    lastc0 = ci - 1;
                 if (active) ring_release(ring);
                 if (iblk < args.nblk) {
                     const int ti = 4 * iblk + r;
@@ -482,7 +498,7 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
                     advance(iblk, ilu);
                 }
             }
-            while (cc < ci) consume();
+            if (pnh) read_back();
             // block end: sets 1.. hand their sums to set 0 (each set's own x
             // image is free: its groups are all read back), which adds them in
             // set order and stores the rows (or, in a cluster, leaves them for
@@ -600,7 +616,6 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
 template <typename C>
 size_t tc_smem_bytes(int depth) {
     return (size_t)C::SETS * 2 * C::XBYTES + (size_t)C::CW * depth * kStageBytes +
-           (size_t)C::CW * C::P * 32 * 4 +
            (size_t)(C::CW * depth + 2 * C::SETS * C::Q + C::SETS) * 8 + 16;
 }
 
