@@ -855,10 +855,46 @@ void item_shape(const Geometry &g, int64_t target, int *ppc, int *tpc) {
     *tpc = kPersistWarps / best_p;
 }
 
-// Item byte target: about 8 items per CTA, at least 64 KB.
-int64_t item_target(int64_t total, int ncta) {
-    const int64_t t = total / ((int64_t)ncta * 8);
+// Item byte target: about `per_cta` items per CTA, at least 64 KB.
+int64_t item_target(int64_t total, int ncta, int per_cta) {
+    const int64_t t = total / ((int64_t)ncta * per_cta);
     return t < 65536 ? 65536 : t;
+}
+
+// A CTA whose range crosses into another matrix restages x there, a few
+// microseconds of its stream; the split counts each change as this many bytes.
+constexpr int64_t kRestageBytes = 192 * 1024;
+
+// Contiguous item ranges of about equal cost (bytes, plus kRestageBytes per
+// matrix change): boundary c goes to the item edge nearest c / ncta of the
+// total, so a CTA is off its share by at most half an item.
+void split_ctas(PersistArgs &args, int count, int ncta, int items) {
+    int64_t total = 0;
+    for (int i = 0; i < count; ++i) {
+        const Prob &a = args.probs[i];
+        total += (int64_t)a.T * tile_bytes(Geometry::of(a.n, a.k, a.n_o)) + (i > 0 ? kRestageBytes : 0);
+    }
+    int64_t acc = 0;
+    int c = 1;
+    args.cta_first[0] = 0;
+    for (int i = 0; i < count && c < ncta; ++i) {
+        const Prob &a = args.probs[i];
+        const int64_t tb = tile_bytes(Geometry::of(a.n, a.k, a.n_o));
+        for (int it = 0; it < a.items && c < ncta; ++it) {
+            const int idx = args.item_start[i] + it;
+            const int64_t cost = (int64_t)min(a.tpc, a.T - it * a.tpc) * tb +
+                                 (it == 0 && i > 0 ? kRestageBytes : 0);
+            // boundaries whose ideal position falls inside this item
+            while (c < ncta && (acc + cost) * ncta >= total * (int64_t)c) {
+                const int64_t before = total * (int64_t)c - acc * ncta;
+                const int64_t after = (acc + cost) * ncta - total * (int64_t)c;
+                args.cta_first[c] = (before < after && idx > args.cta_first[c - 1]) ? idx : idx + 1;
+                ++c;
+            }
+            acc += cost;
+        }
+    }
+    while (c <= ncta) args.cta_first[c++] = items;
 }
 
 // The persistent launch over the `count` problems filled in args.probs.
@@ -872,7 +908,9 @@ spectra_status run_persistent(PersistArgs &args, int count, const DeviceInfo &de
         const Prob &a = args.probs[i];
         total += (int64_t)a.T * tile_bytes(Geometry::of(a.n, a.k, a.n_o));
     }
-    const int64_t target = item_target(total, dev.sm_count);
+    // items of a few per cent of a CTA's share: narrower items would split
+    // tiles into more slices (idle warps on short tiles, a reduction per item)
+    const int64_t target = item_target(total, dev.sm_count, 8);
     total = 0;
     for (int i = 0; i < count; ++i) {
         Prob &a = args.probs[i];
@@ -883,7 +921,6 @@ spectra_status run_persistent(PersistArgs &args, int count, const DeviceInfo &de
         a.items = (int)cdiv(a.T, a.tpc);
         args.item_start[i] = items;
         items += a.items;
-        total += (int64_t)a.T * tile_bytes(g);
         sm.xg = max(sm.xg, 8 * a.S);
         sm.xo = max(sm.xo, 8 * kOB * (a.U - a.S));
     }
@@ -897,21 +934,7 @@ spectra_status run_persistent(PersistArgs &args, int count, const DeviceInfo &de
     int ncta = dev.sm_count;
     if (ncta > kMaxCtas) ncta = kMaxCtas;
     if (ncta > items) ncta = items;
-    // contiguous item ranges of about equal bytes
-    int64_t acc = 0;
-    int c = 1;
-    args.cta_first[0] = 0;
-    for (int i = 0; i < count && c < ncta; ++i) {
-        const Prob &a = args.probs[i];
-        const Geometry g = Geometry::of(a.n, a.k, a.n_o);
-        for (int it = 0; it < a.items && c < ncta; ++it) {
-            const int tiles = min(a.tpc, a.T - it * a.tpc);
-            acc += (int64_t)tiles * tile_bytes(g);
-            while (c < ncta && acc * ncta >= total * (int64_t)c)
-                args.cta_first[c++] = args.item_start[i] + it + 1;
-        }
-    }
-    while (c <= ncta) args.cta_first[c++] = items;
+    split_ctas(args, count, ncta, items);
     cudaError_t e = prepare_kernel(gemv_persistent_kernel<MB>, done, dev);
     if (e != cudaSuccess) return SPECTRA_ERR_CUDA;
     e = launch_kernel(gemv_persistent_kernel<MB>, args, (unsigned)ncta,
@@ -944,7 +967,7 @@ spectra_status run_one(const Prob &a, const DeviceInfo &dev, cudaStream_t s) {
     const Geometry g = Geometry::of(a.n, a.k, a.n_o);
     const int64_t total = (int64_t)g.T * tile_bytes(g);
     int ppc, tpc;
-    item_shape(g, item_target(total, dev.sm_count), &ppc, &tpc);
+    item_shape(g, item_target(total, dev.sm_count, 8), &ppc, &tpc);
     const int64_t items = cdiv(g.T, tpc);
     if (items >= 4LL * dev.sm_count && total >= (int64_t)dev.sm_count * 512 * 1024) {
         static std::mutex mu;
