@@ -85,6 +85,10 @@ def _declare(L):
     L.spectra_ref_dequant.restype = None
     L.spectra_ref_gemm.argtypes = [i32, i32, P, P, P, P, P, i32, P, i32, P, P]
     L.spectra_ref_gemm.restype = None
+    L.spectra_ref_double_to_bf16.argtypes = [f64]
+    L.spectra_ref_double_to_bf16.restype = u16
+    L.spectra_ref_embed.argtypes = [i32, i32, P, P, P, P, P, i32, P, i32, P]
+    L.spectra_ref_embed.restype = ctypes.c_int
 
 
 def _p(a: np.ndarray | None):
@@ -243,6 +247,28 @@ def pack(w_bits: np.ndarray, gain: np.ndarray | None, tau: float) -> Layer:
     idx = split(kap, tau)
     can = quantize(w_bits, idx)
     return Layer(kap, idx, can, pack_layout(can, w_bits, idx))
+
+
+def double_to_bf16(values) -> np.ndarray:
+    v = np.asarray(values, dtype=np.float64).ravel()
+    f = lib().spectra_ref_double_to_bf16
+    return np.array([f(float(a)) for a in v], dtype=np.uint16).reshape(np.shape(values))
+
+
+def embed(can: Canonical, w_bits: np.ndarray, idx: np.ndarray, ids) -> np.ndarray:
+    """Rows ids of the reconstructed table (FP64 [m, k]); w_bits: uint16 [n, k]."""
+    w = _c(w_bits, np.uint16)
+    n, k = w.shape
+    ix = _c(idx, np.int32)
+    tok = _c(np.asarray(ids).ravel(), np.int32)
+    out = np.zeros((tok.size, k), dtype=np.float64)
+    st = lib().spectra_ref_embed(n, k, _p(_c(can.codes, np.uint8)), _p(_c(can.scales, np.uint16)),
+                                 _p(_c(can.zeros, np.uint8)), _p(w), _p(ix) if ix.size else None,
+                                 ix.size, _p(tok) if tok.size else None, tok.size,
+                                 _p(out) if tok.size else None)
+    if st != OK:
+        raise OracleError(st)
+    return out
 
 
 def tolerance(bound: np.ndarray) -> np.ndarray:

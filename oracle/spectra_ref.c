@@ -369,3 +369,79 @@ void spectra_ref_gemm(int32_t n, int32_t k, const uint8_t *codes, const uint16_t
         }
     }
 }
+
+/* ---------------------------------------------------------------- embedding */
+
+/*
+ * double -> bfloat16 (the upper half of an IEEE binary32 word: 8 exponent
+ * bits, bias 127, 7 fraction bits) with ONE round-to-nearest-even step,
+ * subnormals kept, overflow to infinity.  As for binary16 above, an exact
+ * power-of-two scaling makes the kept bits an integer and rint() rounds once.
+ */
+uint16_t spectra_ref_double_to_bf16(double v)
+{
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (isnan(v))
+        return (uint16_t)(sign | 0x7FC0);
+    if (isinf(v))
+        return (uint16_t)(sign | 0x7F80);
+    if (a < ldexp(1.0, -126)) {
+        /* subnormal range: multiples of 2^-133; q == 128 encodes 2^-126 */
+        double q = rint(ldexp(a, 133));
+        return (uint16_t)(sign | (uint16_t)q);
+    }
+    int e2;
+    frexp(a, &e2);            /* a = f * 2^e2, f in [0.5, 1) */
+    int E = e2 - 1;           /* a in [2^E, 2^(E+1)) */
+    if (E > 127)
+        return (uint16_t)(sign | 0x7F80);
+    double q = rint(ldexp(a, 7 - E)); /* in [128, 256] */
+    if (q == 256.0) {
+        q = 128.0;
+        E += 1;
+    }
+    if (E > 127)
+        return (uint16_t)(sign | 0x7F80);
+    return (uint16_t)(sign | (uint16_t)(((E + 127) << 7) | ((int)q - 128)));
+}
+
+/*
+ * Row gather of the reconstructed table (abstract and highlight 5:
+ * SpectraFusedEmbedding keeps vocabulary tables in the 4-bit Group-32 format
+ * and dequantises the rows it needs while the forward pass runs).  The table
+ * E[n][k] (n = vocabulary, k = hidden) is a packed layer like any other; its
+ * reconstruction is
+ *   E_hat[i][j] = W[i][j]                   for j in O (stored bit-exact),
+ *   E_hat[i][j] = (c_ij - z_ig) * S_ig      otherwise (g = j / 32),
+ * and out[r][.] = E_hat[ids[r]][.] in double (every value is exact).  The
+ * codes, scales and zero points are the canonical arrays of the quantiser.
+ * An id outside [0, n) rejects the call before anything is written.
+ */
+int spectra_ref_embed(int32_t n, int32_t k, const uint8_t *codes, const uint16_t *scales,
+                      const uint8_t *zeros, const uint16_t *w, const int32_t *idx, int32_t n_o,
+                      const int32_t *ids, int32_t m, double *out)
+{
+    if (n < 1 || k < 32 || k % 32 != 0 || m < 0 || n_o < 0 || n_o > k)
+        return REF_ERR_INVALID_ARG;
+    if (m == 0)
+        return REF_OK;
+    if (!codes || !scales || !zeros || !ids || !out || (n_o > 0 && (!w || !idx)))
+        return REF_ERR_INVALID_ARG;
+    for (int32_t r = 0; r < m; ++r)
+        if (ids[r] < 0 || ids[r] >= n)
+            return REF_ERR_INVALID_ARG;
+    const int64_t ngroups = k / 32;
+    for (int64_t r = 0; r < m; ++r) {
+        const int64_t row = ids[r];
+        double *dst = out + r * k;
+        for (int64_t col = 0; col < k; ++col) {
+            const int64_t grp = row * ngroups + col / 32;
+            double S = spectra_ref_fp16_to_double(scales[grp]);
+            dst[col] = ((double)codes[row * k + col] - (double)zeros[grp]) * S;
+        }
+        for (int64_t t = 0; t < n_o; ++t)
+            dst[idx[t]] = spectra_ref_bf16_to_double(w[row * k + idx[t]]);
+    }
+    return REF_OK;
+}

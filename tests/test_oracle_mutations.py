@@ -39,6 +39,15 @@ MUTATIONS = {
                           "double wd = ((double)codes[i * k + kk] + (double)zeros"),
     "gemm_outlier_x_index": ("double xv = spectra_ref_bf16_to_double(xr[idx[t]]);",
                              "double xv = spectra_ref_bf16_to_double(xr[t]);"),
+    "bf16_truncates": ("double q = rint(ldexp(a, 7 - E));", "double q = floor(ldexp(a, 7 - E));"),
+    "bf16_subnormal_step": ("double q = rint(ldexp(a, 133));", "double q = rint(ldexp(a, 134));"),
+    "embed_row_from_position": ("const int64_t row = ids[r];", "const int64_t row = r;"),
+    "embed_group_of_column": ("const int64_t grp = row * ngroups + col / 32;",
+                              "const int64_t grp = row * ngroups + col % ngroups;"),
+    "embed_outlier_value_slot": ("dst[idx[t]] = spectra_ref_bf16_to_double(w[row * k + idx[t]]);",
+                                 "dst[idx[t]] = spectra_ref_bf16_to_double(w[row * k + t]);"),
+    "embed_zero_point_sign": ("dst[col] = ((double)codes[row * k + col] - (double)zeros[grp]) * S;",
+                              "dst[col] = ((double)codes[row * k + col] + (double)zeros[grp]) * S;"),
 }
 
 PIN_FUNCS = [
@@ -55,6 +64,10 @@ PIN_FUNCS = [
     pins.test_gemm_brute_force_8x32,
     pins.test_gemm_all_outliers_is_dense_product,
     pins.test_gemm_unit_vectors_extract_columns,
+    pins.test_bf16_golden_cases,
+    pins.test_embed_all_outliers_is_row_indexing,
+    pins.test_embed_exact_grid_rows,
+    pins.test_embed_rows_agree_with_gemm,
 ]
 _PARAMS = {
     "test_quantizer_exact_grid": [{"S": 2.0 ** -7, "z": 5}],

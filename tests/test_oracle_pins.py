@@ -454,3 +454,117 @@ def test_pack_pipeline_counts_bytes(ref):
     bulk = p.codes.nbytes + p.scales.nbytes + p.zeros.nbytes
     assert bulk * 8 == 512 * 512 * 4.625
     assert p.outliers.nbytes == 512 * (-(-n_o // 8) * 8) * 2
+
+
+# ----------------------------------------------------------------- embedding
+
+def test_bf16_golden_cases(ref, golden_dir):
+    for line in open(os.path.join(golden_dir, "bf16_rounding_cases.txt")):
+        line = line.split("#")[0].strip() if not line.lstrip().startswith("#") else ""
+        if not line:
+            continue
+        expr, hexbits = line.split()[:2]
+        v = float(eval(expr, {"__builtins__": {}}))
+        assert int(ref.double_to_bf16([v])[0]) == int(hexbits, 16), expr
+
+
+def test_bf16_midpoints_match_torch(ref):
+    # every midpoint between adjacent positive finite BF16 values is exact in
+    # float32, so torch's float32 -> bfloat16 (round to nearest even) decides
+    # the ties; one double ulp either side must give the lower / upper value
+    pos = np.arange(0, 0x7F7F, dtype=np.uint16)
+    lo = _bf16_values(pos)
+    hi = _bf16_values((pos + 1).astype(np.uint16))
+    mid = (lo + hi) / 2.0
+    assert np.array_equal(ref.double_to_bf16(mid), _bf16_bits(mid))
+    assert np.array_equal(ref.double_to_bf16(np.nextafter(mid, -np.inf)), pos)
+    assert np.array_equal(ref.double_to_bf16(np.nextafter(mid, np.inf)), pos + 1)
+    neg = ref.double_to_bf16(-mid)
+    assert np.array_equal(neg, _bf16_bits(-mid))
+
+
+def test_bf16_random_floats_match_torch(ref):
+    rng = np.random.default_rng(8)
+    e = rng.uniform(-140, 127, 40000)
+    vals = (np.exp2(e) * rng.choice([-1.0, 1.0], e.size)).astype(np.float32).astype(np.float64)
+    assert np.array_equal(ref.double_to_bf16(vals), _bf16_bits(vals))
+
+
+def _table(ref, n, k, n_t, seed, tau):
+    spec = wl.MatrixSpec("lm_head", n, k, n_t)
+    wb = wl.bits(wl.weight(spec, seed=seed))
+    g = wl.gain(spec, seed=seed).numpy()
+    return wb, ref.pack(wb, g, tau)
+
+
+def test_embed_all_outliers_is_row_indexing(ref):
+    # every column kept in BF16: the gather is plain row indexing of W
+    wb, layer = _table(ref, 70, 96, 3, 21, -np.inf)
+    assert layer.idx.size == 96
+    ids = np.array([0, 69, 5, 5, 33, 32, 31])
+    out = ref.embed(layer.can, wb, layer.idx, ids)
+    expect = _bf16_values(wb)[ids]
+    assert np.array_equal(out, expect)
+    assert np.array_equal(np.signbit(out), np.signbit(expect))
+
+
+def test_embed_exact_grid_rows(ref):
+    # a table whose groups are exact quantiser grids comes back exactly
+    S = 2.0 ** -7
+    vals = np.stack([_grid_row(S, 6, s) for s in range(16)])
+    vals = np.concatenate([vals, vals[:, ::-1]], axis=1)  # [16, 64]
+    w = _bf16_bits(vals)
+    can = ref.quantize(w, np.array([], dtype=np.int32))
+    ids = np.array([15, 0, 7, 7, 3])
+    out = ref.embed(can, w, np.array([], dtype=np.int32), ids)
+    assert np.array_equal(out, vals[ids])
+
+
+def test_embed_rows_agree_with_gemm(ref):
+    # row i of the reconstruction dotted with x is y_i of the matvec oracle:
+    # a transposed index, a wrong group or a misplaced outlier breaks it
+    for tau in (3.0, 6.0):
+        wb, layer = _table(ref, 80, 256, 6, 22, tau)
+        assert 0 < layer.idx.size < 256
+        xb = wl.bits(wl.activations(256, 1, seed=23))
+        y, bound = ref.gemm(layer.can, wb, layer.idx, xb)
+        ids = np.arange(80)[::-1]
+        rows = ref.embed(layer.can, wb, layer.idx, ids)
+        dots = rows @ _bf16_values(xb)[0]
+        assert np.all(np.abs(dots - y[0, ids]) <= 1e-13 * bound[0, ids])
+
+
+def test_embed_brute_force_8x32(ref):
+    wb, layer = _table(ref, 8, 64, 2, 24, 3.0)
+    assert 0 < layer.idx.size < 64
+    codes, sc, ze = layer.can.codes, layer.can.scales, layer.can.zeros
+    S = sc.view(np.float16).astype(np.float64)
+    wv = _bf16_values(wb)
+    ids = [3, 0, 7, 3]
+    out = ref.embed(layer.can, wb, layer.idx, np.array(ids))
+    for r, i in enumerate(ids):
+        for j in range(64):
+            if j in layer.idx:
+                expect = float(wv[i, j])
+            else:
+                expect = (float(codes[i, j]) - float(ze[i, j // 32])) * float(S[i, j // 32])
+            assert out[r, j] == expect
+
+
+def test_embed_keeps_negative_zero_of_outlier_columns(ref):
+    vals = np.zeros((4, 32), dtype=np.float32)
+    vals[:, 5] = [-0.0, 1.5, -2.0, 0.0]
+    w = _bf16_bits(vals)
+    idx = np.array([5], dtype=np.int32)
+    can = ref.quantize(w, idx)
+    out = ref.embed(can, w, idx, np.array([0, 3]))
+    assert np.signbit(out[0, 5]) and not np.signbit(out[1, 5])
+    assert np.all(out[:, np.arange(32) != 5] == 0.0)
+
+
+def test_embed_rejects_ids_outside_table(ref):
+    wb, layer = _table(ref, 10, 32, 0, 25, 6.0)
+    for bad in ([10], [-1], [0, 3, 10]):
+        with pytest.raises(ref.OracleError):
+            ref.embed(layer.can, wb, layer.idx, np.array(bad))
+    assert ref.embed(layer.can, wb, layer.idx, np.array([], dtype=np.int32)).shape == (0, 32)
