@@ -61,6 +61,13 @@ def algorithmic_bytes(n: int, k: int, n_o: int, m: int = 1, y_bytes: int = 4) ->
             + 2 * m * k + y_bytes * m * n)
 
 
+def embed_bytes(k: int, n_o: int, m: int, out_bytes: int = 2) -> int:
+    """Bytes an embedding gather of m rows must move: each row's codes, scales
+    and zero points (4.625 bits per column), its BF16 outlier values, the
+    outlier index list, the ids and the dequantised rows written out."""
+    return m * (k // 2 + k // 16 + k // 64 + 2 * n_o + 4 + out_bytes * k) + 4 * n_o
+
+
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -362,6 +369,22 @@ def extras(device, stream, peak_gbs, tau):
                          "gbs": round(b / us * 1e-3, 1), "frac": round(b / us * 1e-3 / peak_gbs, 3),
                          "tflops": round(2 * m * spec.n * spec.k / us * 1e-6, 2)})
         out["lm_head_batch_131072x3072"] = rows
+        # the same packed buffers as an embedding table (tied LM head): rows
+        # gathered and dequantised to BF16 for M token ids
+        rows = []
+        for m in (1, 64, 4096):
+            ids = torch.from_numpy(np.random.default_rng(m).integers(0, spec.n, m).astype(np.int32)).to(device)
+            o = torch.empty((m, spec.k), dtype=torch.bfloat16, device=device)
+            us, p10, p90 = time_single(
+                lambda: sp.spectra_embed(lay, ids, o, view=v, stream=stream), stream, 30, flush)
+            us_r = time_rotating([lambda: sp.spectra_embed(lay, ids, o, view=v, stream=stream)],
+                                 stream, 200)
+            b = embed_bytes(spec.k, lay.n_outliers, m)
+            rows.append({"m": m, "n_outliers": lay.n_outliers, "us_single_flushed": round(us, 2),
+                         "us_back_to_back": round(us_r, 2), "bytes": b,
+                         "gbs_single_flushed": round(b / us * 1e-3, 1),
+                         "frac_single_flushed": round(b / us * 1e-3 / peak_gbs, 3)})
+        out["embed_rows_131072x3072_bf16"] = rows
         del w, lay
     return out
 

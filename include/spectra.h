@@ -258,11 +258,40 @@ SPECTRA_API spectra_status spectra_gemv_batched(const spectra_layer *layers,
                                                 void *stream);
 
 /*
- * Health of the matvec kernels on the current device.  Their waits for the
- * asynchronous weight copies are bounded: a wait that gives up raises a
- * per-device flag instead of hanging, and the outputs of that launch are
- * invalid.  Returns SPECTRA_ERR_INTERNAL if the flag was raised since the
- * last call (and clears it), SPECTRA_OK otherwise.  Synchronous on `stream`.
+ * Embedding-row gather over a packed table (abstract: "Dynamic vocabulary
+ * embedding dequantization (SpectraFusedEmbedding)"; highlight 5: vocabulary
+ * tables stored in the 4-bit Group-32 format, rows gathered and dequantised
+ * during the forward pass).
+ *   table  HOST struct viewing a packed layer of the table E[n][k] (n =
+ *          vocabulary rows, k = hidden size), packed by spectra_pack_plan +
+ *          spectra_pack like any layer; a tied LM head's buffers serve as is
+ *   ids    device int32 [m] row ids
+ *   m      number of rows, >= 0; m == 0 returns SPECTRA_OK without touching
+ *          CUDA
+ *   out    device [m][k] of out_dtype, 16-byte aligned
+ * out[r][j] = (c - z) * s of row ids[r] for bulk columns j (exact in FP32;
+ * BF16 output rounds it once, to nearest even) and the stored BF16 value
+ * W[ids[r]][j], bit for bit, for outlier columns j.  An id outside [0, n)
+ * yields a zero row and raises the device flag that spectra_device_status
+ * reports as SPECTRA_ERR_INVALID_ARG; nothing is read or written out of
+ * bounds.  Asynchronous, allocates nothing, graph-capturable; launched with
+ * programmatic dependent launch (it reads ids only after the previous kernel
+ * on the stream has completed).
+ * Errors: INVALID_ARG, SHAPE (m < 0, or a bad table shape), ALIGN,
+ * UNSUPPORTED, CUDA.
+ */
+SPECTRA_API spectra_status spectra_embed(const spectra_layer *table, const int32_t *ids, int32_t m,
+                                         void *out, spectra_dtype out_dtype, void *stream);
+
+/*
+ * Health of the kernels on the current device.  The matvec kernels' waits
+ * for the asynchronous weight copies are bounded: a wait that gives up
+ * raises a per-device flag instead of hanging, and the outputs of that
+ * launch are invalid.  The embedding gather raises its own flag for an id
+ * outside the table (or an outlier index outside [0, k)).  Returns
+ * SPECTRA_ERR_INTERNAL if a wait gave up, else SPECTRA_ERR_INVALID_ARG if the
+ * gather saw a bad id, since the last call (and clears both flags),
+ * SPECTRA_OK otherwise.  Synchronous on `stream`.
  */
 SPECTRA_API spectra_status spectra_device_status(void *stream);
 

@@ -22,7 +22,8 @@ from ._lib import Layer, Sizes
 
 __all__ = ["SpectraError", "PackedLayer", "spectra_status_string", "spectra_version",
            "spectra_packed_sizes", "spectra_pack_plan", "spectra_pack", "spectra_unpack",
-           "spectra_gemv", "spectra_gemm_small", "spectra_gemv_batched", "spectra_device_status",
+           "spectra_gemv", "spectra_gemm_small", "spectra_gemv_batched", "spectra_embed",
+           "spectra_device_status",
            "pack_layer", "library"]
 
 class _Lazy:
@@ -194,6 +195,20 @@ def spectra_gemm_small(layer: PackedLayer, x: torch.Tensor, y: torch.Tensor | No
     _check(_L.spectra_gemm_small(ctypes.byref(v), _ptr(x), m, _ptr(y), _DT[y.dtype],
                                  _stream(stream)), "spectra_gemm_small")
     return y
+
+
+def spectra_embed(table: PackedLayer, ids: torch.Tensor, out: torch.Tensor | None = None, *,
+                  out_dtype=torch.bfloat16, view: Layer | None = None,
+                  stream=None) -> torch.Tensor:
+    """Rows ids (int32 [m]) of a packed table, dequantised: out [m, k]."""
+    m = int(ids.numel())
+    if out is None:
+        out = torch.empty((m, table.k), dtype=out_dtype, device=ids.device)
+    v = table.view() if view is None else view
+    _check(_L.spectra_embed(ctypes.byref(v), _ptr(ids) if m else None, m,
+                            _ptr(out) if m else None, _DT[out.dtype], _stream(stream)),
+           "spectra_embed")
+    return out
 
 
 class BatchViews:

@@ -53,6 +53,7 @@ SIGNATURES = {
     "spectra_gemm_small": (ctypes.c_int, [LP, P, i32, P, ctypes.c_int, P]),
     "spectra_gemv_batched": (ctypes.c_int, [LP, P, P, i32, ctypes.c_int, P]),
     "spectra_device_status": (ctypes.c_int, [P]),
+    "spectra_embed": (ctypes.c_int, [LP, P, i32, P, ctypes.c_int, P]),
     "spectra_pack_plan_noalloc": (ctypes.c_int, [P, P, i32, i32, f64, P, P, ctypes.POINTER(i32), P]),
 }
 

@@ -90,7 +90,7 @@ const char *spectra_status_string(spectra_status s) {
     return "unknown status";
 }
 
-int32_t spectra_version(void) { return 100; }
+int32_t spectra_version(void) { return 101; }
 
 spectra_status spectra_packed_sizes(int32_t n, int32_t k, int32_t n_outliers, spectra_sizes *out) {
     if (!out) return SPECTRA_ERR_INVALID_ARG;
@@ -250,6 +250,21 @@ spectra_status spectra_gemv_batched(const spectra_layer *layers, const uint16_t 
     return launch_gemv_batched(layers, x, y, count, (int)y_dtype, (cudaStream_t)stream, dev);
 }
 
+spectra_status spectra_embed(const spectra_layer *table, const int32_t *ids, int32_t m, void *out,
+                             spectra_dtype out_dtype, void *stream) {
+    spectra_status st = check_layer(table);
+    if (st != SPECTRA_OK) return st;
+    if (out_dtype != SPECTRA_F32 && out_dtype != SPECTRA_BF16) return SPECTRA_ERR_INVALID_ARG;
+    if (m < 0) return SPECTRA_ERR_SHAPE;
+    if (m == 0) return SPECTRA_OK;
+    if (!ids || !out) return SPECTRA_ERR_INVALID_ARG;
+    if (!aligned4(ids) || !aligned16(out)) return SPECTRA_ERR_ALIGN;
+    DeviceInfo dev;
+    st = current_device(&dev);
+    if (st != SPECTRA_OK) return st;
+    return launch_embed(*table, ids, m, out, (int)out_dtype, (cudaStream_t)stream, dev);
+}
+
 spectra_status spectra_device_status(void *stream) {
     DeviceInfo dev;
     spectra_status st = current_device(&dev);
@@ -257,7 +272,11 @@ spectra_status spectra_device_status(void *stream) {
     bool raised = false;
     st = device_error(&raised, (cudaStream_t)stream);
     if (st != SPECTRA_OK) return st;
-    return raised ? SPECTRA_ERR_INTERNAL : SPECTRA_OK;
+    unsigned int embed_bits = 0;
+    st = embed_device_error(&embed_bits, (cudaStream_t)stream);
+    if (st != SPECTRA_OK) return st;
+    if (raised) return SPECTRA_ERR_INTERNAL;
+    return embed_bits ? SPECTRA_ERR_INVALID_ARG : SPECTRA_OK;
 }
 
 }  // extern "C"

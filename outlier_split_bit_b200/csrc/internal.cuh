@@ -81,4 +81,12 @@ spectra_status launch_tc(const spectra_layer &l, const uint16_t *x, int m, void 
 // Reads (and clears) the tensor-core kernel's bounded-wait error flag.
 spectra_status tc_device_error(bool *raised, cudaStream_t s);
 
+// ---- embedding-row gather (embed.cu) ----
+// Rows ids[0..m) of a packed table, dequantised (1 <= m).
+spectra_status launch_embed(const spectra_layer &l, const int32_t *ids, int m, void *out,
+                            int out_type, cudaStream_t s, const DeviceInfo &dev);
+// Reads (and clears) the gather's flag: bit 0 a token id outside the table,
+// bit 1 an outlier index outside [0, k).
+spectra_status embed_device_error(unsigned int *bits, cudaStream_t s);
+
 }  // namespace spectra

@@ -139,3 +139,17 @@ def test_product_path_does_not_reference_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
                 assert "spectra_ref" not in text, f
+
+
+def test_embed_argument_checks(L):
+    lay = ctypes.byref(_layer())
+    assert L.spectra_embed(None, FAKE, 1, FAKE, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.spectra_embed(ctypes.byref(_layer(k=100)), FAKE, 1, FAKE, 0, None) == _lib.ERR_SHAPE
+    assert L.spectra_embed(lay, FAKE, -1, FAKE, 0, None) == _lib.ERR_SHAPE
+    assert L.spectra_embed(lay, FAKE, 1, FAKE, 5, None) == _lib.ERR_INVALID_ARG
+    assert L.spectra_embed(lay, None, 1, FAKE, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.spectra_embed(lay, FAKE, 1, None, 1, None) == _lib.ERR_INVALID_ARG
+    assert L.spectra_embed(lay, FAKE + 2, 1, FAKE, 0, None) == _lib.ERR_ALIGN
+    assert L.spectra_embed(lay, FAKE, 1, FAKE + 4, 1, None) == _lib.ERR_ALIGN
+    # no rows: nothing to do, and CUDA is never touched (this machine may have no GPU)
+    assert L.spectra_embed(lay, None, 0, None, 1, None) == _lib.OK

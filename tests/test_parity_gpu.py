@@ -16,7 +16,8 @@ import oracle
 import outlier_split_bit_b200 as sp
 from outlier_split_bit_b200 import workload as wl
 
-from gpu_helpers import (DEV, check_gemv, draw, np_gain, oracle_rows, tile_slices, u8, u16, u32)
+from gpu_helpers import (DEV, check_gemv, draw, np_gain, oracle_rows, oracle_split, tile_slices,
+                         u8, u16, u32)
 
 pytestmark = pytest.mark.gpu
 
@@ -168,21 +169,20 @@ def test_lm_head_full_size_sampled(frac):
     wb = wl.bits(w)
     idx_np = idx.cpu().numpy()
     kap = kappa.cpu().numpy()
-    assert np.array_equal(idx_np, np.flatnonzero(kap > 6.0))
-    rng = np.random.default_rng(0)
-    cols = np.unique(np.concatenate([rng.choice(spec.k, 48, replace=False), idx_np[:16]]))
-    gn = np_gain(g)
-    kref = oracle.kurtosis(np.ascontiguousarray(wb[:, cols]), None if gn is None else gn[cols])
-    assert np.array_equal(kap[cols].view(np.uint64), kref.view(np.uint64))
+    # the oracle's own split of the whole matrix: kurtosis bit-exact on every
+    # column, and the oracle's indices (never the GPU's) feed its packing
+    kref, ref_idx = oracle_split(wb, np_gain(g), 6.0, key=("lm_head", frac))
+    assert np.array_equal(kap.view(np.uint64), kref.view(np.uint64))
+    assert np.array_equal(idx_np, ref_idx)
     # heavy columns are found: at 131072 rows every Student-t(3) column passes
-    assert idx_np.size >= spec.n_t
+    assert ref_idx.size >= spec.n_t
     T = spec.n // 32
     tiles = [0, 1, T // 2, T - 1]
-    rows, can, packed = oracle_rows(wb, idx_np, tiles)
+    rows, can, packed = oracle_rows(wb, ref_idx, tiles)
     got = tile_slices(lay, tiles)
     for key in ("codes", "scales", "zeros", "outliers"):
         assert np.array_equal(got[key], packed[key]), key
-    y_ref, bound = oracle.gemm(can, np.ascontiguousarray(wb[rows]), idx_np, wl.bits(x))
+    y_ref, bound = oracle.gemm(can, np.ascontiguousarray(wb[rows]), ref_idx, wl.bits(x))
     check_gemv(y[rows], y_ref[0], bound[0])
 
 
@@ -361,11 +361,12 @@ def test_decoder_layer_4b_tensor_cores(spec, m):
     torch.cuda.synchronize()
     sp.spectra_device_status()
     wb = wl.bits(w)
-    idx_np = lay.outlier_idx[: lay.n_outliers].cpu().numpy() if lay.n_outliers else np.zeros(0, np.int32)
+    _, ref_idx = oracle_split(wb, np_gain(g), 6.0)
+    assert np.array_equal(lay.outlier_idx[: lay.n_outliers].cpu().numpy(), ref_idx)
     T = -(-spec.n // 32)
     tiles = sorted({0, 1, T // 2, T - 1})
-    rows, can, packed = oracle_rows(wb, idx_np, tiles)
-    y_ref, bound = oracle.gemm(can, np.ascontiguousarray(wb[rows]), idx_np, wl.bits(x))
+    rows, can, packed = oracle_rows(wb, ref_idx, tiles)
+    y_ref, bound = oracle.gemm(can, np.ascontiguousarray(wb[rows]), ref_idx, wl.bits(x))
     check_gemv(y[:, rows], y_ref, bound)
 
 
@@ -402,11 +403,12 @@ def test_tensor_cores_persistent_blocks(m, tau):
     torch.cuda.synchronize()
     sp.spectra_device_status()
     wb = wl.bits(w)
-    idx_np = lay.outlier_idx[: lay.n_outliers].cpu().numpy() if lay.n_outliers else np.zeros(0, np.int32)
+    _, ref_idx = oracle_split(wb, np_gain(g), tau)
+    assert np.array_equal(lay.outlier_idx[: lay.n_outliers].cpu().numpy(), ref_idx)
     T = -(-spec.n // 32)
     tiles = sorted({0, 1, 2, 3, 4, 300, 301, T - 2, T - 1})
-    rows, can, packed = oracle_rows(wb, idx_np, tiles)
-    y_ref, bound = oracle.gemm(can, np.ascontiguousarray(wb[rows]), idx_np, wl.bits(x))
+    rows, can, packed = oracle_rows(wb, ref_idx, tiles)
+    y_ref, bound = oracle.gemm(can, np.ascontiguousarray(wb[rows]), ref_idx, wl.bits(x))
     check_gemv(y[:, rows], y_ref, bound)
 
 
