@@ -89,6 +89,16 @@ def _declare(L):
     L.spectra_ref_double_to_bf16.restype = u16
     L.spectra_ref_embed.argtypes = [i32, i32, P, P, P, P, P, i32, P, i32, P]
     L.spectra_ref_embed.restype = ctypes.c_int
+    L.spectra_ref_bulk_columns.argtypes = [i32, P, i32, P]
+    L.spectra_ref_bulk_columns.restype = i32
+    L.spectra_ref_gather_bulk.argtypes = [P, i32, i32, P, i32, P]
+    L.spectra_ref_gather_bulk.restype = None
+    L.spectra_ref_pack_outliers.argtypes = [i32, i32, P, P, i32, P]
+    L.spectra_ref_pack_outliers.restype = None
+    L.spectra_ref_gemm_compact.argtypes = [i32, i32, i32, P, P, P, P, P, P, i32, P, i32, P, P]
+    L.spectra_ref_gemm_compact.restype = None
+    L.spectra_ref_embed_compact.argtypes = [i32, i32, i32, P, P, P, P, P, P, i32, P, i32, P]
+    L.spectra_ref_embed_compact.restype = ctypes.c_int
 
 
 def _p(a: np.ndarray | None):
@@ -266,6 +276,98 @@ def embed(can: Canonical, w_bits: np.ndarray, idx: np.ndarray, ids) -> np.ndarra
                                  _p(_c(can.zeros, np.uint8)), _p(w), _p(ix) if ix.size else None,
                                  ix.size, _p(tok) if tok.size else None, tok.size,
                                  _p(out) if tok.size else None)
+    if st != OK:
+        raise OracleError(st)
+    return out
+
+
+# ------------------------------------------------------------------ bulk compaction
+
+def bulk_columns(k: int, idx: np.ndarray):
+    """(k_bulk, bulk_idx int32 [k_bulk]) of the compacted bulk."""
+    ix = _c(idx, np.int32)
+    out = np.full(max(32, k + 31), -7, dtype=np.int32)
+    kb = lib().spectra_ref_bulk_columns(k, _p(ix) if ix.size else None, ix.size, _p(out))
+    if kb < 0:
+        raise OracleError(ERR_INVALID_ARG)
+    return kb, out[:kb].copy()
+
+
+def gather_bulk(w_bits: np.ndarray, bulk_idx: np.ndarray) -> np.ndarray:
+    w = _c(w_bits, np.uint16)
+    n, k = w.shape
+    bi = _c(bulk_idx, np.int32)
+    out = np.empty((n, bi.size), dtype=np.uint16)
+    lib().spectra_ref_gather_bulk(_p(w), n, k, _p(bi), bi.size, _p(out))
+    return out
+
+
+def pack_outliers(w_bits: np.ndarray, idx: np.ndarray) -> np.ndarray:
+    w = _c(w_bits, np.uint16)
+    n, k = w.shape
+    ix = _c(idx, np.int32)
+    sz = layout_sizes(n, 32, ix.size)["outliers"]
+    out = np.zeros(max(1, sz), dtype=np.uint16)
+    lib().spectra_ref_pack_outliers(n, k, _p(w), _p(ix) if ix.size else None, ix.size, _p(out))
+    return out[:sz]
+
+
+@dataclass
+class CompactLayer:
+    """Everything the oracle derives from one matrix with a compacted bulk."""
+    kappa: np.ndarray
+    idx: np.ndarray
+    k_bulk: int
+    bulk_idx: np.ndarray  # int32 [k_bulk], -1 = padding
+    can: Canonical        # bulk [n, k_bulk]
+    packed: Packed        # bulk layout over k_bulk columns + outlier block
+
+
+def pack_compact(w_bits: np.ndarray, gain: np.ndarray | None, tau: float) -> CompactLayer:
+    """Saliency split, compaction of the bulk, group quantiser of the compacted
+    bulk, packed layout: in that order."""
+    w = _c(w_bits, np.uint16)
+    kap = kurtosis(w, gain)
+    idx = split(kap, tau)
+    k_bulk, bidx = bulk_columns(w.shape[1], idx)
+    wb = gather_bulk(w, bidx)
+    can = quantize(wb, np.zeros(0, np.int32))
+    bulk = pack_layout(can, wb, np.zeros(0, np.int32))
+    packed = Packed(bulk.codes, bulk.scales, bulk.zeros, pack_outliers(w, idx), idx.copy(),
+                    w.shape[0], w.shape[1])
+    return CompactLayer(kap, idx, k_bulk, bidx, can, packed)
+
+
+def gemm_compact(lay: CompactLayer, w_bits: np.ndarray, x_bits: np.ndarray):
+    """(y [m, n], bound [m, n]) of a compacted layer in FP64."""
+    w = _c(w_bits, np.uint16)
+    n, k = w.shape
+    x = _c(x_bits, np.uint16).reshape(-1, k)
+    m = x.shape[0]
+    ix = _c(lay.idx, np.int32)
+    y = np.empty((m, n), dtype=np.float64)
+    b = np.empty((m, n), dtype=np.float64)
+    lib().spectra_ref_gemm_compact(n, k, lay.k_bulk, _p(_c(lay.can.codes, np.uint8)),
+                                   _p(_c(lay.can.scales, np.uint16)), _p(_c(lay.can.zeros, np.uint8)),
+                                   _p(_c(lay.bulk_idx, np.int32)), _p(w),
+                                   _p(ix) if ix.size else None, ix.size, _p(x), m, _p(y), _p(b))
+    return y, b
+
+
+def embed_compact(lay: CompactLayer, w_bits: np.ndarray, ids) -> np.ndarray:
+    """Rows ids of the reconstructed compacted table (FP64 [m, k])."""
+    w = _c(w_bits, np.uint16)
+    n, k = w.shape
+    ix = _c(lay.idx, np.int32)
+    tok = _c(np.asarray(ids).ravel(), np.int32)
+    out = np.full((tok.size, k), np.nan, dtype=np.float64)
+    st = lib().spectra_ref_embed_compact(n, k, lay.k_bulk, _p(_c(lay.can.codes, np.uint8)),
+                                         _p(_c(lay.can.scales, np.uint16)),
+                                         _p(_c(lay.can.zeros, np.uint8)),
+                                         _p(_c(lay.bulk_idx, np.int32)), _p(w),
+                                         _p(ix) if ix.size else None, ix.size,
+                                         _p(tok) if tok.size else None, tok.size,
+                                         _p(out) if tok.size else None)
     if st != OK:
         raise OracleError(st)
     return out

@@ -445,3 +445,132 @@ int spectra_ref_embed(int32_t n, int32_t k, const uint8_t *codes, const uint16_t
     }
     return REF_OK;
 }
+
+/* ---------------------------------------------------------------- bulk compaction */
+
+/*
+ * Compacted bulk (abstract: the heavy-tailed coordinates are decoupled into
+ * bit-exact storage and the residual bulk is quantised; this variant removes
+ * the outlier columns from the bulk instead of masking them to +0 in place).
+ * The bulk then holds the k - n_o non-outlier columns in ascending order,
+ * padded with all-zero columns to a multiple of 32 and to at least one group:
+ *   k_bulk = max(32, 32 * ceil((k - n_o) / 32)),
+ *   bulk_idx[p] = the p-th non-outlier column for p < k - n_o, -1 after.
+ * Returns k_bulk, or -1 when idx is not strictly ascending within [0, k).
+ * bulk_idx must hold max(32, k + 31) entries.
+ */
+int32_t spectra_ref_bulk_columns(int32_t k, const int32_t *idx, int32_t n_o, int32_t *bulk_idx)
+{
+    if (k < 1 || n_o < 0 || n_o > k || (n_o > 0 && !idx) || !bulk_idx)
+        return -1;
+    for (int32_t t = 0; t < n_o; ++t)
+        if (idx[t] < 0 || idx[t] >= k || (t > 0 && idx[t - 1] >= idx[t]))
+            return -1;
+    const int32_t nb = k - n_o;
+    const int32_t k_bulk = nb <= 32 ? 32 : (int32_t)(cdiv(nb, 32) * 32);
+    int32_t p = 0, t = 0;
+    for (int32_t j = 0; j < k; ++j) {
+        if (t < n_o && idx[t] == j) {
+            ++t;
+            continue;
+        }
+        bulk_idx[p++] = j;
+    }
+    for (; p < k_bulk; ++p)
+        bulk_idx[p] = -1;
+    return k_bulk;
+}
+
+/* W_b[i][p] = W[i][bulk_idx[p]] as BF16 bits, +0 at padding positions. */
+void spectra_ref_gather_bulk(const uint16_t *w, int32_t n, int32_t k, const int32_t *bulk_idx,
+                             int32_t k_bulk, uint16_t *w_b)
+{
+    for (int64_t i = 0; i < n; ++i)
+        for (int64_t p = 0; p < k_bulk; ++p)
+            w_b[i * k_bulk + p] = bulk_idx[p] < 0 ? 0 : w[i * k + bulk_idx[p]];
+}
+
+/* The outlier block alone, in the RT32 order of spectra_ref_pack_layout. */
+void spectra_ref_pack_outliers(int32_t n, int32_t k, const uint16_t *w, const int32_t *idx,
+                               int32_t n_o, uint16_t *poutl)
+{
+    const int64_t O8 = cdiv(n_o, 8), np = cdiv(n, 32) * 32;
+    if (n_o == 0)
+        return;
+    memset(poutl, 0, (size_t)(np * O8 * 8) * 2);
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t t = i / 32, r = i % 32;
+        for (int64_t slot = 0; slot < n_o; ++slot)
+            poutl[((t * O8 + slot / 8) * 32 + r) * 8 + slot % 8] = w[i * k + idx[slot]];
+    }
+}
+
+/*
+ * Matvec over a compacted layer: codes/scales/zeros are the canonical arrays
+ * of the bulk [n][k_bulk], w the original BF16 matrix [n][k], x [m][k]:
+ *   y[m][i] = sum_p w_hat_b[i][p] * x[m][bulk_idx[p]]   (p ascending, padding skipped)
+ *           + sum_t W[i][idx[t]] * x[m][idx[t]]         (t ascending)
+ * in double; bound is the same sum over absolute values (may be NULL).
+ */
+void spectra_ref_gemm_compact(int32_t n, int32_t k, int32_t k_bulk, const uint8_t *codes,
+                              const uint16_t *scales, const uint8_t *zeros,
+                              const int32_t *bulk_idx, const uint16_t *w, const int32_t *idx,
+                              int32_t n_o, const uint16_t *x, int32_t m, double *y, double *bound)
+{
+    const int64_t Gb = k_bulk / 32;
+    for (int64_t mm = 0; mm < m; ++mm) {
+        const uint16_t *xr = x + mm * k;
+        for (int64_t i = 0; i < n; ++i) {
+            double acc = 0.0, b = 0.0;
+            for (int64_t p = 0; p < k_bulk; ++p) {
+                if (bulk_idx[p] < 0)
+                    continue;
+                double S = spectra_ref_fp16_to_double(scales[i * Gb + p / 32]);
+                double wb = ((double)codes[i * k_bulk + p] - (double)zeros[i * Gb + p / 32]) * S;
+                double xb = spectra_ref_bf16_to_double(xr[bulk_idx[p]]);
+                acc = acc + wb * xb;
+                b = b + fabs(wb) * fabs(xb);
+            }
+            for (int64_t t = 0; t < n_o; ++t) {
+                double wo = spectra_ref_bf16_to_double(w[i * k + idx[t]]);
+                double xo = spectra_ref_bf16_to_double(xr[idx[t]]);
+                acc = acc + wo * xo;
+                b = b + fabs(wo) * fabs(xo);
+            }
+            y[mm * n + i] = acc;
+            if (bound)
+                bound[mm * n + i] = b;
+        }
+    }
+}
+
+/*
+ * Row gather of a compacted table: out[r][bulk_idx[p]] = (c - z) * S of bulk
+ * column p of row ids[r], out[r][idx[t]] = W[ids[r]][idx[t]] (bit-exact); the
+ * two sets of columns partition [0, k).  An id outside [0, n) rejects the call.
+ */
+int spectra_ref_embed_compact(int32_t n, int32_t k, int32_t k_bulk, const uint8_t *codes,
+                              const uint16_t *scales, const uint8_t *zeros,
+                              const int32_t *bulk_idx, const uint16_t *w, const int32_t *idx,
+                              int32_t n_o, const int32_t *ids, int32_t m, double *out)
+{
+    if (n < 1 || k < 1 || k_bulk < 32 || k_bulk % 32 != 0 || m < 0 || n_o < 0 || n_o > k)
+        return REF_ERR_INVALID_ARG;
+    for (int32_t r = 0; r < m; ++r)
+        if (ids[r] < 0 || ids[r] >= n)
+            return REF_ERR_INVALID_ARG;
+    const int64_t Gb = k_bulk / 32;
+    for (int64_t r = 0; r < m; ++r) {
+        const int64_t i = ids[r];
+        double *orow = out + r * k;
+        for (int64_t p = 0; p < k_bulk; ++p) {
+            if (bulk_idx[p] < 0)
+                continue;
+            double S = spectra_ref_fp16_to_double(scales[i * Gb + p / 32]);
+            orow[bulk_idx[p]] = ((double)codes[i * k_bulk + p] - (double)zeros[i * Gb + p / 32]) * S;
+        }
+        for (int64_t t = 0; t < n_o; ++t)
+            orow[idx[t]] = spectra_ref_bf16_to_double(w[i * k + idx[t]]);
+    }
+    return REF_OK;
+}

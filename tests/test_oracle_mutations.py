@@ -46,6 +46,15 @@ MUTATIONS = {
                               "const int64_t grp = row * ngroups + col % ngroups;"),
     "embed_outlier_value_slot": ("dst[idx[t]] = spectra_ref_bf16_to_double(w[row * k + idx[t]]);",
                                  "dst[idx[t]] = spectra_ref_bf16_to_double(w[row * k + t]);"),
+    "bulk_columns_skip_first": ("        bulk_idx[p++] = j;\n    }", "        if (j > 0) bulk_idx[p++] = j;\n    }"),
+    "bulk_columns_pad_zero": ("        bulk_idx[p] = -1;\n", "        bulk_idx[p] = 0;\n"),
+    "gather_bulk_by_position": ("w_b[i * k_bulk + p] = bulk_idx[p] < 0 ? 0 : w[i * k + bulk_idx[p]];",
+                                "w_b[i * k_bulk + p] = bulk_idx[p] < 0 ? 0 : w[i * k + p];"),
+    "gemm_compact_x_by_position": ("double xb = spectra_ref_bf16_to_double(xr[bulk_idx[p]]);",
+                                   "double xb = spectra_ref_bf16_to_double(xr[p]);"),
+    "gemm_compact_group_of_bulk": ("double wb = ((double)codes[i * k_bulk + p] - (double)zeros[i * Gb + p / 32]) * S;",
+                                   "double wb = ((double)codes[i * k_bulk + p] - (double)zeros[i * Gb + p % Gb]) * S;"),
+    "pack_outliers_slot_reversed": ("= w[i * k + idx[slot]];", "= w[i * k + idx[n_o - 1 - slot]];"),
     "embed_zero_point_sign": ("dst[col] = ((double)codes[row * k + col] - (double)zeros[grp]) * S;",
                               "dst[col] = ((double)codes[row * k + col] + (double)zeros[grp]) * S;"),
 }
@@ -68,6 +77,11 @@ PIN_FUNCS = [
     pins.test_embed_all_outliers_is_row_indexing,
     pins.test_embed_exact_grid_rows,
     pins.test_embed_rows_agree_with_gemm,
+    pins.test_bulk_columns_are_the_complement,
+    pins.test_gemm_compact_brute_force_8x64,
+    pins.test_gemm_compact_exact_grid_bulk_is_dense_product,
+    pins.test_gemm_compact_unit_vectors_extract_columns,
+    pins.test_compact_outlier_block_is_the_masked_one,
 ]
 _PARAMS = {
     "test_quantizer_exact_grid": [{"S": 2.0 ** -7, "z": 5}],

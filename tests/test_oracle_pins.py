@@ -568,3 +568,122 @@ def test_embed_rejects_ids_outside_table(ref):
         with pytest.raises(ref.OracleError):
             ref.embed(layer.can, wb, layer.idx, np.array(bad))
     assert ref.embed(layer.can, wb, layer.idx, np.array([], dtype=np.int32)).shape == (0, 32)
+
+
+# ----------------------------------------------------------------- bulk compaction
+
+def test_bulk_columns_are_the_complement(ref):
+    rng = np.random.default_rng(30)
+    for k, n_o in [(64, 0), (64, 1), (96, 95), (96, 96), (1536, 23), (1536, 720), (8960, 4193), (32, 7)]:
+        idx = np.sort(rng.choice(k, n_o, replace=False)).astype(np.int32)
+        kb, bidx = ref.bulk_columns(k, idx)
+        rest = np.setdiff1d(np.arange(k), idx)
+        assert kb == max(32, -(-rest.size // 32) * 32)
+        assert np.array_equal(bidx[: rest.size], rest)
+        assert np.all(bidx[rest.size:] == -1)
+    for bad in ([3, 3], [5, 2], [-1], [64]):
+        with pytest.raises(ref.OracleError):
+            ref.bulk_columns(64, np.array(bad, dtype=np.int32))
+
+
+def test_compaction_without_outliers_is_the_masked_pack(ref):
+    wb, layer = _table(ref, 70, 256, 0, 31, np.inf)
+    c = ref.pack_compact(wb, wl.gain(wl.MatrixSpec("lm_head", 70, 256, 0), seed=31).numpy(), np.inf)
+    assert c.k_bulk == 256 and np.array_equal(c.bulk_idx, np.arange(256))
+    for a, b in [(c.can.codes, layer.can.codes), (c.can.scales, layer.can.scales),
+                 (c.can.zeros, layer.can.zeros), (c.packed.codes, layer.packed.codes),
+                 (c.packed.scales, layer.packed.scales), (c.packed.zeros, layer.packed.zeros)]:
+        assert np.array_equal(a, b)
+
+
+def _compact_problem(ref, n, k, n_t, seed, tau, m=1):
+    spec = wl.MatrixSpec("single", n, k, n_t)
+    wb = wl.bits(wl.weight(spec, seed=seed))
+    g = wl.gain(spec, seed=seed).numpy()
+    lay = ref.pack_compact(wb, g, tau)
+    xb = wl.bits(wl.activations(k, m, seed=seed))
+    return wb, lay, xb
+
+
+def test_gemm_compact_brute_force_8x64(ref):
+    wb, lay, xb = _compact_problem(ref, 8, 64, 2, 24, 3.0)
+    assert 0 < lay.idx.size < 64 and lay.k_bulk == 32 * -(-(64 - lay.idx.size) // 32)
+    y, b = ref.gemm_compact(lay, wb, xb)
+    codes, sc, ze = lay.can.codes, lay.can.scales, lay.can.zeros
+    S = sc.view(np.float16).astype(np.float64)
+    wv, xv = _bf16_values(wb), _bf16_values(xb)[0]
+    bulk = [j for j in range(64) if j not in lay.idx]
+    for i in range(8):
+        acc = 0.0
+        for p, j in enumerate(bulk):
+            acc += (float(codes[i, p]) - float(ze[i, p // 32])) * float(S[i, p // 32]) * float(xv[j])
+        for j in lay.idx:
+            acc += float(wv[i, j]) * float(xv[j])
+        assert y[0, i] == acc
+
+
+def test_gemm_compact_exact_grid_bulk_is_dense_product(ref):
+    # heavy outlier columns anywhere, the remaining columns (in order) forming
+    # exact quantiser grids: the compacted reconstruction is exact, so y is
+    # the dense product -- a bulk column matched with the wrong x breaks it
+    S = 2.0 ** -7
+    rng = np.random.default_rng(32)
+    n, k, n_o = 16, 96, 32
+    idx = np.sort(rng.choice(k, n_o, replace=False)).astype(np.int32)
+    rest = np.setdiff1d(np.arange(k), idx)
+    vals = np.zeros((n, k))
+    grid = np.stack([np.concatenate([_grid_row(S, 6, s), _grid_row(S, 9, s + 50)]) for s in range(n)])
+    vals[:, rest] = grid
+    vals[:, idx] = rng.standard_t(3, (n, n_o)) * 0.5
+    w = _bf16_bits(vals)
+    kb, bidx = ref.bulk_columns(k, idx)
+    can = ref.quantize(ref.gather_bulk(w, bidx), np.zeros(0, np.int32))
+    lay = ref.CompactLayer(None, idx, kb, bidx, can, None)
+    xb = wl.bits(wl.activations(k, 3, seed=33))
+    y, _ = ref.gemm_compact(lay, w, xb)
+    wvals = _bf16_values(w)
+    dense = _bf16_values(xb) @ wvals.T
+    assert np.all(np.abs(y - dense) <= 1e-13 * (np.abs(_bf16_values(xb)) @ np.abs(wvals).T))
+
+
+def test_gemm_compact_unit_vectors_extract_columns(ref):
+    wb, lay, _ = _compact_problem(ref, 40, 128, 4, 34, 3.0)
+    what = ref.dequant(lay.can)  # [n, k_bulk]
+    wv = _bf16_values(wb)
+    pos = {int(j): p for p, j in enumerate(lay.bulk_idx) if j >= 0}
+    for j in [0, 31, 32, 77, 127] + lay.idx[:6].tolist():
+        x = np.zeros((1, 128), dtype=np.uint16)
+        x[0, j] = 0x3F80  # 1.0
+        y, _ = ref.gemm_compact(lay, wb, x)
+        expect = wv[:, j] if j in lay.idx else what[:, pos[j]]
+        assert np.array_equal(y[0], expect)
+
+
+def test_gemm_compact_all_outliers_is_dense_product(ref):
+    wb, lay, xb = _compact_problem(ref, 48, 96, 3, 35, -np.inf, m=2)
+    assert lay.idx.size == 96 and lay.k_bulk == 32 and np.all(lay.bulk_idx == -1)
+    y, _ = ref.gemm_compact(lay, wb, xb)
+    dense = _bf16_values(xb) @ _bf16_values(wb).T
+    assert np.all(np.abs(y - dense) <= 1e-13 * (np.abs(_bf16_values(xb)) @ np.abs(_bf16_values(wb)).T))
+
+
+def test_embed_compact_rows_agree_with_gemm(ref):
+    wb, lay, xb = _compact_problem(ref, 64, 256, 6, 36, 3.0)
+    y, bound = ref.gemm_compact(lay, wb, xb)
+    ids = np.arange(64)[::-1].astype(np.int32)
+    rows = ref.embed_compact(lay, wb, ids)
+    assert not np.isnan(rows).any()  # the bulk and outlier columns cover every column
+    dots = rows @ _bf16_values(xb)[0]
+    assert np.all(np.abs(dots - y[0, ids]) <= 1e-13 * bound[0, ids])
+
+
+def test_compact_outlier_block_is_the_masked_one(ref):
+    # compaction changes only the bulk: the BF16 outlier block (pinned by the
+    # layout offsets) is the same array
+    for tau in (3.0, 6.0):
+        spec = wl.MatrixSpec("single", 45, 192, 5)
+        wb = wl.bits(wl.weight(spec, seed=37))
+        g = wl.gain(spec, seed=37).numpy()
+        masked, comp = ref.pack(wb, g, tau), ref.pack_compact(wb, g, tau)
+        assert np.array_equal(masked.idx, comp.idx) and comp.idx.size > 0
+        assert np.array_equal(masked.packed.outliers, comp.packed.outliers)
