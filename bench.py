@@ -61,6 +61,23 @@ def algorithmic_bytes(n: int, k: int, n_o: int, m: int = 1, y_bytes: int = 4) ->
             + 2 * m * k + y_bytes * m * n)
 
 
+def algorithmic_bytes_compact(n: int, k: int, k_bulk: int, n_o: int, m: int = 1,
+                              y_bytes: int = 4) -> int:
+    """algorithmic_bytes for a compacted bulk: 4.625 bits per weight over the
+    k_bulk bulk columns only, the bulk column list (4 bytes per bulk column),
+    BF16 outlier columns, outlier indices, x (all k columns), y."""
+    n_pad = -(-n // 32) * 32
+    return (n_pad * k_bulk // 2 + n_pad * k_bulk // 16 + n_pad * k_bulk // 64 + 4 * k_bulk
+            + 2 * n * n_o + 4 * n_o + 2 * m * k + y_bytes * m * n)
+
+
+def layer_bytes(lay, m: int = 1, y_bytes: int = 4) -> int:
+    """Algorithmic bytes of one matvec over a packed layer (masked or compacted)."""
+    if lay.compact:
+        return algorithmic_bytes_compact(lay.n, lay.k, lay.k_bulk, lay.n_outliers, m, y_bytes)
+    return algorithmic_bytes(lay.n, lay.k, lay.n_outliers, m, y_bytes)
+
+
 def embed_bytes(k: int, n_o: int, m: int, out_bytes: int = 2) -> int:
     """Bytes an embedding gather of m rows must move: each row's codes, scales
     and zero points (4.625 bits per column), its BF16 outlier values, the
@@ -141,7 +158,7 @@ class ClockSampler:
 class Stream:
     """The packed 28-layer weight stream with its activation and output buffers."""
 
-    def __init__(self, device, seed: int, tau: float):
+    def __init__(self, device, seed: int, tau: float, compact: bool = False):
         import outlier_split_bit_b200 as sp
         self.sp = sp
         specs = [(layer, s) for layer in range(N_LAYERS) for s in wl.LAYER_1P5B]
@@ -156,7 +173,7 @@ class Stream:
         for layer, spec in specs:
             w = wl.weight(spec, seed, layer, device=device)
             g = wl.gain(spec, seed, layer, device=device)
-            lay = sp.pack_layer(w, g, tau)
+            lay = sp.pack_layer(w, g, tau, compact=compact)
             del w
             x = self.x_all[xo:xo + spec.k]
             x.copy_(wl.activations(spec.k, 1, seed, layer, slot=wl.PROJ.index(spec.name),
@@ -165,7 +182,7 @@ class Stream:
             xo += spec.k
             yo += spec.n
             self.items.append((spec, lay, x, y, lay.view()))
-            self.bytes += algorithmic_bytes(spec.n, spec.k, lay.n_outliers)
+            self.bytes += layer_bytes(lay)
             self.n_outliers += lay.n_outliers
         self.launches = len(self.items)
 
@@ -238,7 +255,8 @@ def copies_of(lay, min_total_bytes):
     out = [lay]
     while sum(c.nbytes for c in out) < min_total_bytes:
         out.append(sp.PackedLayer(lay.n, lay.k, lay.n_outliers, lay.codes.clone(), lay.scales.clone(),
-                                  lay.zeros.clone(), lay.outlier_idx.clone(), lay.outlier_w.clone()))
+                                  lay.zeros.clone(), lay.outlier_idx.clone(), lay.outlier_w.clone(),
+                                  None if lay.bulk_idx is None else lay.bulk_idx.clone(), lay.k_bulk))
     return out
 
 
@@ -329,6 +347,22 @@ def extras(device, stream, peak_gbs, tau):
                          "bits_per_weight": round(8 * lay.nbytes / (spec.n * spec.k), 3)})
             del w, lay, dense
         out["lm_head_131072x3072"] = rows
+        # the compacted bulk on the same matrix (1 % Student-t columns)
+        spec = wl.lm_head_spec(0.01)
+        w = wl.weight(spec, 0, 0, device=device)
+        g = wl.gain(spec, 0, 0, device=device)
+        lay = sp.pack_layer(w, g, tau, compact=True)
+        x = wl.activations(spec.k, 1, device=device)[0]
+        y = torch.empty(spec.n, device=device)
+        v = lay.view()
+        us, p10, p90 = time_single(lambda: sp.spectra_gemv(lay, x, y, view=v, stream=stream),
+                                   stream, 20, flush)
+        b = layer_bytes(lay)
+        out["lm_head_131072x3072_compact_bulk"] = {
+            "frac_t_columns": 0.01, "n_outliers": lay.n_outliers, "k_bulk": lay.k_bulk, "us": round(us, 2),
+            "gbs": round(b / us * 1e-3, 1), "frac": round(b / us * 1e-3 / peak_gbs, 3), "bytes": b,
+            "bits_per_weight": round(8 * lay.nbytes / (spec.n * spec.k), 3)}
+        del w, lay
         rows = []
         spec = wl.LAYER_4B[4]
         w = wl.weight(spec, 0, 0, device=device)
@@ -566,7 +600,7 @@ def run_ours(args):
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_done = [torch.cuda.Event() for _ in range(2)]
     ev_out = [torch.cuda.Event() for _ in range(2)]
-    e2e_steps = max(2, min(args.steps, 200))
+    e2e_steps = max(2, args.steps)
     barrier()
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -626,6 +660,29 @@ def run_ours(args):
         "frac": round(st.bytes / (chain_ms * 1e-3) * 1e-9 / peak, 4),
         "us_per_launch": round(chain_ms * 1e3 / chain_launches, 3)}}
     if rank == 0 and not args.quick:
+        # the same stream with the outlier columns removed from the 4-bit bulk
+        st_c = Stream(device, seed=rank, tau=args.tau, compact=True)
+        graph_c, _ = st_c.capture(stream, "batched")
+        for _ in range(args.warmup):
+            graph_c.replay()
+        stream.synchronize()
+        c_steps = max(3, min(args.steps, 500))
+        with torch.cuda.stream(stream):
+            c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            c0.record(stream)
+            for _ in range(c_steps):
+                graph_c.replay()
+            c1.record(stream)
+        c1.synchronize()
+        c_ms = c0.elapsed_time(c1) / c_steps
+        extra["decode_stream_compact_bulk"] = {
+            "tau": args.tau, "launches_per_step": 1, "us_per_step": round(c_ms * 1e3, 2),
+            "bytes_per_step": st_c.bytes, "gbs": round(st_c.bytes / (c_ms * 1e-3) * 1e-9, 1),
+            "frac": round(st_c.bytes / (c_ms * 1e-3) * 1e-9 / peak, 4),
+            "us_per_step_masked_bulk": round(step_ms * 1e3, 2),
+            "bytes_per_step_masked_bulk": st.bytes,
+            "steps": c_steps}
+        del graph_c, st_c
         extra.update(extras(device, stream, peak, args.tau))
 
     cpu = None

@@ -49,6 +49,19 @@
  *             W[32t + r][idx[j]] for outlier slot j.
  *   Padding rows, groups and outlier slots are zero.  Bulk storage is
  *   4.625 bits per weight (0.578 bytes) plus 16 bits per outlier element.
+ *
+ * Two forms of the bulk:
+ *   masked (spectra_pack): the bulk keeps all k columns and the outlier
+ *     columns are set to +0 in it before quantisation (their codes decode to
+ *     exactly 0); G = k/32.
+ *   compacted (spectra_pack_compact): the outlier columns are removed from
+ *     the bulk, which holds the k - n_outliers other columns in ascending
+ *     order, padded with all-zero columns to k_bulk = max(32, 32 *
+ *     ceil((k - n_outliers)/32)); bulk_idx[p] is the column of W held by
+ *     bulk column p (-1 for padding); G = k_bulk/32.  Groups of 32 are then
+ *     32 consecutive *bulk* columns.  The layout above applies with k_bulk in
+ *     place of k; x keeps its k columns and the kernels gather it through
+ *     bulk_idx.
  */
 #ifndef SPECTRA_H
 #define SPECTRA_H
@@ -97,6 +110,9 @@ typedef struct {
     const uint32_t *zeros;       /* device, 8 zero points per word */
     const int32_t *outlier_idx;  /* device, ascending column indices [n_outliers] */
     const uint16_t *outlier_w;   /* device, BF16 bits, RT32 outlier block */
+    int32_t k_bulk;              /* compacted: bulk columns; masked: 0 or k */
+    const int32_t *bulk_idx;     /* device [k_bulk], 16-byte aligned, compacted
+                                    only; NULL selects the masked bulk */
 } spectra_layer;
 
 /* Byte sizes of the packed buffers of one layer. */
@@ -107,6 +123,8 @@ typedef struct {
     size_t zeros_bytes;
     size_t outlier_idx_bytes;
     size_t outlier_w_bytes;
+    int32_t k_bulk;              /* columns of the bulk (k when masked) */
+    size_t bulk_idx_bytes;       /* 0 when masked */
 } spectra_sizes;
 
 /* Human-readable name of a status value (static string, never NULL). */
@@ -120,6 +138,13 @@ SPECTRA_API int32_t spectra_version(void);
  * columns (layout above).  Host only, no CUDA call.
  */
 SPECTRA_API spectra_status spectra_packed_sizes(int32_t n, int32_t k, int32_t n_outliers, spectra_sizes *out);
+
+/*
+ * The same for a compacted bulk (k_bulk columns, plus the bulk column list).
+ * Host only, no CUDA call.
+ */
+SPECTRA_API spectra_status spectra_packed_sizes_compact(int32_t n, int32_t k, int32_t n_outliers,
+                                                        spectra_sizes *out);
 
 /* Device workspace bytes that spectra_pack_plan needs for in_features k. */
 SPECTRA_API size_t spectra_pack_plan_workspace_size(int32_t k);
@@ -199,9 +224,30 @@ SPECTRA_API spectra_status spectra_pack(const uint16_t *w, int32_t n, int32_t k,
                             size_t workspace_bytes, spectra_layer *layer_out, void *stream);
 
 /*
+ * spectra_pack with a compacted bulk (abstract: the heavy-tailed coordinates
+ * are decoupled into bit-exact storage and the residual bulk quantised; here
+ * the outlier columns leave the 4-bit bulk instead of staying in it as
+ * zeros, which saves 4.625 bits per outlier element).  Arguments as
+ * spectra_pack, sized by spectra_packed_sizes_compact, plus
+ *   bulk_idx  device int32 [k_bulk] output, 16-byte aligned: the column of W
+ *             held by each bulk column, -1 for padding
+ * The quantiser is spectra_pack's, applied to the compacted bulk: per row
+ * and group of 32 consecutive bulk columns.  layer_out (HOST, may be NULL)
+ * receives the view with k_bulk and bulk_idx set.  Bit-identical to the
+ * oracle.  Synchronous.  Errors: as spectra_pack.
+ */
+SPECTRA_API spectra_status spectra_pack_compact(const uint16_t *w, int32_t n, int32_t k,
+                                                const int32_t *idx, int32_t n_outliers,
+                                                uint8_t *codes, uint16_t *scales, uint32_t *zeros,
+                                                uint16_t *outlier_w, int32_t *bulk_idx,
+                                                void *workspace, size_t workspace_bytes,
+                                                spectra_layer *layer_out, void *stream);
+
+/*
  * Inverse of the layout step, for tests: packed layer -> canonical row-major
- * arrays codes [n][k] (one code per byte), scales [n][k/32] (FP16 bits),
- * zeros [n][k/32] (one zero point per byte), all device.  Asynchronous.
+ * arrays codes [n][kb] (one code per byte), scales [n][kb/32] (FP16 bits),
+ * zeros [n][kb/32] (one zero point per byte), all device, where kb is k for
+ * a masked bulk and k_bulk for a compacted one.  Asynchronous.
  */
 SPECTRA_API spectra_status spectra_unpack(const spectra_layer *layer, uint8_t *codes, uint16_t *scales,
                               uint8_t *zeros, void *stream);

@@ -21,7 +21,8 @@ from . import _lib
 from ._lib import Layer, Sizes
 
 __all__ = ["SpectraError", "PackedLayer", "spectra_status_string", "spectra_version",
-           "spectra_packed_sizes", "spectra_pack_plan", "spectra_pack", "spectra_unpack",
+           "spectra_packed_sizes", "spectra_packed_sizes_compact", "spectra_pack_plan",
+           "spectra_pack", "spectra_pack_compact", "spectra_unpack",
            "spectra_gemv", "spectra_gemm_small", "spectra_gemv_batched", "spectra_embed",
            "spectra_device_status",
            "pack_layer", "library"]
@@ -77,12 +78,23 @@ def spectra_device_status(*, stream=None) -> None:
     _check(_L.spectra_device_status(_stream(stream)), "spectra_device_status")
 
 
+def _sizes(s: Sizes) -> dict:
+    return {"n_pad": s.n_pad, "codes": s.codes_bytes, "scales": s.scales_bytes,
+            "zeros": s.zeros_bytes, "outlier_idx": s.outlier_idx_bytes,
+            "outlier_w": s.outlier_w_bytes, "k_bulk": s.k_bulk, "bulk_idx": s.bulk_idx_bytes}
+
+
 def spectra_packed_sizes(n: int, k: int, n_outliers: int) -> dict:
     s = Sizes()
     _check(_L.spectra_packed_sizes(n, k, n_outliers, ctypes.byref(s)), "spectra_packed_sizes")
-    return {"n_pad": s.n_pad, "codes": s.codes_bytes, "scales": s.scales_bytes,
-            "zeros": s.zeros_bytes, "outlier_idx": s.outlier_idx_bytes,
-            "outlier_w": s.outlier_w_bytes}
+    return _sizes(s)
+
+
+def spectra_packed_sizes_compact(n: int, k: int, n_outliers: int) -> dict:
+    s = Sizes()
+    _check(_L.spectra_packed_sizes_compact(n, k, n_outliers, ctypes.byref(s)),
+           "spectra_packed_sizes_compact")
+    return _sizes(s)
 
 
 def spectra_pack_plan(w: torch.Tensor, gain: torch.Tensor | None, tau: float, *,
@@ -112,18 +124,30 @@ class PackedLayer:
     zeros: torch.Tensor        # int32 storage of u32 words
     outlier_idx: torch.Tensor  # int32
     outlier_w: torch.Tensor    # int16 storage of BF16 bits
+    bulk_idx: torch.Tensor | None = None  # int32 [k_bulk]: compacted bulk only
+    k_bulk: int = 0                       # bulk columns (k when masked)
+
+    def __post_init__(self):
+        if self.k_bulk == 0:
+            self.k_bulk = self.k
+
+    @property
+    def compact(self) -> bool:
+        return self.bulk_idx is not None
 
     def view(self) -> Layer:
         return Layer(self.n, self.k, self.n_outliers, _ptr(self.codes), _ptr(self.scales),
                      _ptr(self.zeros), _ptr(self.outlier_idx) if self.n_outliers else None,
-                     _ptr(self.outlier_w) if self.n_outliers else None)
+                     _ptr(self.outlier_w) if self.n_outliers else None,
+                     self.k_bulk, _ptr(self.bulk_idx))
 
     @property
     def nbytes(self) -> int:
         """Bytes a matvec streams from these buffers (codes, scales, zeros,
-        outlier weights and indices)."""
+        outlier weights and indices, and the bulk column list)."""
         return (self.codes.numel() + 2 * self.scales.numel() + 4 * self.zeros.numel()
-                + 4 * self.n_outliers + 2 * self.outlier_w.numel())
+                + 4 * self.n_outliers + 2 * self.outlier_w.numel()
+                + (4 * self.bulk_idx.numel() if self.compact else 0))
 
 
 def _alloc(nbytes: int, dtype, dev):
@@ -151,17 +175,43 @@ def spectra_pack(w: torch.Tensor, idx: torch.Tensor, *, stream=None) -> PackedLa
     return PackedLayer(n, k, n_o, codes, scales, zeros, idx_c, outw)
 
 
-def pack_layer(w: torch.Tensor, gain: torch.Tensor | None, tau: float, *, stream=None):
-    """spectra_pack_plan followed by spectra_pack."""
+def spectra_pack_compact(w: torch.Tensor, idx: torch.Tensor, *, stream=None) -> PackedLayer:
+    """Quantise and pack W with the outlier columns removed from the bulk."""
+    n, k = w.shape
+    n_o = int(idx.numel())
+    dev = w.device
+    sz = spectra_packed_sizes_compact(n, k, n_o)
+    codes = _alloc(sz["codes"], torch.uint8, dev)
+    scales = _alloc(sz["scales"], torch.int16, dev)
+    zeros = _alloc(sz["zeros"], torch.int32, dev)
+    outw = _alloc(sz["outlier_w"], torch.int16, dev)
+    bidx = torch.empty(sz["k_bulk"], dtype=torch.int32, device=dev)
+    idx_c = idx.contiguous() if n_o else torch.zeros(1, dtype=torch.int32, device=dev)
+    ws_bytes = _L.spectra_pack_workspace_size()
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    view = Layer()
+    _check(_L.spectra_pack_compact(_ptr(w), n, k, _ptr(idx_c) if n_o else None, n_o, _ptr(codes),
+                                   _ptr(scales), _ptr(zeros), _ptr(outw) if n_o else None,
+                                   _ptr(bidx), _ptr(ws), ws_bytes, ctypes.byref(view),
+                                   _stream(stream)), "spectra_pack_compact")
+    return PackedLayer(n, k, n_o, codes, scales, zeros, idx_c, outw, bidx, sz["k_bulk"])
+
+
+def pack_layer(w: torch.Tensor, gain: torch.Tensor | None, tau: float, *, compact: bool = False,
+               stream=None):
+    """spectra_pack_plan followed by spectra_pack (or spectra_pack_compact)."""
     idx, _ = spectra_pack_plan(w, gain, tau, stream=stream)
+    if compact:
+        return spectra_pack_compact(w, idx, stream=stream)
     return spectra_pack(w, idx, stream=stream)
 
 
 def spectra_unpack(layer: PackedLayer, *, stream=None):
-    """Canonical (codes u8 [n,k], scales int16-bits [n,k/32], zeros u8 [n,k/32])."""
+    """Canonical (codes u8 [n,kb], scales int16-bits [n,kb/32], zeros u8 [n,kb/32]),
+    kb = k_bulk (k for a masked bulk)."""
     dev = layer.codes.device
-    G = layer.k // 32
-    codes = torch.empty((layer.n, layer.k), dtype=torch.uint8, device=dev)
+    G = layer.k_bulk // 32
+    codes = torch.empty((layer.n, layer.k_bulk), dtype=torch.uint8, device=dev)
     scales = torch.empty((layer.n, G), dtype=torch.int16, device=dev)
     zeros = torch.empty((layer.n, G), dtype=torch.uint8, device=dev)
     v = layer.view()

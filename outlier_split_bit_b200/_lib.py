@@ -27,13 +27,15 @@ class Layer(ctypes.Structure):
     """spectra_layer: a view of caller-owned device buffers."""
     _fields_ = [("n", ctypes.c_int32), ("k", ctypes.c_int32), ("n_outliers", ctypes.c_int32),
                 ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("zeros", ctypes.c_void_p),
-                ("outlier_idx", ctypes.c_void_p), ("outlier_w", ctypes.c_void_p)]
+                ("outlier_idx", ctypes.c_void_p), ("outlier_w", ctypes.c_void_p),
+                ("k_bulk", ctypes.c_int32), ("bulk_idx", ctypes.c_void_p)]
 
 
 class Sizes(ctypes.Structure):
     _fields_ = [("n_pad", ctypes.c_int64), ("codes_bytes", ctypes.c_size_t),
                 ("scales_bytes", ctypes.c_size_t), ("zeros_bytes", ctypes.c_size_t),
-                ("outlier_idx_bytes", ctypes.c_size_t), ("outlier_w_bytes", ctypes.c_size_t)]
+                ("outlier_idx_bytes", ctypes.c_size_t), ("outlier_w_bytes", ctypes.c_size_t),
+                ("k_bulk", ctypes.c_int32), ("bulk_idx_bytes", ctypes.c_size_t)]
 
 
 # name -> (restype, argtypes), mirroring spectra.h
@@ -48,6 +50,8 @@ SIGNATURES = {
     "spectra_pack_workspace_size": (sz, []),
     "spectra_pack_plan": (ctypes.c_int, [P, P, i32, i32, f64, P, P, ctypes.POINTER(i32), P, sz, P]),
     "spectra_pack": (ctypes.c_int, [P, i32, i32, P, i32, P, P, P, P, P, sz, LP, P]),
+    "spectra_packed_sizes_compact": (ctypes.c_int, [i32, i32, i32, ctypes.POINTER(Sizes)]),
+    "spectra_pack_compact": (ctypes.c_int, [P, i32, i32, P, i32, P, P, P, P, P, P, sz, LP, P]),
     "spectra_unpack": (ctypes.c_int, [LP, P, P, P, P]),
     "spectra_gemv": (ctypes.c_int, [LP, P, P, ctypes.c_int, P]),
     "spectra_gemm_small": (ctypes.c_int, [LP, P, i32, P, ctypes.c_int, P]),

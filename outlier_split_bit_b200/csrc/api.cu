@@ -40,7 +40,26 @@ spectra_status check_layer(const spectra_layer *l) {
         return SPECTRA_ERR_ALIGN;
     if (l->n_outliers > 0 && (!aligned16(l->outlier_w) || !aligned4(l->outlier_idx)))
         return SPECTRA_ERR_ALIGN;
+    if (l->bulk_idx) {
+        if (l->k_bulk != compact_width(l->k, l->n_outliers)) return SPECTRA_ERR_INVALID_ARG;
+        if (!aligned16(l->bulk_idx)) return SPECTRA_ERR_ALIGN;
+    } else if (l->k_bulk != 0 && l->k_bulk != l->k) {
+        return SPECTRA_ERR_INVALID_ARG;
+    }
     return SPECTRA_OK;
+}
+
+void fill_sizes(int32_t n, int32_t kb, int32_t n_outliers, spectra_sizes *out) {
+    const Geometry g = Geometry::of(n, kb, n_outliers);
+    const int64_t np = (int64_t)g.T * 32;
+    out->n_pad = np;
+    out->codes_bytes = (size_t)(np * kb / 2);
+    out->scales_bytes = (size_t)(np * g.S * 8 * 2);
+    out->zeros_bytes = (size_t)(np * g.S * 4);
+    out->outlier_idx_bytes = (size_t)n_outliers * 4;
+    out->outlier_w_bytes = (size_t)(np * g.O8 * 8 * 2);
+    out->k_bulk = kb;
+    out->bulk_idx_bytes = 0;
 }
 }  // namespace
 
@@ -90,21 +109,26 @@ const char *spectra_status_string(spectra_status s) {
     return "unknown status";
 }
 
-int32_t spectra_version(void) { return 101; }
+int32_t spectra_version(void) { return 200; }
 
 spectra_status spectra_packed_sizes(int32_t n, int32_t k, int32_t n_outliers, spectra_sizes *out) {
     if (!out) return SPECTRA_ERR_INVALID_ARG;
     spectra_status st = check_shape(n, k);
     if (st != SPECTRA_OK) return st;
     if (n_outliers < 0 || n_outliers > k) return SPECTRA_ERR_INVALID_ARG;
-    const Geometry g = Geometry::of(n, k, n_outliers);
-    const int64_t np = (int64_t)g.T * 32;
-    out->n_pad = np;
-    out->codes_bytes = (size_t)(np * k / 2);
-    out->scales_bytes = (size_t)(np * g.S * 8 * 2);
-    out->zeros_bytes = (size_t)(np * g.S * 4);
-    out->outlier_idx_bytes = (size_t)n_outliers * 4;
-    out->outlier_w_bytes = (size_t)(np * g.O8 * 8 * 2);
+    fill_sizes(n, k, n_outliers, out);
+    return SPECTRA_OK;
+}
+
+spectra_status spectra_packed_sizes_compact(int32_t n, int32_t k, int32_t n_outliers,
+                                            spectra_sizes *out) {
+    if (!out) return SPECTRA_ERR_INVALID_ARG;
+    spectra_status st = check_shape(n, k);
+    if (st != SPECTRA_OK) return st;
+    if (n_outliers < 0 || n_outliers > k) return SPECTRA_ERR_INVALID_ARG;
+    const int32_t kb = compact_width(k, n_outliers);
+    fill_sizes(n, kb, n_outliers, out);
+    out->bulk_idx_bytes = (size_t)kb * 4;
     return SPECTRA_OK;
 }
 
@@ -188,6 +212,62 @@ spectra_status spectra_pack(const uint16_t *w, int32_t n, int32_t k, const int32
         layer_out->zeros = zeros;
         layer_out->outlier_idx = idx;
         layer_out->outlier_w = outlier_w;
+        layer_out->k_bulk = k;
+        layer_out->bulk_idx = nullptr;
+    }
+    return SPECTRA_OK;
+}
+
+spectra_status spectra_pack_compact(const uint16_t *w, int32_t n, int32_t k, const int32_t *idx,
+                                    int32_t n_outliers, uint8_t *codes, uint16_t *scales,
+                                    uint32_t *zeros, uint16_t *outlier_w, int32_t *bulk_idx,
+                                    void *workspace, size_t workspace_bytes,
+                                    spectra_layer *layer_out, void *stream) {
+    if (!w || !codes || !scales || !zeros || !bulk_idx || !workspace)
+        return SPECTRA_ERR_INVALID_ARG;
+    spectra_status st = check_shape(n, k);
+    if (st != SPECTRA_OK) return st;
+    if (n_outliers < 0 || n_outliers > k) return SPECTRA_ERR_INVALID_ARG;
+    if (n_outliers > 0 && (!idx || !outlier_w)) return SPECTRA_ERR_INVALID_ARG;
+    if (!aligned16(w) || !aligned16(codes) || !aligned16(scales) || !aligned16(zeros) ||
+        !aligned16(bulk_idx) || !aligned16(workspace) ||
+        (n_outliers > 0 && (!aligned16(outlier_w) || !aligned4(idx))))
+        return SPECTRA_ERR_ALIGN;
+    if (workspace_bytes < spectra_pack_workspace_size()) return SPECTRA_ERR_BUFFER_TOO_SMALL;
+    DeviceInfo dev;
+    st = current_device(&dev);
+    if (st != SPECTRA_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int kb = compact_width(k, n_outliers);
+    const Geometry gb = Geometry::of(n, kb, n_outliers);
+    int *err = (int *)workspace;
+    if (cudaMemsetAsync(err, 0, sizeof(int), s) != cudaSuccess) return SPECTRA_ERR_CUDA;
+    if (launch_bulk_columns(n_outliers > 0 ? idx : nullptr, n_outliers, k, kb, bulk_idx, err, s) !=
+        cudaSuccess)
+        return SPECTRA_ERR_CUDA;
+    if (launch_quantize_pack_compact(w, k, gb, bulk_idx, codes, scales, zeros, err, s) !=
+        cudaSuccess)
+        return SPECTRA_ERR_CUDA;
+    if (launch_outlier_gather(w, Geometry::of(n, k, n_outliers), idx, outlier_w, s) != cudaSuccess)
+        return SPECTRA_ERR_CUDA;
+    int host = 0;
+    if (cudaMemcpyAsync(&host, err, sizeof host, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return SPECTRA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SPECTRA_ERR_CUDA;
+    if (host & kErrBadIndex) return SPECTRA_ERR_INVALID_ARG;
+    if (host & kErrNonfinite) return SPECTRA_ERR_NONFINITE;
+    if (host & kErrRange) return SPECTRA_ERR_RANGE;
+    if (layer_out) {
+        layer_out->n = n;
+        layer_out->k = k;
+        layer_out->n_outliers = n_outliers;
+        layer_out->codes = codes;
+        layer_out->scales = scales;
+        layer_out->zeros = zeros;
+        layer_out->outlier_idx = idx;
+        layer_out->outlier_w = outlier_w;
+        layer_out->k_bulk = kb;
+        layer_out->bulk_idx = bulk_idx;
     }
     return SPECTRA_OK;
 }

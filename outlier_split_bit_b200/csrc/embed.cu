@@ -8,24 +8,32 @@
 // k = hidden columns, outlier columns kept bit-exact in BF16), so a tied
 // LM head's buffers serve as the embedding table as they are.
 //
-// Work decomposition.  One CTA per requested row (grid-stride over the ids);
-// thread g of the CTA decodes group g of the row: its 16-byte code record
-// (lane r = id % 32 of tile id / 32, one record per group), its FP16 scale
-// and its zero-point nibble, and writes the 32 values (c - z) * s -- exact in
-// FP32 (a 5-bit signed integer times an 11-bit significand) -- as eight
-// 16-byte FP32 stores or four 16-byte BF16 stores (one rounding to nearest
-// even).  The bulk holds exact zeros at the outlier columns; after a block
-// barrier the threads overwrite those columns with the stored BF16 values,
-// so they come back bit for bit.  Each row's records lie 512 bytes apart
-// (the RT32 layout serves the matvec, where a warp reads whole tiles), so a
-// lone row moves 32-byte sectors for 16-byte records; ids in one tile share
-// sectors through L2.
+// Work decomposition.  One CTA per requested row (grid-stride over the
+// ids).  The row is assembled in shared memory, then written out once with
+// 16-byte coalesced stores:
+//   1. thread g decodes bulk group g of the row: its 16-byte code record
+//      (lane r = id % 32 of tile id / 32), its FP16 scale and zero-point
+//      nibble, giving (c - z) * s exact in FP32 (a 5-bit signed integer times
+//      an 11-bit significand), rounded once to nearest even for BF16 output;
+//      a masked bulk fills columns 32g..32g+31 (zeros at the outlier
+//      columns), a compacted bulk scatters its values to the columns its
+//      bulk column list names;
+//   2. after a block barrier, each thread takes outlier octets: one 16-byte
+//      load of the row's 8 BF16 values and their 8 column indices, written
+//      into the row, so those columns come back bit for bit;
+//   3. after a second barrier the row goes out, and a third barrier frees
+//      the buffer for the next row.
+// Each row's records lie 512 bytes apart (the RT32 layout serves the matvec,
+// where a warp reads whole tiles), so a lone row moves 32-byte sectors for
+// its 16-byte records; ids in one tile share sectors through L2.
 //
 // An id outside [0, n) yields a zero row and raises bit 0 of a device flag;
-// an outlier index outside [0, k) is skipped and raises bit 1.  Neither
-// reads or writes out of bounds.
+// a column index outside [0, k) (outlier list or bulk column list) is
+// skipped and raises bit 1.  Neither reads or writes out of bounds.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+
+#include <mutex>
 
 #include "internal.cuh"
 
@@ -33,9 +41,9 @@ namespace spectra {
 namespace {
 
 constexpr int kEmbedMaxThreads = 256;
-constexpr int kEmbedCtasPerSm = 16;
+constexpr int kEmbedCtasPerSm = 8;
 
-// bit 0: a token id outside the table; bit 1: an outlier index outside [0, k).
+// bit 0: a token id outside the table; bit 1: a column index outside [0, k).
 __device__ unsigned int g_embed_error;
 
 struct EmbedArgs {
@@ -43,14 +51,26 @@ struct EmbedArgs {
     const uint16_t *scales;
     const uint32_t *zeros;
     const int32_t *oidx;
-    const uint16_t *outw;
+    const uint4 *outw;
+    const int32_t *bidx;  // bulk column list (compacted bulk), nullptr when masked
     const int32_t *ids;
     void *out;
     int n, k, G, S, O8, n_o, m;
 };
 
 template <bool kBF16>
+__device__ __forceinline__ void put(uint8_t *row, int col, float v) {
+    if constexpr (kBF16)
+        reinterpret_cast<__nv_bfloat16 *>(row)[col] = __float2bfloat16_rn(v);
+    else
+        reinterpret_cast<float *>(row)[col] = v;
+}
+
+template <bool kBF16>
 __global__ void __launch_bounds__(kEmbedMaxThreads) embed_kernel(const EmbedArgs a) {
+    extern __shared__ uint4 rowbuf[];  // one output row: k * (2 or 4) bytes
+    uint8_t *row = reinterpret_cast<uint8_t *>(rowbuf);
+    constexpr int kEsz = kBF16 ? 2 : 4;
     // the table is constant, but which rows are needed is known only from the
     // ids, which the previous kernel on the stream may still be writing
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -60,6 +80,7 @@ __global__ void __launch_bounds__(kEmbedMaxThreads) embed_kernel(const EmbedArgs
         const bool ok = id >= 0 && id < a.n;
         if (!ok && threadIdx.x == 0) atomicOr(&g_embed_error, 1u);
         const int t = ok ? (id >> 5) : 0, lane = ok ? (id & 31) : 0;
+        // 1. bulk groups
         for (int g = threadIdx.x; g < a.G; g += blockDim.x) {
             float v[32];
             if (ok) {
@@ -77,55 +98,83 @@ __global__ void __launch_bounds__(kEmbedMaxThreads) embed_kernel(const EmbedArgs
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = 0.f;
             }
-            if constexpr (kBF16) {
-                uint4 *dst = reinterpret_cast<uint4 *>(
-                    reinterpret_cast<__nv_bfloat16 *>(a.out) + (size_t)r * a.k + 32 * g);
+            if (a.bidx == nullptr) {
+                uint4 *dst = reinterpret_cast<uint4 *>(row + (size_t)32 * kEsz * g);
+                if constexpr (kBF16) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t p[4];
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t p[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(v[8 * q + 2 * e]));
-                        const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(v[8 * q + 2 * e + 1]));
-                        p[e] = lo | (hi << 16);
+                        for (int e = 0; e < 4; ++e) {
+                            const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(v[8 * q + 2 * e]));
+                            const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(v[8 * q + 2 * e + 1]));
+                            p[e] = lo | (hi << 16);
+                        }
+                        dst[q] = make_uint4(p[0], p[1], p[2], p[3]);
                     }
-                    dst[q] = make_uint4(p[0], p[1], p[2], p[3]);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        dst[q] = make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
+                                            __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
                 }
             } else {
-                float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(a.out) +
-                                                         (size_t)r * a.k + 32 * g);
+                const int4 *bc = reinterpret_cast<const int4 *>(a.bidx + 32 * g);
 #pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-            }
-        }
-        if (a.n_o > 0) {
-            // the bulk stores of this row (zeros at the outlier columns) land
-            // before the outlier values replace them
-            __syncthreads();
-            for (int j = threadIdx.x; j < a.n_o; j += blockDim.x) {
-                const int col = a.oidx[j];
-                if (col < 0 || col >= a.k) {
-                    atomicOr(&g_embed_error, 2u);
-                    continue;
+                for (int q = 0; q < 8; ++q) {
+                    const int4 c4 = __ldg(bc + q);
+                    const int c[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        if (c[e] < 0) continue;  // padding column
+                        if (c[e] >= a.k) {
+                            atomicOr(&g_embed_error, 2u);
+                            continue;
+                        }
+                        put<kBF16>(row, c[e], v[4 * q + e]);
+                    }
                 }
-                const uint16_t b =
-                    ok ? a.outw[(((size_t)t * a.O8 + (j >> 3)) * 32 + lane) * 8 + (j & 7)] : 0;
-                if constexpr (kBF16)
-                    reinterpret_cast<uint16_t *>(a.out)[(size_t)r * a.k + col] = b;
-                else
-                    reinterpret_cast<uint32_t *>(a.out)[(size_t)r * a.k + col] = (uint32_t)b << 16;
             }
         }
+        // 2. outlier columns, an octet per thread at a time
+        if (a.n_o > 0) {
+            __syncthreads();
+            for (int o = threadIdx.x; o < a.O8; o += blockDim.x) {
+                const uint4 wv = ok ? a.outw[((size_t)t * a.O8 + o) * 32 + lane] : make_uint4(0, 0, 0, 0);
+                const uint32_t w4[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int j = 8 * o + e;
+                    if (j >= a.n_o) break;
+                    const int col = __ldg(a.oidx + j);
+                    if (col < 0 || col >= a.k) {
+                        atomicOr(&g_embed_error, 2u);
+                        continue;
+                    }
+                    const uint32_t b = (w4[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+                    if constexpr (kBF16)
+                        reinterpret_cast<uint16_t *>(row)[col] = (uint16_t)b;
+                    else
+                        reinterpret_cast<uint32_t *>(row)[col] = b << 16;
+                }
+            }
+        }
+        __syncthreads();
+        // 3. the row, 16 bytes per thread and store
+        uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(a.out) + (size_t)r * a.k * kEsz);
+        const int nvec = a.k * kEsz / 16;
+        for (int i = threadIdx.x; i < nvec; i += blockDim.x) dst[i] = rowbuf[i];
+        __syncthreads();
     }
 }
 
 template <bool kBF16>
-cudaError_t launch(const EmbedArgs &args, unsigned grid, unsigned threads, cudaStream_t s) {
+cudaError_t launch(const EmbedArgs &args, unsigned grid, unsigned threads, size_t smem,
+                   cudaStream_t s) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid, 1, 1);
     cfg.blockDim = dim3(threads, 1, 1);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr;
     attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -135,17 +184,36 @@ cudaError_t launch(const EmbedArgs &args, unsigned grid, unsigned threads, cudaS
     return cudaLaunchKernelEx(&cfg, embed_kernel<kBF16>, args);
 }
 
+std::mutex g_embed_mu;
+bool g_embed_ready[2][64];
+
+// Raise the dynamic shared-memory limit of the kernel once per device.
+template <bool kBF16>
+cudaError_t prepare(const DeviceInfo &dev) {
+    std::lock_guard<std::mutex> lock(g_embed_mu);
+    if (dev.device < 0 || dev.device >= 64) return cudaErrorInvalidDevice;
+    if (g_embed_ready[kBF16][dev.device]) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(
+        embed_kernel<kBF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dev.smem_optin);
+    if (e == cudaSuccess) g_embed_ready[kBF16][dev.device] = true;
+    return e;
+}
+
 }  // namespace
 
 spectra_status launch_embed(const spectra_layer &l, const int32_t *ids, int m, void *out,
                             int out_type, cudaStream_t s, const DeviceInfo &dev) {
-    const Geometry g = Geometry::of(l.n, l.k, l.n_outliers);
+    const bool bf16 = out_type == SPECTRA_BF16;
+    const size_t smem = (size_t)l.k * (bf16 ? 2 : 4);
+    if (smem > dev.smem_optin) return SPECTRA_ERR_SHAPE;
+    const Geometry g = Geometry::of(l.n, bulk_cols(l), l.n_outliers);
     EmbedArgs a;
     a.codes = reinterpret_cast<const uint4 *>(l.codes);
     a.scales = l.scales;
     a.zeros = l.zeros;
     a.oidx = l.outlier_idx;
-    a.outw = l.outlier_w;
+    a.outw = reinterpret_cast<const uint4 *>(l.outlier_w);
+    a.bidx = l.bulk_idx;
     a.ids = ids;
     a.out = out;
     a.n = l.n;
@@ -155,14 +223,18 @@ spectra_status launch_embed(const spectra_layer &l, const int32_t *ids, int m, v
     a.O8 = g.O8;
     a.n_o = l.n_outliers;
     a.m = m;
-    // one thread per group (rounded up to whole warps), one CTA per row up to
-    // a few waves of the device, the rest by grid stride
+    // a thread per bulk group (whole warps, at least 128 threads for the
+    // outlier octets and the row store), one CTA per row up to a few CTAs
+    // per SM, the rest by grid stride
     int threads = (int)cdiv(g.G, 32) * 32;
+    if (threads < 128) threads = 128;
     if (threads > kEmbedMaxThreads) threads = kEmbedMaxThreads;
     const int64_t cap = (int64_t)dev.sm_count * kEmbedCtasPerSm;
     const unsigned grid = (unsigned)(m < cap ? m : cap);
-    const cudaError_t e = out_type == SPECTRA_BF16 ? launch<true>(a, grid, (unsigned)threads, s)
-                                                   : launch<false>(a, grid, (unsigned)threads, s);
+    cudaError_t e = bf16 ? prepare<true>(dev) : prepare<false>(dev);
+    if (e != cudaSuccess) return SPECTRA_ERR_CUDA;
+    e = bf16 ? launch<true>(a, grid, (unsigned)threads, smem, s)
+             : launch<false>(a, grid, (unsigned)threads, smem, s);
     return e == cudaSuccess ? SPECTRA_OK : SPECTRA_ERR_CUDA;
 }
 

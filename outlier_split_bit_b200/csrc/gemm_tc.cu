@@ -170,7 +170,9 @@ __device__ __forceinline__ void tc_load_x(const Prob &a, int u, int tid, TcX<MB>
 #pragma unroll
         for (int i = 0; i < MB / 4; ++i) {
             const int c = tid + 128 * i, m = min(c % MB, a.m - 1), W = min(c / MB, nw - 1);
-            xp.v[i] = __ldg(reinterpret_cast<const uint4 *>(a.x + (size_t)m * a.k + 256 * u + 8 * W));
+            xp.v[i] = a.bidx == nullptr
+                          ? __ldg(reinterpret_cast<const uint4 *>(a.x + (size_t)m * a.kx + 256 * u + 8 * W))
+                          : bulk_x8_gather(a, m, 256 * u + 8 * W);
         }
     } else {
         const int ob = u - a.S;
@@ -182,7 +184,7 @@ __device__ __forceinline__ void tc_load_x(const Prob &a, int u, int tid, TcX<MB>
 #pragma unroll
             for (int e = 0; e < 8; ++e) ix[e] = (j0 + e < a.n_o) ? __ldg(a.oidx + j0 + e) : -1;
             // padding slots read column 0 and are zeroed when stored
-            const uint16_t *row = a.x + (size_t)min(m, a.m - 1) * a.k;
+            const uint16_t *row = a.x + (size_t)min(m, a.m - 1) * a.kx;
             uint32_t h[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) h[e] = (uint32_t)__ldg(row + max(ix[e], 0));
@@ -656,7 +658,7 @@ spectra_status run_tc(const Prob &a0, const DeviceInfo &dev, cudaStream_t s) {
 
 spectra_status launch_tc(const spectra_layer &l, const uint16_t *x, int m, void *y, int ytype,
                          cudaStream_t s, const DeviceInfo &dev) {
-    const Geometry g = Geometry::of(l.n, l.k, l.n_outliers);
+    const Geometry g = Geometry::of(l.n, bulk_cols(l), l.n_outliers);
     Prob a;
     fill_prob(a, l, g, x, m, y, ytype);
     return m <= 16 ? run_tc<TcCfg16>(a, dev, s) : run_tc<TcCfg32>(a, dev, s);

@@ -208,9 +208,14 @@ __device__ __forceinline__ void stage_x_load(const Prob &a, const XRange &xr, co
     {
         const int c = threadIdx.x, gl = c / MB, m = c - gl * MB, g = xr.g0 + gl;
         if (c < ng * MB && g < a.G && m < a.m) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)m * a.k + 32 * g);
+            if (a.bidx == nullptr) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)m * a.kx + 32 * g);
 #pragma unroll
-            for (int w = 0; w < 4; ++w) f.v0[w] = src[w];
+                for (int w = 0; w < 4; ++w) f.v0[w] = src[w];
+            } else {
+#pragma unroll
+                for (int w = 0; w < 4; ++w) f.v0[w] = bulk_x8_gather(a, m, 32 * g + 8 * w);
+            }
         }
     }
 #pragma unroll
@@ -218,8 +223,8 @@ __device__ __forceinline__ void stage_x_load(const Prob &a, const XRange &xr, co
         const int c = threadIdx.x + i * nth;
         const int m = c % MB;
         const bool mv = c < np * MB && m < a.m;
-        f.lo[i] = (mv && xi.i0[i] >= 0) ? a.x[(size_t)m * a.k + xi.i0[i]] : 0u;
-        f.hi[i] = (mv && xi.i1[i] >= 0) ? a.x[(size_t)m * a.k + xi.i1[i]] : 0u;
+        f.lo[i] = (mv && xi.i0[i] >= 0) ? a.x[(size_t)m * a.kx + xi.i0[i]] : 0u;
+        f.hi[i] = (mv && xi.i1[i] >= 0) ? a.x[(size_t)m * a.kx + xi.i1[i]] : 0u;
     }
 }
 
@@ -242,10 +247,13 @@ __device__ void stage_x_store(const Prob &a, const Stage<MB> &st, const XRange &
             if (c == (int)threadIdx.x) {
 #pragma unroll
                 for (int w = 0; w < 4; ++w) v[w] = f.v0[w];
-            } else {
-                const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)m * a.k + 32 * g);
+            } else if (a.bidx == nullptr) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)m * a.kx + 32 * g);
 #pragma unroll
                 for (int w = 0; w < 4; ++w) v[w] = src[w];
+            } else {
+#pragma unroll
+                for (int w = 0; w < 4; ++w) v[w] = bulk_x8_gather(a, m, 32 * g + 8 * w);
             }
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
@@ -287,8 +295,8 @@ __device__ void stage_x_store(const Prob &a, const Stage<MB> &st, const XRange &
             if (c < np * MB) {
                 const int m = c % MB;
                 const bool mv = m < a.m;
-                const uint32_t l = (i0[i] >= 0 && mv) ? a.x[(size_t)m * a.k + i0[i]] : 0u;
-                const uint32_t h = (i1[i] >= 0 && mv) ? a.x[(size_t)m * a.k + i1[i]] : 0u;
+                const uint32_t l = (i0[i] >= 0 && mv) ? a.x[(size_t)m * a.kx + i0[i]] : 0u;
+                const uint32_t h = (i1[i] >= 0 && mv) ? a.x[(size_t)m * a.kx + i1[i]] : 0u;
                 st.xo[c] = l | (h << 16);
             }
         }
@@ -1010,7 +1018,7 @@ spectra_status launch_gemv(const spectra_layer &l, const uint16_t *x, int m, voi
     // 8 or more batch rows: a real dense contraction, on the tensor cores
     // (measured faster than the CUDA-core decode from 8 rows on)
     if (m >= 8) return launch_tc(l, x, m, y, ytype, s, dev);
-    const Geometry g = Geometry::of(l.n, l.k, l.n_outliers);
+    const Geometry g = Geometry::of(l.n, bulk_cols(l), l.n_outliers);
     int done = 0;
     while (done < m) {
         const int mc = (m - done) > 8 ? 8 : (m - done);
@@ -1040,7 +1048,7 @@ spectra_status launch_gemv_batched(const spectra_layer *layers, const uint16_t *
     static PersistArgs args;  // large: kept off the stack, guarded by the mutex
     std::lock_guard<std::mutex> lock(mu);
     for (int i = 0; i < count; ++i) {
-        const Geometry g = Geometry::of(layers[i].n, layers[i].k, layers[i].n_outliers);
+        const Geometry g = Geometry::of(layers[i].n, bulk_cols(layers[i]), layers[i].n_outliers);
         fill_prob(args.probs[i], layers[i], g, xs[i], 1, ys[i], ytype);
     }
     return run_persistent<1>(args, count, dev, s);

@@ -47,6 +47,16 @@ struct Geometry {
     }
 };
 
+// Columns of a compacted bulk: the k - n_o non-outlier columns, padded to a
+// multiple of 32 and to at least one group.
+inline int compact_width(int k, int n_o) {
+    const int nb = k - n_o;
+    return nb <= 32 ? 32 : (int)cdiv(nb, 32) * 32;
+}
+
+// Columns of a layer's bulk (the geometry of its codes, scales and zeros).
+inline int bulk_cols(const spectra_layer &l) { return l.bulk_idx ? l.k_bulk : l.k; }
+
 // ---- packing (pack.cu) ----
 cudaError_t launch_kurtosis(const uint16_t *w, const float *gain, int n, int k, double *kappa,
                             int *err, cudaStream_t s);
@@ -55,6 +65,15 @@ cudaError_t launch_split(const double *kappa, int k, double tau, int32_t *idx, i
 cudaError_t launch_quantize_pack(const uint16_t *w, const Geometry &g, const int32_t *idx,
                                  uint8_t *codes, uint16_t *scales, uint32_t *zeros, int *err,
                                  cudaStream_t s);
+// Compacted bulk: the column list (validating idx) and the quantiser over
+// the bulk columns; `g` is the geometry of the bulk (k_bulk columns), `k` the
+// row stride of W.
+cudaError_t launch_bulk_columns(const int32_t *idx, int n_o, int k, int k_bulk, int32_t *bulk_idx,
+                                int *err, cudaStream_t s);
+cudaError_t launch_quantize_pack_compact(const uint16_t *w, int k, const Geometry &g,
+                                         const int32_t *bulk_idx, uint8_t *codes,
+                                         uint16_t *scales, uint32_t *zeros, int *err,
+                                         cudaStream_t s);
 cudaError_t launch_outlier_gather(const uint16_t *w, const Geometry &g, const int32_t *idx,
                                   uint16_t *outlier_w, cudaStream_t s);
 cudaError_t launch_unpack(const spectra_layer &l, uint8_t *codes, uint16_t *scales, uint8_t *zeros,

@@ -101,28 +101,65 @@ __device__ __forceinline__ double clamp015(double v) {
     return v < 0.0 ? 0.0 : (v > 15.0 ? 15.0 : v);
 }
 
+// Column list of a compacted bulk, one thread per column j of W: a
+// non-outlier column j is bulk column j - (number of outliers below j), found
+// by binary search in the ascending outlier list; positions from k - n_o to
+// k_bulk are padding (-1).  Threads j < n_o also check that the list is
+// strictly ascending within [0, k).  A bad list only ever writes inside
+// [0, k_bulk) and is reported through err.
+__global__ void __launch_bounds__(256) bulk_columns_kernel(const int32_t *__restrict__ idx,
+                                                           int n_o, int k, int k_bulk,
+                                                           int32_t *__restrict__ bulk_idx,
+                                                           int *__restrict__ err) {
+    const int j = blockIdx.x * blockDim.x + threadIdx.x;
+    if (j < n_o) {
+        const int c = idx[j];
+        if (c < 0 || c >= k || (j > 0 && idx[j - 1] >= c)) atomicOr(err, kErrBadIndex);
+    }
+    if (j < k) {
+        int lo = 0, hi = n_o;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (idx[mid] < j)
+                lo = mid + 1;
+            else
+                hi = mid;
+        }
+        const bool outlier = lo < n_o && idx[lo] == j;
+        const int p = j - lo;
+        if (!outlier && p >= 0 && p < k_bulk) bulk_idx[p] = j;
+    }
+    if (j >= k - n_o && j < k_bulk) bulk_idx[j] = -1;
+}
+
 // One thread per (tile t, super-group sg, lane r): quantises the 8 groups of
 // row 32t + r in that super-group and writes its 8 code records, one 16-byte
-// scale vector and one zero-point word.
+// scale vector and one zero-point word.  Masked bulk (kCompact false): `cols`
+// is the outlier list, whose columns read as +0.  Compacted bulk: `cols` is
+// the bulk column list, bulk column p of the row reads W[row][cols[p]] (+0
+// for padding); G and S count bulk groups and k is the row stride of W.
+template <bool kCompact>
 __global__ void __launch_bounds__(128) quantize_pack_kernel(
     const uint16_t *__restrict__ w, int n, int k, int T, int G, int S,
-    const int32_t *__restrict__ idx, int n_o, uint4 *__restrict__ codes,
+    const int32_t *__restrict__ cols, int n_o, uint4 *__restrict__ codes,
     uint4 *__restrict__ scales, uint32_t *__restrict__ zeros, int *__restrict__ err) {
-    extern __shared__ uint32_t omask[];  // k bits: outlier columns
-    const int words = k / 32;
-    for (int i = threadIdx.x; i < words; i += blockDim.x) omask[i] = 0u;
-    __syncthreads();
-    bool bad_idx = false;
-    for (int i = threadIdx.x; i < n_o; i += blockDim.x) {
-        const int j = idx[i];
-        if (j < 0 || j >= k || (i > 0 && idx[i - 1] >= j)) {
-            bad_idx = true;
-        } else {
-            atomicOr(&omask[j >> 5], 1u << (j & 31));
+    extern __shared__ uint32_t omask[];  // masked: k bits, the outlier columns
+    if constexpr (!kCompact) {
+        const int words = k / 32;
+        for (int i = threadIdx.x; i < words; i += blockDim.x) omask[i] = 0u;
+        __syncthreads();
+        bool bad_idx = false;
+        for (int i = threadIdx.x; i < n_o; i += blockDim.x) {
+            const int j = cols[i];
+            if (j < 0 || j >= k || (i > 0 && cols[i - 1] >= j)) {
+                bad_idx = true;
+            } else {
+                atomicOr(&omask[j >> 5], 1u << (j & 31));
+            }
         }
+        __syncthreads();
+        if (bad_idx) atomicOr(err, kErrBadIndex);
     }
-    __syncthreads();
-    if (bad_idx) atomicOr(err, kErrBadIndex);
 
     const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;  // (t, sg) pair
     const int r = threadIdx.x & 31;
@@ -137,22 +174,33 @@ __global__ void __launch_bounds__(128) quantize_pack_kernel(
         if (g >= G) break;
         uint32_t rec[4] = {0u, 0u, 0u, 0u};
         if (row < n) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(w + (size_t)row * k + 32 * g);
-            uint32_t raw[16];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint4 u = src[q];
-                raw[4 * q + 0] = u.x; raw[4 * q + 1] = u.y;
-                raw[4 * q + 2] = u.z; raw[4 * q + 3] = u.w;
-            }
-            const uint32_t m = omask[g];
             double v[32];
+            if constexpr (kCompact) {
+                const int32_t *bc = cols + 32 * g;
 #pragma unroll
-            for (int kk = 0; kk < 32; ++kk) {
-                const uint32_t b = (kk & 1) ? (raw[kk >> 1] >> 16) : (raw[kk >> 1] & 0xFFFFu);
-                if (bf16_nonfinite(b)) flags |= kErrNonfinite;
-                const double x = ((m >> kk) & 1u) ? 0.0 : bf16_to_double(b);
-                v[kk] = __dadd_rn(x, 0.0);  // -0 + +0 = +0
+                for (int kk = 0; kk < 32; ++kk) {
+                    const int c = bc[kk];
+                    const uint32_t b = (c >= 0 && c < k) ? (uint32_t)w[(size_t)row * k + c] : 0u;
+                    if (bf16_nonfinite(b)) flags |= kErrNonfinite;
+                    v[kk] = __dadd_rn(bf16_to_double(b), 0.0);  // -0 + +0 = +0
+                }
+            } else {
+                const uint4 *src = reinterpret_cast<const uint4 *>(w + (size_t)row * k + 32 * g);
+                uint32_t raw[16];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 u = src[q];
+                    raw[4 * q + 0] = u.x; raw[4 * q + 1] = u.y;
+                    raw[4 * q + 2] = u.z; raw[4 * q + 3] = u.w;
+                }
+                const uint32_t m = omask[g];
+#pragma unroll
+                for (int kk = 0; kk < 32; ++kk) {
+                    const uint32_t b = (kk & 1) ? (raw[kk >> 1] >> 16) : (raw[kk >> 1] & 0xFFFFu);
+                    if (bf16_nonfinite(b)) flags |= kErrNonfinite;
+                    const double x = ((m >> kk) & 1u) ? 0.0 : bf16_to_double(b);
+                    v[kk] = __dadd_rn(x, 0.0);  // -0 + +0 = +0
+                }
             }
             double lo = v[0], hi = v[0];
 #pragma unroll
@@ -252,12 +300,29 @@ cudaError_t launch_quantize_pack(const uint16_t *w, const Geometry &g, const int
     const int64_t threads = (int64_t)g.T * g.S * 32;
     const size_t smem = (size_t)(g.k / 32) * sizeof(uint32_t);
     if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(quantize_pack_kernel,
+        cudaError_t e = cudaFuncSetAttribute(quantize_pack_kernel<false>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    quantize_pack_kernel<<<(unsigned)cdiv(threads, 128), 128, smem, s>>>(
+    quantize_pack_kernel<false><<<(unsigned)cdiv(threads, 128), 128, smem, s>>>(
         w, g.n, g.k, g.T, g.G, g.S, idx, g.n_o, reinterpret_cast<uint4 *>(codes),
+        reinterpret_cast<uint4 *>(scales), zeros, err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bulk_columns(const int32_t *idx, int n_o, int k, int k_bulk, int32_t *bulk_idx,
+                                int *err, cudaStream_t s) {
+    bulk_columns_kernel<<<(unsigned)cdiv(k, 256), 256, 0, s>>>(idx, n_o, k, k_bulk, bulk_idx, err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_pack_compact(const uint16_t *w, int k, const Geometry &g,
+                                         const int32_t *bulk_idx, uint8_t *codes,
+                                         uint16_t *scales, uint32_t *zeros, int *err,
+                                         cudaStream_t s) {
+    const int64_t threads = (int64_t)g.T * g.S * 32;
+    quantize_pack_kernel<true><<<(unsigned)cdiv(threads, 128), 128, 0, s>>>(
+        w, g.n, k, g.T, g.G, g.S, bulk_idx, 0, reinterpret_cast<uint4 *>(codes),
         reinterpret_cast<uint4 *>(scales), zeros, err);
     return cudaGetLastError();
 }
@@ -273,10 +338,10 @@ cudaError_t launch_outlier_gather(const uint16_t *w, const Geometry &g, const in
 
 cudaError_t launch_unpack(const spectra_layer &l, uint8_t *codes, uint16_t *scales, uint8_t *zeros,
                           cudaStream_t s) {
-    const Geometry g = Geometry::of(l.n, l.k, l.n_outliers);
+    const Geometry g = Geometry::of(l.n, bulk_cols(l), l.n_outliers);
     const int64_t threads = (int64_t)l.n * g.G;
     unpack_kernel<<<(unsigned)cdiv(threads, 128), 128, 0, s>>>(
-        reinterpret_cast<const uint4 *>(l.codes), l.scales, l.zeros, l.n, l.k, g.G, g.S, codes,
+        reinterpret_cast<const uint4 *>(l.codes), l.scales, l.zeros, l.n, g.k, g.G, g.S, codes,
         scales, zeros);
     return cudaGetLastError();
 }

@@ -39,8 +39,10 @@ struct Prob {
     const uint4 *outw;
     const int32_t *oidx;
     const uint16_t *x;
+    const int32_t *bidx;  // bulk column list of a compacted bulk, nullptr when masked
     void *y;
-    int n, k, m, G, S, O8, n_o, T;
+    int n, k, m, G, S, O8, n_o, T;  // k: bulk columns (the geometry of the codes)
+    int kx;                         // columns of x (its row stride)
     int U;         // units per tile
     int ppc, tpc;  // slices per tile, tiles per CTA item
     int lgp;       // log2(ppc) where ppc is a power of two (persistent kernel)
@@ -130,6 +132,21 @@ __device__ __forceinline__ void issue_unit(const Prob &a, int t, int u, uint32_t
 template <int sh>
 __device__ __forceinline__ uint32_t code_pair(uint32_t w) {
     return ((w >> (4 * sh)) & 0x000F000Fu) | 0x43004300u;
+}
+
+// x of 8 consecutive columns c0..c0+7 of a compacted bulk for batch row m,
+// as 4 BF16 pairs in column order: gathered through the bulk column list,
+// padding (and any entry outside [0, kx)) read as +0.  c0 is a multiple of 8.
+__device__ __forceinline__ uint4 bulk_x8_gather(const Prob &a, int m, int c0) {
+    const uint16_t *xr = a.x + (size_t)m * a.kx;
+    const int4 b0 = __ldg(reinterpret_cast<const int4 *>(a.bidx + c0));
+    const int4 b1 = __ldg(reinterpret_cast<const int4 *>(a.bidx + c0 + 4));
+    const int c[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+    uint32_t h[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) h[e] = ((unsigned)c[e] < (unsigned)a.kx) ? (uint32_t)xr[c[e]] : 0u;
+    return make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16),
+                      h[6] | (h[7] << 16));
 }
 
 __device__ __forceinline__ void store_y(const Prob &a, int t, int lane, int m, float v) {
@@ -232,9 +249,11 @@ void fill_prob(Prob &a, const spectra_layer &l, const Geometry &g, const uint16_
     a.outw = reinterpret_cast<const uint4 *>(l.outlier_w);
     a.oidx = l.outlier_idx;
     a.x = x;
+    a.bidx = l.bulk_idx;
     a.y = y;
     a.n = l.n;
-    a.k = l.k;
+    a.k = g.k;
+    a.kx = l.k;
     a.m = mc;
     a.G = g.G;
     a.S = g.S;

@@ -84,23 +84,24 @@ def check_gemv(y_gpu: torch.Tensor, y_ref: np.ndarray, bound: np.ndarray, bf16: 
     return float((err / tol).max())
 
 
-_SPLIT_CACHE = {}
+_KAPPA_CACHE = {}
 
 
 def oracle_split(wb: np.ndarray, gain, tau: float, key=None):
     """The oracle's kurtosis and outlier indices of a large matrix.  Kurtosis
     is computed per column, so the oracle is called on contiguous blocks of 64
     columns (the same values, read with unit stride instead of one cache miss
-    per element).  `key` caches the result for matrices drawn more than once."""
-    if key is not None and (key, tau) in _SPLIT_CACHE:
-        return _SPLIT_CACHE[(key, tau)]
-    k = wb.shape[1]
-    kap = np.empty(k, dtype=np.float64)
-    for j0 in range(0, k, 64):
-        j1 = min(k, j0 + 64)
-        kap[j0:j1] = oracle.kurtosis(np.ascontiguousarray(wb[:, j0:j1]),
-                                     None if gain is None else gain[j0:j1])
-    out = (kap, oracle.split(kap, tau))
-    if key is not None:
-        _SPLIT_CACHE[(key, tau)] = out
-    return out
+    per element).  `key` caches the kurtosis of a matrix drawn more than once
+    (it does not depend on tau)."""
+    if key is not None and key in _KAPPA_CACHE:
+        kap = _KAPPA_CACHE[key]
+    else:
+        k = wb.shape[1]
+        kap = np.empty(k, dtype=np.float64)
+        for j0 in range(0, k, 64):
+            j1 = min(k, j0 + 64)
+            kap[j0:j1] = oracle.kurtosis(np.ascontiguousarray(wb[:, j0:j1]),
+                                         None if gain is None else gain[j0:j1])
+        if key is not None:
+            _KAPPA_CACHE[key] = kap
+    return kap, oracle.split(kap, tau)

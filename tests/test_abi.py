@@ -153,3 +153,39 @@ def test_embed_argument_checks(L):
     assert L.spectra_embed(lay, FAKE, 1, FAKE + 4, 1, None) == _lib.ERR_ALIGN
     # no rows: nothing to do, and CUDA is never touched (this machine may have no GPU)
     assert L.spectra_embed(lay, None, 0, None, 1, None) == _lib.OK
+
+
+def test_packed_sizes_compact(L):
+    s = _lib.Sizes()
+    assert L.spectra_packed_sizes_compact(512, 512, 100, ctypes.byref(s)) == _lib.OK
+    assert s.k_bulk == 416 and s.bulk_idx_bytes == 416 * 4
+    assert s.codes_bytes == 512 * 416 // 2 and s.scales_bytes == 512 * 2 * 8 * 2
+    assert s.zeros_bytes == 512 * 2 * 4 and s.outlier_w_bytes == 512 * 13 * 8 * 2
+    assert L.spectra_packed_sizes_compact(40, 96, 96, ctypes.byref(s)) == _lib.OK
+    assert s.k_bulk == 32 and s.n_pad == 64  # every column BF16: one all-zero group
+    assert L.spectra_packed_sizes_compact(40, 96, 70, ctypes.byref(s)) == _lib.OK
+    assert s.k_bulk == 32
+    assert L.spectra_packed_sizes_compact(40, 96, 0, ctypes.byref(s)) == _lib.OK
+    assert s.k_bulk == 96
+    assert L.spectra_packed_sizes(40, 96, 3, ctypes.byref(s)) == _lib.OK
+    assert s.k_bulk == 96 and s.bulk_idx_bytes == 0
+    assert L.spectra_packed_sizes_compact(40, 96, 97, ctypes.byref(s)) == _lib.ERR_INVALID_ARG
+
+
+def test_compacted_layer_checks(L):
+    y = FAKE
+    # a compacted view's k_bulk must be max(32, ceil32(k - n_outliers)): 128 here
+    bad = _lib.Layer(64, 128, 3, FAKE, FAKE, FAKE, FAKE, FAKE, 96, FAKE)
+    assert L.spectra_gemv(ctypes.byref(bad), FAKE, y, 0, None) == _lib.ERR_INVALID_ARG
+    bad = _lib.Layer(64, 128, 40, FAKE, FAKE, FAKE, FAKE, FAKE, 96, FAKE + 4)
+    assert L.spectra_gemv(ctypes.byref(bad), FAKE, y, 0, None) == _lib.ERR_ALIGN
+    bad = _lib.Layer(64, 128, 3, FAKE, FAKE, FAKE, FAKE, FAKE, 7, None)  # masked: 0 or k
+    assert L.spectra_gemv(ctypes.byref(bad), FAKE, y, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.spectra_embed(ctypes.byref(bad), FAKE, 1, FAKE, 0, None) == _lib.ERR_INVALID_ARG
+    wsb = L.spectra_pack_workspace_size()
+    assert L.spectra_pack_compact(FAKE, 8, 128, FAKE, 2, FAKE, FAKE, FAKE, FAKE, None, FAKE, wsb,
+                                  None, None) == _lib.ERR_INVALID_ARG
+    assert L.spectra_pack_compact(FAKE, 8, 128, FAKE, 2, FAKE, FAKE, FAKE, FAKE, FAKE + 4, FAKE,
+                                  wsb, None, None) == _lib.ERR_ALIGN
+    assert L.spectra_pack_compact(FAKE, 8, 120, FAKE, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, wsb,
+                                  None, None) == _lib.ERR_SHAPE
