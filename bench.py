@@ -513,6 +513,11 @@ def job_gbs(bytes_per_rank_step: int, steps: int, world: int, max_ms: float) -> 
 
 # ---------------------------------------------------------------- our arm
 
+# committed ncu summaries of the stream launch's DRAM traffic (masked and
+# compacted bulk), machine-read for roofline.traffic
+TRAFFIC_PROFILES = ("gemv_decode_stream_traffic.md", "gemv_decode_stream_compact_traffic.md")
+
+
 def kernel_source_digest() -> str:
     """Digest of the source the matvec kernels are compiled from (gemv.cu and
     the streaming machinery it includes); the tensor-core kernel lives apart."""
@@ -528,23 +533,25 @@ def profiled_traffic(digest: str, algorithmic_bytes=None):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the current kernel source and (when given) on a launch with the same
     algorithmic bytes, i.e. the same workload and threshold."""
-    p = os.path.join(ROOT, "profiles", "gemv_decode_stream_traffic.md")
-    if not os.path.exists(p):
-        return None
-    vals = {}
-    for line in open(p):
-        if ":" in line and line.startswith("- "):
-            k, v = line[2:].split(":", 1)
-            vals[k.strip()] = v.strip().strip("`")
-    if vals.get("kernel_source_sha256_16") != digest:
-        return None
-    try:
-        if algorithmic_bytes is not None and \
-                int(vals["algorithmic_bytes_per_launch"]) != int(algorithmic_bytes):
-            return None
-        return float(vals["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
-        return None
+    for name in TRAFFIC_PROFILES:
+        p = os.path.join(ROOT, "profiles", name)
+        if not os.path.exists(p):
+            continue
+        vals = {}
+        for line in open(p):
+            if ":" in line and line.startswith("- "):
+                k, v = line[2:].split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+        if vals.get("kernel_source_sha256_16") != digest:
+            continue
+        try:
+            if algorithmic_bytes is not None and \
+                    int(vals["algorithmic_bytes_per_launch"]) != int(algorithmic_bytes):
+                continue
+            return float(vals["dram_bytes_per_launch"])
+        except (KeyError, ValueError):
+            continue
+    return None
 
 
 def run_ours(args):
@@ -565,7 +572,7 @@ def run_ours(args):
     peaks = measured_peaks()
     peak = float(peaks["hbm_gbs"])
     stream = torch.cuda.Stream(device=device)
-    st = Stream(device, seed=rank, tau=args.tau)
+    st = Stream(device, seed=rank, tau=args.tau, compact=args.compact)
     graph, launches_per_step = st.capture(stream, "batched")
     for _ in range(args.warmup):
         graph.replay()
@@ -659,14 +666,14 @@ def run_ours(args):
         "gbs": round(st.bytes / (chain_ms * 1e-3) * 1e-9, 1),
         "frac": round(st.bytes / (chain_ms * 1e-3) * 1e-9 / peak, 4),
         "us_per_launch": round(chain_ms * 1e3 / chain_launches, 3)}}
-    if rank == 0 and not args.quick:
+    if rank == 0 and not args.quick and not args.compact:
         # the same stream with the outlier columns removed from the 4-bit bulk
         st_c = Stream(device, seed=rank, tau=args.tau, compact=True)
         graph_c, _ = st_c.capture(stream, "batched")
         for _ in range(args.warmup):
             graph_c.replay()
         stream.synchronize()
-        c_steps = max(3, min(args.steps, 500))
+        c_steps = max(50, min(args.steps, 500))
         with torch.cuda.stream(stream):
             c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             c0.record(stream)
@@ -683,6 +690,7 @@ def run_ours(args):
             "bytes_per_step_masked_bulk": st.bytes,
             "steps": c_steps}
         del graph_c, st_c
+    if rank == 0 and not args.quick:
         extra.update(extras(device, stream, peak, args.tau))
 
     cpu = None
@@ -712,6 +720,8 @@ def run_ours(args):
             "config": {"workload": WORKLOAD, "matrices_per_step": st.launches,
                        "bytes_per_step": st.bytes, "n_outliers_per_step": st.n_outliers,
                        "tau": args.tau, "m": 1,
+                       "bulk": "compacted (outlier columns removed)" if args.compact
+                               else "masked (outlier columns set to +0 in place)",
                        "launch": "one spectra_gemv_batched launch per step (CUDA graph replay)",
                        "l2": "inputs larger than L2 (0.76 GB of packed weights per step)",
                        "parallelism": f"replicas x{world}"},
@@ -747,7 +757,7 @@ def run_single(args):
     spec = wl.MatrixSpec("lm_head", args.n, args.k, args.nt)
     w = wl.weight(spec, 0, 0, device=device)
     g = wl.gain(spec, 0, 0, device=device)
-    lay = sp.pack_layer(w, g, args.tau)
+    lay = sp.pack_layer(w, g, args.tau, compact=args.compact)
     del w
     x = wl.activations(spec.k, args.m, device=device)
     y = torch.empty((args.m, spec.n), device=device)
@@ -760,11 +770,45 @@ def run_single(args):
         for _ in range(args.warmup):
             fn()
         us, p10, p90 = time_single(fn, stream, args.steps, flush)
-    b = algorithmic_bytes(spec.n, spec.k, lay.n_outliers, m=args.m)
+    b = layer_bytes(lay, m=args.m)
     print(json.dumps({"case": "single", "n": spec.n, "k": spec.k, "m": args.m, "tau": args.tau,
+                      "compact": args.compact,
                       "n_outliers": lay.n_outliers, "us": round(us, 2), "us_p10": round(p10, 2),
                       "us_p90": round(p90, 2), "bytes": b, "gbs": round(b / us * 1e-3, 1),
                       "frac": round(b / us * 1e-3 / peak, 4)}), flush=True)
+    return 0
+
+
+def run_embed(args):
+    """Embedding-row gather of m random ids from an n x k packed table (BF16
+    rows out), timed alone with L2 flushed before every launch; prints one
+    JSON line.  Also the small case of profiler captures of the gather."""
+    import outlier_split_bit_b200 as sp
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    peak = float(measured_peaks()["hbm_gbs"])
+    spec = wl.MatrixSpec("lm_head", args.n, args.k, args.nt)
+    w = wl.weight(spec, 0, 0, device=device)
+    g = wl.gain(spec, 0, 0, device=device)
+    lay = sp.pack_layer(w, g, args.tau, compact=args.compact)
+    del w
+    ids = torch.from_numpy(np.random.default_rng(args.m).integers(0, spec.n, args.m)
+                           .astype(np.int32)).to(device)
+    out = torch.empty((args.m, spec.k), dtype=torch.bfloat16, device=device)
+    v = lay.view()
+    stream = torch.cuda.Stream(device=device)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+    fn = lambda: sp.spectra_embed(lay, ids, out, view=v, stream=stream)  # noqa: E731
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            fn()
+        us, p10, p90 = time_single(fn, stream, args.steps, flush)
+    b = embed_bytes(spec.k, lay.n_outliers, args.m)
+    print(json.dumps({"case": "embed", "n": spec.n, "k": spec.k, "m": args.m, "tau": args.tau,
+                      "compact": args.compact, "n_outliers": lay.n_outliers, "us": round(us, 2),
+                      "us_p10": round(p10, 2), "us_p90": round(p90, 2), "bytes": b,
+                      "gbs": round(b / us * 1e-3, 1), "frac": round(b / us * 1e-3 / peak, 4)}),
+          flush=True)
     return 0
 
 
@@ -777,8 +821,11 @@ def main():
     ap.add_argument("--tau", type=float, default=3.0)
     ap.add_argument("--quick", action="store_true", help="skip the per-matrix / LM-head / batch rows")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["stream", "single"], default="stream",
-                    help="stream: the decode-step weight stream (the benchmark); single: one matrix")
+    ap.add_argument("--case", choices=["stream", "single", "embed"], default="stream",
+                    help="stream: the decode-step weight stream (the benchmark); single: one "
+                         "matrix; embed: the embedding-row gather of --m ids")
+    ap.add_argument("--compact", action="store_true",
+                    help="pack with the outlier columns removed from the 4-bit bulk")
     ap.add_argument("--n", type=int, default=wl.LM_HEAD_N)
     ap.add_argument("--k", type=int, default=wl.LM_HEAD_K)
     ap.add_argument("--nt", type=int, default=0, help="Student-t columns of the single matrix")
@@ -790,6 +837,8 @@ def main():
         return run_reference(args)
     if args.case == "single":
         return run_single(args)
+    if args.case == "embed":
+        return run_embed(args)
     return run_ours(args)
 
 

@@ -9,8 +9,8 @@
  * 4-bit codes with one FP16 scale and one bit-packed 4-bit zero point per
  * group of 32 consecutive weights of a row.  Decoding happens in registers
  * inside the matrix-vector kernel, which also runs the dense matvec of the
- * BF16 outlier columns in the same pass (abstract: fused dequantisation
- * "within register pipelines").
+ * BF16 outlier columns in the same pass (abstract: the dequantisation is
+ * fused into the kernels' register pipelines).
  *
  * Conventions shared by every entry point:
  *   - All pointers named *_dev or documented as "device" are CUDA device
@@ -304,8 +304,8 @@ SPECTRA_API spectra_status spectra_gemv_batched(const spectra_layer *layers,
                                                 void *stream);
 
 /*
- * Embedding-row gather over a packed table (abstract: "Dynamic vocabulary
- * embedding dequantization (SpectraFusedEmbedding)"; highlight 5: vocabulary
+ * Embedding-row gather over a packed table (abstract: SpectraFusedEmbedding,
+ * dequantisation of vocabulary embeddings on demand; highlight 5: vocabulary
  * tables stored in the 4-bit Group-32 format, rows gathered and dequantised
  * during the forward pass).
  *   table  HOST struct viewing a packed layer of the table E[n][k] (n =

@@ -117,7 +117,7 @@ static int is_finite_bf16(uint16_t b) { return ((b >> 7) & 0xFF) != 0xFF; }
 /*
  * Pearson kurtosis (m4 / m2^2, population moments, not excess) of each
  * column of the gain-scaled matrix a[i][j] = W[i][j] * g[j]
- * (abstract: "fourth-moment kurtosis", computed with the upstream
+ * (abstract: the channel's fourth-moment kurtosis, computed with the upstream
  * normalisation gain).  gain == NULL means g = 1.
  * Order: S = sum_i a_i (i ascending), mu = S/N; then for i ascending
  * d = a_i - mu, q = d*d, m2 += q, m4 += q*q; m2 /= N, m4 /= N,
