@@ -2,7 +2,7 @@
 //
 // Method: "SPECTRA: Sparse-Precision Exact Channel Tensor Reconstruction
 // Architecture" (Dev.to abstract), abstract paragraph and highlight 5
-// ("SpectraFusedEmbedding"): vocabulary tables stay in the 4-bit Group-32
+// (SpectraFusedEmbedding): vocabulary tables stay in the 4-bit Group-32
 // format and the rows a forward pass needs are gathered and dequantised on
 // the fly.  The table is a packed layer like any other (n = vocabulary rows,
 // k = hidden columns, outlier columns kept bit-exact in BF16), so a tied
