@@ -89,7 +89,9 @@ typedef enum {
     SPECTRA_ERR_BUFFER_TOO_SMALL = 6, /* workspace smaller than the stated size */
     SPECTRA_ERR_CUDA = 7,             /* a CUDA runtime call failed */
     SPECTRA_ERR_UNSUPPORTED = 8,      /* the current device is not compute capability 10.0 */
-    SPECTRA_ERR_INTERNAL = 9          /* a kernel reported an inconsistent state */
+    SPECTRA_ERR_INTERNAL = 9,         /* a kernel reported an inconsistent state */
+    SPECTRA_ERR_IO = 10,              /* a container file could not be opened, read or written */
+    SPECTRA_ERR_FORMAT = 11           /* a container is not TRDC, is truncated, or fails a checksum */
 } spectra_status;
 
 typedef enum { SPECTRA_F32 = 0, SPECTRA_BF16 = 1 } spectra_dtype;
@@ -340,6 +342,114 @@ SPECTRA_API spectra_status spectra_embed(const spectra_layer *table, const int32
  * SPECTRA_OK otherwise.  Synchronous on `stream`.
  */
 SPECTRA_API spectra_status spectra_device_status(void *stream);
+
+/*
+ * TRDC container (abstract: every weight, scale and offset is serialised
+ * into one self-contained binary container that is streamed straight into
+ * GPU memory, so that initialisation has a bounded memory spike).  The
+ * pages give no byte format; this one is the library's own.  Little-endian
+ * throughout:
+ *   file header, 64 bytes:
+ *     0  "TRDC"   4  u32 version (1)   8  u32 layer count L
+ *     12 u32 header bytes H = 64 + 256 * L   16 u64 file bytes
+ *     24 u32 CRC-32 of the L layer records   28..63 zero
+ *   L layer records of 256 bytes each, from byte 64:
+ *     0   name, 96 bytes, NUL-padded (at most 95 characters)
+ *     96  i32 n, i32 k, i32 n_outliers, i32 k_bulk (0: masked bulk)
+ *     112 f64 tau (the threshold the layer was split at; informative)
+ *     120 u32 flags (bit 0: compacted bulk), u32 zero
+ *     128 six (u64 offset, u64 bytes) pairs: codes, scales, zeros,
+ *         outlier_idx, outlier_w, bulk_idx (bytes 0 where absent)
+ *     224 six u32 CRC-32 of those buffers (0 where absent)
+ *     248 u64 zero
+ *   buffers at offsets that are multiples of 4096, in layer and buffer
+ *   order, zero padding between them; their sizes are those of
+ *   spectra_packed_sizes (masked) or spectra_packed_sizes_compact.
+ * CRC-32 is the IEEE 802.3 polynomial, reflected (0xEDB88320), initial and
+ * final XOR 0xFFFFFFFF (the checksum of zlib and PNG).
+ *
+ * Host memory: every entry streams through a caller-owned staging buffer
+ * (pinned host memory for device transfers) in chunks of half its size,
+ * double-buffered (the file read of one chunk overlaps the copy of the
+ * other).  The library allocates no host memory proportional to the
+ * model: only the reader handle (the layer records).
+ */
+typedef enum { SPECTRA_MEM_DEVICE = 0, SPECTRA_MEM_HOST = 1 } spectra_memory;
+
+/* The 256-byte layer record of a container, as read. */
+typedef struct {
+    char name[96];
+    int32_t n, k, n_outliers, k_bulk;
+    double tau;
+    uint32_t flags;
+    uint64_t offset[6];
+    uint64_t bytes[6];
+    uint32_t crc32[6];
+} spectra_trdc_layer;
+
+/* Opaque reader handle. */
+typedef struct spectra_trdc spectra_trdc;
+
+/* CRC-32 of a host buffer (as stored in containers); `crc` is 0 to start. */
+SPECTRA_API uint32_t spectra_crc32(uint32_t crc, const void *data, size_t bytes);
+
+/*
+ * Write a container of `count` packed layers.
+ *   path     HOST string; the file is created or truncated
+ *   names    HOST array [count] of NUL-terminated names (< 96 bytes each)
+ *   layers   HOST array [count] of layer views; their buffers are device
+ *            memory (mem = SPECTRA_MEM_DEVICE) or host memory
+ *            (SPECTRA_MEM_HOST: no CUDA call is made)
+ *   taus     HOST array [count], or NULL (stored as 0)
+ *   staging  HOST buffer of staging_bytes (>= 8192, pinned for device
+ *            memory); buffers move through it in chunks of half its size.
+ *            Required for device memory; for host memory it may be NULL
+ *            (buffers are written directly) or given (same chunked path)
+ * Synchronous (device copies run on `stream`).  Errors: INVALID_ARG,
+ * SHAPE, BUFFER_TOO_SMALL, IO, CUDA.
+ */
+SPECTRA_API spectra_status spectra_trdc_write(const char *path, int32_t count,
+                                              const char *const *names,
+                                              const spectra_layer *layers, const double *taus,
+                                              spectra_memory mem, void *staging,
+                                              size_t staging_bytes, void *stream);
+
+/*
+ * Open a container: reads and checks the header and the layer records
+ * (magic, version, record checksum, every layer's shape, buffer sizes and
+ * offsets within the file).  *out receives a handle to release with
+ * spectra_trdc_close.  Errors: INVALID_ARG, IO, FORMAT.
+ */
+SPECTRA_API spectra_status spectra_trdc_open(const char *path, spectra_trdc **out);
+
+/* Number of layers in an open container (0 for NULL). */
+SPECTRA_API int32_t spectra_trdc_count(const spectra_trdc *t);
+
+/* Record of layer i (INVALID_ARG when i is out of range). */
+SPECTRA_API spectra_status spectra_trdc_info(const spectra_trdc *t, int32_t i,
+                                             spectra_trdc_layer *out);
+
+/*
+ * Stream layer i into caller-allocated buffers sized by its record
+ * (codes, scales, zeros; outlier_idx and outlier_w when n_outliers > 0;
+ * bulk_idx when compacted; the others may be NULL), in device memory
+ * (mem = SPECTRA_MEM_DEVICE, 16-byte aligned) or host memory
+ * (SPECTRA_MEM_HOST: no CUDA call).  staging as for spectra_trdc_write
+ * (required for device memory, optional for host memory).  verify != 0
+ * checks every buffer's
+ * CRC-32 while it streams (FORMAT on a mismatch).  layer_out (HOST, may be
+ * NULL) receives the view of the loaded buffers.  Synchronous.  Errors:
+ * INVALID_ARG, ALIGN, BUFFER_TOO_SMALL, IO, FORMAT, CUDA.
+ */
+SPECTRA_API spectra_status spectra_trdc_load(const spectra_trdc *t, int32_t i, uint8_t *codes,
+                                             uint16_t *scales, uint32_t *zeros,
+                                             int32_t *outlier_idx, uint16_t *outlier_w,
+                                             int32_t *bulk_idx, spectra_memory mem,
+                                             void *staging, size_t staging_bytes, int32_t verify,
+                                             spectra_layer *layer_out, void *stream);
+
+/* Release a reader handle (NULL is ignored). */
+SPECTRA_API void spectra_trdc_close(spectra_trdc *t);
 
 #ifdef __cplusplus
 }

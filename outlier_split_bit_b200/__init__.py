@@ -18,14 +18,14 @@ from dataclasses import dataclass
 import torch
 
 from . import _lib
-from ._lib import Layer, Sizes
+from ._lib import Layer, Sizes, TrdcLayer
 
 __all__ = ["SpectraError", "PackedLayer", "spectra_status_string", "spectra_version",
            "spectra_packed_sizes", "spectra_packed_sizes_compact", "spectra_pack_plan",
            "spectra_pack", "spectra_pack_compact", "spectra_unpack",
            "spectra_gemv", "spectra_gemm_small", "spectra_gemv_batched", "spectra_embed",
            "spectra_device_status",
-           "pack_layer", "library"]
+           "pack_layer", "library", "spectra_crc32", "write_container", "Container"]
 
 class _Lazy:
     """Loads libspectra.so on first attribute access."""
@@ -285,3 +285,90 @@ def spectra_gemv_batched(layers=None, xs=None, ys=None, *, views: BatchViews | N
     _check(_L.spectra_gemv_batched(v.layers, v.xs, v.ys, v.count, v.y_dtype, _stream(stream)),
            "spectra_gemv_batched")
     return v
+
+
+# ---------------------------------------------------------------- TRDC container
+
+_BUFFERS = ("codes", "scales", "zeros", "outlier_idx", "outlier_w", "bulk_idx")
+
+
+def spectra_crc32(data, crc: int = 0) -> int:
+    """CRC-32 of a bytes-like object (the checksum stored in containers)."""
+    buf = (ctypes.c_char * len(data)).from_buffer_copy(bytes(data))
+    return int(_L.spectra_crc32(crc, buf, len(data)))
+
+
+def _pinned(nbytes: int) -> torch.Tensor:
+    return torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+
+
+def write_container(path: str, layers, names, taus=None, *, staging_bytes: int = 64 << 20,
+                    stream=None) -> None:
+    """Write packed layers (device buffers) into a TRDC container, streaming
+    them through a pinned staging buffer of staging_bytes."""
+    n = len(layers)
+    views = (Layer * n)(*[l.view() for l in layers])
+    cnames = (ctypes.c_char_p * n)(*[nm.encode() for nm in names])
+    ctaus = (ctypes.c_double * n)(*(taus if taus is not None else [0.0] * n))
+    staging = _pinned(staging_bytes)
+    _check(_L.spectra_trdc_write(str(path).encode(), n, cnames, views, ctaus, _lib.MEM_DEVICE,
+                                 _ptr(staging), staging_bytes, _stream(stream)),
+           "spectra_trdc_write")
+
+
+class Container:
+    """An open TRDC container: layer records, and layers streamed into device
+    buffers that this binding allocates with torch."""
+
+    def __init__(self, path: str):
+        h = ctypes.c_void_p()
+        _check(_L.spectra_trdc_open(str(path).encode(), ctypes.byref(h)), "spectra_trdc_open")
+        self._h = h
+
+    def close(self):
+        if self._h:
+            _L.spectra_trdc_close(self._h)
+            self._h = None
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        self.close()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __len__(self) -> int:
+        return int(_L.spectra_trdc_count(self._h))
+
+    def info(self, i: int) -> dict:
+        r = TrdcLayer()
+        _check(_L.spectra_trdc_info(self._h, i, ctypes.byref(r)), "spectra_trdc_info")
+        return {"name": r.name.decode(), "n": r.n, "k": r.k, "n_outliers": r.n_outliers,
+                "k_bulk": r.k_bulk, "tau": r.tau, "compact": bool(r.flags & 1),
+                "offset": list(r.offset), "bytes": list(r.bytes), "crc32": list(r.crc32)}
+
+    def load(self, i: int, device="cuda", *, staging: torch.Tensor | None = None,
+             staging_bytes: int = 64 << 20, verify: bool = True, stream=None) -> PackedLayer:
+        """Stream layer i into new device buffers; returns the PackedLayer."""
+        inf = self.info(i)
+        nb = dict(zip(_BUFFERS, inf["bytes"]))
+        codes = _alloc(nb["codes"], torch.uint8, device)
+        scales = _alloc(nb["scales"], torch.int16, device)
+        zeros = _alloc(nb["zeros"], torch.int32, device)
+        oidx = _alloc(max(nb["outlier_idx"], 4), torch.int32, device)
+        outw = _alloc(max(nb["outlier_w"], 2), torch.int16, device)
+        bidx = _alloc(nb["bulk_idx"], torch.int32, device) if inf["compact"] else None
+        if staging is None:
+            staging = _pinned(staging_bytes)
+        view = Layer()
+        _check(_L.spectra_trdc_load(self._h, i, _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(oidx),
+                                    _ptr(outw), _ptr(bidx), _lib.MEM_DEVICE, _ptr(staging),
+                                    staging.numel(), 1 if verify else 0, ctypes.byref(view),
+                                    _stream(stream)), "spectra_trdc_load")
+        return PackedLayer(inf["n"], inf["k"], inf["n_outliers"], codes, scales, zeros, oidx, outw,
+                           bidx, inf["k_bulk"] if inf["compact"] else 0)

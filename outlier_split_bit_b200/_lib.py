@@ -18,6 +18,11 @@ ERR_BUFFER_TOO_SMALL = 6
 ERR_CUDA = 7
 ERR_UNSUPPORTED = 8
 ERR_INTERNAL = 9
+ERR_IO = 10
+ERR_FORMAT = 11
+
+MEM_DEVICE = 0
+MEM_HOST = 1
 
 F32 = 0
 BF16 = 1
@@ -36,6 +41,14 @@ class Sizes(ctypes.Structure):
                 ("scales_bytes", ctypes.c_size_t), ("zeros_bytes", ctypes.c_size_t),
                 ("outlier_idx_bytes", ctypes.c_size_t), ("outlier_w_bytes", ctypes.c_size_t),
                 ("k_bulk", ctypes.c_int32), ("bulk_idx_bytes", ctypes.c_size_t)]
+
+
+class TrdcLayer(ctypes.Structure):
+    """spectra_trdc_layer: one layer record of a TRDC container."""
+    _fields_ = [("name", ctypes.c_char * 96), ("n", ctypes.c_int32), ("k", ctypes.c_int32),
+                ("n_outliers", ctypes.c_int32), ("k_bulk", ctypes.c_int32), ("tau", ctypes.c_double),
+                ("flags", ctypes.c_uint32), ("offset", ctypes.c_uint64 * 6),
+                ("bytes", ctypes.c_uint64 * 6), ("crc32", ctypes.c_uint32 * 6)]
 
 
 # name -> (restype, argtypes), mirroring spectra.h
@@ -59,6 +72,13 @@ SIGNATURES = {
     "spectra_device_status": (ctypes.c_int, [P]),
     "spectra_embed": (ctypes.c_int, [LP, P, i32, P, ctypes.c_int, P]),
     "spectra_pack_plan_noalloc": (ctypes.c_int, [P, P, i32, i32, f64, P, P, ctypes.POINTER(i32), P]),
+    "spectra_crc32": (ctypes.c_uint32, [ctypes.c_uint32, P, sz]),
+    "spectra_trdc_write": (ctypes.c_int, [ctypes.c_char_p, i32, P, LP, P, ctypes.c_int, P, sz, P]),
+    "spectra_trdc_open": (ctypes.c_int, [ctypes.c_char_p, ctypes.POINTER(P)]),
+    "spectra_trdc_count": (i32, [P]),
+    "spectra_trdc_info": (ctypes.c_int, [P, i32, ctypes.POINTER(TrdcLayer)]),
+    "spectra_trdc_load": (ctypes.c_int, [P, i32, P, P, P, P, P, P, ctypes.c_int, P, sz, i32, LP, P]),
+    "spectra_trdc_close": (None, [P]),
 }
 
 NOALLOC_MAX_K = 65536

@@ -1,4 +1,5 @@
-"""Compile the sm_100a CUDA sources into the in-tree shared library libspectra.so.
+"""Compile the sm_100a CUDA sources (and the host C++ of the container I/O)
+into the in-tree shared library libspectra.so.
 
     python -m outlier_split_bit_b200.build [--force]
 
@@ -29,7 +30,7 @@ NVCC_FLAGS = [
 
 
 def sources():
-    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
 
 
 def _stale() -> bool:

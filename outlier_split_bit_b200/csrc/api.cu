@@ -105,6 +105,8 @@ const char *spectra_status_string(spectra_status s) {
         case SPECTRA_ERR_CUDA: return "CUDA runtime error";
         case SPECTRA_ERR_UNSUPPORTED: return "device is not compute capability 10.0";
         case SPECTRA_ERR_INTERNAL: return "internal error";
+        case SPECTRA_ERR_IO: return "container file could not be opened, read or written";
+        case SPECTRA_ERR_FORMAT: return "not a valid TRDC container, or a checksum failed";
     }
     return "unknown status";
 }
