@@ -99,6 +99,12 @@ def _declare(L):
     L.spectra_ref_gemm_compact.restype = None
     L.spectra_ref_embed_compact.argtypes = [i32, i32, i32, P, P, P, P, P, P, i32, P, i32, P]
     L.spectra_ref_embed_compact.restype = ctypes.c_int
+    L.spectra_ref_kv_quantize.argtypes = [P, i32, i32, i32, i32, i32, P, P, P]
+    L.spectra_ref_kv_quantize.restype = ctypes.c_int
+    L.spectra_ref_attention.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P, P, P, f64, P, P, P]
+    L.spectra_ref_attention.restype = ctypes.c_int
+    L.spectra_ref_kv_pack.argtypes = [i32, i32, i32, P, P, P, P, P, P]
+    L.spectra_ref_kv_pack.restype = None
 
 
 def _p(a: np.ndarray | None):
@@ -371,6 +377,73 @@ def embed_compact(lay: CompactLayer, w_bits: np.ndarray, ids) -> np.ndarray:
     if st != OK:
         raise OracleError(st)
     return out
+
+
+# ------------------------------------------------------------------ KV cache
+
+@dataclass
+class KVCache:
+    """Canonical 4-bit cache of one of K or V: [H][cap][D] codes, [H][cap][D/32]
+    scales (FP16 bits) and zero points."""
+    codes: np.ndarray
+    scales: np.ndarray
+    zeros: np.ndarray
+
+    @property
+    def shape(self):
+        return self.codes.shape  # (H, cap, D)
+
+
+def kv_cache(H: int, cap: int, D: int) -> KVCache:
+    return KVCache(np.zeros((H, cap, D), np.uint8), np.zeros((H, cap, D // 32), np.uint16),
+                   np.zeros((H, cap, D // 32), np.uint8))
+
+
+def kv_quantize(cache: KVCache, x_bits: np.ndarray, pos: int) -> None:
+    """Quantise tokens x [n_tok, H, D] (BF16 bits) into positions pos.. of cache."""
+    H, cap, D = cache.shape
+    x = _c(x_bits, np.uint16).reshape(-1, H, D)
+    st = lib().spectra_ref_kv_quantize(_p(x), x.shape[0], H, D, pos, cap, _p(cache.codes),
+                                       _p(cache.scales), _p(cache.zeros))
+    if st != OK:
+        raise OracleError(st)
+
+
+def kv_pack(cache: KVCache):
+    """(codes bytes, scales u16, zeros u32) in the packed KV layout."""
+    H, cap, D = cache.shape
+    pc = np.zeros(H * cap * D // 2, np.uint8)
+    ps = np.zeros(H * cap * (D // 32), np.uint16)
+    pz = np.zeros(H * cap, np.uint32)
+    lib().spectra_ref_kv_pack(H, cap, D, _p(cache.codes), _p(cache.scales), _p(cache.zeros),
+                              _p(pc), _p(ps), _p(pz))
+    return pc, ps, pz
+
+
+def attention(kc: KVCache, vc: KVCache, q_bits: np.ndarray, T: int, scale: float):
+    """(out [Hq, D], vbound [Hq, D], smax [Hq]) of decode attention in FP64."""
+    H, cap, D = kc.shape
+    q = _c(q_bits, np.uint16).reshape(-1, D)
+    Hq = q.shape[0]
+    out = np.empty((Hq, D)); vb = np.empty((Hq, D)); sm = np.empty(Hq)
+    st = lib().spectra_ref_attention(Hq, H, D, T, cap, _p(kc.codes), _p(kc.scales), _p(kc.zeros),
+                                     _p(vc.codes), _p(vc.scales), _p(vc.zeros), _p(q), float(scale),
+                                     _p(out), _p(vb), _p(sm))
+    if st != OK:
+        raise OracleError(st)
+    return out, vb, sm
+
+
+def attention_tolerance(vbound: np.ndarray, smax: np.ndarray) -> np.ndarray:
+    """Acceptance bound of a GPU decode-attention output.  Each score is a dot
+    product held to the matvec's budget, |ds_t| <= 2e-3 * S_t with
+    S_t = scale * sum_d |q_d k_hat_td| (so |ds_t| <= D_s = 2e-3 * max_t S_t);
+    score errors of at most D_s move every softmax weight by a factor within
+    [exp(-2 D_s), exp(2 D_s)], so the output moves by at most
+    (exp(2 D_s) - 1) * sum_t p_t |v_hat_td|; the weighted sum over V has its
+    own 2e-3 * sum_t p_t |v_hat_td|.  Plus 1e-5 absolute."""
+    ds = 2e-3 * smax[:, None]
+    return (2e-3 + np.expm1(2.0 * ds)) * vbound + 1e-5
 
 
 def tolerance(bound: np.ndarray) -> np.ndarray:

@@ -574,3 +574,142 @@ int spectra_ref_embed_compact(int32_t n, int32_t k, int32_t k_bulk, const uint8_
     }
     return REF_OK;
 }
+
+/* ---------------------------------------------------------------- KV cache */
+
+/*
+ * Group-32 4-bit key-value cache (abstract: microscaled Group-32 4-bit KV
+ * caching keeps long contexts resident).  Read as the weight quantiser
+ * applied to every token's vector of one KV head: the D channels of token t
+ * and head h form one row of D/32 groups, each with an FP16 scale and a
+ * 4-bit zero point, codes by the same formula (spectra_ref_quantize, no
+ * outlier columns).  x is [n_tok][H][D] BF16 (the layout a K or V
+ * projection writes); the canonical outputs are indexed by (h, t):
+ *   codes  [H][cap][D], scales [H][cap][D/32], zeros [H][cap][D/32],
+ * and tokens go to positions pos .. pos + n_tok - 1 of a capacity cap.
+ */
+int spectra_ref_kv_quantize(const uint16_t *x, int32_t n_tok, int32_t H, int32_t D, int32_t pos,
+                            int32_t cap, uint8_t *codes, uint16_t *scales, uint8_t *zeros)
+{
+    if (!x || n_tok < 1 || H < 1 || D < 32 || D % 32 != 0 || pos < 0 || pos + n_tok > cap)
+        return REF_ERR_INVALID_ARG;
+    const int64_t G = D / 32;
+    uint8_t *c = (uint8_t *)malloc((size_t)D);
+    uint16_t *s = (uint16_t *)malloc((size_t)G * 2);
+    uint8_t *z = (uint8_t *)malloc((size_t)G);
+    if (!c || !s || !z) {
+        free(c); free(s); free(z);
+        return REF_ERR_INVALID_ARG;
+    }
+    int st = REF_OK;
+    for (int64_t t = 0; t < n_tok && st == REF_OK; ++t)
+        for (int64_t h = 0; h < H && st == REF_OK; ++h) {
+            st = spectra_ref_quantize(x + (t * H + h) * D, 1, D, NULL, 0, c, s, z);
+            if (st != REF_OK)
+                break;
+            const int64_t slot = h * cap + pos + t;
+            memcpy(codes + slot * D, c, (size_t)D);
+            memcpy(scales + slot * G, s, (size_t)G * 2);
+            memcpy(zeros + slot * G, z, (size_t)G);
+        }
+    free(c); free(s); free(z);
+    return st;
+}
+
+/*
+ * Decode attention over the 4-bit cache, in double:
+ *   k_hat[h][t][d] = (c - z) * S (and v_hat likewise), exact;
+ *   for query head i (KV head h = i / (Hq / Hkv)) and tokens t < T:
+ *     s_t = scale * sum_d q[i][d] * k_hat[h][t][d]     (d ascending)
+ *     p_t = exp(s_t - max_t s_t) / sum_t exp(s_t - max_t s_t)
+ *     out[i][d] = sum_t p_t * v_hat[h][t][d]            (t ascending)
+ * Also, for the acceptance test: vbound[i][d] = sum_t p_t |v_hat[h][t][d]|
+ * and smax[i] = max_t scale * sum_d |q[i][d]| |k_hat[h][t][d]| (either may
+ * be NULL).  Caches are canonical arrays of capacity cap (see above).
+ */
+int spectra_ref_attention(int32_t Hq, int32_t Hkv, int32_t D, int32_t T, int32_t cap,
+                          const uint8_t *kc, const uint16_t *ks, const uint8_t *kz,
+                          const uint8_t *vc, const uint16_t *vs, const uint8_t *vz,
+                          const uint16_t *q, double scale, double *out, double *vbound,
+                          double *smax)
+{
+    if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || D < 32 || D % 32 != 0 || T < 1 || T > cap)
+        return REF_ERR_INVALID_ARG;
+    const int64_t G = D / 32, grp = Hq / Hkv;
+    double *sc = (double *)malloc((size_t)T * sizeof(double));
+    double *sa = (double *)malloc((size_t)T * sizeof(double));
+    if (!sc || !sa) {
+        free(sc); free(sa);
+        return REF_ERR_INVALID_ARG;
+    }
+    for (int64_t i = 0; i < Hq; ++i) {
+        const int64_t h = i / grp;
+        double m = -INFINITY, sm = 0.0;
+        for (int64_t t = 0; t < T; ++t) {
+            const int64_t slot = h * cap + t;
+            double acc = 0.0, ab = 0.0;
+            for (int64_t d = 0; d < D; ++d) {
+                double S = spectra_ref_fp16_to_double(ks[slot * G + d / 32]);
+                double kv = ((double)kc[slot * D + d] - (double)kz[slot * G + d / 32]) * S;
+                double qv = spectra_ref_bf16_to_double(q[i * D + d]);
+                acc = acc + qv * kv;
+                ab = ab + fabs(qv) * fabs(kv);
+            }
+            sc[t] = scale * acc;
+            sa[t] = fabs(scale) * ab;
+            if (sc[t] > m) m = sc[t];
+            if (sa[t] > sm) sm = sa[t];
+        }
+        double l = 0.0;
+        for (int64_t t = 0; t < T; ++t) {
+            sc[t] = exp(sc[t] - m);
+            l = l + sc[t];
+        }
+        for (int64_t d = 0; d < D; ++d) {
+            double o = 0.0, b = 0.0;
+            for (int64_t t = 0; t < T; ++t) {
+                const int64_t slot = h * cap + t;
+                double S = spectra_ref_fp16_to_double(vs[slot * G + d / 32]);
+                double vv = ((double)vc[slot * D + d] - (double)vz[slot * G + d / 32]) * S;
+                o = o + (sc[t] / l) * vv;
+                b = b + (sc[t] / l) * fabs(vv);
+            }
+            out[i * D + d] = o;
+            if (vbound)
+                vbound[i * D + d] = b;
+        }
+        if (smax)
+            smax[i] = sm;
+    }
+    free(sc); free(sa);
+    return REF_OK;
+}
+
+/*
+ * Packed KV cache (repository-defined, like RT32): one slot per (head h,
+ * position t), slot = h*cap + t, G = D/32 groups:
+ *   codes : 16-byte record per (slot, group g) at byte (slot*G + g)*16; word
+ *           w, nibble j holds the code of channel 32g + 8w + j;
+ *   scales: FP16 bits, element slot*G + g;
+ *   zeros : u32 word slot, nibble g (D <= 256).
+ * Slots and nibbles not covered by the canonical arrays stay zero.
+ */
+void spectra_ref_kv_pack(int32_t H, int32_t cap, int32_t D, const uint8_t *codes,
+                         const uint16_t *scales, const uint8_t *zeros, uint8_t *pcodes,
+                         uint16_t *pscales, uint32_t *pzeros)
+{
+    const int64_t G = D / 32, slots = (int64_t)H * cap;
+    memset(pcodes, 0, (size_t)(slots * D / 2));
+    memset(pscales, 0, (size_t)(slots * G) * 2);
+    memset(pzeros, 0, (size_t)slots * 4);
+    for (int64_t slot = 0; slot < slots; ++slot)
+        for (int64_t ch = 0; ch < D; ++ch) {
+            const int64_t grp = ch / 32, in = ch % 32, word = in / 8, nib = in % 8;
+            const uint8_t c = codes[slot * D + ch] & 0xF;
+            pcodes[(slot * G + grp) * 16 + word * 4 + nib / 2] |= (uint8_t)((nib % 2) ? (c << 4) : c);
+            if (in == 0) {
+                pscales[slot * G + grp] = scales[slot * G + grp];
+                pzeros[slot] |= (uint32_t)(zeros[slot * G + grp] & 0xF) << (4 * grp);
+            }
+        }
+}

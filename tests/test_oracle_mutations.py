@@ -55,6 +55,13 @@ MUTATIONS = {
     "gemm_compact_group_of_bulk": ("double wb = ((double)codes[i * k_bulk + p] - (double)zeros[i * Gb + p / 32]) * S;",
                                    "double wb = ((double)codes[i * k_bulk + p] - (double)zeros[i * Gb + p % Gb]) * S;"),
     "pack_outliers_slot_reversed": ("= w[i * k + idx[slot]];", "= w[i * k + idx[n_o - 1 - slot]];"),
+    "kv_pack_nibble_swapped": ("(uint8_t)((nib % 2) ? (c << 4) : c);", "(uint8_t)((nib % 2) ? c : (c << 4));"),
+    "kv_slot_transposed": ("const int64_t slot = h * cap + pos + t;", "const int64_t slot = t * H + h + pos;"),
+    "attention_head_mapping": ("const int64_t h = i / grp;", "const int64_t h = i % Hkv;"),
+    "attention_unnormalised": ("o = o + (sc[t] / l) * vv;", "o = o + sc[t] * vv;"),
+    "attention_key_zero_index": ("double kv = ((double)kc[slot * D + d] - (double)kz[slot * G + d / 32]) * S;",
+                                 "double kv = ((double)kc[slot * D + d] - (double)kz[slot * G + d % G]) * S;"),
+    "attention_scale_dropped": ("sc[t] = scale * acc;", "sc[t] = acc;"),
     "embed_zero_point_sign": ("dst[col] = ((double)codes[row * k + col] - (double)zeros[grp]) * S;",
                               "dst[col] = ((double)codes[row * k + col] + (double)zeros[grp]) * S;"),
 }
@@ -82,6 +89,10 @@ PIN_FUNCS = [
     pins.test_gemm_compact_exact_grid_bulk_is_dense_product,
     pins.test_gemm_compact_unit_vectors_extract_columns,
     pins.test_compact_outlier_block_is_the_masked_one,
+    pins.test_kv_quantize_is_the_weight_quantiser_per_token,
+    pins.test_attention_exact_grid_is_textbook,
+    pins.test_attention_one_token_and_zero_query,
+    pins.test_kv_pack_golden_offsets,
 ]
 _PARAMS = {
     "test_quantizer_exact_grid": [{"S": 2.0 ** -7, "z": 5}],

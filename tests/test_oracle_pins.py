@@ -687,3 +687,115 @@ def test_compact_outlier_block_is_the_masked_one(ref):
         masked, comp = ref.pack(wb, g, tau), ref.pack_compact(wb, g, tau)
         assert np.array_equal(masked.idx, comp.idx) and comp.idx.size > 0
         assert np.array_equal(masked.packed.outliers, comp.packed.outliers)
+
+
+# ----------------------------------------------------------------- KV cache
+
+def _kv_tokens(n_tok, H, D, seed):
+    return wl.bits(wl.activations(H * D, n_tok, seed=seed)).reshape(n_tok, H, D)
+
+
+def test_kv_quantize_is_the_weight_quantiser_per_token(ref):
+    H, cap, D = 3, 20, 96
+    x = _kv_tokens(7, H, D, 40)
+    c = ref.kv_cache(H, cap, D)
+    ref.kv_quantize(c, x, pos=5)
+    for t in range(7):
+        for h in range(H):
+            row = ref.quantize(x[t, h][None, :], np.zeros(0, np.int32))
+            assert np.array_equal(c.codes[h, 5 + t], row.codes[0])
+            assert np.array_equal(c.scales[h, 5 + t], row.scales[0])
+            assert np.array_equal(c.zeros[h, 5 + t], row.zeros[0])
+    assert not c.codes[:, :5].any() and not c.codes[:, 12:].any()
+    with pytest.raises(ref.OracleError):
+        ref.kv_quantize(c, x, pos=14)  # past the capacity
+
+
+def _grid_cache(ref, H, T, D, seed, S=2.0 ** -6):
+    """A cache whose token vectors are exact quantiser grids: dequantisation
+    returns them exactly."""
+    rng = np.random.default_rng(seed)
+    vals = np.stack([np.concatenate([_grid_row(S, int(rng.integers(0, 16)), int(rng.integers(1e6)))
+                                     for _ in range(D // 32)]) for _ in range(T * H)]).reshape(T, H, D)
+    c = ref.kv_cache(H, T, D)
+    ref.kv_quantize(c, _bf16_bits(vals), 0)
+    return c, vals
+
+
+def _textbook_attention(q, K, V, scale, Hq, Hkv):
+    from scipy.special import softmax
+    grp = Hq // Hkv
+    out = np.empty((Hq, K.shape[2]))
+    for i in range(Hq):
+        h = i // grp
+        p = softmax(scale * (K[:, h, :] @ q[i]))
+        out[i] = p @ V[:, h, :]
+    return out
+
+
+def test_attention_exact_grid_is_textbook(ref):
+    Hq, Hkv, T, D = 6, 2, 50, 64
+    kc, K = _grid_cache(ref, Hkv, T, D, 41)
+    vc, V = _grid_cache(ref, Hkv, T, D, 42)
+    qb = wl.bits(wl.activations(D, Hq, seed=43))
+    out, vb, sm = ref.attention(kc, vc, qb, T, 1.0 / np.sqrt(D))
+    want = _textbook_attention(_bf16_values(qb), K, V, 1.0 / np.sqrt(D), Hq, Hkv)
+    assert np.allclose(out, want, rtol=1e-12, atol=1e-14)
+    assert np.all(vb >= np.abs(out) - 1e-15) and np.all(sm > 0)
+
+
+def test_attention_one_token_and_zero_query(ref):
+    Hkv, D = 2, 64
+    kc, K = _grid_cache(ref, Hkv, 9, D, 44)
+    vc, V = _grid_cache(ref, Hkv, 9, D, 45)
+    qb = wl.bits(wl.activations(D, 4, seed=46))
+    out, _, _ = ref.attention(kc, vc, qb, 1, 0.125)
+    assert np.array_equal(out[:2], np.stack([V[0, 0]] * 2)) and np.array_equal(out[2:], np.stack([V[0, 1]] * 2))
+    out, _, _ = ref.attention(kc, vc, np.zeros((4, D), np.uint16), 9, 0.125)
+    assert np.allclose(out[0], V[:, 0].mean(0), rtol=0, atol=1e-15)
+    assert np.allclose(out[3], V[:, 1].mean(0), rtol=0, atol=1e-15)
+
+
+def test_kv_pack_golden_offsets(ref, golden_dir):
+    H, cap, D = 2, 3, 64
+    c = ref.kv_cache(H, cap, D)
+    rng = np.random.default_rng(47)
+    c.codes[:] = rng.integers(0, 16, c.codes.shape)
+    c.scales[:] = rng.integers(0, 1 << 15, c.scales.shape)
+    c.zeros[:] = rng.integers(0, 16, c.zeros.shape)
+    pc, ps, pz = ref.kv_pack(c)
+    n = 0
+    for line in open(os.path.join(golden_dir, "kv_layout_offsets.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        h, t, ch, byte, hi, se, zw, zs = (int(v) for v in line.split()[:8])
+        got = (pc[byte] >> 4) if hi else (pc[byte] & 0xF)
+        assert got == c.codes[h, t, ch]
+        assert ps[se] == c.scales[h, t, ch // 32]
+        assert ((pz[zw] >> zs) & 0xF) == c.zeros[h, t, ch // 32]
+        n += 1
+    assert n == 4
+
+
+def test_attention_tolerance_covers_its_budget(ref):
+    # perturb every score by up to 2e-3 S_t and every weighted-sum term by up
+    # to 2e-3 of its size, in the worst direction; the output stays inside
+    # the stated tolerance
+    Hq, Hkv, T, D = 2, 1, 40, 64
+    kc, K = _grid_cache(ref, Hkv, T, D, 48)
+    vc, V = _grid_cache(ref, Hkv, T, D, 49)
+    qb = wl.bits(wl.activations(D, Hq, seed=50))
+    scale = 1.0 / np.sqrt(D)
+    out, vb, sm = ref.attention(kc, vc, qb, T, scale)
+    tol = ref.attention_tolerance(vb, sm)
+    q = _bf16_values(qb)
+    for i in range(Hq):
+        s = scale * (K[:, 0, :] @ q[i])
+        S = scale * (np.abs(K[:, 0, :]) @ np.abs(q[i]))
+        for d in range(D):
+            for sign in (1, -1):
+                bump = sign * np.sign(V[:, 0, d] - out[i, d])  # raise the weights that move o_d away
+                s2 = s + 2e-3 * S * bump
+                p = np.exp(s2 - s2.max()); p /= p.sum()
+                o2 = p @ V[:, 0, d] + sign * 2e-3 * (p @ np.abs(V[:, 0, d]))
+                assert abs(o2 - out[i, d]) <= tol[i, d]
