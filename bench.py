@@ -420,7 +420,44 @@ def extras(device, stream, peak_gbs, tau):
                          "frac_single_flushed": round(b / us * 1e-3 / peak_gbs, 3)})
         out["embed_rows_131072x3072_bf16"] = rows
         del w, lay
+        out["kv_attention_decode_8192"] = kv_rows(device, stream, peak_gbs, flush)
     return out
+
+
+def kv_rows(device, stream, peak_gbs, flush, T: int = 8192):
+    """Decode attention of one token over T cached positions (Group-32 4-bit K
+    and V) for the 1.5B-class (12 query / 2 KV heads) and 4B-class (32 / 8)
+    shapes, head_dim 128.  Back-to-back launches cycle over cache copies that
+    together exceed twice the L2, so every call reads its cache from DRAM."""
+    import outlier_split_bit_b200 as sp
+    rows = []
+    for name, hq, hkv, d in (("1.5B-class", 12, 2, 128), ("4B-class", 32, 8, 128)):
+        k0, v0 = sp.KVCache(hkv, d, T, device), sp.KVCache(hkv, d, T, device)
+        k0.append(wl.activations(hkv * d, T, seed=1, device=device).reshape(T, hkv, d), 0)
+        v0.append(wl.activations(hkv * d, T, seed=2, device=device).reshape(T, hkv, d), 0)
+        per = k0.nbytes + v0.nbytes
+        copies = [(k0, v0)]
+        while len(copies) * per < L2_ROTATE_BYTES:
+            k1, v1 = sp.KVCache(hkv, d, T, device), sp.KVCache(hkv, d, T, device)
+            for a, b in ((k1, k0), (v1, v0)):
+                a.codes.copy_(b.codes); a.scales.copy_(b.scales); a.zeros.copy_(b.zeros)
+            copies.append((k1, v1))
+        q = wl.activations(d, hq, seed=3, device=device)
+        o = torch.empty((hq, d), device=device)
+        ws = torch.empty(sp.library().spectra_attention_workspace_size(hq, d, T), dtype=torch.uint8,
+                         device=device)
+        fns = [(lambda kk=kk, vv=vv: sp.spectra_attention_decode(kk, vv, q, T, None, o, workspace=ws,
+                                                                 stream=stream)) for kk, vv in copies]
+        us, p10, p90 = time_single(fns[0], stream, 30, flush)
+        us_r = time_rotating(fns, stream, 200)
+        b = per + hq * d * 2 + hq * d * 4
+        rows.append({"shape": name, "n_q_heads": hq, "n_kv_heads": hkv, "head_dim": d, "positions": T,
+                     "cache_bytes": per, "us_single_flushed": round(us, 2),
+                     "us_back_to_back": round(us_r, 2), "gbs_back_to_back": round(b / us_r * 1e-3, 1),
+                     "frac_back_to_back": round(b / us_r * 1e-3 / peak_gbs, 3),
+                     "launches_per_call": 2})
+        del copies, k0, v0
+    return rows
 
 
 # ---------------------------------------------------------------- oracle leg
@@ -857,6 +894,20 @@ def run_embed(args):
     return 0
 
 
+def run_kv(args):
+    """Decode attention over the 4-bit KV cache alone (the kv rows of the
+    benchmark); prints one JSON line."""
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    peak = float(measured_peaks()["hbm_gbs"])
+    stream = torch.cuda.Stream(device=device)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+    with torch.cuda.stream(stream):
+        rows = kv_rows(device, stream, peak, flush, T=args.positions)
+    print(json.dumps({"case": "kv", "rows": rows}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -866,9 +917,11 @@ def main():
     ap.add_argument("--tau", type=float, default=3.0)
     ap.add_argument("--quick", action="store_true", help="skip the per-matrix / LM-head / batch rows")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["stream", "single", "embed"], default="stream",
+    ap.add_argument("--case", choices=["stream", "single", "embed", "kv"], default="stream",
                     help="stream: the decode-step weight stream (the benchmark); single: one "
-                         "matrix; embed: the embedding-row gather of --m ids")
+                         "matrix; embed: the embedding-row gather of --m ids; kv: decode "
+                         "attention over the 4-bit KV cache")
+    ap.add_argument("--positions", type=int, default=8192, help="cached positions (--case kv)")
     ap.add_argument("--compact", action="store_true",
                     help="pack with the outlier columns removed from the 4-bit bulk")
     ap.add_argument("--n", type=int, default=wl.LM_HEAD_N)
@@ -884,6 +937,8 @@ def main():
         return run_single(args)
     if args.case == "embed":
         return run_embed(args)
+    if args.case == "kv":
+        return run_kv(args)
     return run_ours(args)
 
 

@@ -336,12 +336,82 @@ SPECTRA_API spectra_status spectra_embed(const spectra_layer *table, const int32
  * for the asynchronous weight copies are bounded: a wait that gives up
  * raises a per-device flag instead of hanging, and the outputs of that
  * launch are invalid.  The embedding gather raises its own flag for an id
- * outside the table (or an outlier index outside [0, k)).  Returns
+ * outside the table (or an outlier index outside [0, k)), and the KV append
+ * for a non-finite value or an FP16 scale overflow.  Returns, for what
+ * happened since the last call (and clears every flag):
  * SPECTRA_ERR_INTERNAL if a wait gave up, else SPECTRA_ERR_INVALID_ARG if the
- * gather saw a bad id, since the last call (and clears both flags),
- * SPECTRA_OK otherwise.  Synchronous on `stream`.
+ * gather saw a bad id, else SPECTRA_ERR_NONFINITE or SPECTRA_ERR_RANGE from
+ * the KV append, else SPECTRA_OK.  Synchronous on `stream`.
  */
 SPECTRA_API spectra_status spectra_device_status(void *stream);
+
+/*
+ * Group-32 4-bit KV cache (abstract: microscaled Group-32 4-bit key-value
+ * caching keeps long contexts resident).  Each token's vector of one KV head
+ * (head_dim = D channels, D a multiple of 32, at most 256) is quantised with
+ * the weight quantiser of spectra_pack: D/32 groups of 32 consecutive
+ * channels, an FP16 scale and a 4-bit zero point each.  One cache holds K
+ * or V.  Layout, slot = head * capacity + position, G = D/32:
+ *   codes : 16-byte record per (slot, group g) at byte (slot*G + g)*16;
+ *           word w, nibble j = code of channel 32g + 8w + j (a token's codes
+ *           are D/2 contiguous bytes);
+ *   scales: FP16 bits, element slot*G + g;
+ *   zeros : u32 word slot, nibble g.
+ * 4.625 bits per cached value instead of 16.
+ */
+typedef struct {
+    int32_t n_heads;     /* KV heads */
+    int32_t head_dim;    /* D */
+    int32_t capacity;    /* positions per head */
+    uint8_t *codes;      /* device, 16-byte aligned, n_heads*capacity*D/2 bytes */
+    uint16_t *scales;    /* device, n_heads*capacity*D/32 FP16 */
+    uint32_t *zeros;     /* device, n_heads*capacity words */
+} spectra_kv;
+
+/* Byte sizes of a cache's three buffers (host only, no CUDA call). */
+SPECTRA_API spectra_status spectra_kv_sizes(int32_t n_heads, int32_t head_dim, int32_t capacity,
+                                            size_t *codes_bytes, size_t *scales_bytes,
+                                            size_t *zeros_bytes);
+
+/*
+ * Quantise n_tok new tokens into positions pos .. pos + n_tok - 1:
+ *   x  device, BF16 bits [n_tok][n_heads][head_dim] (a K or V projection's
+ *      output layout)
+ * Bit-identical to the oracle (the weight quantiser per token and head).
+ * A group holding a NaN or infinity, or whose scale overflows FP16, is
+ * stored as zeros and raises the flag that spectra_device_status reports
+ * (NONFINITE, RANGE).  n_tok == 0 returns SPECTRA_OK without touching CUDA.
+ * Asynchronous.  Errors: INVALID_ARG, SHAPE (pos + n_tok > capacity), ALIGN,
+ * UNSUPPORTED, CUDA.
+ */
+SPECTRA_API spectra_status spectra_kv_append(const spectra_kv *cache, const uint16_t *x,
+                                             int32_t n_tok, int32_t pos, void *stream);
+
+/* Device workspace bytes that spectra_attention_decode needs. */
+SPECTRA_API size_t spectra_attention_workspace_size(int32_t n_q_heads, int32_t head_dim,
+                                                    int32_t length);
+
+/*
+ * Decode attention of one query token over positions 0 .. length - 1 of a
+ * K and a V cache of the same geometry (grouped-query heads: query head i
+ * reads KV head i / (n_q_heads / n_heads), at most 8 query heads per KV head):
+ *   s_t = scale * sum_d q[i][d] * k_hat[t][d],  p = softmax(s),
+ *   out[i][d] = sum_t p_t * v_hat[t][d],  x_hat = (c - z) * s dequantised
+ *   in registers (exact in FP32), FP32 accumulation and softmax.
+ *   q    device, BF16 bits [n_q_heads][head_dim]
+ *   out  device, float [n_q_heads][head_dim]
+ *   workspace  device, 16-byte aligned, >= spectra_attention_workspace_size
+ * Accepted results stay within (2e-3 + expm1(4e-3 * S_max)) * sum_t p_t
+ * |v_hat_td| + 1e-5 of the FP64 oracle, S_max = max_t scale * sum_d |q_d
+ * k_hat_td| (the matvec's 2e-3 per dot product carried through the softmax).
+ * Asynchronous, allocates nothing, deterministic.  Errors: INVALID_ARG,
+ * SHAPE, ALIGN, BUFFER_TOO_SMALL, UNSUPPORTED, CUDA.
+ */
+SPECTRA_API spectra_status spectra_attention_decode(const spectra_kv *k, const spectra_kv *v,
+                                                    const uint16_t *q, int32_t n_q_heads,
+                                                    int32_t length, float scale, float *out,
+                                                    void *workspace, size_t workspace_bytes,
+                                                    void *stream);
 
 /*
  * TRDC container (abstract: every weight, scale and offset is serialised

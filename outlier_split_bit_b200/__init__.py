@@ -18,14 +18,15 @@ from dataclasses import dataclass
 import torch
 
 from . import _lib
-from ._lib import Layer, Sizes, TrdcLayer
+from ._lib import KV, Layer, Sizes, TrdcLayer
 
 __all__ = ["SpectraError", "PackedLayer", "spectra_status_string", "spectra_version",
            "spectra_packed_sizes", "spectra_packed_sizes_compact", "spectra_pack_plan",
            "spectra_pack", "spectra_pack_compact", "spectra_unpack",
            "spectra_gemv", "spectra_gemm_small", "spectra_gemv_batched", "spectra_embed",
            "spectra_device_status",
-           "pack_layer", "library", "spectra_crc32", "write_container", "Container"]
+           "pack_layer", "library", "spectra_crc32", "write_container", "Container", "KVCache",
+           "spectra_attention_decode"]
 
 class _Lazy:
     """Loads libspectra.so on first attribute access."""
@@ -372,3 +373,54 @@ class Container:
                                     _stream(stream)), "spectra_trdc_load")
         return PackedLayer(inf["n"], inf["k"], inf["n_outliers"], codes, scales, zeros, oidx, outw,
                            bidx, inf["k_bulk"] if inf["compact"] else 0)
+
+
+# ---------------------------------------------------------------- KV cache
+
+class KVCache:
+    """One Group-32 4-bit KV cache (K or V) in device buffers allocated here
+    with torch: n_heads x capacity positions of head_dim channels."""
+
+    def __init__(self, n_heads: int, head_dim: int, capacity: int, device="cuda"):
+        cb, sb, zb = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+        _check(_L.spectra_kv_sizes(n_heads, head_dim, capacity, ctypes.byref(cb), ctypes.byref(sb),
+                                   ctypes.byref(zb)), "spectra_kv_sizes")
+        self.n_heads, self.head_dim, self.capacity = n_heads, head_dim, capacity
+        self.codes = torch.zeros(cb.value, dtype=torch.uint8, device=device)
+        self.scales = torch.zeros(sb.value // 2, dtype=torch.int16, device=device)
+        self.zeros = torch.zeros(zb.value // 4, dtype=torch.int32, device=device)
+        self._view = KV(n_heads, head_dim, capacity, _ptr(self.codes), _ptr(self.scales),
+                        _ptr(self.zeros))
+
+    def view(self) -> KV:
+        return self._view
+
+    @property
+    def nbytes(self) -> int:
+        return self.codes.numel() + 2 * self.scales.numel() + 4 * self.zeros.numel()
+
+    def append(self, x: torch.Tensor, pos: int, *, stream=None) -> None:
+        """Quantise x (BF16 [n_tok, n_heads, head_dim]) into positions pos.."""
+        n_tok = x.shape[0] if x.numel() else 0
+        _check(_L.spectra_kv_append(ctypes.byref(self._view), _ptr(x) if n_tok else None, n_tok, pos,
+                                    _stream(stream)), "spectra_kv_append")
+
+
+def spectra_attention_decode(k: KVCache, v: KVCache, q: torch.Tensor, length: int,
+                             scale: float | None = None, out: torch.Tensor | None = None, *,
+                             workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Decode attention of q (BF16 [n_q_heads, head_dim]) over positions
+    0..length-1 of the caches; returns float [n_q_heads, head_dim]."""
+    hq, d = q.shape
+    if scale is None:
+        scale = 1.0 / d ** 0.5
+    if out is None:
+        out = torch.empty((hq, d), dtype=torch.float32, device=q.device)
+    need = _L.spectra_attention_workspace_size(hq, d, length)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(_L.spectra_attention_decode(ctypes.byref(k.view()), ctypes.byref(v.view()), _ptr(q), hq,
+                                       length, float(scale), _ptr(out), _ptr(workspace),
+                                       workspace.numel(), _stream(stream)),
+           "spectra_attention_decode")
+    return out

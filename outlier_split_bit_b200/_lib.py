@@ -43,6 +43,13 @@ class Sizes(ctypes.Structure):
                 ("k_bulk", ctypes.c_int32), ("bulk_idx_bytes", ctypes.c_size_t)]
 
 
+class KV(ctypes.Structure):
+    """spectra_kv: a view of one packed 4-bit KV cache (device buffers)."""
+    _fields_ = [("n_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("capacity", ctypes.c_int32), ("codes", ctypes.c_void_p),
+                ("scales", ctypes.c_void_p), ("zeros", ctypes.c_void_p)]
+
+
 class TrdcLayer(ctypes.Structure):
     """spectra_trdc_layer: one layer record of a TRDC container."""
     _fields_ = [("name", ctypes.c_char * 96), ("n", ctypes.c_int32), ("k", ctypes.c_int32),
@@ -73,6 +80,12 @@ SIGNATURES = {
     "spectra_embed": (ctypes.c_int, [LP, P, i32, P, ctypes.c_int, P]),
     "spectra_pack_plan_noalloc": (ctypes.c_int, [P, P, i32, i32, f64, P, P, ctypes.POINTER(i32), P]),
     "spectra_crc32": (ctypes.c_uint32, [ctypes.c_uint32, P, sz]),
+    "spectra_kv_sizes": (ctypes.c_int, [i32, i32, i32, ctypes.POINTER(sz), ctypes.POINTER(sz),
+                                        ctypes.POINTER(sz)]),
+    "spectra_kv_append": (ctypes.c_int, [ctypes.POINTER(KV), P, i32, i32, P]),
+    "spectra_attention_workspace_size": (sz, [i32, i32, i32]),
+    "spectra_attention_decode": (ctypes.c_int, [ctypes.POINTER(KV), ctypes.POINTER(KV), P, i32, i32,
+                                                ctypes.c_float, P, P, sz, P]),
     "spectra_trdc_write": (ctypes.c_int, [ctypes.c_char_p, i32, P, LP, P, ctypes.c_int, P, sz, P]),
     "spectra_trdc_open": (ctypes.c_int, [ctypes.c_char_p, ctypes.POINTER(P)]),
     "spectra_trdc_count": (i32, [P]),

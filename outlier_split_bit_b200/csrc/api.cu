@@ -5,6 +5,7 @@
 // tested on a machine without a GPU.
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <mutex>
 
 #include "internal.cuh"
@@ -347,6 +348,77 @@ spectra_status spectra_embed(const spectra_layer *table, const int32_t *ids, int
     return launch_embed(*table, ids, m, out, (int)out_dtype, (cudaStream_t)stream, dev);
 }
 
+static spectra_status check_kv(const spectra_kv *c) {
+    if (!c) return SPECTRA_ERR_INVALID_ARG;
+    if (c->n_heads < 1 || c->capacity < 1 || c->head_dim < 32 || c->head_dim > 256 ||
+        c->head_dim % 32 != 0)
+        return SPECTRA_ERR_SHAPE;
+    if ((int64_t)c->n_heads * c->capacity * c->head_dim > ((int64_t)1 << 40)) return SPECTRA_ERR_SHAPE;
+    if (!c->codes || !c->scales || !c->zeros) return SPECTRA_ERR_INVALID_ARG;
+    if (!aligned16(c->codes) || ((uintptr_t)c->scales & 1u) || !aligned4(c->zeros))
+        return SPECTRA_ERR_ALIGN;
+    return SPECTRA_OK;
+}
+
+spectra_status spectra_kv_sizes(int32_t n_heads, int32_t head_dim, int32_t capacity,
+                                size_t *codes_bytes, size_t *scales_bytes, size_t *zeros_bytes) {
+    if (!codes_bytes || !scales_bytes || !zeros_bytes) return SPECTRA_ERR_INVALID_ARG;
+    if (n_heads < 1 || capacity < 1 || head_dim < 32 || head_dim > 256 || head_dim % 32 != 0)
+        return SPECTRA_ERR_SHAPE;
+    const int64_t slots = (int64_t)n_heads * capacity;
+    if (slots * head_dim > ((int64_t)1 << 40)) return SPECTRA_ERR_SHAPE;
+    *codes_bytes = (size_t)(slots * head_dim / 2);
+    *scales_bytes = (size_t)(slots * (head_dim / 32) * 2);
+    *zeros_bytes = (size_t)(slots * 4);
+    return SPECTRA_OK;
+}
+
+spectra_status spectra_kv_append(const spectra_kv *cache, const uint16_t *x, int32_t n_tok,
+                                 int32_t pos, void *stream) {
+    spectra_status st = check_kv(cache);
+    if (st != SPECTRA_OK) return st;
+    if (n_tok < 0 || pos < 0) return SPECTRA_ERR_INVALID_ARG;
+    if ((int64_t)pos + n_tok > cache->capacity) return SPECTRA_ERR_SHAPE;
+    if (n_tok == 0) return SPECTRA_OK;
+    if (!x) return SPECTRA_ERR_INVALID_ARG;
+    if ((uintptr_t)x & 1u) return SPECTRA_ERR_ALIGN;
+    if ((int64_t)n_tok * cache->n_heads > ((int64_t)1 << 30)) return SPECTRA_ERR_SHAPE;
+    DeviceInfo dev;
+    st = current_device(&dev);
+    if (st != SPECTRA_OK) return st;
+    return launch_kv_append(*cache, x, n_tok, pos, (cudaStream_t)stream);
+}
+
+size_t spectra_attention_workspace_size(int32_t n_q_heads, int32_t head_dim, int32_t length) {
+    if (n_q_heads < 1 || head_dim < 1 || length < 1) return 0;
+    return attention_workspace_bytes(n_q_heads, head_dim, length);
+}
+
+spectra_status spectra_attention_decode(const spectra_kv *k, const spectra_kv *v, const uint16_t *q,
+                                        int32_t n_q_heads, int32_t length, float scale, float *out,
+                                        void *workspace, size_t workspace_bytes, void *stream) {
+    spectra_status st = check_kv(k);
+    if (st != SPECTRA_OK) return st;
+    st = check_kv(v);
+    if (st != SPECTRA_OK) return st;
+    if (k->n_heads != v->n_heads || k->head_dim != v->head_dim || k->capacity != v->capacity)
+        return SPECTRA_ERR_SHAPE;
+    if (!q || !out || !workspace) return SPECTRA_ERR_INVALID_ARG;
+    if (!(scale == scale) || scale == INFINITY || scale == -INFINITY) return SPECTRA_ERR_INVALID_ARG;
+    if (n_q_heads < 1 || n_q_heads % k->n_heads != 0 ||
+        n_q_heads / k->n_heads > attention_max_group())
+        return SPECTRA_ERR_SHAPE;
+    if (length < 1 || length > k->capacity) return SPECTRA_ERR_SHAPE;
+    if (((uintptr_t)q & 1u) || !aligned4(out) || !aligned16(workspace)) return SPECTRA_ERR_ALIGN;
+    if (workspace_bytes < attention_workspace_bytes(n_q_heads, k->head_dim, length))
+        return SPECTRA_ERR_BUFFER_TOO_SMALL;
+    DeviceInfo dev;
+    st = current_device(&dev);
+    if (st != SPECTRA_OK) return st;
+    return launch_attention(*k, *v, q, n_q_heads, length, scale, out, workspace,
+                            (cudaStream_t)stream);
+}
+
 spectra_status spectra_device_status(void *stream) {
     DeviceInfo dev;
     spectra_status st = current_device(&dev);
@@ -354,11 +426,16 @@ spectra_status spectra_device_status(void *stream) {
     bool raised = false;
     st = device_error(&raised, (cudaStream_t)stream);
     if (st != SPECTRA_OK) return st;
-    unsigned int embed_bits = 0;
+    unsigned int embed_bits = 0, kv_bits = 0;
     st = embed_device_error(&embed_bits, (cudaStream_t)stream);
     if (st != SPECTRA_OK) return st;
+    st = kv_device_error(&kv_bits, (cudaStream_t)stream);
+    if (st != SPECTRA_OK) return st;
     if (raised) return SPECTRA_ERR_INTERNAL;
-    return embed_bits ? SPECTRA_ERR_INVALID_ARG : SPECTRA_OK;
+    if (embed_bits) return SPECTRA_ERR_INVALID_ARG;
+    if (kv_bits & 1u) return SPECTRA_ERR_NONFINITE;
+    if (kv_bits & 2u) return SPECTRA_ERR_RANGE;
+    return SPECTRA_OK;
 }
 
 }  // extern "C"

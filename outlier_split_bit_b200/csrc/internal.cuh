@@ -108,4 +108,14 @@ spectra_status launch_embed(const spectra_layer &l, const int32_t *ids, int m, v
 // bit 1 an outlier index outside [0, k).
 spectra_status embed_device_error(unsigned int *bits, cudaStream_t s);
 
+// ---- KV cache (kv.cu) ----
+spectra_status launch_kv_append(const spectra_kv &c, const uint16_t *x, int n_tok, int pos,
+                                cudaStream_t s);
+spectra_status launch_attention(const spectra_kv &k, const spectra_kv &v, const uint16_t *q, int Hq,
+                                int T, float scale, float *out, void *ws, cudaStream_t s);
+size_t attention_workspace_bytes(int Hq, int D, int T);
+int attention_max_group();
+// Reads (and clears) the append's flag: bit 0 non-finite value, bit 1 FP16 range.
+spectra_status kv_device_error(unsigned int *bits, cudaStream_t s);
+
 }  // namespace spectra

@@ -15,6 +15,7 @@
 #include <cuda_fp16.h>
 
 #include "internal.cuh"
+#include "quant.cuh"
 
 namespace spectra {
 namespace {
@@ -95,10 +96,6 @@ __global__ void __launch_bounds__(1024) split_kernel(const double *__restrict__ 
         __syncthreads();
     }
     if (threadIdx.x == 0) *count = base;
-}
-
-__device__ __forceinline__ double clamp015(double v) {
-    return v < 0.0 ? 0.0 : (v > 15.0 ? 15.0 : v);
 }
 
 // Column list of a compacted bulk, one thread per column j of W: a
@@ -202,27 +199,9 @@ __global__ void __launch_bounds__(128) quantize_pack_kernel(
                     v[kk] = __dadd_rn(x, 0.0);  // -0 + +0 = +0
                 }
             }
-            double lo = v[0], hi = v[0];
-#pragma unroll
-            for (int kk = 1; kk < 32; ++kk) {
-                if (v[kk] < lo) lo = v[kk];
-                if (v[kk] > hi) hi = v[kk];
-            }
-            const double q15 = __ddiv_rn(__dsub_rn(hi, lo), 15.0);
             unsigned short hbits;
-            asm("cvt.rn.f16.f64 %0, %1;" : "=h"(hbits) : "d"(q15));
-            if ((hbits & 0x7FFFu) == 0x7C00u) flags |= kErrRange;
-            const double Sd = (double)__half2float(__ushort_as_half(hbits));
             uint32_t z = 0;
-            if (Sd != 0.0 && !(flags & kErrRange)) {
-                const double zd = clamp015(rint(__ddiv_rn(-lo, Sd)));
-                z = (uint32_t)zd;
-#pragma unroll
-                for (int kk = 0; kk < 32; ++kk) {
-                    const double c = clamp015(__dadd_rn(rint(__ddiv_rn(v[kk], Sd)), zd));
-                    rec[kk >> 3] |= (uint32_t)c << (4 * (kk & 7));
-                }
-            }
+            if (!quantize_group32(v, rec, &hbits, &z, (flags & kErrRange) != 0)) flags |= kErrRange;
             sc[gg >> 1] |= (uint32_t)hbits << (16 * (gg & 1));
             zw |= z << (4 * gg);
         }

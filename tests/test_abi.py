@@ -189,3 +189,33 @@ def test_compacted_layer_checks(L):
                                   wsb, None, None) == _lib.ERR_ALIGN
     assert L.spectra_pack_compact(FAKE, 8, 120, FAKE, 2, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, wsb,
                                   None, None) == _lib.ERR_SHAPE
+
+
+def test_kv_argument_checks(L):
+    cb, sb, zb = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    assert L.spectra_kv_sizes(2, 128, 100, ctypes.byref(cb), ctypes.byref(sb), ctypes.byref(zb)) == _lib.OK
+    assert (cb.value, sb.value, zb.value) == (2 * 100 * 64, 2 * 100 * 4 * 2, 2 * 100 * 4)
+    assert L.spectra_kv_sizes(2, 96, 10, ctypes.byref(cb), ctypes.byref(sb), ctypes.byref(zb)) == _lib.OK
+    assert L.spectra_kv_sizes(2, 100, 10, ctypes.byref(cb), ctypes.byref(sb), ctypes.byref(zb)) == _lib.ERR_SHAPE
+    assert L.spectra_kv_sizes(2, 288, 10, ctypes.byref(cb), ctypes.byref(sb), ctypes.byref(zb)) == _lib.ERR_SHAPE
+    kv = _lib.KV(2, 128, 100, FAKE, FAKE, FAKE)
+    k = ctypes.byref(kv)
+    assert L.spectra_kv_append(k, None, 0, 5, None) == _lib.OK  # nothing to do: no CUDA call
+    assert L.spectra_kv_append(k, FAKE, 10, 95, None) == _lib.ERR_SHAPE
+    assert L.spectra_kv_append(k, FAKE, 1, -1, None) == _lib.ERR_INVALID_ARG
+    assert L.spectra_kv_append(k, FAKE + 1, 1, 0, None) == _lib.ERR_ALIGN
+    assert L.spectra_kv_append(ctypes.byref(_lib.KV(2, 128, 100, FAKE + 8, FAKE, FAKE)), FAKE, 1, 0,
+                               None) == _lib.ERR_ALIGN
+    ws = L.spectra_attention_workspace_size(12, 128, 100)
+    assert ws >= 12 * 130 * 4
+    att = L.spectra_attention_decode
+    other = ctypes.byref(_lib.KV(2, 128, 99, FAKE, FAKE, FAKE))
+    assert att(k, other, FAKE, 12, 50, 0.1, FAKE, FAKE, ws, None) == _lib.ERR_SHAPE
+    assert att(k, k, FAKE, 13, 50, 0.1, FAKE, FAKE, ws, None) == _lib.ERR_SHAPE  # not a multiple
+    assert att(k, k, FAKE, 18, 50, 0.1, FAKE, FAKE, ws, None) == _lib.ERR_SHAPE  # 9 per KV head
+    assert att(k, k, FAKE, 12, 0, 0.1, FAKE, FAKE, ws, None) == _lib.ERR_SHAPE
+    assert att(k, k, FAKE, 12, 101, 0.1, FAKE, FAKE, ws, None) == _lib.ERR_SHAPE
+    assert att(k, k, FAKE, 12, 100, float("nan"), FAKE, FAKE, ws, None) == _lib.ERR_INVALID_ARG
+    assert att(k, k, FAKE, 12, 100, 0.1, FAKE, FAKE, ws - 1, None) == _lib.ERR_BUFFER_TOO_SMALL
+    assert att(k, k, FAKE, 12, 100, 0.1, FAKE + 2, FAKE, ws, None) == _lib.ERR_ALIGN
+    assert att(k, k, None, 12, 100, 0.1, FAKE, FAKE, ws, None) == _lib.ERR_INVALID_ARG
