@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(kChunk) attn_partial_kernel(const AttnArgs a) 
     constexpr int kVStage = kChunk * (NG * 16 + NG * 2 + 4);
     constexpr int kRed = kWarps * kMaxGroup * D * 4;
     constexpr int kPool = kVStage > kRed ? kVStage : kRed;
-    __shared__ float qs[kMaxGroup][D];
+    __shared__ __align__(16) float qs[kMaxGroup][D];
     __shared__ float sc[kMaxGroup][kChunk];
     __shared__ __align__(16) unsigned char pool[kPool];
     __shared__ float wmax[kWarps][kMaxGroup], wsum[kWarps][kMaxGroup];
@@ -142,10 +142,20 @@ __global__ void __launch_bounds__(kChunk) attn_partial_kernel(const AttnArgs a) 
             vsr[g] = 0;
         }
     }
-    // query rows of the group, FP32
-    for (int i = tid; i < grp * D; i += kChunk) {
-        const int gi = i / D, d = i - gi * D;
-        qs[gi][d] = __uint_as_float((uint32_t)a.q[(size_t)(h * grp + gi) * D + d] << 16);
+    // query rows of the group, FP32: every load issued before the first store
+    // (a load-store loop would wait out one round trip per element)
+    constexpr int kQPer = kMaxGroup * D / kChunk;
+    uint32_t qraw[kQPer];
+    const uint16_t *qh = a.q + (size_t)h * grp * D;  // the group's rows are contiguous
+#pragma unroll
+    for (int u = 0; u < kQPer; ++u) {
+        const int i = tid + u * kChunk;
+        qraw[u] = i < grp * D ? (uint32_t)qh[i] : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < kQPer; ++u) {
+        const int i = tid + u * kChunk;
+        if (i < grp * D) qs[i / D][i % D] = __uint_as_float(qraw[u] << 16);
     }
     __syncthreads();
 
@@ -160,17 +170,30 @@ __global__ void __launch_bounds__(kChunk) attn_partial_kernel(const AttnArgs a) 
         for (int g = 0; g < NG; ++g) {
             const uint4 rec = a.kc[slot * NG + g];
             const float sg = __half2float(__ushort_as_half(a.ks[slot * NG + g]));
-            const int z = (int)((zw >> (4 * g)) & 0xFu);
+            const float nzs = -(float)((zw >> (4 * g)) & 0xFu) * sg;  // -z * s, exact
             const uint32_t wv[4] = {rec.x, rec.y, rec.z, rec.w};
 #pragma unroll
             for (int w = 0; w < 4; ++w)
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float kval = (float)((int)((wv[w] >> (4 * j)) & 0xFu) - z) * sg;
-                    const int d = 32 * g + 8 * w + j;
+                for (int j4 = 0; j4 < 2; ++j4) {
+                    // channels 32g + 8w + 4*j4 .. +3: (c - z) * s = fma(c, s, -z * s),
+                    // exact; c as a float by the 2^23 mantissa trick
+                    float kv[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const uint32_t code = (wv[w] >> (4 * (4 * j4 + u))) & 0xFu;
+                        kv[u] = fmaf(__uint_as_float(0x4B000000u | code) - 8388608.f, sg, nzs);
+                    }
+                    const int d4 = (32 * g + 8 * w + 4 * j4) / 4;
 #pragma unroll
                     for (int gi = 0; gi < kMaxGroup; ++gi)
-                        if (gi < grp) s[gi] = fmaf(kval, qs[gi][d], s[gi]);
+                        if (gi < grp) {
+                            const float4 qv = reinterpret_cast<const float4 *>(qs[gi])[d4];
+                            s[gi] = fmaf(kv[0], qv.x, s[gi]);
+                            s[gi] = fmaf(kv[1], qv.y, s[gi]);
+                            s[gi] = fmaf(kv[2], qv.z, s[gi]);
+                            s[gi] = fmaf(kv[3], qv.w, s[gi]);
+                        }
                 }
         }
     }
@@ -264,13 +287,13 @@ __global__ void __launch_bounds__(kChunk) attn_partial_kernel(const AttnArgs a) 
     }
 }
 
-// Merge of the chunk partials, one CTA per query head.  The chunk weights
-// exp(m_c - M) and the normaliser L are computed once by the whole CTA
-// (fixed-order reductions) and kept in shared memory in slices of kMergeSlice
-// chunks; each thread then sums its channel over the chunks in order, eight
-// independent loads in flight.
+// Merge of the chunk partials, one CTA per query head.  M (the largest chunk
+// maximum) and L = sum_c exp(m_c - M) l_c come from fixed-order block
+// reductions; the partial sums are staged slice by slice in shared memory
+// with independent 16-byte loads (one round trip per slice), and thread d
+// then sums channel d over the slice's chunks in order.
 constexpr int kMergeThreads = 256;
-constexpr int kMergeSlice = 1024;
+constexpr int kMergeFloats = 8192;  // one slice: 32 KB of partial sums
 
 __device__ float block_max(float v, float *red) {
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -295,7 +318,8 @@ __device__ float block_sum(float v, float *red) {
 }
 
 __global__ void __launch_bounds__(kMergeThreads) attn_combine_kernel(const AttnArgs a, int D) {
-    __shared__ float wt[kMergeSlice];
+    __shared__ __align__(16) float buf[kMergeFloats];
+    __shared__ float wt[kMergeFloats / 32];
     __shared__ float red[kMergeThreads / 32];
     const int i = blockIdx.x, tid = threadIdx.x;
     const int nch = a.nch;
@@ -306,27 +330,29 @@ __global__ void __launch_bounds__(kMergeThreads) attn_combine_kernel(const AttnA
     float l = 0.f;
     for (int c = tid; c < nch; c += kMergeThreads) l += expf(ml[2 * c] - M) * ml[2 * c + 1];
     const float L = block_sum(l, red);
-    float o[1] = {0.f};  // channel tid (head_dim <= 256 = kMergeThreads)
-    const float *acc = a.ws_acc + (size_t)i * nch * D;
-    for (int c0 = 0; c0 < nch; c0 += kMergeSlice) {
-        const int nc = min(kMergeSlice, nch - c0);
+    const int per = kMergeFloats / D;  // chunks per slice
+    float o = 0.f;
+    for (int c0 = 0; c0 < nch; c0 += per) {
+        const int nc = min(per, nch - c0);
+        const float4 *src = reinterpret_cast<const float4 *>(a.ws_acc + ((size_t)i * nch + c0) * D);
+        float4 *dst = reinterpret_cast<float4 *>(buf);
+        const int n4 = nc * D / 4;
+        int j = tid;
+        for (; j + 7 * kMergeThreads < n4; j += 8 * kMergeThreads) {
+            float4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = src[j + u * kMergeThreads];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) dst[j + u * kMergeThreads] = v[u];
+        }
+        for (; j < n4; j += kMergeThreads) dst[j] = src[j];
         for (int c = tid; c < nc; c += kMergeThreads) wt[c] = expf(ml[2 * (c0 + c)] - M);
         __syncthreads();
-        if (tid < D) {
-            const float *p = acc + (size_t)c0 * D + tid;
-            int c = 0;
-            for (; c + 8 <= nc; c += 8) {
-                float v[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) v[u] = p[(size_t)(c + u) * D];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) o[0] = fmaf(wt[c + u], v[u], o[0]);
-            }
-            for (; c < nc; ++c) o[0] = fmaf(wt[c], p[(size_t)c * D], o[0]);
-        }
+        if (tid < D)
+            for (int c = 0; c < nc; ++c) o = fmaf(wt[c], buf[c * D + tid], o);
         __syncthreads();
     }
-    if (tid < D) a.out[(size_t)i * D + tid] = o[0] / L;
+    if (tid < D) a.out[(size_t)i * D + tid] = o / L;
 }
 
 template <int NG>
@@ -340,9 +366,13 @@ cudaError_t launch_attn(const AttnArgs &args, cudaStream_t s) {
 
 }  // namespace
 
+// Workspace: [Hq][nch][2] chunk statistics, then (from a 16-byte boundary)
+// [Hq][nch][D] partial sums.
+size_t ml_floats(int Hq, int64_t nch) { return (size_t)((Hq * nch * 2 + 3) / 4 * 4); }
+
 size_t attention_workspace_bytes(int Hq, int D, int T) {
     const int64_t nch = cdiv(T, kChunk);
-    return (size_t)Hq * nch * (2 + D) * sizeof(float);
+    return (ml_floats(Hq, nch) + (size_t)Hq * nch * D) * sizeof(float);
 }
 
 int attention_max_group() { return kMaxGroup; }
@@ -374,7 +404,7 @@ spectra_status launch_attention(const spectra_kv &k, const spectra_kv &v, const 
     a.cap = k.capacity;
     a.nch = (int)cdiv(T, kChunk);
     a.ws_ml = static_cast<float *>(ws);
-    a.ws_acc = a.ws_ml + (size_t)Hq * a.nch * 2;
+    a.ws_acc = a.ws_ml + ml_floats(Hq, a.nch);
     a.out = out;
     cudaError_t e;
     switch (k.head_dim / 32) {
