@@ -8,6 +8,7 @@ statically, so the library needs only the NVIDIA driver at run time.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import glob
 import os
 import subprocess
@@ -46,14 +47,21 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
         return LIB
     objdir = os.path.join(PKG, "_build")
     os.makedirs(objdir, exist_ok=True)
-    objs = []
+    cmds, objs = [], []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
-        cmd = [NVCC, *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
+        cmds.append([NVCC, *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj])
+        objs.append(obj)
+    # one nvcc per source file, concurrently (outputs in file order)
+    with concurrent.futures.ThreadPoolExecutor(max_workers=max(1, min(len(cmds), os.cpu_count() or 1))) as ex:
+        results = list(ex.map(lambda c: subprocess.run(c, capture_output=True, text=True), cmds))
+    for cmd, r in zip(cmds, results):
         if verbose:
             print(" ".join(cmd), file=sys.stderr)
-        subprocess.check_call(cmd)
-        objs.append(obj)
+        if r.stdout or r.stderr:
+            print(r.stdout + r.stderr, file=sys.stderr, end="")
+        if r.returncode != 0:
+            raise subprocess.CalledProcessError(r.returncode, cmd)
     tmp = LIB + f".tmp{os.getpid()}"
     subprocess.check_call([NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared",
                            "-cudart", "static", "-o", tmp, *objs])

@@ -23,6 +23,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <thread>
 
 #include "internal.cuh"
 #include "spectra.h"
@@ -48,7 +49,8 @@ constexpr int kBuffers = 6;  // codes, scales, zeros, outlier_idx, outlier_w, bu
 
 // Reflected CRC-32 with the IEEE polynomial, eight bytes per step (the
 // "slicing" tables: tab[t][b] is the CRC contribution of byte b followed by
-// t zero bytes).
+// t zero bytes).  Buffers of 4 MB and more are split over up to eight
+// threads and the slices' CRCs combined (crc_concat).
 uint32_t g_tab[8][256];
 std::once_flag g_tab_once;
 
@@ -79,9 +81,71 @@ uint32_t crc_step(uint32_t s, const uint8_t *p, size_t n) {
     return s;
 }
 
-uint32_t crc(uint32_t prev, const void *data, size_t n) {
+uint32_t crc_serial(uint32_t prev, const void *data, size_t n) {
     std::call_once(g_tab_once, build_tables);
     return ~crc_step(~prev, static_cast<const uint8_t *>(data), n);
+}
+
+// Multiplication modulo the CRC polynomial in the reflected representation
+// (bit 31 is the coefficient of x^0, bit 0 that of x^31).
+uint32_t mulmod(uint32_t a, uint32_t b) {
+    uint32_t p = 0;
+    for (uint32_t m = 1u << 31; m; m >>= 1) {
+        if (a & m) p ^= b;
+        b = (b & 1u) ? (b >> 1) ^ 0xEDB88320u : b >> 1;  // b *= x
+    }
+    return p;
+}
+
+// x^(8n) modulo the polynomial: the operator that runs a CRC register
+// through n zero bytes.
+uint32_t x8n(uint64_t n) {
+    uint32_t r = 1u << 31;          // 1
+    uint32_t sq = 1u << 23;         // x^8
+    for (; n; n >>= 1) {
+        if (n & 1u) r = mulmod(r, sq);
+        sq = mulmod(sq, sq);
+    }
+    return r;
+}
+
+// CRC of A followed by B from the CRCs of the two parts: the register of A,
+// run through |B| zero bytes, XOR the CRC of B (the initial and final
+// inversions cancel out of the combination).
+uint32_t crc_concat(uint32_t crc_a, uint32_t crc_b, uint64_t len_b) {
+    return mulmod(x8n(len_b), crc_a) ^ crc_b;
+}
+
+// Large buffers are checksummed in slices on several threads and combined.
+constexpr size_t kParallelCrcBytes = 4u << 20;
+
+uint32_t crc(uint32_t prev, const void *data, size_t n) {
+    const unsigned hw = std::thread::hardware_concurrency();
+    if (n < kParallelCrcBytes || hw < 2) return crc_serial(prev, data, n);
+    std::call_once(g_tab_once, build_tables);
+    size_t parts = n / (1u << 20);
+    if (parts > 8) parts = 8;
+    if (parts > hw) parts = hw;
+    const size_t slice = (n / parts + 63) & ~(size_t)63;
+    uint32_t part_crc[8] = {0};
+    size_t part_len[8] = {0};
+    std::thread pool[8];
+    const uint8_t *p = static_cast<const uint8_t *>(data);
+    size_t used = 0;
+    for (size_t i = 0; i < parts; ++i) {
+        const size_t len = (i + 1 == parts) ? n - used : (slice < n - used ? slice : n - used);
+        part_len[i] = len;
+        const uint8_t *q = p + used;
+        uint32_t *out = &part_crc[i];
+        pool[i] = std::thread([q, len, out] { *out = crc_serial(0, q, len); });
+        used += len;
+    }
+    uint32_t c = prev;
+    for (size_t i = 0; i < parts; ++i) {
+        pool[i].join();
+        c = crc_concat(c, part_crc[i], part_len[i]);
+    }
+    return c;
 }
 
 // ---------------------------------------------------------------- layout
@@ -227,30 +291,65 @@ struct HostCopier {
     void drain() {}
 };
 
+// Checksum of one staged chunk, computed on a thread of its own.
+struct CrcJob {
+    std::thread t;
+    uint32_t value = 0;
+    size_t len = 0;
+    bool active = false;
+    void start(const uint8_t *p, size_t n) {
+        len = n;
+        active = true;
+        t = std::thread([this, p, n] { value = crc(0, p, n); });
+    }
+    // folds this chunk into the running CRC (chunks must be folded in order)
+    void finish(uint32_t *running) {
+        if (!active) return;
+        t.join();
+        *running = crc_concat(*running, value, len);
+        active = false;
+    }
+    ~CrcJob() {
+        if (t.joinable()) t.join();
+    }
+};
+
 // One buffer from the file into the caller's memory through the staging
-// halves: the file read of chunk j overlaps the copy of chunk j - 1.
+// halves.  Chunk j: wait until half j % 2 is free (its copy and its checksum
+// done), read the chunk into it, start its copy, and checksum it on a
+// thread while chunk j + 1 is read into the other half.  Checksums are
+// folded into the running CRC in chunk order.
 template <typename Copier>
 spectra_status load_buffer(int fd, uint64_t off, uint64_t bytes, uint8_t *dst, uint8_t *staging,
                            size_t half, bool verify, uint32_t *crc_out, Copier &cp) {
     uint32_t c = 0;
     bool pending[2] = {false, false};
+    CrcJob job[2];
     spectra_status st = SPECTRA_OK;
     for (uint64_t done = 0, j = 0; done < bytes && st == SPECTRA_OK; done += half, ++j) {
         const int k = (int)(j & 1);
         const size_t len = (size_t)((bytes - done) < half ? (bytes - done) : half);
         if (pending[k] && (st = cp.wait(k)) != SPECTRA_OK) break;
+        job[k].finish(&c);  // chunk j - 2 (chunk j - 1, if any, is still running)
         uint8_t *buf = staging + (size_t)k * half;
         if (!pread_all(fd, buf, len, off + done)) {
             st = SPECTRA_ERR_IO;
             break;
         }
-        if (verify) c = crc(c, buf, len);
         st = cp.copy(dst + done, buf, len, true, k);
         pending[k] = true;
+        if (verify && st == SPECTRA_OK) job[k].start(buf, len);
     }
+    // fold the remaining chunks in order: the earlier one is in the half of
+    // the second-to-last chunk
+    const uint64_t nchunks = bytes == 0 ? 0 : (bytes + half - 1) / half;
+    if (nchunks >= 2) job[(nchunks - 2) & 1].finish(&c);
+    if (nchunks >= 1) job[(nchunks - 1) & 1].finish(&c);
     for (int k = 0; k < 2 && st == SPECTRA_OK; ++k)
         if (pending[k]) st = cp.wait(k);
     if (st != SPECTRA_OK) {
+        job[0].finish(&c);
+        job[1].finish(&c);
         cp.drain();
         return st;
     }

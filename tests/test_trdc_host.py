@@ -188,3 +188,30 @@ def test_argument_checks(L, tmp_path):
     L.spectra_trdc_close(h)
     assert L.spectra_trdc_count(None) == 0
     L.spectra_trdc_close(None)
+
+
+def test_crc32_of_large_buffers_matches_zlib(L):
+    # 4 MB and more are checksummed in slices on several threads and combined
+    rng = np.random.default_rng(6)
+    for n in [4 << 20, (4 << 20) + 13, (17 << 20) + 5]:
+        data = rng.integers(0, 256, n, dtype=np.uint8).tobytes()
+        for prev in (0, 0xDEADBEEF):
+            assert L.spectra_crc32(prev, data, n) == zlib.crc32(data, prev)
+
+
+def test_large_buffer_container_round_trip(L, tmp_path):
+    # one 8.4 MB code buffer moving through 16 MB staging halves (threaded CRC)
+    spec = wl.MatrixSpec("single", 8192, 2080, 31)
+    wb = wl.bits(wl.weight(spec, seed=9))
+    p = oracle.pack(wb, wl.gain(spec, seed=9).numpy(), 6.0)
+    entries = [trdc.entry_from_packed("big", p.packed, 6.0)]
+    assert len(entries[0].buffers["codes"]) > 8 << 20
+    path = tmp_path / "big.trdc"
+    assert _write(L, path, entries, 32 << 20) == _lib.OK
+    assert path.read_bytes() == trdc.write_bytes(entries)
+    st, h = _open(L, path)
+    assert st == _lib.OK
+    st, dst, _ = _load(L, h, 0, _info(L, h, 0), 32 << 20)
+    L.spectra_trdc_close(h)
+    assert st == _lib.OK
+    assert dst["codes"].tobytes() == entries[0].buffers["codes"]
