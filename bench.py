@@ -728,7 +728,10 @@ def run_ours(args):
             "steps": c_steps}
         del graph_c, st_c
     if rank == 0 and not args.quick:
-        extra["trdc_container_4_layers"] = container_row(st, stream)
+        try:
+            extra["trdc_container_4_layers"] = container_row(st, stream)
+        except Exception as exc:  # an auxiliary row: report it, keep the benchmark line
+            extra["trdc_container_4_layers"] = {"error": f"{type(exc).__name__}: {exc}"}
         extra.update(extras(device, stream, peak, args.tau))
 
     cpu = None
