@@ -27,8 +27,12 @@
  *   - Device pointers must be 16-byte aligned (SPECTRA_ERR_ALIGN otherwise).
  *   - Results are bit-identical from run to run: every reduction has a fixed
  *     order.
- *   - No exception crosses the ABI.  The only library state is a per-device
- *     cache of device properties, filled on first use under a lock.
+ *   - No exception crosses the ABI.  Library state: a per-device cache of
+ *     device properties (filled on first use under a lock), per-device
+ *     status flags that kernels raise and spectra_device_status reads and
+ *     clears, the CRC-32 tables (built once), and the fixed scratch array of
+ *     spectra_pack_plan_noalloc.  Container readers are handles the caller
+ *     owns (spectra_trdc_open / spectra_trdc_close).
  *
  * Shapes: n = out_features (rows of W), k = in_features (columns), m = batch
  * rows of x.  k must be a positive multiple of 32; n >= 1.
