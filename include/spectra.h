@@ -329,8 +329,11 @@ SPECTRA_API spectra_status spectra_gemv_batched(const spectra_layer *layers,
  * bounds.  Asynchronous, allocates nothing, graph-capturable; launched with
  * programmatic dependent launch (it reads ids only after the previous kernel
  * on the stream has completed).
- * Errors: INVALID_ARG, SHAPE (m < 0, or a bad table shape), ALIGN,
- * UNSUPPORTED, CUDA.
+ * Each row is assembled in shared memory, so k * (4 for FP32, 2 for BF16)
+ * must fit the device's shared memory per block (B200: k <= 58112 for FP32,
+ * 116224 for BF16 rows).
+ * Errors: INVALID_ARG, SHAPE (m < 0, a bad table shape, or a row too large
+ * for shared memory), ALIGN, UNSUPPORTED, CUDA.
  */
 SPECTRA_API spectra_status spectra_embed(const spectra_layer *table, const int32_t *ids, int32_t m,
                                          void *out, spectra_dtype out_dtype, void *stream);
