@@ -219,3 +219,14 @@ def test_kv_argument_checks(L):
     assert att(k, k, FAKE, 12, 100, 0.1, FAKE, FAKE, ws - 1, None) == _lib.ERR_BUFFER_TOO_SMALL
     assert att(k, k, FAKE, 12, 100, 0.1, FAKE + 2, FAKE, ws, None) == _lib.ERR_ALIGN
     assert att(k, k, None, 12, 100, 0.1, FAKE, FAKE, ws, None) == _lib.ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path, monkeypatch):
+    # no fallback: with the shared library absent, the first call raises
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "libspectra.so"))
+    monkeypatch.setattr(_lib, "_lib", None)
+    import outlier_split_bit_b200 as sp
+    with pytest.raises(ImportError):
+        sp.spectra_version()
+    with pytest.raises(ImportError):
+        sp.spectra_packed_sizes(32, 64, 0)
