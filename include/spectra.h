@@ -450,6 +450,11 @@ SPECTRA_API spectra_status spectra_attention_decode(const spectra_kv *k, const s
  * double-buffered (the file read of one chunk overlaps the copy of the
  * other).  The library allocates no host memory proportional to the
  * model: only the reader handle (the layer records).
+ * Threads: checksums of chunks of 4 MB and more are computed on up to eight
+ * short-lived helper threads (and, while loading, on a thread that runs
+ * beside the next file read); every thread is joined before the call
+ * returns.  A reader handle may serve concurrent spectra_trdc_load calls
+ * (reads use explicit offsets); spectra_trdc_close must not overlap them.
  */
 typedef enum { SPECTRA_MEM_DEVICE = 0, SPECTRA_MEM_HOST = 1 } spectra_memory;
 
