@@ -735,6 +735,10 @@ def run_ours(args):
             extra["decode_stream_tau6"] = {"error": f"{type(exc).__name__}: {exc}"}
     if rank == 0 and not args.quick:
         try:
+            extra["tau_sweep_1p5b_layer0"] = tau_sweep_rows(device, stream)
+        except Exception as exc:  # an auxiliary row: report it, keep the benchmark line
+            extra["tau_sweep_1p5b_layer0"] = {"error": f"{type(exc).__name__}: {exc}"}
+        try:
             extra["trdc_container_4_layers"] = container_row(st, stream)
         except Exception as exc:  # an auxiliary row: report it, keep the benchmark line
             extra["trdc_container_4_layers"] = {"error": f"{type(exc).__name__}: {exc}"}
@@ -791,6 +795,47 @@ def run_ours(args):
     if world > 1:
         dist.destroy_process_group()
     return 0
+
+
+def tau_sweep_rows(device, stream, taus=(2.0, 3.0, 4.0, 5.0, 6.0, 8.0, float("inf"))):
+    """The threshold sweep over the seven matrices of layer 0 of the
+    1.5B-class stack: outlier columns, bits per weight of the masked and the
+    compacted bulk (and the size against BF16, the pages' container ratio,
+    which they quote as 2.80-3.31x on their models), and the matvec's
+    relative error against the dense BF16 product, ||y - W x|| / ||W x||."""
+    import outlier_split_bit_b200 as sp
+    mats = []
+    for spec in wl.LAYER_1P5B:
+        w = wl.weight(spec, 0, 0, device=device)
+        g = wl.gain(spec, 0, 0, device=device)
+        x = wl.activations(spec.k, 1, device=device)[0]
+        mats.append((spec, w, g, x, (w.float() @ x.float())))
+    torch.cuda.synchronize()  # inputs come from the default stream
+    weights = sum(s.n * s.k for s, *_ in mats)
+    rows = []
+    with torch.cuda.stream(stream):
+        for tau in taus:
+            row = {"tau": tau if tau != float("inf") else "inf", "n_outliers": 0}
+            for compact in (False, True):
+                nbytes, num, den = 0, 0.0, 0.0
+                for spec, w, g, x, dense in mats:
+                    lay = sp.pack_layer(w, g, tau, compact=compact, stream=stream)
+                    y = sp.spectra_gemv(lay, x, stream=stream)
+                    stream.synchronize()
+                    nbytes += lay.nbytes
+                    num += float(torch.linalg.vector_norm(y - dense)) ** 2
+                    den += float(torch.linalg.vector_norm(dense)) ** 2
+                    if not compact:
+                        row["n_outliers"] += lay.n_outliers
+                    del lay, y
+                key = "compacted" if compact else "masked"
+                row[f"bits_per_weight_{key}"] = round(8 * nbytes / weights, 3)
+                row[f"ratio_vs_bf16_{key}"] = round(16 * weights / (8 * nbytes), 3)
+                row[f"rel_err_{key}"] = round((num / den) ** 0.5, 5)
+            row["outlier_fraction"] = round(row["n_outliers"] / sum(s.k for s, *_ in mats), 4)
+            rows.append(row)
+    del mats
+    return rows
 
 
 def stream_row(device, stream, rank, tau, args, peak):
