@@ -17,6 +17,13 @@ from HBM.  The per-matrix and batch rows time back-to-back launches cycling
 over copies of the matrix that together exceed twice the L2 (each launch
 reads DRAM, launch latency overlaps as in a decode stream); the single-launch
 time with the L2 flushed beforehand is reported beside them.
+Further rows of the same line: the stream with the compacted bulk and at
+tau = 6.0, the threshold sweep (outlier columns, bits per weight, matvec
+error against the dense BF16 product), the TRDC container written and
+streamed back, the LM head at M = 1 (four outlier fractions, masked and
+compacted) and at 16 / 32 rows on the tensor cores, the 4B-class batch
+sweep, the embedding-row gather and decode attention over the 4-bit KV
+cache.  --case single|embed|kv times one workload alone.
 Rank 0 prints one JSON line.  For N > 1 every rank (one per GPU) runs its own
 replica of the stream: the problems are independent, there is no data-path
 collective, and the value is the bytes of all ranks over the slowest rank's
