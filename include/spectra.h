@@ -10,7 +10,10 @@
  * group of 32 consecutive weights of a row.  Decoding happens in registers
  * inside the matrix-vector kernel, which also runs the dense matvec of the
  * BF16 outlier columns in the same pass (abstract: the dequantisation is
- * fused into the kernels' register pipelines).
+ * fused into the kernels' register pipelines).  Around the matvec: the
+ * packing steps, a compacted form of the bulk, rows of a packed table
+ * gathered as embeddings, the Group-32 4-bit KV cache with decode attention
+ * over it, and the self-contained container the layers are stored in.
  *
  * Conventions shared by every entry point:
  *   - All pointers named *_dev or documented as "device" are CUDA device
@@ -24,7 +27,8 @@
  *     status and leaves every output untouched.  Launch failures return
  *     SPECTRA_ERR_CUDA.  Faults of asynchronous work surface at the caller's
  *     next synchronisation.
- *   - Device pointers must be 16-byte aligned (SPECTRA_ERR_ALIGN otherwise).
+ *   - Device pointers must be 16-byte aligned unless an entry states a
+ *     weaker rule (SPECTRA_ERR_ALIGN otherwise).
  *   - Results are bit-identical from run to run: every reduction has a fixed
  *     order.
  *   - No exception crosses the ABI.  Library state: a per-device cache of
@@ -85,10 +89,13 @@ extern "C" {
 
 typedef enum {
     SPECTRA_OK = 0,
-    SPECTRA_ERR_INVALID_ARG = 1,      /* null pointer, negative count, bad enum value */
-    SPECTRA_ERR_SHAPE = 2,            /* k % 32 != 0, k < 32, n < 1, m outside [1, 32], too large */
-    SPECTRA_ERR_ALIGN = 3,            /* a device pointer is not 16-byte aligned */
-    SPECTRA_ERR_NONFINITE = 4,        /* NaN or infinity in W or in the gain */
+    SPECTRA_ERR_INVALID_ARG = 1,      /* null pointer, negative count, bad enum value; a
+                                         gathered id outside the table (device status) */
+    SPECTRA_ERR_SHAPE = 2,            /* k % 32 != 0, k < 32, n < 1, m outside [1, 32], a KV
+                                         shape or length out of range, too large */
+    SPECTRA_ERR_ALIGN = 3,            /* a pointer is not aligned as its entry requires */
+    SPECTRA_ERR_NONFINITE = 4,        /* NaN or infinity in W, in the gain, or in appended
+                                         K/V values (device status) */
     SPECTRA_ERR_RANGE = 5,            /* a group's scale (max-min)/15 overflows FP16 */
     SPECTRA_ERR_BUFFER_TOO_SMALL = 6, /* workspace smaller than the stated size */
     SPECTRA_ERR_CUDA = 7,             /* a CUDA runtime call failed */
