@@ -204,9 +204,9 @@ SPECTRA_API spectra_status spectra_pack_plan(const uint16_t *w, const float *gai
  *     contents.  Calls that overlap on the GPU (issued on two streams or from
  *     two host threads for the same device) race on it: serialise them.
  *     Each call clears the words that must start at zero.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before capturing a stream into a graph.
+ *   - Every call looks up the array's device address (cudaGetSymbolAddress)
+ *     on the current device, so an address is never reused after a reset of
+ *     the device's context moved the array.
  * Synchronous, like spectra_pack_plan.
  */
 SPECTRA_API spectra_status spectra_pack_plan_noalloc(const uint16_t *w, const float *gain,
@@ -358,6 +358,18 @@ SPECTRA_API spectra_status spectra_embed(const spectra_layer *table, const int32
  * the KV append, else SPECTRA_OK.  Synchronous on `stream`.
  */
 SPECTRA_API spectra_status spectra_device_status(void *stream);
+
+/*
+ * Exercises the failure path of the kernels' bounded waits without a fault.
+ * kind 0 launches one warp that acquires a stage of a weight ring (the
+ * cp.async.bulk + mbarrier ring of the matvec kernels) that no copy ever
+ * fills.  Its wait gives up after the kernels' limit (one second of
+ * %globaltimer time), the launch raises the flag that spectra_device_status
+ * then reports as SPECTRA_ERR_INTERNAL, and the context stays usable.
+ * For tests of callers' error handling; asynchronous, allocates nothing.
+ * Errors: INVALID_ARG (unknown kind), UNSUPPORTED, CUDA.
+ */
+SPECTRA_API spectra_status spectra_selftest_wait(int32_t kind, void *stream);
 
 /*
  * Group-32 4-bit KV cache (abstract: microscaled Group-32 4-bit key-value

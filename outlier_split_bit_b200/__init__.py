@@ -79,6 +79,12 @@ def spectra_device_status(*, stream=None) -> None:
     _check(_L.spectra_device_status(_stream(stream)), "spectra_device_status")
 
 
+def spectra_selftest_wait(kind: int = 0, *, stream=None) -> None:
+    """Launch a kernel whose bounded wait can never be satisfied; the next
+    spectra_device_status reports SPECTRA_ERR_INTERNAL."""
+    _check(_L.spectra_selftest_wait(int(kind), _stream(stream)), "spectra_selftest_wait")
+
+
 def _sizes(s: Sizes) -> dict:
     return {"n_pad": s.n_pad, "codes": s.codes_bytes, "scales": s.scales_bytes,
             "zeros": s.zeros_bytes, "outlier_idx": s.outlier_idx_bytes,

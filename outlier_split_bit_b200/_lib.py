@@ -77,6 +77,7 @@ SIGNATURES = {
     "spectra_gemm_small": (ctypes.c_int, [LP, P, i32, P, ctypes.c_int, P]),
     "spectra_gemv_batched": (ctypes.c_int, [LP, P, P, i32, ctypes.c_int, P]),
     "spectra_device_status": (ctypes.c_int, [P]),
+    "spectra_selftest_wait": (ctypes.c_int, [i32, P]),
     "spectra_embed": (ctypes.c_int, [LP, P, i32, P, ctypes.c_int, P]),
     "spectra_pack_plan_noalloc": (ctypes.c_int, [P, P, i32, i32, f64, P, P, ctypes.POINTER(i32), P]),
     "spectra_crc32": (ctypes.c_uint32, [ctypes.c_uint32, P, sz]),

@@ -419,6 +419,14 @@ spectra_status spectra_attention_decode(const spectra_kv *k, const spectra_kv *v
                             (cudaStream_t)stream);
 }
 
+spectra_status spectra_selftest_wait(int32_t kind, void *stream) {
+    if (kind != 0) return SPECTRA_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    spectra_status st = current_device(&dev);
+    if (st != SPECTRA_OK) return st;
+    return launch_wait_selftest(kind, (cudaStream_t)stream);
+}
+
 spectra_status spectra_device_status(void *stream) {
     DeviceInfo dev;
     spectra_status st = current_device(&dev);

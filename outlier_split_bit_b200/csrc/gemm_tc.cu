@@ -111,36 +111,15 @@ __device__ __forceinline__ int tc_unit(const Prob &a, int sg0, int nsg, int ob0,
     return lu < nsg ? sg0 + lu : a.S + ob0 + (lu - nsg);
 }
 
-// Shared state of a CTA that turns every later wait into a no-op once one
-// has timed out.
-__device__ __forceinline__ uint64_t global_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    return t;
-}
-
-constexpr uint64_t kTcWaitNs = 1000000000ull;  // a wait gives up after one second
-
+// A bounded mbarrier wait that also turns every later wait of the CTA into a
+// no-op once one has timed out (`abort` is CTA-shared).
 __device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile int *abort) {
-    uint64_t t0 = 0;
-    for (uint32_t i = 0;; ++i) {
-        uint32_t ok;
-        // the thread sleeps until the phase completes or the hint expires, so
-        // a waiting lane leaves the issue slots to the warps that build operands
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(ok)
-            : "r"(bar), "r"(parity), "r"(kSuspendNs)
-            : "memory");
-        if (ok) return true;
+    if (mbar_try(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 0; i < kWaitRounds; ++i) {
+        if (mbar_try(bar, parity)) return true;
         if (*abort) return false;
-        const uint64_t now = global_ns();
-        if (i == 0)
-            t0 = now;
-        else if (now - t0 > kTcWaitNs)
-            break;
+        if (global_ns() - t0 > kWaitNs) break;
     }
     *abort = 1;
     atomicOr(&g_device_error, 1u);

@@ -989,6 +989,20 @@ spectra_status run_one(const Prob &a, const DeviceInfo &dev, cudaStream_t s) {
     return run_cluster<MB>(a, p, dev, s);
 }
 
+// One warp acquires the first stage of a one-stage weight ring that no copy
+// ever fills: the ring's bounded wait gives up after its limit and raises
+// this translation unit's error flag, exactly as in a matvec kernel.
+__global__ void ring_wait_selftest_kernel() {
+    __shared__ __align__(16) uint8_t stage[16];
+    __shared__ __align__(8) uint64_t bar[1];
+    const int lane = threadIdx.x & 31;
+    Ring r;
+    ring_init(r, stage, bar, 1, lane);
+    (void)ring_acquire(r, lane);
+    ring_release(r);
+    ring_drain(r);
+}
+
 }  // namespace
 
 // This translation unit's error word (the matvec kernels), then the
@@ -1052,6 +1066,12 @@ spectra_status launch_gemv_batched(const spectra_layer *layers, const uint16_t *
         fill_prob(args.probs[i], layers[i], g, xs[i], 1, ys[i], ytype);
     }
     return run_persistent<1>(args, count, dev, s);
+}
+
+spectra_status launch_wait_selftest(int kind, cudaStream_t s) {
+    if (kind != 0) return SPECTRA_ERR_INVALID_ARG;
+    ring_wait_selftest_kernel<<<1, 32, 0, s>>>();
+    return cudaGetLastError() == cudaSuccess ? SPECTRA_OK : SPECTRA_ERR_CUDA;
 }
 
 }  // namespace spectra

@@ -88,6 +88,9 @@ spectra_status launch_gemv(const spectra_layer &l, const uint16_t *x, int m, voi
 // Reads (and clears) the flag the matvec kernels raise when a bounded wait
 // for a weight copy gives up.
 spectra_status device_error(bool *raised, cudaStream_t s);
+// A kernel whose bounded wait can never be satisfied (kind 0: the weight
+// ring's mbarrier wait); it gives up after its limit and raises the flag.
+spectra_status launch_wait_selftest(int kind, cudaStream_t s);
 // Independent batch-1 matvecs in one launch (count <= kMaxBatch).
 spectra_status launch_gemv_batched(const spectra_layer *layers, const uint16_t *const *xs,
                                    void *const *ys, int count, int ytype, cudaStream_t s,

@@ -10,8 +10,6 @@
 // fixed array that the library itself holds, so the call allocates nothing.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "internal.cuh"
 #include "spectra.h"
 
@@ -26,21 +24,16 @@ constexpr size_t kScratchBytes = kKappaBytes + 256;
 // Each device that loads the library keeps it until the process exits.
 __device__ __align__(256) unsigned char g_plan_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-unsigned char *g_scratch_addr[kMaxDevices];  // device address of g_plan_scratch, per device
-
 // Device address of the scratch array on the current device.  The symbol's
 // name in host code is only a host-side handle, so the address comes from
-// cudaGetSymbolAddress, once per device, with that device current.
-spectra_status scratch_address(int dev, unsigned char **out) {
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_plan_scratch) != cudaSuccess || !p) return SPECTRA_ERR_CUDA;
-        g_scratch_addr[dev] = static_cast<unsigned char *>(p);
-    }
-    *out = g_scratch_addr[dev];
+// cudaGetSymbolAddress, with the device current.  It is looked up on every
+// call (the lookup allocates nothing): after a reset of the device's primary
+// context the module is loaded again and the array may sit elsewhere, so a
+// cached address could point into another allocation.
+spectra_status scratch_address(unsigned char **out) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_plan_scratch) != cudaSuccess || !p) return SPECTRA_ERR_CUDA;
+    *out = static_cast<unsigned char *>(p);
     return SPECTRA_OK;
 }
 
@@ -66,7 +59,7 @@ extern "C" spectra_status spectra_pack_plan_noalloc(const uint16_t *w, const flo
     spectra_status st = current_device(&dev);
     if (st != SPECTRA_OK) return st;
     unsigned char *scratch = nullptr;
-    st = scratch_address(dev.device, &scratch);
+    st = scratch_address(&scratch);
     if (st != SPECTRA_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
     double *kappa = kappa_out ? kappa_out : reinterpret_cast<double *>(scratch);

@@ -24,8 +24,9 @@ constexpr int kOB = 8;                         // outlier octets per unit
 constexpr int kSgBytes = 8 * 512 + 512 + 128;  // codes + scales + zeros of a warp per super-group
 constexpr int kOctBytes = 512;                 // outlier bytes of a warp per octet
 constexpr int kStageBytes = kSgBytes;          // one ring stage (16-byte multiple)
-constexpr uint32_t kSpinLimit = 1u << 12;      // try_wait rounds before a wait gives up
-constexpr uint32_t kSuspendNs = 500000;        // per-round suspend hint: the limit is ~2 s
+constexpr uint64_t kWaitNs = 1000000000ull;    // a wait gives up after one second (%globaltimer)
+constexpr uint32_t kWaitRounds = 1u << 22;      // backstop on try_wait rounds
+constexpr uint32_t kSuspendNs = 500000;        // per-round suspend hint (an upper bound only)
 
 // Set (bit 0) when a bounded wait in a kernel gave up; read and cleared by
 // spectra_device_status().
@@ -90,20 +91,37 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
         : "memory");
 }
 
-// Wait for phase `parity` of an mbarrier; gives up after kSpinLimit rounds.
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// One try of phase `parity` of an mbarrier.  The thread sleeps until the
+// phase completes or the suspend hint expires (it may also return earlier),
+// so waiting warps leave the issue slots to the computing ones.
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(kSuspendNs)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for phase `parity` of an mbarrier.  Bounded by elapsed time: it gives
+// up once kWaitNs of %globaltimer time have passed since the first failed
+// try (the count of tries is only a backstop, since a try may return before
+// its hint expires).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kSpinLimit; ++i) {
-        uint32_t ok;
-        // the thread sleeps until the phase completes or the hint expires,
-        // so waiting warps leave the issue slots to the computing ones
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(ok)
-            : "r"(bar), "r"(parity), "r"(kSuspendNs)
-            : "memory");
-        if (ok) return true;
+    if (mbar_try(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 0; i < kWaitRounds; ++i) {
+        if (mbar_try(bar, parity)) return true;
+        if (global_ns() - t0 > kWaitNs) return false;
     }
     return false;
 }

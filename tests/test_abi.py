@@ -230,3 +230,10 @@ def test_binding_fails_loudly_without_the_library(tmp_path, monkeypatch):
         sp.spectra_version()
     with pytest.raises(ImportError):
         sp.spectra_packed_sizes(32, 64, 0)
+
+
+def test_selftest_wait_argument_checks(L):
+    # unknown kinds are rejected on the host, before any CUDA call
+    for kind in (-1, 1, 7):
+        assert L.spectra_selftest_wait(kind, None) == _lib.ERR_INVALID_ARG
+

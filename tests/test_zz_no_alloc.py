@@ -31,12 +31,22 @@ def _noalloc(L, w, g, tau, kappa_out):
     torch.cuda.synchronize()
     gc.collect()  # no collection of earlier tests' tensors inside the measured call
     gc.disable()
+    args = (w.data_ptr(), None if g is None else g.data_ptr(), n, k, float(tau),
+            None if kappa_out is None else kappa_out.data_ptr(), idx.data_ptr(), ctypes.byref(n_o),
+            stream)
     try:
+        # one call first: the library's code and its fixed array are loaded on
+        # first use, which the device-wide count below would otherwise see
+        assert L.spectra_pack_plan_noalloc(*args) == _lib.OK
         before = torch.cuda.memory_allocated()
-        st = L.spectra_pack_plan_noalloc(w.data_ptr(), None if g is None else g.data_ptr(), n, k,
-                                         float(tau), None if kappa_out is None else kappa_out.data_ptr(),
-                                         idx.data_ptr(), ctypes.byref(n_o), stream)
+        reserved = torch.cuda.memory_reserved()
+        # device-wide free bytes also see a cudaMalloc inside the library,
+        # which torch's allocator counters cannot
+        free = torch.cuda.mem_get_info()[0]
+        st = L.spectra_pack_plan_noalloc(*args)
         assert torch.cuda.memory_allocated() == before
+        assert torch.cuda.memory_reserved() == reserved
+        assert torch.cuda.mem_get_info()[0] == free
     finally:
         gc.enable()
     assert st == _lib.OK, sp.spectra_status_string(st)
