@@ -370,29 +370,28 @@ def extras(device, stream, peak_gbs, tau):
             "gbs": round(b / us * 1e-3, 1), "frac": round(b / us * 1e-3 / peak_gbs, 3), "bytes": b,
             "bits_per_weight": round(8 * lay.nbytes / (spec.n * spec.k), 3)}
         del w, lay
+        # the batch sweep over all seven 4B-class projections (M >= 8 on the
+        # tensor cores), back to back over copies larger than twice the L2
         rows = []
-        spec = wl.LAYER_4B[4]
-        w = wl.weight(spec, 0, 0, device=device)
-        g = wl.gain(spec, 0, 0, device=device)
-        lay = sp.pack_layer(w, g, tau)
-        v = lay.view()
-        cps = copies_of(lay, L2_ROTATE_BYTES)
-        vs = [c.view() for c in cps]
-        for m in wl.BATCH_SWEEP:
-            x = wl.activations(spec.k, m, device=device)
-            y = torch.empty((m, spec.n), device=device)
-            us, p10, p90 = time_single(
-                lambda: sp.spectra_gemm_small(lay, x, y, view=v, stream=stream), stream, 30, flush)
-            fns = [(lambda c=c, vv=vv: sp.spectra_gemm_small(c, x, y, view=vv, stream=stream))
-                   for c, vv in zip(cps, vs)]
-            us_r = time_rotating(fns, stream, max(2, 200 // len(fns)))
-            b = algorithmic_bytes(spec.n, spec.k, lay.n_outliers, m=m)
-            rows.append({"m": m, "us": round(us_r, 2), "gbs": round(b / us_r * 1e-3, 1),
-                         "frac": round(b / us_r * 1e-3 / peak_gbs, 3),
-                         "tflops": round(2 * m * spec.n * spec.k / us_r * 1e-6, 2),
-                         "us_single_flushed": round(us, 2)})
-        out["batch_sweep_4b_gate_9728x2560"] = rows
-        del w, lay, cps
+        for spec in wl.LAYER_4B:
+            w = wl.weight(spec, 0, 0, device=device)
+            g = wl.gain(spec, 0, 0, device=device)
+            lay = sp.pack_layer(w, g, tau)
+            del w
+            cps = copies_of(lay, L2_ROTATE_BYTES)
+            vs = [c.view() for c in cps]
+            for m in wl.BATCH_SWEEP:
+                x = wl.activations(spec.k, m, device=device)
+                y = torch.empty((m, spec.n), device=device)
+                fns = [(lambda c=c, vv=vv: sp.spectra_gemm_small(c, x, y, view=vv, stream=stream))
+                       for c, vv in zip(cps, vs)]
+                us_r = time_rotating(fns, stream, max(2, 200 // len(fns)))
+                b = algorithmic_bytes(spec.n, spec.k, lay.n_outliers, m=m)
+                rows.append({"matrix": spec.name, "m": m, "us": round(us_r, 2),
+                             "gbs": round(b / us_r * 1e-3, 1), "frac": round(b / us_r * 1e-3 / peak_gbs, 3),
+                             "tflops": round(2 * m * spec.n * spec.k / us_r * 1e-6, 2)})
+            del lay, cps, vs
+        out["batch_sweep_4b"] = rows
         # the tensor-core path on the large matrix (1 % Student-t columns)
         rows = []
         spec = wl.lm_head_spec(0.01)
@@ -428,7 +427,44 @@ def extras(device, stream, peak_gbs, tau):
         out["embed_rows_131072x3072_bf16"] = rows
         del w, lay
         out["kv_attention_decode_8192"] = kv_rows(device, stream, peak_gbs, flush)
+        out["single_512x512"] = single_512_rows(device, stream, peak_gbs, flush)
     return out
+
+
+def single_512_rows(device, stream, peak_gbs, flush):
+    """The 512 x 512 layer (10 Student-t columns, gain, seed 0) at M = 1 and
+    both thresholds: a launch alone after an L2 flush, back to back on the same
+    (L2-resident, 0.15 MB) buffers, and the CPU oracle's matvec of the same
+    packed layer (unpack + FP64 product, one thread) beside it."""
+    import oracle
+    import outlier_split_bit_b200 as sp
+    oracle.build()
+    spec = wl.SINGLE_512
+    w = wl.weight(spec, 0, 0, device=device)
+    g = wl.gain(spec, 0, 0, device=device)
+    x = wl.activations(spec.k, 1, device=device)
+    wb, xb, gn = wl.bits(w), wl.bits(x), g.cpu().numpy()
+    rows = []
+    for tau in (3.0, 6.0):
+        lay = sp.pack_layer(w, g, tau)
+        y = torch.empty(spec.n, device=device)
+        v = lay.view()
+        fn = lambda: sp.spectra_gemv(lay, x[0], y, view=v, stream=stream)  # noqa: E731
+        us, _, _ = time_single(fn, stream, 50, flush)
+        us_r = time_rotating([fn], stream, 400)
+        ref = oracle.pack(wb, gn, tau)
+        reps, t0 = 0, time.perf_counter()
+        while reps < 3 or time.perf_counter() - t0 < 0.5:
+            oracle.gemm(oracle.unpack_layout(ref.packed), wb, ref.idx, xb)
+            reps += 1
+        o_us = (time.perf_counter() - t0) / reps * 1e6
+        b = algorithmic_bytes(spec.n, spec.k, lay.n_outliers)
+        rows.append({"tau": tau, "n_outliers": lay.n_outliers, "bytes": b,
+                     "us_back_to_back": round(us_r, 2), "us_single_flushed": round(us, 2),
+                     "gbs_back_to_back": round(b / us_r * 1e-3, 1),
+                     "oracle_us_1thread": round(o_us, 1)})
+        del lay
+    return rows
 
 
 def kv_rows(device, stream, peak_gbs, flush, T: int = 8192):
@@ -469,68 +505,160 @@ def kv_rows(device, stream, peak_gbs, flush, T: int = 8192):
 
 # ---------------------------------------------------------------- oracle leg
 
-def oracle_sample(seed: int, tau: float, tiles_per_matrix: int, reps: int = 1):
-    """Time the CPU oracle's matvec (unpack of the packed layout + FP64 product)
-    on whole 32-row tiles of each matrix of one layer.  Returns (bytes, seconds,
-    description)."""
+def host_cpu():
+    """(usable cores, CPU model) of this host."""
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return cores, model
+
+
+def oracle_layer(tau: float):
+    """The seven matrices of layer 0 of the 1.5B-class stack drawn on the host
+    (weights, gain, x as raw bits), in workload order."""
+    mats = []
+    for spec in wl.LAYER_1P5B:
+        w = wl.weight(spec, 0, 0, device="cpu")
+        g = wl.gain(spec, 0, 0, device="cpu")
+        x = wl.bits(wl.activations(spec.k, 1, 0, 0, slot=wl.PROJ.index(spec.name)))
+        mats.append((spec, wl.bits(w), None if g is None else g.numpy(), x))
+    return mats
+
+
+def matvec_items(mats, packed, tiles_per_item: int = 8):
+    """Work items of the oracle's matvec: blocks of row tiles of one matrix."""
+    items = []
+    for (spec, wb, gn, x), lay in zip(mats, packed):
+        T = -(-spec.n // 32)
+        for ta in range(0, T, tiles_per_item):
+            items.append((spec, lay, wb, x, ta, min(T, ta + tiles_per_item)))
+    return items
+
+
+def oracle_matvec(item):
+    """Unpack one block of row tiles from the oracle's packed layout and
+    multiply it in FP64; returns its algorithmic bytes."""
+    import oracle
+    spec, lay, wb, x, ta, tb = item
+    p = lay.packed
+    G, S = spec.k // 32, -(-(spec.k // 32) // 8)
+    r0, r1 = 32 * ta, min(spec.n, 32 * tb)
+    sub = oracle.Packed(p.codes[ta * G * 512:tb * G * 512], p.scales[ta * S * 256:tb * S * 256],
+                        p.zeros[ta * S * 32:tb * S * 32], p.outliers, p.idx, r1 - r0, spec.k)
+    oracle.gemm(oracle.unpack_layout(sub), wb[r0:r1], lay.idx, x)
+    return algorithmic_bytes(r1 - r0, spec.k, lay.idx.size)
+
+
+def cpu_baseline(tau: float, budget_s: float = 4.0):
+    """The oracle, as it stands, on this host's cores: the matvec (unpack of
+    the packed layout + FP64 product) and the pack (kurtosis, split, group
+    quantiser, layout) of the seven matrices of one 1.5B-class layer, each
+    timed on one thread and on every usable core (a thread per core; the
+    oracle's C routines release the interpreter lock).  Matvec throughput is
+    algorithmic GB/s, as on the GPU; pack throughput is weights per second."""
+    import concurrent.futures
     import oracle
     oracle.build()
-    prepared = []
-    for spec in wl.LAYER_1P5B:
-        w = wl.weight(spec, seed, 0, device="cpu")
-        g = wl.gain(spec, seed, 0, device="cpu")
-        wb = wl.bits(w)
-        lay = oracle.pack(wb, None if g is None else g.numpy(), tau)
-        x = wl.bits(wl.activations(spec.k, 1, seed, 0, slot=wl.PROJ.index(spec.name)))
-        T = -(-spec.n // 32)
-        tiles = np.linspace(0, T - 1, num=min(T, tiles_per_matrix)).astype(int)
-        prepared.append((spec, lay, wb, x, tiles))
-    return prepared
+    cores, model = host_cpu()
+    mats = oracle_layer(tau)
+    weights = sum(sp_.n * sp_.k for sp_, *_ in mats)
 
+    def pack_one(item):
+        spec, wb, gn, x = item
+        return oracle.pack(wb, gn, tau)
 
-def oracle_time(prepared):
-    import oracle
-    total_b, t0 = 0, time.perf_counter()
-    for spec, lay, wb, x, tiles in prepared:
-        p = lay.packed
-        G, S = spec.k // 32, -(-(spec.k // 32) // 8)
-        for t in tiles:
-            nr = min(spec.n, 32 * t + 32) - 32 * t
-            sub = oracle.Packed(p.codes[t * G * 512:(t + 1) * G * 512],
-                                p.scales[t * S * 256:(t + 1) * S * 256],
-                                p.zeros[t * S * 32:(t + 1) * S * 32], p.outliers, p.idx, nr, spec.k)
-            can = oracle.unpack_layout(sub)
-            oracle.gemm(can, wb[32 * t:32 * t + nr], lay.idx, x)
-            total_b += algorithmic_bytes(nr, spec.k, lay.idx.size)
-    return total_b, time.perf_counter() - t0
+    # pack, one thread: every matrix in turn
+    t0 = time.perf_counter()
+    packed = [pack_one(it) for it in mats]
+    pack_1t = time.perf_counter() - t0
+
+    # pack, all cores: kurtosis over column blocks, then the quantiser and the
+    # layout over row blocks, each block on a thread
+    def pack_parallel(ex, item):
+        spec, wb, gn, x = item
+        blocks = [(j, min(spec.k, j + 64)) for j in range(0, spec.k, 64)]
+        kap = np.concatenate(list(ex.map(
+            lambda b: oracle.kurtosis(np.ascontiguousarray(wb[:, b[0]:b[1]]),
+                                      None if gn is None else gn[b[0]:b[1]]), blocks)))
+        idx = oracle.split(kap, tau)
+        rb = [(r, min(spec.n, r + 256)) for r in range(0, spec.n, 256)]
+        list(ex.map(lambda r: oracle.pack_layout(oracle.quantize(wb[r[0]:r[1]], idx),
+                                                 wb[r[0]:r[1]], idx), rb))
+
+    with concurrent.futures.ThreadPoolExecutor(max_workers=cores) as ex:
+        t0 = time.perf_counter()
+        for it in mats:
+            pack_parallel(ex, it)
+        pack_all = time.perf_counter() - t0
+
+        items = matvec_items(mats, packed)
+        # one thread: items in turn until the budget is spent
+        b1, t0 = 0, time.perf_counter()
+        i = 0
+        while time.perf_counter() - t0 < budget_s:
+            b1 += oracle_matvec(items[i % len(items)])
+            i += 1
+        mv_1t = b1 / (time.perf_counter() - t0) * 1e-9
+        # all cores: whole passes over the layer until the budget is spent
+        ball, passes, t0 = 0, 0, time.perf_counter()
+        while passes < 1 or time.perf_counter() - t0 < budget_s:
+            ball += sum(ex.map(oracle_matvec, items))
+            passes += 1
+        mv_all = ball / (time.perf_counter() - t0) * 1e-9
+    return {"value": round(mv_all, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "cpu_model": model,
+            "sample": (f"the 7 matrices of one 1.5B-class layer ({weights} weights, tau {tau}): "
+                       f"matvec = unpack + FP64 product over 256-row blocks, {passes} whole passes "
+                       f"on {cores} threads in {budget_s:.0f}+ s; pack = kurtosis + split + "
+                       "quantiser + layout of all 7 matrices"),
+            "matvec_gbs_1thread": round(mv_1t, 4), "matvec_gbs_all_cores": round(mv_all, 4),
+            "pack_mweights_per_s_1thread": round(weights / pack_1t * 1e-6, 2),
+            "pack_mweights_per_s_all_cores": round(weights / pack_all * 1e-6, 2),
+            "pack_s_1thread": round(pack_1t, 3), "pack_s_all_cores": round(pack_all, 3)}
 
 
 def run_reference(args):
+    """The reference arm: the CPU oracle, as it stands, on every host core (a
+    thread per core).  A step is one whole pass of the oracle's matvec over
+    the seven matrices of layer 0 of the stack (1/28 of the GPU step's
+    weights), unpacked from the oracle's own packed layout and multiplied in
+    FP64.  Under torchrun only rank 0 works and prints."""
+    import concurrent.futures
+    import oracle
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    prepared = oracle_sample(0, args.tau, 1)
-    b1, t1 = oracle_time(prepared)
-    budget_s = 120.0
-    per_step = budget_s / max(1, args.steps + args.warmup)
-    tiles = int(max(1, min(64, per_step / max(t1, 1e-6))))
-    prepared = oracle_sample(0, args.tau, tiles)
-    for _ in range(args.warmup):
-        oracle_time(prepared)
-    tot_b, tot_t = 0, 0.0
-    for _ in range(args.steps):
-        b, t = oracle_time(prepared)
-        tot_b += b
-        tot_t += t
+    oracle.build()
+    cores, model = host_cpu()
+    mats = oracle_layer(args.tau)
+    packed = [oracle.pack(wb, gn, args.tau) for spec, wb, gn, x in mats]
+    items = matvec_items(mats, packed)
+    with concurrent.futures.ThreadPoolExecutor(max_workers=cores) as ex:
+        for _ in range(args.warmup):
+            sum(ex.map(oracle_matvec, items))
+        tot_b, t0 = 0, time.perf_counter()
+        for _ in range(args.steps):
+            tot_b += sum(ex.map(oracle_matvec, items))
+        tot_t = time.perf_counter() - t0
     gbs = tot_b / tot_t * 1e-9
-    sample = (f"{tiles} row tile(s) of 32 rows from each of the 7 matrices of layer 0 per step "
-              f"({tot_b // max(1, args.steps)} algorithmic bytes per step)")
+    sample = (f"per step one pass over the 7 matrices of layer 0 ({tot_b // max(1, args.steps)} "
+              f"algorithmic bytes), 256-row blocks on {cores} threads ({model})")
     line = {"impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(tot_t / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": WORKLOAD, "tau": args.tau, "m": 1},
-            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -753,15 +881,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        prepared = oracle_sample(0, args.tau, 8)
-        b_s, t_s = 0, 0.0
-        while t_s < 10.0:
-            bb, tt = oracle_time(prepared)
-            b_s += bb
-            t_s += tt
-        cpu = {"value": round(b_s / t_s * 1e-9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": "8 row tiles of 32 rows from each of the 7 matrices of one 1.5B-class "
-                         f"layer, repeated for {t_s:.1f} s (unpack + FP64 matvec, one thread)"}
+        cpu = cpu_baseline(args.tau)
 
     digest = kernel_source_digest()
     launch_bytes = st.bytes / launches_per_step
@@ -797,11 +917,65 @@ def run_ours(args):
         }
         if extra:
             line["rows"] = extra
+        # last key: the figures a reader needs, short enough to survive a tail
+        line["summary"] = summary_of(line, extra, cpu)
         print(json.dumps(line), flush=True)
     del graph
     if world > 1:
         dist.destroy_process_group()
     return 0
+
+
+def summary_of(line, extra, cpu):
+    """A compact digest of the line (its last key): the headline and the rows
+    behind the bar of >= 75 % of peak on matrices of 8 MB and more."""
+    def r(v, n=3):
+        return None if v is None else round(v, n)
+    out = {"stream_tau3": {"us": line["us_per_step"], "frac": line["roofline"]["frac"],
+                           "e2e_gbs": line["e2e"]["value"]}}
+    t6 = extra.get("decode_stream_tau6")
+    if isinstance(t6, dict) and "frac" in t6:
+        out["stream_tau6"] = {"us": t6["us_per_step"], "frac": r(t6["frac"])}
+    ch = extra.get("decode_stream_dependent_chain")
+    if ch:
+        out["chain"] = {"us": ch["us_per_step"], "frac": r(ch["frac"]), "us_per_launch": ch["us_per_launch"]}
+    big = {}
+    for row in extra.get("per_matrix_1p5b", []):
+        if row["bytes"] >= 8_000_000:
+            big[f"1p5b_{row['matrix']}"] = row["frac"]
+    for row in extra.get("batch_sweep_4b", []):
+        if row["m"] == 1 and row["matrix"] in ("gate", "up", "down"):
+            big[f"4b_{row['matrix']}"] = row["frac"]
+    for row in extra.get("lm_head_131072x3072", []):
+        big[f"lm_head_t{row['frac_t_columns']}"] = row["frac"]
+    if big:
+        out["ge8MB_m1_frac"] = big
+    tc = {}
+    for row in extra.get("batch_sweep_4b", []):
+        if row["matrix"] == "gate" and row["m"] >= 8:
+            tc[f"4b_gate_m{row['m']}"] = row["frac"]
+    for row in extra.get("lm_head_batch_131072x3072", []):
+        if row["m"] >= 16:
+            tc[f"lm_head_m{row['m']}"] = row["frac"]
+    if tc:
+        out["tc_frac"] = tc
+    s5 = extra.get("single_512x512")
+    if s5:
+        out["cfg_512x512_us"] = {f"tau{row['tau']:g}": [row["us_back_to_back"], row["oracle_us_1thread"]]
+                                 for row in s5}
+    tr = extra.get("trdc_container_4_layers")
+    if isinstance(tr, dict) and "load_gbs" in tr:
+        out["trdc_load_gbs"] = tr["load_gbs"]
+    kv = extra.get("kv_attention_decode_8192")
+    if kv:
+        out["attn_8192_us"] = [row["us_back_to_back"] for row in kv]
+    em = extra.get("embed_rows_131072x3072_bf16")
+    if em:
+        out["embed_4096_frac"] = em[-1]["frac_single_flushed"]
+    if cpu:
+        out["cpu"] = {"cores": cpu["cores"], "matvec_gbs": [cpu["matvec_gbs_1thread"], cpu["matvec_gbs_all_cores"]],
+                      "pack_mw_s": [cpu["pack_mweights_per_s_1thread"], cpu["pack_mweights_per_s_all_cores"]]}
+    return out
 
 
 def tau_sweep_rows(device, stream, taus=(2.0, 3.0, 4.0, 5.0, 6.0, 8.0, float("inf"))):

@@ -2,6 +2,7 @@
 committed ncu summaries is attached only to the launch it was captured on,
 and the algorithmic byte counts of every row are what their formulas say."""
 import bench
+from outlier_split_bit_b200 import workload as wl
 
 
 def test_traffic_needs_matching_source_digest():
@@ -69,3 +70,33 @@ def test_embedding_bytes():
     # 64 * 4.625 / 8 = 37 B of codes, scales and zeros, 6 B of outliers, a
     # 4-byte id and 128 B written; plus the 3 indices once
     assert bench.embed_bytes(64, 3, 2) == 2 * (32 + 4 + 1 + 6 + 4 + 128) + 12
+
+
+def test_summary_is_last_and_short():
+    """The line's last key digests the rows a reader needs; the driver keeps
+    only the tail of a long line, so the digest stays under 1400 characters
+    with every row present."""
+    import json
+    line = {"us_per_step": 324.1, "roofline": {"frac": 0.9562}, "e2e": {"value": 6118.7}}
+    per = [{"matrix": s.name, "bytes": 9_000_000 + i, "frac": 0.543} for i, s in enumerate(wl.LAYER_1P5B)]
+    sweep = [{"matrix": s.name, "m": m, "frac": 0.123} for s in wl.LAYER_4B for m in wl.BATCH_SWEEP]
+    extra = {
+        "decode_stream_tau6": {"us_per_step": 197.31, "frac": 0.6212},
+        "decode_stream_dependent_chain": {"us_per_step": 1148.22, "frac": 0.2712, "us_per_launch": 5.858},
+        "per_matrix_1p5b": per, "batch_sweep_4b": sweep,
+        "lm_head_131072x3072": [{"frac_t_columns": f, "frac": 0.801} for f in wl.LM_HEAD_FRACTIONS],
+        "lm_head_batch_131072x3072": [{"m": m, "frac": 0.371} for m in (1, 16, 32)],
+        "single_512x512": [{"tau": t, "us_back_to_back": 3.12, "oracle_us_1thread": 912.3} for t in (3.0, 6.0)],
+        "trdc_container_4_layers": {"load_gbs": 1.84},
+        "kv_attention_decode_8192": [{"us_back_to_back": 16.72}, {"us_back_to_back": 26.45}],
+        "embed_rows_131072x3072_bf16": [{"frac_single_flushed": 0.16}],
+    }
+    cpu = {"cores": 224, "matvec_gbs_1thread": 0.1396, "matvec_gbs_all_cores": 12.3456,
+           "pack_mweights_per_s_1thread": 30.84, "pack_mweights_per_s_all_cores": 1575.53}
+    s = bench.summary_of(line, extra, cpu)
+    text = json.dumps({"summary": s})
+    assert len(text) < 1400, len(text)
+    assert set(s["ge8MB_m1_frac"]) >= {"1p5b_gate", "4b_gate", "4b_up", "4b_down", "lm_head_t0.1"}
+    assert s["tc_frac"]["4b_gate_m16"] == 0.123 and s["tc_frac"]["lm_head_m32"] == 0.371
+    assert s["chain"]["us_per_launch"] == 5.858 and s["stream_tau6"]["frac"] == 0.621
+    assert s["cpu"]["matvec_gbs"] == [0.1396, 12.3456]

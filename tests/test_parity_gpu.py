@@ -155,14 +155,16 @@ def test_decoder_layer_4b_batch(spec, m):
     check_gemv(y[:, rows], y_ref, bound)
 
 
+@pytest.mark.parametrize("tau", [3.0, 6.0])
 @pytest.mark.parametrize("frac", wl.LM_HEAD_FRACTIONS)
-def test_lm_head_full_size_sampled(frac):
-    """131072 x 3072 LM head: kurtosis on sampled columns, packing and matvec on
-    sampled tiles (the first two, a middle one and the last), in the launch
-    configuration of the benchmark."""
+def test_lm_head_full_size_sampled(frac, tau):
+    """131072 x 3072 LM head at both thresholds (tau 3.0 is the benchmark's
+    setting, about half the columns BF16): kurtosis bit-exact on every column,
+    packing and matvec on sampled tiles (the first two, a middle one and the
+    last), in the launch configuration of the benchmark."""
     spec = wl.lm_head_spec(frac)
     w, g, x = draw(spec)
-    idx, kappa = sp.spectra_pack_plan(w, g, 6.0, want_kappa=True)
+    idx, kappa = sp.spectra_pack_plan(w, g, tau, want_kappa=True)
     lay = sp.spectra_pack(w, idx)
     y = sp.spectra_gemv(lay, x[0])
     torch.cuda.synchronize()
@@ -171,7 +173,7 @@ def test_lm_head_full_size_sampled(frac):
     kap = kappa.cpu().numpy()
     # the oracle's own split of the whole matrix: kurtosis bit-exact on every
     # column, and the oracle's indices (never the GPU's) feed its packing
-    kref, ref_idx = oracle_split(wb, np_gain(g), 6.0, key=("lm_head", frac))
+    kref, ref_idx = oracle_split(wb, np_gain(g), tau, key=("lm_head", frac))
     assert np.array_equal(kap.view(np.uint64), kref.view(np.uint64))
     assert np.array_equal(idx_np, ref_idx)
     # heavy columns are found: at 131072 rows every Student-t(3) column passes
@@ -295,10 +297,11 @@ def test_matvec_allocates_nothing():
         gc.enable()
 
 
-def test_batched_equals_single_launches():
-    """One grouped launch of independent matvecs gives bit-identical results to
-    one launch per matrix (same per-problem plan and reduction order)."""
-    layers, xs, ys, ref = [], [], [], []
+def test_batched_two_layers_against_oracle():
+    """One grouped launch over the 7 projections of two layers (14 matrices of
+    five shapes, tau 3.0): every output of every matrix against the oracle's
+    full packing of that matrix; a replay of the same views is bit-identical."""
+    layers, xs, ys, refs = [], [], [], []
     for layer in range(2):
         for spec in wl.LAYER_1P5B:
             w, g, x = draw(spec, seed=3, layer=layer)
@@ -306,15 +309,14 @@ def test_batched_equals_single_launches():
             layers.append(lay)
             xs.append(x[0])
             ys.append(torch.full((spec.n,), float("nan"), device=DEV))
+            refs.append((wl.bits(w), np_gain(g), wl.bits(x)))
     views = sp.spectra_gemv_batched(layers, xs, ys)
     torch.cuda.synchronize()
-    for lay, x, y in zip(layers, xs, ys):
-        single = sp.spectra_gemv(lay, x)
-        torch.cuda.synchronize()
-        assert torch.isfinite(y).all()
-        # the grouped launch uses single-CTA (no cluster) plans: compare to the oracle
-        # through the single launch's tolerance check instead of bit equality
-        assert torch.allclose(y, single, rtol=1e-5, atol=1e-5)
+    for lay, y, (wb, gn, xb) in zip(layers, ys, refs):
+        ref = oracle.pack(wb, gn, 3.0)
+        assert np.array_equal(lay.outlier_idx[: lay.n_outliers].cpu().numpy(), ref.idx)
+        y_ref, bound = oracle.gemm(ref.can, wb, ref.idx, xb)
+        check_gemv(y, y_ref[0], bound[0])
     # replay the same call twice: deterministic
     y0 = [y.clone() for y in ys]
     sp.spectra_gemv_batched(views=views)
@@ -326,12 +328,15 @@ def test_batched_equals_single_launches():
 @pytest.mark.parametrize("spec", [wl.LAYER_1P5B[4], wl.LAYER_1P5B[6], wl.LAYER_4B[1]],
                          ids=["gate", "down", "k4b"])
 def test_batched_against_oracle(spec):
-    w, g, x, idx, kappa, lay, wb, ref = _full_pack(spec, 3.0, True)
-    y = torch.empty(spec.n, device=DEV)
-    sp.spectra_gemv_batched([lay, lay], [x[0], x[0]], [y, torch.empty_like(y)])
+    """The same matrix twice in one grouped launch, with two different x: both
+    outputs against the oracle."""
+    w, g, x, idx, kappa, lay, wb, ref = _full_pack(spec, 3.0, True, m=2)
+    y = [torch.full((spec.n,), float("nan"), device=DEV) for _ in range(2)]
+    sp.spectra_gemv_batched([lay, lay], [x[0], x[1]], y)
     torch.cuda.synchronize()
     y_ref, bound = oracle.gemm(ref.can, wb, ref.idx, wl.bits(x))
-    check_gemv(y, y_ref[0], bound[0])
+    for r in range(2):
+        check_gemv(y[r], y_ref[r], bound[r])
 
 
 def test_device_status_clear_after_all_launches():
@@ -355,17 +360,19 @@ def test_gemm_small_tensor_cores(spec, tau, m):
     check_gemv(y, y_ref, bound)
 
 
-@pytest.mark.parametrize("spec", [wl.LAYER_4B[4], wl.LAYER_4B[6], wl.LAYER_4B[1]], ids=["gate", "down", "k"])
+@pytest.mark.parametrize("spec", wl.LAYER_4B, ids=[s.name for s in wl.LAYER_4B])
 @pytest.mark.parametrize("m", [16, 32])
-def test_decoder_layer_4b_tensor_cores(spec, m):
-    """4B-class shapes at M = 16 and 32 (batch sweep rows): sampled tiles against the oracle."""
+@pytest.mark.parametrize("tau", [3.0, 6.0])
+def test_decoder_layer_4b_tensor_cores(spec, m, tau):
+    """All seven 4B-class projections at M = 16 and 32 (the batch sweep's
+    tensor-core rows) at both thresholds: sampled tiles against the oracle."""
     w, g, x = draw(spec, m=m)
-    lay = sp.pack_layer(w, g, 6.0)
+    lay = sp.pack_layer(w, g, tau)
     y = sp.spectra_gemm_small(lay, x)
     torch.cuda.synchronize()
     sp.spectra_device_status()
     wb = wl.bits(w)
-    _, ref_idx = oracle_split(wb, np_gain(g), 6.0)
+    _, ref_idx = oracle_split(wb, np_gain(g), tau, key=("4b", spec.name))
     assert np.array_equal(lay.outlier_idx[: lay.n_outliers].cpu().numpy(), ref_idx)
     T = -(-spec.n // 32)
     tiles = sorted({0, 1, T // 2, T - 1})
