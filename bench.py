@@ -1112,6 +1112,7 @@ def run_single(args):
         for _ in range(args.warmup):
             fn()
         us, p10, p90 = time_single(fn, stream, args.steps, flush)
+    sp.spectra_device_status(stream=stream)  # a wait that gave up fails the run
     b = layer_bytes(lay, m=args.m)
     print(json.dumps({"case": "single", "n": spec.n, "k": spec.k, "m": args.m, "tau": args.tau,
                       "compact": args.compact,

@@ -288,8 +288,14 @@ SPECTRA_API spectra_status spectra_gemv(const spectra_layer *layer, const uint16
  *   x  device, BF16 bits [m_rows][k] row-major;  y  device [m_rows][n].
  * Same formula and tolerance as spectra_gemv per batch row.  m_rows <= 7 runs
  * on CUDA cores (m_rows accumulators per lane); 8..32 runs the tensor-core
- * path (weights dequantised in registers to exact integer BF16 operands, MMA
- * with FP32 accumulation per group of 32 columns, scale applied in FP32).
+ * path: the bulk weights are dequantised in registers to FP16 operands
+ * s * (c - z) (one round-to-nearest-even rounding, relative 2^-11) against x
+ * converted to FP16, the outlier columns enter as exact BF16 products, and
+ * each 128-row block accumulates in FP32 in tensor memory.  The FP16
+ * operands bound the inputs: an x value beyond 65504 in a bulk column, or a
+ * group scale of 4368 or more, yields non-finite outputs, which the kernel
+ * reports through spectra_device_status as SPECTRA_ERR_RANGE (the CUDA-core
+ * path, m_rows <= 7, computes in FP32 and has no such bound).
  * Asynchronous, allocates nothing.
  */
 SPECTRA_API spectra_status spectra_gemm_small(const spectra_layer *layer, const uint16_t *x, int32_t m_rows,
@@ -315,6 +321,38 @@ SPECTRA_API spectra_status spectra_gemv_batched(const spectra_layer *layers,
                                                 const uint16_t *const *x, void *const *y,
                                                 int32_t count, spectra_dtype y_dtype,
                                                 void *stream);
+
+/*
+ * A dependent sequence of batch-1 matvecs in ONE launch: y[i] = W_i x[i] for
+ * i = 0, 1, ..., count - 1 in that order, where x[i] may be (or may overlap)
+ * the output of any earlier matvec of the call (e.g. x[i] = y[i - 1] with
+ * y_dtype SPECTRA_BF16), as in a decode step whose layers feed one another.
+ * The abstract's decode runs such a step replayed as a CUDA graph; this entry
+ * point removes the launch per matrix: one launch of one CTA per SM spreads
+ * every matvec over all SMs, and a CTA reads x[i] only after every
+ * CTA has stored its rows of y[i - 1] (a device counter, release/acquire at
+ * GPU scope).  The weights keep streaming across that wait.  Same formula,
+ * tolerance and output type as spectra_gemv; arrays as spectra_gemv_batched,
+ * 1 <= count <= SPECTRA_MAX_BATCH.  No y[i] may overlap another y[j] or an
+ * x[j] with j <= i.
+ *   workspace  device, >= spectra_gemv_chain_workspace_size() bytes, 16-byte
+ *              aligned; the call zeroes its counter on `stream` first
+ *              (cudaMemsetAsync), so consecutive calls may share it when
+ *              they run in stream order.
+ * Every wait on the counter is bounded (one second of %globaltimer time); a
+ * wait that gives up raises the flag that spectra_device_status reports as
+ * SPECTRA_ERR_INTERNAL and the launch's outputs are invalid.  The CTAs wait
+ * on one another, so all of them must be resident at once: they are when no
+ * kernel of another stream occupies SMs during the call; otherwise the waits
+ * give up as above.  Asynchronous, allocates nothing.
+ * Errors: INVALID_ARG, SHAPE, ALIGN, BUFFER_TOO_SMALL, UNSUPPORTED, CUDA.
+ */
+SPECTRA_API size_t spectra_gemv_chain_workspace_size(void);
+SPECTRA_API spectra_status spectra_gemv_chain(const spectra_layer *layers,
+                                              const uint16_t *const *x, void *const *y,
+                                              int32_t count, spectra_dtype y_dtype,
+                                              void *workspace, size_t workspace_bytes,
+                                              void *stream);
 
 /*
  * Embedding-row gather over a packed table (abstract: SpectraFusedEmbedding,
@@ -354,8 +392,10 @@ SPECTRA_API spectra_status spectra_embed(const spectra_layer *table, const int32
  * for a non-finite value or an FP16 scale overflow.  Returns, for what
  * happened since the last call (and clears every flag):
  * SPECTRA_ERR_INTERNAL if a wait gave up, else SPECTRA_ERR_INVALID_ARG if the
- * gather saw a bad id, else SPECTRA_ERR_NONFINITE or SPECTRA_ERR_RANGE from
- * the KV append, else SPECTRA_OK.  Synchronous on `stream`.
+ * gather saw a bad id, else SPECTRA_ERR_NONFINITE from the KV append, else
+ * SPECTRA_ERR_RANGE from the KV append (a scale overflowing FP16) or from the
+ * tensor-core matmul (an FP16 operand out of range), else SPECTRA_OK.
+ * Synchronous on `stream`.
  */
 SPECTRA_API spectra_status spectra_device_status(void *stream);
 
@@ -363,9 +403,11 @@ SPECTRA_API spectra_status spectra_device_status(void *stream);
  * Exercises the failure path of the kernels' bounded waits without a fault.
  * kind 0 launches one warp that acquires a stage of a weight ring (the
  * cp.async.bulk + mbarrier ring of the matvec kernels) that no copy ever
- * fills.  Its wait gives up after the kernels' limit (one second of
- * %globaltimer time), the launch raises the flag that spectra_device_status
- * then reports as SPECTRA_ERR_INTERNAL, and the context stays usable.
+ * fills; kind 1 launches a thread that waits, as a CTA of spectra_gemv_chain
+ * waits for the others, on a device counter that nothing increments.  The
+ * wait gives up after the kernels' limit (one second of %globaltimer time),
+ * the launch raises the flag that spectra_device_status then reports as
+ * SPECTRA_ERR_INTERNAL, and the context stays usable.
  * For tests of callers' error handling; asynchronous, allocates nothing.
  * Errors: INVALID_ARG (unknown kind), UNSUPPORTED, CUDA.
  */

@@ -294,6 +294,24 @@ def spectra_gemv_batched(layers=None, xs=None, ys=None, *, views: BatchViews | N
     return v
 
 
+def spectra_gemv_chain(layers=None, xs=None, ys=None, *, views: BatchViews | None = None,
+                       workspace: torch.Tensor | None = None, stream=None) -> BatchViews:
+    """Dependent batch-1 matvecs ys[i] = W_i xs[i], i in order, in one launch;
+    xs[i] may be an earlier ys[j].  `workspace` (device, >=
+    spectra_gemv_chain_workspace_size() bytes) holds the launch's counter."""
+    v = views if views is not None else BatchViews(layers, xs, ys)
+    if workspace is None:
+        workspace = getattr(v, "_chain_ws", None)
+    if workspace is None:
+        dev = v._keep[2][0].device
+        workspace = torch.empty(_L.spectra_gemv_chain_workspace_size(), dtype=torch.uint8, device=dev)
+        v._chain_ws = workspace
+    _check(_L.spectra_gemv_chain(v.layers, v.xs, v.ys, v.count, v.y_dtype, workspace.data_ptr(),
+                                 workspace.numel() * workspace.element_size(), _stream(stream)),
+           "spectra_gemv_chain")
+    return v
+
+
 # ---------------------------------------------------------------- TRDC container
 
 _BUFFERS = ("codes", "scales", "zeros", "outlier_idx", "outlier_w", "bulk_idx")

@@ -333,6 +333,31 @@ spectra_status spectra_gemv_batched(const spectra_layer *layers, const uint16_t 
     return launch_gemv_batched(layers, x, y, count, (int)y_dtype, (cudaStream_t)stream, dev);
 }
 
+size_t spectra_gemv_chain_workspace_size(void) { return 256; }
+
+spectra_status spectra_gemv_chain(const spectra_layer *layers, const uint16_t *const *x,
+                                  void *const *y, int32_t count, spectra_dtype y_dtype,
+                                  void *workspace, size_t workspace_bytes, void *stream) {
+    if (!layers || !x || !y || !workspace) return SPECTRA_ERR_INVALID_ARG;
+    if (count < 1 || count > SPECTRA_MAX_BATCH) return SPECTRA_ERR_SHAPE;
+    if (y_dtype != SPECTRA_F32 && y_dtype != SPECTRA_BF16) return SPECTRA_ERR_INVALID_ARG;
+    if (workspace_bytes < spectra_gemv_chain_workspace_size()) return SPECTRA_ERR_BUFFER_TOO_SMALL;
+    if (!aligned16(workspace)) return SPECTRA_ERR_ALIGN;
+    for (int32_t i = 0; i < count; ++i) {
+        spectra_status st = check_layer(&layers[i]);
+        if (st != SPECTRA_OK) return st;
+        if (!x[i] || !y[i]) return SPECTRA_ERR_INVALID_ARG;
+        if (!aligned16(x[i])) return SPECTRA_ERR_ALIGN;
+        if (y_dtype == SPECTRA_F32 ? !aligned4(y[i]) : ((uintptr_t)y[i] & 1u))
+            return SPECTRA_ERR_ALIGN;
+    }
+    DeviceInfo dev;
+    spectra_status st = current_device(&dev);
+    if (st != SPECTRA_OK) return st;
+    return launch_gemv_chain(layers, x, y, count, (int)y_dtype,
+                             static_cast<unsigned int *>(workspace), (cudaStream_t)stream, dev);
+}
+
 spectra_status spectra_embed(const spectra_layer *table, const int32_t *ids, int32_t m, void *out,
                              spectra_dtype out_dtype, void *stream) {
     spectra_status st = check_layer(table);
@@ -420,7 +445,7 @@ spectra_status spectra_attention_decode(const spectra_kv *k, const spectra_kv *v
 }
 
 spectra_status spectra_selftest_wait(int32_t kind, void *stream) {
-    if (kind != 0) return SPECTRA_ERR_INVALID_ARG;
+    if (kind != 0 && kind != 1) return SPECTRA_ERR_INVALID_ARG;
     DeviceInfo dev;
     spectra_status st = current_device(&dev);
     if (st != SPECTRA_OK) return st;
@@ -431,18 +456,18 @@ spectra_status spectra_device_status(void *stream) {
     DeviceInfo dev;
     spectra_status st = current_device(&dev);
     if (st != SPECTRA_OK) return st;
-    bool raised = false;
-    st = device_error(&raised, (cudaStream_t)stream);
+    unsigned int mv_bits = 0;
+    st = device_error(&mv_bits, (cudaStream_t)stream);
     if (st != SPECTRA_OK) return st;
     unsigned int embed_bits = 0, kv_bits = 0;
     st = embed_device_error(&embed_bits, (cudaStream_t)stream);
     if (st != SPECTRA_OK) return st;
     st = kv_device_error(&kv_bits, (cudaStream_t)stream);
     if (st != SPECTRA_OK) return st;
-    if (raised) return SPECTRA_ERR_INTERNAL;
+    if (mv_bits & 1u) return SPECTRA_ERR_INTERNAL;
     if (embed_bits) return SPECTRA_ERR_INVALID_ARG;
     if (kv_bits & 1u) return SPECTRA_ERR_NONFINITE;
-    if (kv_bits & 2u) return SPECTRA_ERR_RANGE;
+    if ((kv_bits & 2u) || (mv_bits & 2u)) return SPECTRA_ERR_RANGE;
     return SPECTRA_OK;
 }
 

@@ -12,71 +12,70 @@
 namespace spectra {
 namespace {
 
-// ---------------------------------------------------------------- tensor-core path (M = 16..32)
+// ---------------------------------------------------------------- design
 //
-// y[m][n] for 8 <= m_rows <= 32 (MB = 16 or 32 batch rows) on the fifth-
-// generation tensor cores.  A CTA owns blocks of 128 rows (4 tiles; TMEM
-// lane = row) and streams their units (super-groups, outlier batches) with
-// two kinds of warps:
+// A CTA owns blocks of 128 rows (4 tiles; TMEM lane = row) and streams their
+// units (super-groups of 8 groups, outlier batches of up to 8 octets) with:
 //
-//  * SETS sets of four compute warps (three at 16 rows, two at 32).  Set j
-//    takes every SETS-th unit of the block; warp 4j + r owns tile r (rows
-//    32r..32r+31) and keeps its own cp.async.bulk ring of that tile's units.
-//    Per group of 32 columns it writes the exact integer weights c - z as a
-//    BF16 A operand (128 rows x 32 columns) into a TMEM buffer, and later
-//    reads back that group's FP32 product D = (c - z) x from TMEM and adds
-//    s * D to its rows' sums.  The outlier columns enter the same way with
-//    their BF16 weights and s = 1.
-//  * one MMA warp per set, whose elected lane issues two tcgen05.mma
-//    kind::f16 (M = 128, N = MB, K = 16) per group into the group's own D
-//    buffer.
+//  * SETS sets of four compute warps.  Set j takes every SETS-th unit of the
+//    block; warp 4j + r owns tile r (rows 32r..32r+31) and keeps its own
+//    cp.async.bulk ring of that tile's units.  Per group of 32 columns each
+//    lane writes its row of the A operand into TMEM: the dequantised weights
+//    s * (c - z) rounded once to FP16 (c - z is exact in FP16, then one
+//    round-to-nearest-even multiply by the FP16 scale).  Outlier columns enter
+//    with their exact BF16 weights.  The set's threads also stage x as the B
+//    operand: FP16 for the bulk (BF16 x converted, exact in FP16's normal
+//    range), BF16 for the outlier columns.
+//  * one MMA warp whose elected lane issues every tcgen05.mma of the CTA
+//    (kind::f16, M = 128, N = MB, K = 16; A from TMEM, B from shared memory)
+//    into the block's FP32 accumulator in TMEM, so the scales need no FP32
+//    epilogue per group: the whole row sum stays in the tensor core until the
+//    block ends.  Consecutive MMAs rotate over NCH accumulators (independent
+//    dependency chains, so the tensor pipe overlaps them), summed in a fixed
+//    order when the block is read back.
 //
-// Groups travel in chunks of H: the compute warps store H groups' A operands
-// and arrive once, the MMA lane waits once, issues 2H MMAs and commits once,
-// and the compute warps wait once before reading the H D buffers back.  Each
-// mbarrier operation costs the issuing thread on the order of a hundred
-// cycles, more than one group's two MMAs, so handshakes per group would pace
-// the kernel.
+// Groups travel in chunks of H: the warps of a set store H groups' A operands
+// into one of the set's Q = 2 TMEM slots and arrive once on full[slot]; the
+// MMA lane waits, issues 2H MMAs and commits to done[slot].  A slot (and the
+// x image of the unit two units back) is rewritten only after done[] of the
+// chunk that last used it, so the MMAs that read them have completed.  At a
+// block end the MMA lane commits to dready[block & 1]; set 0 reads the
+// accumulator back (deferred until it has built the next block's first chunk,
+// so the MMA pipe stays fed) and arrives on dfree[block & 1], which the MMA
+// lane awaits before the block two later overwrites that accumulator.
 //
-// The products are exact: c - z is an integer in [-15, 15] and x is BF16, so
-// each product has at most 12 significant bits; D holds FP32 sums of 32 of
-// them and the per-group scale is applied in FP32 afterwards, as in the
-// CUDA-core path.  The B operand (x) of each unit is staged by the set's
-// threads in shared memory in the K-major canonical layout (8 x 16-byte core
-// matrices, K halves 128 B apart, 8-row groups 256 B apart), in the order
-// the decoder pairs the codes: the two BF16 halves of TMEM column 4w + s are
-// columns 8w + s and 8w + s + 4 of the group.
-//
-// Handshakes, per set and chunk slot q (Q slots of H TMEM buffers, used
-// round robin): full[q] (one arrival per compute warp, after its TMEM stores
-// and x writes) -> MMA issue -> done[q] (tcgen05.commit) -> compute threads
-// read the chunk's D buffers.  A slot is rebuilt only after its previous
-// chunk was read back, so the MMAs that read its A operands have completed.  Every wait is bounded; a timeout raises the
-// device error bit and turns the remaining waits into no-ops.
+// Accuracy: each weight carries one FP16 rounding (relative 2^-11) and FP32
+// accumulation, well inside |y - y_ref| <= 2e-3 * sum|w_hat x| + 1e-5; with x
+// a unit vector e_j, y is column j of W_hat rounded to FP16 (exactly), plus
+// the column's BF16 weight when j is an outlier.  Range: an FP16 operand that
+// overflows (|x| > 65504 in a bulk column, or a group scale of 4368 or more)
+// makes the row's sum non-finite; the read-back raises the RANGE flag of
+// spectra_device_status for any non-finite output.  Every wait is bounded by
+// a one-second %globaltimer limit and sleeps on the mbarrier's suspend hint.
 constexpr int kTcTmemCols = 512;
 
-template <int MB_, int SETS_, int H_, int Q_>
+template <int MB_, int SETS_, int H_, int NCH_>
 struct TcCfg {
     static constexpr int MB = MB_;
-    static constexpr int SETS = SETS_;               // warp sets
-    static constexpr int H = H_;                     // groups per handshake (a chunk)
-    static constexpr int Q = Q_;                     // chunk slots per set
-    static constexpr int P = H * Q;                  // TMEM group buffers per set
-    static constexpr int CW = 4 * SETS;              // compute warps
-    static constexpr int WARPS = CW + SETS;          // + one MMA warp per set
-    static constexpr int DCOL = (SETS * P * 16 + 31) / 32 * 32;  // A buffers below, D from here
-    static constexpr int XBYTES = 256 * MB * 2;      // x image of one super-group
-    static constexpr int KSTEP = MB * 32;            // bytes of one 16-column K step of x
-    static_assert(DCOL + SETS * P * MB <= kTcTmemCols, "TMEM budget");
-    static_assert(DCOL % 32 == 0, "D alignment");
-    static_assert(H >= 1 && H <= 8 && Q >= 2 && Q <= 8, "chunk shape");
+    static constexpr int SETS = SETS_;             // warp sets
+    static constexpr int H = H_;                   // groups per handshake (a chunk)
+    static constexpr int Q = 2;                    // chunk slots per set
+    static constexpr int NCH = NCH_;               // accumulator chains per block
+    static constexpr int CW = 4 * SETS;            // compute warps
+    static constexpr int WARPS = CW + 1;           // + the MMA warp
+    static constexpr int ACOLS = H * 16;           // TMEM columns of one chunk's A operands
+    static constexpr int DCOL = SETS * Q * ACOLS;  // A slots below, accumulators from here
+    static constexpr int XBYTES = 256 * MB * 2;    // x image of one unit (256 columns)
+    static constexpr int KSTEP = MB * 32;          // bytes of one 16-column K step of x
+    static_assert(DCOL % 32 == 0, "accumulator alignment");
+    static_assert(DCOL + 2 * NCH * MB <= kTcTmemCols, "TMEM budget");
+    static_assert(H >= 1 && H <= 8 && NCH >= 1 && NCH <= 4, "chunk shape");
 };
 
-// 16 rows: three sets of four compute warps (four warps per sub-partition
-// keep each thread within 128 registers), chunks of two groups, two chunk
-// slots per set.  32 rows: the D buffers are twice as wide, so two sets.
-using TcCfg16 = TcCfg<16, 3, 2, 2>;
-using TcCfg32 = TcCfg<32, 2, 2, 2>;
+// 16 rows: three sets; 32 rows: two sets.  Chunks of four groups, four
+// accumulator chains.
+using TcCfg16 = TcCfg<16, 3, 4, 4>;
+using TcCfg32 = TcCfg<32, 2, 4, 4>;
 
 struct TcArgs {
     Prob p;
@@ -91,11 +90,13 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
 }
 
+// Instruction descriptor of kind::f16: D = F32 (bits 4-5 = 1), A and B of the
+// same type (format at bits 7 and 10: 0 = F16, 1 = BF16), both K-major,
+// N = MB (>> 3 at bit 17), M = 128 (>> 4 at bit 24).
 template <int MB>
-__device__ __forceinline__ uint32_t bf16_idesc() {
-    // D = F32 (bits 4-5 = 1), A = B = BF16 (format 1 at bits 7 and 10), both
-    // K-major, N = MB (>> 3 at bit 17), M = 128 (>> 4 at bit 24)
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(MB >> 3) << 17) | (8u << 24);
+__device__ __forceinline__ uint32_t f16_idesc(bool bf16) {
+    const uint32_t t = bf16 ? 1u : 0u;
+    return (1u << 4) | (t << 7) | (t << 10) | ((uint32_t)(MB >> 3) << 17) | (8u << 24);
 }
 
 // Groups (of 32 columns) in unit u: a super-group has up to 8, an outlier
@@ -130,6 +131,12 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+        : "memory");
+}
+
 // x of one unit for one thread of a set (tid in [0, 128)), loaded one unit
 // ahead into registers.  Super-group: MB/4 chunks of 8 consecutive columns
 // (chunk c = tid + 128 i: row m = c % MB, word W = c / MB).  Outlier batch:
@@ -144,7 +151,7 @@ __device__ __forceinline__ void tc_load_x(const Prob &a, int u, int tid, TcX<MB>
     if (u < a.S) {
         // only valid addresses: batch rows past m_rows read row m_rows - 1 and
         // chunks past the super-group's end read its last chunk (their
-        // products land in D columns, or groups, that are never used)
+        // products land in accumulator columns, or K steps, that are never used)
         const int nw = 4 * min(8, a.G - 8 * u);
 #pragma unroll
         for (int i = 0; i < MB / 4; ++i) {
@@ -173,9 +180,17 @@ __device__ __forceinline__ void tc_load_x(const Prob &a, int u, int tid, TcX<MB>
     }
 }
 
+// FP16 pair (lo, hi) of two BF16 values given in the high halves of 32-bit
+// words (each exact as FP32; one rounding to FP16).
+__device__ __forceinline__ uint32_t f16_pair(uint32_t lo_bits, uint32_t hi_bits) {
+    const __half2 h = __floats2half2_rn(__uint_as_float(lo_bits), __uint_as_float(hi_bits));
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
 // Write the prefetched x of unit u as the B image: chunk W goes to K step
-// W / 2, core-matrix column W % 2.  Super-group chunks are reordered to
-// (x0, x4, x1, x5, x2, x6, x3, x7), the decoder's pairing.
+// W / 2, core-matrix column W % 2.  Super-group chunks become FP16 pairs in
+// the decoder's order (x0, x4), (x1, x5), (x2, x6), (x3, x7); outlier chunks
+// stay BF16 in slot order.
 template <int MB>
 __device__ __forceinline__ void tc_store_x(const Prob &a, int u, int tid, const TcX<MB> &xp,
                                            uint8_t *xb) {
@@ -183,9 +198,11 @@ __device__ __forceinline__ void tc_store_x(const Prob &a, int u, int tid, const 
 #pragma unroll
         for (int i = 0; i < MB / 4; ++i) {
             const int c = tid + 128 * i, m = c % MB, W = c / MB;
-            const uint4 v = xp.v[i];
-            const uint4 p = make_uint4(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632),
-                                       __byte_perm(v.y, v.w, 0x5410), __byte_perm(v.y, v.w, 0x7632));
+            const uint4 v = xp.v[i];  // (x0, x1), (x2, x3), (x4, x5), (x6, x7)
+            const uint4 p = make_uint4(f16_pair(v.x << 16, v.z << 16),
+                                       f16_pair(v.x & 0xFFFF0000u, v.z & 0xFFFF0000u),
+                                       f16_pair(v.y << 16, v.w << 16),
+                                       f16_pair(v.y & 0xFFFF0000u, v.w & 0xFFFF0000u));
             *reinterpret_cast<uint4 *>(xb + (W >> 1) * (MB * 32) + (m >> 3) * 256 +
                                        (W & 1) * 128 + (m & 7) * 16) = p;
         }
@@ -207,9 +224,15 @@ __device__ __forceinline__ void tc_store_x(const Prob &a, int u, int tid, const 
     }
 }
 
-__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+__device__ __forceinline__ uint32_t f16x2_sub(uint32_t a, uint32_t b) {
     uint32_t d;
-    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t f16x2_mul(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
 }
 
@@ -237,6 +260,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *v) {
         : "memory");
 }
 
+// MB consecutive FP32 accumulator columns of this warp's 32 lanes.
 template <int MB>
 __device__ __forceinline__ void tmem_ld_d(uint32_t taddr, float *d) {
     uint32_t r[MB];
@@ -268,43 +292,42 @@ __device__ __forceinline__ void tmem_ld_d(uint32_t taddr, float *d) {
     for (int i = 0; i < MB; ++i) d[i] = __uint_as_float(r[i]);
 }
 
-// The A operand of group g of a unit for one row (lane): 16 TMEM columns of
-// BF16 pairs, and the group's scale.
-__device__ __forceinline__ float tc_build_a(const Prob &a, int u, int g, const uint8_t *stage,
-                                            int lane, uint32_t *av) {
-    if (!stage) {
+// The A operand of bulk group g for one row (lane): 16 TMEM columns of FP16
+// pairs s * (c - z), column 4w + s holding the codes of columns 8w + s (low)
+// and 8w + s + 4 (high) of the group.  1024 + c is exact in FP16 (10
+// mantissa bits), so the subtraction of 1024 + z is exact and the multiply
+// by the scale is the one rounding.
+__device__ __forceinline__ void tc_build_a_bulk(uint32_t sa, int g, int lane, uint32_t *av) {
+    const uint4 q = lds128(sa + g * 512 + lane * 16);
+    const uint32_t sw = lds32(sa + 4096 + lane * 16 + (g >> 1) * 4);
+    const uint32_t zw = lds32(sa + 4608 + lane * 4);
+    const uint32_t ss = __byte_perm(sw, 0u, (g & 1) ? 0x3232u : 0x1010u);    // (s, s)
+    const uint32_t zz = (0x6400u | ((zw >> (4 * g)) & 0xFu)) * 0x00010001u;  // (1024 + z, 1024 + z)
+    const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-        for (int i = 0; i < 16; ++i) av[i] = 0u;
-        return 0.f;
-    }
-    if (u < a.S) {
-        const uint32_t sa = smem_u32(stage);
-        const uint4 q = lds128(sa + g * 512 + lane * 16);
-        const uint32_t sw = lds32(sa + 4096 + lane * 16 + (g >> 1) * 4);
-        const uint32_t zw = lds32(sa + 4608 + lane * 4);
-        const uint32_t z = (zw >> (4 * g)) & 0xFu;
-        const uint32_t zz = (0x4300u | z) * 0x00010001u;  // BF16 pair (128 + z, 128 + z)
-        const uint32_t wv[4] = {q.x, q.y, q.z, q.w};
+    for (int w = 0; w < 4; ++w) {
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            av[4 * w + 0] = bf16x2_sub(code_pair<0>(wv[w]), zz);
-            av[4 * w + 1] = bf16x2_sub(code_pair<1>(wv[w]), zz);
-            av[4 * w + 2] = bf16x2_sub(code_pair<2>(wv[w]), zz);
-            av[4 * w + 3] = bf16x2_sub(code_pair<3>(wv[w]), zz);
+        for (int s = 0; s < 4; ++s) {
+            const uint32_t p = ((wv[w] >> (4 * s)) & 0x000F000Fu) | 0x64006400u;  // (1024 + c, 1024 + c')
+            av[4 * w + s] = f16x2_mul(f16x2_sub(p, zz), ss);
         }
-        return __half2float(__ushort_as_half((unsigned short)((g & 1) ? (sw >> 16) : (sw & 0xFFFFu))));
     }
+}
+
+// The A operand of outlier group g (octets 4g..4g+3) of batch unit u: the
+// exact BF16 weights, zero past the batch's last octet.
+__device__ __forceinline__ void tc_build_a_outlier(const Prob &a, int u, int g, uint32_t sa, int lane,
+                                                   uint32_t *av) {
     const int nv = min(kOB, a.O8 - kOB * (u - a.S));
 #pragma unroll
     for (int o = 0; o < 4; ++o) {
         uint4 w4 = make_uint4(0u, 0u, 0u, 0u);
-        if (4 * g + o < nv) w4 = *reinterpret_cast<const uint4 *>(stage + (4 * g + o) * 512 + lane * 16);
+        if (4 * g + o < nv) w4 = lds128(sa + (4 * g + o) * 512 + lane * 16);
         av[4 * o + 0] = w4.x;
         av[4 * o + 1] = w4.y;
         av[4 * o + 2] = w4.z;
         av[4 * o + 3] = w4.w;
     }
-    return 1.f;
 }
 
 template <typename C>
@@ -315,26 +338,32 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cr = (a.cl > 1) ? (int)cg::this_cluster().block_rank() : 0;
     const int D = args.depth;
-    // shared memory: [x images SETS x 2][ring CW x D]
-    // [bars][tmem slot, abort].  At a block end, once every group of the block
-    // has been read back, set j's first x image holds its 128 x MB partial
-    // sums (the same 256 x MB x 2 bytes).
+    // shared memory: [x images SETS x 2][ring CW x D][bars][tmem slot, abort].
+    // In a cluster (one block per CTA) set 0's x images hold the block's
+    // 128 x MB partial sums at the end, once every MMA has completed.
     uint8_t *ximg = tsm;
     uint8_t *ring_base = ximg + (size_t)C::SETS * 2 * C::XBYTES;
-    auto red_of = [&](int set) { return reinterpret_cast<float *>(ximg + (size_t)set * 2 * C::XBYTES); };
+    float *red = reinterpret_cast<float *>(ximg);
     uint64_t *bars = reinterpret_cast<uint64_t *>(ring_base + (size_t)C::CW * D * kStageBytes);
-    uint64_t *full = bars + C::CW * D;      // [SETS][Q]
-    uint64_t *done = full + C::SETS * C::Q;  // [SETS][Q]
-    uint64_t *fin = done + C::SETS * C::Q;   // [SETS]
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(fin + C::SETS);
+    uint64_t *full = bars + C::CW * D;        // [SETS][Q]
+    uint64_t *done = full + C::SETS * C::Q;   // [SETS][Q]
+    uint64_t *dready = done + C::SETS * C::Q; // [2]
+    uint64_t *dfree = dready + 2;             // [2]
+    uint64_t *fin = dfree + 2;                // [1]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(fin + 1);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
-    // this CTA's share of the units of every block it visits
-    const int OB = a.U - a.S;
-    const int sg0 = split_at(a.S, cr, a.cl), ob0 = split_at(OB, cr, a.cl);
-    const int nsg = split_at(a.S, cr + 1, a.cl) - sg0;
-    const int nunits = nsg + (split_at(OB, cr + 1, a.cl) - ob0);
+    // this CTA's share of the units of every block it visits: a contiguous
+    // range of the block's unit list (super-groups, then outlier batches), so
+    // with cl <= U every rank of a cluster has at least one unit
+    const int u0 = split_at(a.U, cr, a.cl), u1 = split_at(a.U, cr + 1, a.cl);
+    const int sg0 = u0, nsg = max(0, min(u1, a.S) - u0);
+    const int ob0 = max(u0, a.S) - a.S;
+    const int nunits = u1 - u0;
     const int bstride = (int)(gridDim.x / a.cl);
+    // MMAs of one block (the same for every block this CTA visits): two per group
+    int nmma = 0;
+    for (int lu = 0; lu < nunits; ++lu) nmma += 2 * tc_groups(a, tc_unit(a, sg0, nsg, ob0, lu));
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -347,7 +376,11 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
             mbar_init(smem_u32(&full[b]), 4u);  // one arrival per compute warp of the set
             mbar_init(smem_u32(&done[b]), 1u);
         }
-        for (int j = 0; j < C::SETS; ++j) mbar_init(smem_u32(&fin[j]), 1u);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&dready[b]), 1u);
+            mbar_init(smem_u32(&dfree[b]), 4u);  // one arrival per warp of set 0
+        }
+        mbar_init(smem_u32(&fin[0]), 1u);
         *abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -388,76 +421,88 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
         if (xblk < args.nblk) tc_load_x<MB>(a, tc_unit(a, sg0, nsg, ob0, xlu), tid, xp);
         advance(xblk, xlu);
 
-        // Two chunk slots: the chunk built last is read back right after the
-        // next one is built, so one chunk is in the MMA while the warp builds
-        // the next.  When a unit starts, every chunk of the unit before the
-        // previous one has been read back, so the MMAs that read the x image
-        // about to be rewritten have completed.
-        static_assert(C::Q == 2, "two chunk slots");
-        int ci = 0, xl = 0;
-        int pnh = 0;       // groups of the pending chunk (0: none)
-        float ps[C::H];    // their scales
-        float y[MB];
-#pragma unroll
-        for (int m = 0; m < MB; ++m) y[m] = 0.f;
-#pragma unroll
-        for (int h = 0; h < C::H; ++h) ps[h] = 0.f;
-        // read back the pending chunk (built as chunk ci - 1, slot (ci - 1) & 1)
-        auto read_back = [&]() {
-            const int q = (ci - 1) & 1;
-            // every lane waits: no divergent branch around the wait
-            tc_wait(smem_u32(&donej[q]), (uint32_t)((ci - 1) >> 1) & 1u, abort);
+        // Set 0 reads each block's accumulator back and stores its rows (or,
+        // in a cluster, leaves them for the rank-ordered reduction).
+        auto read_back = [&](int b, int blk) {
+            tc_wait(smem_u32(&dready[b & 1]), (uint32_t)(b >> 1) & 1u, abort);
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const uint32_t td = tl + (uint32_t)(C::DCOL + (b & 1) * C::NCH * MB);
+            float acc[MB];
+            if (nmma > 0) {  // CTA-uniform; a CTA without units adds zeros
+                tmem_ld_d<MB>(td, acc);
+            } else {
 #pragma unroll
-            for (int h = 0; h < C::H; ++h) {
-                if (h < pnh) {  // warp-uniform
-                    const uint32_t td = tl + (uint32_t)(C::DCOL + (j * C::P + q * C::H + h) * MB);
-                    const float2 s2 = make_float2(ps[h], ps[h]);
+                for (int m = 0; m < MB; ++m) acc[m] = 0.f;
+            }
 #pragma unroll
-                    for (int hh = 0; hh < MB / 16; ++hh) {
-                        float dv[16];
-                        tmem_ld_d<16>(td + 16 * hh, dv);
+            for (int c = 1; c < C::NCH; ++c) {
+                if (c < nmma) {  // CTA-uniform: chain c was written in this block
+                    float t2[MB];
+                    tmem_ld_d<MB>(td + (uint32_t)(c * MB), t2);
 #pragma unroll
-                        for (int m = 0; m < 16; m += 2) {
-                            const float2 r2 = __ffma2_rn(s2, make_float2(dv[m], dv[m + 1]),
-                                                         make_float2(y[16 * hh + m], y[16 * hh + m + 1]));
-                            y[16 * hh + m] = r2.x;
-                            y[16 * hh + m + 1] = r2.y;
-                        }
-                    }
+                    for (int m = 0; m < MB; ++m) acc[m] += t2[m];
                 }
             }
-            pnh = 0;
+            asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&dfree[b & 1]));
+            const int t = 4 * blk + r;
+            if (a.cl > 1) {
+#pragma unroll
+                for (int m = 0; m < MB; ++m) red[(32 * r + lane) * MB + m] = acc[m];
+            } else if (t < a.T) {
+                bool bad = false;
+#pragma unroll
+                for (int m = 0; m < MB; ++m) {
+                    store_y(a, t, lane, m, acc[m]);
+                    bad |= (m < a.m) && !isfinite(acc[m]);
+                }
+                if (bad && 32 * t + lane < a.n) atomicOr(&g_device_error, 2u);
+            }
         };
 
-        for (int blk = blockIdx.x / a.cl; blk < args.nblk; blk += bstride) {
+        int c = 0, xl = 0, b = 0;     // chunks, units and blocks of this set so far
+        int pend = -1, pend_blk = 0;  // set 0: a block whose accumulator is still to be read
+        for (int blk = blockIdx.x / a.cl; blk < args.nblk; blk += bstride, ++b) {
             const int t = 4 * blk + r;
             const bool active = t < a.T;
             for (int lu = j; lu < nunits; lu += C::SETS, ++xl) {
                 const int u = tc_unit(a, sg0, nsg, ob0, lu);
+                const bool bulk = u < a.S;
                 uint8_t *xb = ximg + (size_t)(j * 2 + (xl & 1)) * C::XBYTES;
-                tc_store_x<MB>(a, u, tid, xp, xb);
-                if (xblk < args.nblk) {
-                    tc_load_x<MB>(a, tc_unit(a, sg0, nsg, ob0, xlu), tid, xp);
-                    advance(xblk, xlu);
-                }
                 const uint8_t *stage = nullptr;
                 if (active) stage = ring_acquire(ring, lane);
                 else ring_advance_consume(ring);
                 __syncwarp();
+                const uint32_t sa = stage ? smem_u32(stage) : 0u;
                 const int ngr = tc_groups(a, u);
-                for (int g0 = 0; g0 < ngr; g0 += C::H) {
-                    // one chunk: up to H groups' A operands, then one arrival
-                    const int q = ci & 1;
+                for (int g0 = 0; g0 < ngr; g0 += C::H, ++c) {
+                    const int q = c & 1;
+                    // the slot's previous chunk (and, at a unit's start, every
+                    // MMA that read this x image two units back) has completed
+                    if (c >= C::Q) tc_wait(smem_u32(&donej[q]), (uint32_t)((c - C::Q) >> 1) & 1u, abort);
+                    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                    if (g0 == 0) {
+                        tc_store_x<MB>(a, u, tid, xp, xb);
+                        if (xblk < args.nblk) {
+                            tc_load_x<MB>(a, tc_unit(a, sg0, nsg, ob0, xlu), tid, xp);
+                            advance(xblk, xlu);
+                        }
+                    }
                     const int nh = min(C::H, ngr - g0);
-                    float sc[C::H];
 #pragma unroll
                     for (int h = 0; h < C::H; ++h) {
-                        sc[h] = 0.f;
                         if (h < nh) {  // warp-uniform
                             uint32_t av[16];
-                            sc[h] = tc_build_a(a, u, g0 + h, stage, lane, av);
-                            tmem_st16(tl + (uint32_t)((j * C::P + q * C::H + h) * 16), av);
+                            if (!stage) {
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) av[i] = 0u;
+                            } else if (bulk) {
+                                tc_build_a_bulk(sa, g0 + h, lane, av);
+                            } else {
+                                tc_build_a_outlier(a, u, g0 + h, sa, lane, av);
+                            }
+                            tmem_st16(tl + (uint32_t)((j * C::Q + q) * C::ACOLS + h * 16), av);
                         }
                     }
                     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
@@ -465,11 +510,10 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
                     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
                     __syncwarp();
                     if (lane == 0) mbar_arrive(smem_u32(&fullj[q]));
-                    if (pnh) read_back();
-                    ++ci;
-                    pnh = nh;
-#pragma unroll
-                    for (int h = 0; h < C::H; ++h) ps[h] = sc[h];
+                    if (pend >= 0) {  // set 0 only: the previous block, now that this one is fed
+                        read_back(pend, pend_blk);
+                        pend = -1;
+                    }
                 }
                 if (active) ring_release(ring);
                 if (iblk < args.nblk) {
@@ -479,87 +523,67 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
                     advance(iblk, ilu);
                 }
             }
-            if (pnh) read_back();
-            // block end: sets 1.. hand their sums to set 0 (each set's own x
-            // image is free: its groups are all read back), which adds them in
-            // set order and stores the rows (or, in a cluster, leaves them for
-            // the rank-ordered reduction)
-            if (j > 0) {
-                float *red = red_of(j);
-#pragma unroll
-                for (int m = 0; m < MB; ++m) red[(32 * r + lane) * MB + m] = y[m];
-            }
-            named_sync(1, 32 * C::CW);
             if (j == 0) {
-                for (int o = 1; o < C::SETS; ++o) {
-                    const float *red = red_of(o);
-#pragma unroll
-                    for (int m = 0; m < MB; ++m) y[m] += red[(32 * r + lane) * MB + m];
-                }
-                if (a.cl > 1) {
-                    float *red = red_of(0);
-#pragma unroll
-                    for (int m = 0; m < MB; ++m) red[(32 * r + lane) * MB + m] = y[m];
-                } else if (active) {
-#pragma unroll
-                    for (int m = 0; m < MB; ++m) store_y(a, t, lane, m, y[m]);
-                }
+                pend = b;
+                pend_blk = blk;
             }
-            named_sync(1, 32 * C::CW);
-#pragma unroll
-            for (int m = 0; m < MB; ++m) y[m] = 0.f;
         }
+        if (pend >= 0) read_back(pend, pend_blk);
         ring_drain(ring);
     } else if (lane == 0) {
-        // ------------------------------------------------ MMA issuer of set j (one lane)
-        const int j = warp - C::CW;
-        pdl_wait();
-        const uint32_t idesc = bf16_idesc<MB>();
-        int q = 0, xl = 0;
-        bool any = false;
-        for (int blk = blockIdx.x / a.cl; blk < args.nblk; blk += bstride) {
-            for (int lu = j; lu < nunits; lu += C::SETS, ++xl) {
-                const int ngr = tc_groups(a, tc_unit(a, sg0, nsg, ob0, lu));
-                const uint32_t xs0 = smem_u32(ximg + (size_t)(j * 2 + (xl & 1)) * C::XBYTES);
-                for (int g0 = 0; g0 < ngr; g0 += C::H, ++q) {
-                    const int sl = q % C::Q;
+        // ------------------------------------------------ MMA issuer (one lane)
+        int cj[C::SETS], xj[C::SETS];  // chunks and units of each set so far
+#pragma unroll
+        for (int j = 0; j < C::SETS; ++j) cj[j] = xj[j] = 0;
+        int b = 0;
+        for (int blk = blockIdx.x / a.cl; blk < args.nblk; blk += bstride, ++b) {
+            // the accumulator two blocks back has been read
+            if (b >= 2) tc_wait(smem_u32(&dfree[b & 1]), (uint32_t)((b - 2) >> 1) & 1u, abort);
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            int mi = 0;  // MMAs of this block so far
+            for (int lu = 0; lu < nunits; ++lu) {
+                const int j = lu % C::SETS;
+                const int u = tc_unit(a, sg0, nsg, ob0, lu);
+                const int ngr = tc_groups(a, u);
+                const uint32_t idesc = f16_idesc<MB>(u >= a.S);
+                const uint32_t xs0 = smem_u32(ximg + (size_t)(j * 2 + (xj[j] & 1)) * C::XBYTES);
+                for (int g0 = 0; g0 < ngr; g0 += C::H) {
+                    const int q = cj[j] & 1;
                     const int nh = min(C::H, ngr - g0);
-                    const bool ok = tc_wait(smem_u32(&full[j * C::Q + sl]), (uint32_t)(q / C::Q) & 1u, abort);
+                    const bool ok = tc_wait(smem_u32(&full[j * C::Q + q]), (uint32_t)(cj[j] >> 1) & 1u, abort);
                     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                     if (ok) {
+                        const uint32_t td0 = tmem + (uint32_t)(C::DCOL + (b & 1) * C::NCH * MB);
                         for (int h = 0; h < nh; ++h) {
-                            const int b = sl * C::H + h;
+                            const uint32_t ta = tmem + (uint32_t)((j * C::Q + q) * C::ACOLS + h * 16);
                             const uint32_t xs = xs0 + (uint32_t)(2 * (g0 + h) * C::KSTEP);
-                            const uint32_t ta = tmem + (uint32_t)((j * C::P + b) * 16);
-                            const uint32_t td = tmem + (uint32_t)(C::DCOL + (j * C::P + b) * MB);
 #pragma unroll
                             for (int k = 0; k < 2; ++k) {
                                 const uint64_t bdesc = umma_desc(xs + (uint32_t)(k * C::KSTEP), 128u, 256u);
+                                const uint32_t td = td0 + (uint32_t)((mi % C::NCH) * MB);
+                                // the first product of a chain in this block overwrites it
+                                const uint32_t accum = mi >= C::NCH ? 1u : 0u;
+                                ++mi;
                                 asm volatile(
                                     "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %3, 0;\n\t"
                                     "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p;\n\t}" ::"r"(td),
-                                    "r"(ta + 8u * k), "l"(bdesc), "r"((uint32_t)k), "r"(idesc)
+                                    "r"(ta + 8u * k), "l"(bdesc), "r"(accum), "r"(idesc)
                                     : "memory");
                             }
                         }
-                        any = true;
                     }
-                    // one commit per chunk: done[sl] fires when all its MMAs completed
-                    asm volatile(
-                        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                            smem_u32(&done[j * C::Q + sl]))
-                        : "memory");
+                    // one commit per chunk: done[] fires when all its MMAs completed
+                    mma_commit(smem_u32(&done[j * C::Q + q]));
+                    ++cj[j];
                 }
+                ++xj[j];
             }
+            // the block's accumulator is complete once every MMA so far has completed
+            mma_commit(smem_u32(&dready[b & 1]));
         }
         // every MMA this lane issued has completed before TMEM is released
-        if (any) {
-            asm volatile(
-                "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                    smem_u32(&fin[j]))
-                : "memory");
-            tc_wait(smem_u32(&fin[j]), 0u, abort);
-        }
+        mma_commit(smem_u32(&fin[0]));
+        tc_wait(smem_u32(&fin[0]), 0u, abort);
     }
     __syncwarp();
 
@@ -574,13 +598,18 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
 #pragma unroll
             for (int m = 0; m < MB; ++m) yv[m] = 0.f;
             for (int rk = 0; rk < a.cl; ++rk) {
-                const float *rp = cluster.map_shared_rank(red_of(0), rk) + (32 * warp + lane) * MB;
+                const float *rp = cluster.map_shared_rank(red, rk) + (32 * warp + lane) * MB;
 #pragma unroll
                 for (int m = 0; m < MB; ++m) yv[m] += rp[m];
             }
             if (t < a.T) {
+                bool bad = false;
 #pragma unroll
-                for (int m = 0; m < MB; ++m) store_y(a, t, lane, m, yv[m]);
+                for (int m = 0; m < MB; ++m) {
+                    store_y(a, t, lane, m, yv[m]);
+                    bad |= (m < a.m) && !isfinite(yv[m]);
+                }
+                if (bad && 32 * t + lane < a.n) atomicOr(&g_device_error, 2u);
             }
         }
         cluster.sync();
@@ -597,7 +626,7 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
 template <typename C>
 size_t tc_smem_bytes(int depth) {
     return (size_t)C::SETS * 2 * C::XBYTES + (size_t)C::CW * depth * kStageBytes +
-           (size_t)(C::CW * depth + 2 * C::SETS * C::Q + C::SETS) * 8 + 16;
+           (size_t)(C::CW * depth + 2 * C::SETS * C::Q + 5) * 8 + 16;
 }
 
 template <typename C>
@@ -622,7 +651,7 @@ spectra_status run_tc(const Prob &a0, const DeviceInfo &dev, cudaStream_t s) {
     }
     args.p.cl = cl;
     args.nblk = (int)nblk;
-    int depth = 2;  // two units in flight per warp; a third measured slower (shared memory left to L1)
+    int depth = 2;  // two units in flight per warp
     while (depth > 1 && tc_smem_bytes<C>(depth) > dev.smem_optin) --depth;
     args.depth = depth;
     const size_t smem = tc_smem_bytes<C>(depth);
@@ -643,13 +672,13 @@ spectra_status launch_tc(const spectra_layer &l, const uint16_t *x, int m, void 
     return m <= 16 ? run_tc<TcCfg16>(a, dev, s) : run_tc<TcCfg32>(a, dev, s);
 }
 
-spectra_status tc_device_error(bool *raised, cudaStream_t s) {
+spectra_status tc_device_error(unsigned int *bits, cudaStream_t s) {
     unsigned int v = 0;
     if (cudaMemcpyFromSymbolAsync(&v, g_device_error, sizeof v, 0, cudaMemcpyDeviceToHost, s) !=
         cudaSuccess)
         return SPECTRA_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return SPECTRA_ERR_CUDA;
-    *raised = v != 0;
+    *bits = v;
     if (v != 0) {
         const unsigned int zero = 0;
         if (cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof zero, 0, cudaMemcpyHostToDevice,

@@ -211,7 +211,7 @@ __device__ __forceinline__ void stage_x_load(const Prob &a, const XRange &xr, co
             if (a.bidx == nullptr) {
                 const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)m * a.kx + 32 * g);
 #pragma unroll
-                for (int w = 0; w < 4; ++w) f.v0[w] = src[w];
+                for (int w = 0; w < 4; ++w) f.v0[w] = __ldcg(src + w);
             } else {
 #pragma unroll
                 for (int w = 0; w < 4; ++w) f.v0[w] = bulk_x8_gather(a, m, 32 * g + 8 * w);
@@ -223,11 +223,14 @@ __device__ __forceinline__ void stage_x_load(const Prob &a, const XRange &xr, co
         const int c = threadIdx.x + i * nth;
         const int m = c % MB;
         const bool mv = c < np * MB && m < a.m;
-        f.lo[i] = (mv && xi.i0[i] >= 0) ? a.x[(size_t)m * a.kx + xi.i0[i]] : 0u;
-        f.hi[i] = (mv && xi.i1[i] >= 0) ? a.x[(size_t)m * a.kx + xi.i1[i]] : 0u;
+        f.lo[i] = (mv && xi.i0[i] >= 0) ? __ldcg(a.x + (size_t)m * a.kx + xi.i0[i]) : 0u;
+        f.hi[i] = (mv && xi.i1[i] >= 0) ? __ldcg(a.x + (size_t)m * a.kx + xi.i1[i]) : 0u;
     }
 }
 
+// (x is read with ld.global.cg: it may have been written by other CTAs of
+// the same launch -- the chain kernel -- so it must not come from a stale L1
+// line; read once per CTA, it gains nothing from L1 anyway.)
 // Stage x for a unit range: bulk groups as BF16 pairs in the decoder's order
 // with their FP32 sums X_g (column order), and the BF16 pairs of the outlier
 // slots, gathered through the index list; the first round comes from `f`.
@@ -250,7 +253,7 @@ __device__ void stage_x_store(const Prob &a, const Stage<MB> &st, const XRange &
             } else if (a.bidx == nullptr) {
                 const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)m * a.kx + 32 * g);
 #pragma unroll
-                for (int w = 0; w < 4; ++w) v[w] = src[w];
+                for (int w = 0; w < 4; ++w) v[w] = __ldcg(src + w);
             } else {
 #pragma unroll
                 for (int w = 0; w < 4; ++w) v[w] = bulk_x8_gather(a, m, 32 * g + 8 * w);
@@ -295,8 +298,8 @@ __device__ void stage_x_store(const Prob &a, const Stage<MB> &st, const XRange &
             if (c < np * MB) {
                 const int m = c % MB;
                 const bool mv = m < a.m;
-                const uint32_t l = (i0[i] >= 0 && mv) ? a.x[(size_t)m * a.kx + i0[i]] : 0u;
-                const uint32_t h = (i1[i] >= 0 && mv) ? a.x[(size_t)m * a.kx + i1[i]] : 0u;
+                const uint32_t l = (i0[i] >= 0 && mv) ? __ldcg(a.x + (size_t)m * a.kx + i0[i]) : 0u;
+                const uint32_t h = (i1[i] >= 0 && mv) ? __ldcg(a.x + (size_t)m * a.kx + i1[i]) : 0u;
                 st.xo[c] = l | (h << 16);
             }
         }
@@ -693,6 +696,161 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1)
     ring_drain(ring);
 }
 
+// ---------------------------------------------------------------- chain kernel
+//
+// A sequence of batch-1 matvecs where problem i may read what problems
+// before it wrote (x of one layer = y of the last): one launch of one 16-warp
+// CTA per SM, all resident at once.  Every problem is spread over all CTAs (CTA c takes
+// its items c, c + ncta, ...), and before a CTA reads x of problem i it waits
+// until every CTA has counted problem i - 1 as done on a global counter
+// (release / acquire at GPU scope).  The weight rings keep prefetching across
+// problems while a CTA waits, so the weight stream overlaps the barrier.
+
+struct ChainArgs {
+    Smem sm;
+    int count;                // problems
+    unsigned int *done;       // completion counter (zeroed before the launch)
+    Prob probs[kMaxBatch];    // each with its own item shape (tpc x ppc = 16 warps)
+};
+static_assert(sizeof(ChainArgs) <= 32760, "kernel parameter space");
+
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int *p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void red_release_gpu_add(unsigned int *p, unsigned int v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Wait until *ctr >= target; bounded like the ring waits (one second of
+// %globaltimer time), sleeping between polls.  Returns false on a timeout.
+__device__ __forceinline__ bool counter_wait(const unsigned int *ctr, unsigned int target) {
+    if (ld_acquire_gpu(ctr) >= target) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 0; i < kWaitRounds; ++i) {
+        __nanosleep(128);
+        if (ld_acquire_gpu(ctr) >= target) return true;
+        if (global_ns() - t0 > kWaitNs) return false;
+    }
+    return false;
+}
+
+// One warp's position in the chain's unit sequence: problem, item, tile,
+// slice and local unit.
+struct ChainCursor {
+    int p, item, t, u;
+    Slice sl;
+};
+
+// Move the cursor to the first unit at or after (c.p, c.item) that this warp
+// owns.
+__device__ __forceinline__ void chain_load(const ChainArgs &args, int warp, ChainCursor &c) {
+    while (c.p < args.count) {
+        const Prob &a = args.probs[c.p];
+        if (c.item < a.items) {
+            c.t = c.item * a.tpc + (warp >> a.lgp);
+            if (c.t < a.T) {
+                c.sl = slice_of_pow2(a, warp & (a.ppc - 1), a.lgp);
+                c.u = 0;
+                if (c.sl.nsg + c.sl.nob > 0) return;
+            }
+            c.item += gridDim.x;
+        } else {
+            ++c.p;
+            c.item = blockIdx.x;
+        }
+    }
+}
+
+__device__ __forceinline__ void chain_next(const ChainArgs &args, int warp, ChainCursor &c) {
+    if (++c.u < c.sl.nsg + c.sl.nob) return;
+    c.item += gridDim.x;
+    chain_load(args, warp, c);
+}
+
+__global__ void __launch_bounds__(kPersistWarps * 32, 1) gemv_chain_kernel(const ChainArgs args) {
+    extern __shared__ __align__(16) float smem[];
+    __shared__ int s_abort;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Stage<1> st = carve<1>(smem, args.sm, kPersistWarps);
+    if (threadIdx.x == 0) s_abort = 0;
+    Ring ring;
+    ring_init(ring, st.ring + (size_t)warp * args.sm.depth * kStageBytes,
+              st.bar + warp * args.sm.depth, args.sm.depth, lane);
+    // weights are constant: the ring is filled before any wait
+    ChainCursor ic;
+    ic.p = 0;
+    ic.item = blockIdx.x;
+    chain_load(args, warp, ic);
+    for (int d = 0; d < ring.D && ic.p < args.count; ++d) {
+        ring_issue(ring, args.probs[ic.p], ic.t, unit_id(args.probs[ic.p], ic.sl, ic.u), lane);
+        chain_next(args, warp, ic);
+    }
+    __syncthreads();
+    int rbuf = 0;
+    for (int p = 0; p < args.count; ++p) {
+        const Prob &a = args.probs[p];
+        // every CTA has finished problem p - 1 (its y may be this x)
+        if (p > 0) {
+            if (threadIdx.x == 0) {
+                if (!s_abort && !counter_wait(args.done, (unsigned int)p * gridDim.x)) {
+                    s_abort = 1;
+                    atomicOr(&g_device_error, 1u);
+                }
+                __threadfence();
+            }
+            __syncthreads();
+        }
+        if ((int)blockIdx.x < a.items) {
+            const XRange xr = x_range(a, 0, 1, 1);
+            XIdx xi;
+            load_x_idx(a, xr, 1, xi);
+            stage_x<1>(a, st, xr, xi);
+            __syncthreads();
+            for (int item = blockIdx.x; item < a.items; item += gridDim.x) {
+                const int tl = warp >> a.lgp, sl = warp & (a.ppc - 1);
+                const int t = item * a.tpc + tl;
+                const bool active = t < a.T;
+                const Slice slc = slice_of_pow2(a, sl, a.lgp);
+                const int nunits = active ? slc.nsg + slc.nob : 0;
+                float yacc = 0.f;
+                for (int u = 0; u < nunits; ++u) {
+                    const uint8_t *stage = ring_acquire(ring, lane);
+                    if (stage) compute_unit<1>(a, stage, lane, st, xr, unit_id(a, slc, u), &yacc);
+                    ring_release(ring);
+                    if (ic.p < args.count) {
+                        ring_issue(ring, args.probs[ic.p], ic.t, unit_id(args.probs[ic.p], ic.sl, ic.u), lane);
+                        chain_next(args, warp, ic);
+                    }
+                }
+                if (a.ppc == 1) {
+                    if (active) store_y(a, t, lane, 0, yacc);
+                } else {
+                    // the ppc warps of one tile meet on their own barrier (ids 1..tpc)
+                    float *red = st.red + (size_t)rbuf * kPersistWarps * 32;
+                    red[warp * 32 + lane] = yacc;
+                    named_sync(1 + tl, 32 * a.ppc);
+                    if (active && sl == 0) {
+                        float tot = 0.f;
+                        for (int s2 = 0; s2 < a.ppc; ++s2) tot += red[(tl * a.ppc + s2) * 32 + lane];
+                        store_y(a, t, lane, 0, tot);
+                    }
+                    rbuf ^= 1;
+                }
+            }
+        }
+        // this CTA's rows of problem p are stored: count it done
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            __threadfence();
+            red_release_gpu_add(args.done, 1u);
+        }
+    }
+    ring_drain(ring);
+}
+
 // ---------------------------------------------------------------- host planning
 
 constexpr size_t kSmPerSm = 228 * 1024;  // shared memory of one SM
@@ -950,6 +1108,66 @@ spectra_status run_persistent(PersistArgs &args, int count, const DeviceInfo &de
     return e == cudaSuccess ? SPECTRA_OK : SPECTRA_ERR_CUDA;
 }
 
+// Chain kernel: per problem the item shape that spreads it over the most
+// CTAs with the smallest largest share: tpc tiles x ppc slices per item
+// (tpc x ppc = 16), items dealt round robin over `ncta` CTAs.
+void chain_shape(const Geometry &g, int ncta, int *ppc, int *tpc) {
+    const int OB = (int)cdiv(g.O8, kOB);
+    double best = 1e300;
+    for (int p = 1; p <= kPersistWarps; p *= 2) {
+        const int tp = kPersistWarps / p;
+        const int64_t items = cdiv(g.T, tp);
+        const double per_item = (double)tp * ((double)cdiv(g.S, p) * kSgBytes +
+                                              (double)cdiv(OB, p) * kOB * kOctBytes);
+        // rounds of items on the busiest CTA, each one the slowest slice
+        const double cost = (double)cdiv(items, ncta) * per_item / tp + (p > 1 ? 64.0 * p : 0.0);
+        if (cost < best - 1e-9) {
+            best = cost;
+            *ppc = p;
+            *tpc = tp;
+        }
+    }
+}
+
+spectra_status run_chain(ChainArgs &args, int count, unsigned int *done, const DeviceInfo &dev,
+                         cudaStream_t s) {
+    const int ncta = dev.sm_count;
+    Smem sm = {1, 0, 0, 0};
+    for (int i = 0; i < count; ++i) {
+        Prob &a = args.probs[i];
+        const Geometry g = Geometry::of(a.n, a.k, a.n_o);
+        chain_shape(g, ncta, &a.ppc, &a.tpc);
+        a.lgp = 0;
+        while ((1 << a.lgp) < a.ppc) ++a.lgp;
+        a.items = (int)cdiv(a.T, a.tpc);
+        sm.xg = max(sm.xg, 8 * a.S);
+        sm.xo = max(sm.xo, 8 * kOB * (a.U - a.S));
+    }
+    sm.depth = fit_depth(1, kPersistWarps, sm, dev.smem_optin);
+    if (sm.depth > 2) sm.depth = 2;
+    if (sm.depth == 0) return SPECTRA_ERR_SHAPE;
+    args.sm = sm;
+    args.count = count;
+    args.done = done;
+    const size_t smem = stage_bytes(1, kPersistWarps, sm);
+    // the kernel also has a static shared word: raise the dynamic limit to
+    // what this launch needs (the device maximum would leave no room for it)
+    cudaError_t e = cudaFuncSetAttribute(gemv_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return SPECTRA_ERR_CUDA;
+    // every CTA waits on the others, so all of them must be resident at once:
+    // one CTA per SM, which the device must be able to hold
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_chain_kernel, kPersistWarps * 32,
+                                                      smem) != cudaSuccess)
+        return SPECTRA_ERR_CUDA;
+    if (per_sm < 1) return SPECTRA_ERR_SHAPE;
+    // the counter starts at zero in every launch
+    if (cudaMemsetAsync(done, 0, sizeof(unsigned int), s) != cudaSuccess) return SPECTRA_ERR_CUDA;
+    gemv_chain_kernel<<<(unsigned)ncta, kPersistWarps * 32, smem, s>>>(args);
+    return cudaGetLastError() == cudaSuccess ? SPECTRA_OK : SPECTRA_ERR_CUDA;
+}
+
 template <int MB>
 spectra_status run_cluster(const Prob &a0, const ClusterPlan &p, const DeviceInfo &dev,
                            cudaStream_t s) {
@@ -1003,20 +1221,29 @@ __global__ void ring_wait_selftest_kernel() {
     ring_drain(r);
 }
 
+// A counter that no kernel ever increments.
+__device__ unsigned int g_never_counted;
+
+// One thread waits, as a chain CTA waits for the others, on a counter that
+// never reaches its target: the bounded wait gives up and raises the flag.
+__global__ void counter_wait_selftest_kernel() {
+    if (threadIdx.x == 0 && !counter_wait(&g_never_counted, 1u)) atomicOr(&g_device_error, 1u);
+}
+
 }  // namespace
 
 // This translation unit's error word (the matvec kernels), then the
 // tensor-core kernel's (gemm_tc.cu).
-spectra_status device_error(bool *raised, cudaStream_t s) {
-    bool tc_raised = false;
-    const spectra_status st = tc_device_error(&tc_raised, s);
+spectra_status device_error(unsigned int *bits, cudaStream_t s) {
+    unsigned int tc_bits = 0;
+    const spectra_status st = tc_device_error(&tc_bits, s);
     if (st != SPECTRA_OK) return st;
     unsigned int v = 0;
     if (cudaMemcpyFromSymbolAsync(&v, g_device_error, sizeof v, 0, cudaMemcpyDeviceToHost, s) !=
         cudaSuccess)
         return SPECTRA_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return SPECTRA_ERR_CUDA;
-    *raised = v != 0 || tc_raised;
+    *bits = v | tc_bits;
     if (v != 0) {
         const unsigned int zero = 0;
         if (cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof zero, 0, cudaMemcpyHostToDevice,
@@ -1068,9 +1295,26 @@ spectra_status launch_gemv_batched(const spectra_layer *layers, const uint16_t *
     return run_persistent<1>(args, count, dev, s);
 }
 
+spectra_status launch_gemv_chain(const spectra_layer *layers, const uint16_t *const *xs,
+                                 void *const *ys, int count, int ytype, unsigned int *done,
+                                 cudaStream_t s, const DeviceInfo &dev) {
+    static std::mutex mu;
+    static ChainArgs args;  // large: kept off the stack, guarded by the mutex
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < count; ++i) {
+        const Geometry g = Geometry::of(layers[i].n, bulk_cols(layers[i]), layers[i].n_outliers);
+        fill_prob(args.probs[i], layers[i], g, xs[i], 1, ys[i], ytype);
+    }
+    return run_chain(args, count, done, dev, s);
+}
+
 spectra_status launch_wait_selftest(int kind, cudaStream_t s) {
-    if (kind != 0) return SPECTRA_ERR_INVALID_ARG;
-    ring_wait_selftest_kernel<<<1, 32, 0, s>>>();
+    if (kind == 0)
+        ring_wait_selftest_kernel<<<1, 32, 0, s>>>();
+    else if (kind == 1)
+        counter_wait_selftest_kernel<<<1, 32, 0, s>>>();
+    else
+        return SPECTRA_ERR_INVALID_ARG;
     return cudaGetLastError() == cudaSuccess ? SPECTRA_OK : SPECTRA_ERR_CUDA;
 }
 

@@ -85,9 +85,10 @@ constexpr int kMaxBatch = SPECTRA_MAX_BATCH;
 // tensor cores from 8).
 spectra_status launch_gemv(const spectra_layer &l, const uint16_t *x, int m, void *y, int ytype,
                            cudaStream_t s, const DeviceInfo &dev);
-// Reads (and clears) the flag the matvec kernels raise when a bounded wait
-// for a weight copy gives up.
-spectra_status device_error(bool *raised, cudaStream_t s);
+// Reads (and clears) the matvec kernels' flags: bit 0 a bounded wait for a
+// weight copy gave up, bit 1 the tensor-core path produced a non-finite
+// output (an FP16 operand out of range).
+spectra_status device_error(unsigned int *bits, cudaStream_t s);
 // A kernel whose bounded wait can never be satisfied (kind 0: the weight
 // ring's mbarrier wait); it gives up after its limit and raises the flag.
 spectra_status launch_wait_selftest(int kind, cudaStream_t s);
@@ -96,12 +97,19 @@ spectra_status launch_gemv_batched(const spectra_layer *layers, const uint16_t *
                                    void *const *ys, int count, int ytype, cudaStream_t s,
                                    const DeviceInfo &dev);
 
+// A dependent sequence of batch-1 matvecs in one launch
+// (count <= kMaxBatch): problem i reads x only after problems 0..i-1 have
+// stored y.  `done` is a device counter the call zeroes before the launch.
+spectra_status launch_gemv_chain(const spectra_layer *layers, const uint16_t *const *xs,
+                                 void *const *ys, int count, int ytype, unsigned int *done,
+                                 cudaStream_t s, const DeviceInfo &dev);
+
 // ---- tensor-core matmul (gemm_tc.cu) ----
 // y[m][n] for 8 <= m <= 32 batch rows on the tensor cores.
 spectra_status launch_tc(const spectra_layer &l, const uint16_t *x, int m, void *y, int ytype,
                          cudaStream_t s, const DeviceInfo &dev);
-// Reads (and clears) the tensor-core kernel's bounded-wait error flag.
-spectra_status tc_device_error(bool *raised, cudaStream_t s);
+// Reads (and clears) the tensor-core kernel's flags (bits as device_error).
+spectra_status tc_device_error(unsigned int *bits, cudaStream_t s);
 
 // ---- embedding-row gather (embed.cu) ----
 // Rows ids[0..m) of a packed table, dequantised (1 <= m).

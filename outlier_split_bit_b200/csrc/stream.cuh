@@ -162,7 +162,7 @@ __device__ __forceinline__ uint4 bulk_x8_gather(const Prob &a, int m, int c0) {
     const int c[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
     uint32_t h[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) h[e] = ((unsigned)c[e] < (unsigned)a.kx) ? (uint32_t)xr[c[e]] : 0u;
+    for (int e = 0; e < 8; ++e) h[e] = ((unsigned)c[e] < (unsigned)a.kx) ? (uint32_t)__ldcg(xr + c[e]) : 0u;
     return make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16),
                       h[6] | (h[7] << 16));
 }

@@ -234,6 +234,24 @@ def test_binding_fails_loudly_without_the_library(tmp_path, monkeypatch):
 
 def test_selftest_wait_argument_checks(L):
     # unknown kinds are rejected on the host, before any CUDA call
-    for kind in (-1, 1, 7):
+    for kind in (-1, 2, 7):
         assert L.spectra_selftest_wait(kind, None) == _lib.ERR_INVALID_ARG
+
+
+def test_chain_argument_checks(L):
+    ws = L.spectra_gemv_chain_workspace_size()
+    assert ws >= 4
+    lay = _lib.Layer(64, 128, 0, FAKE, FAKE, FAKE, None, None, 0, None)
+    layers = (_lib.Layer * 1)(lay)
+    xs = (ctypes.c_void_p * 1)(FAKE)
+    ys = (ctypes.c_void_p * 1)(FAKE)
+    # argument errors come back before any CUDA call
+    assert L.spectra_gemv_chain(layers, xs, ys, 1, 0, None, ws, None) == _lib.ERR_INVALID_ARG
+    assert L.spectra_gemv_chain(layers, xs, ys, 1, 0, FAKE, ws - 1, None) == _lib.ERR_BUFFER_TOO_SMALL
+    assert L.spectra_gemv_chain(layers, xs, ys, 1, 0, FAKE + 4, ws, None) == _lib.ERR_ALIGN
+    assert L.spectra_gemv_chain(layers, xs, ys, 0, 0, FAKE, ws, None) == _lib.ERR_SHAPE
+    assert L.spectra_gemv_chain(layers, xs, ys, _lib.MAX_BATCH + 1, 0, FAKE, ws, None) == _lib.ERR_SHAPE
+    assert L.spectra_gemv_chain(layers, xs, ys, 1, 5, FAKE, ws, None) == _lib.ERR_INVALID_ARG
+    bad = (_lib.Layer * 1)(_lib.Layer(64, 100, 0, FAKE, FAKE, FAKE, None, None, 0, None))
+    assert L.spectra_gemv_chain(bad, xs, ys, 1, 0, FAKE, ws, None) == _lib.ERR_SHAPE
 

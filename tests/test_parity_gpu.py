@@ -14,6 +14,7 @@ import torch
 
 import oracle
 import outlier_split_bit_b200 as sp
+from outlier_split_bit_b200 import _lib
 from outlier_split_bit_b200 import workload as wl
 
 from gpu_helpers import (DEV, check_gemv, draw, np_gain, oracle_rows, oracle_split, tile_slices,
@@ -350,8 +351,8 @@ def test_device_status_clear_after_all_launches():
                                       (wl.MatrixSpec("single", 130, 512, 0), np.inf)],
                          ids=["512", "40x96", "300x2080", "130x512-noout"])
 def test_gemm_small_tensor_cores(spec, tau, m):
-    """M = 8..32 runs on tcgen05 (exact BF16 c - z and x operands, FP32 per-group
-    products in TMEM, scales applied in FP32)."""
+    """M = 8..32 runs on tcgen05 (FP16 s * (c - z) and x operands for the bulk,
+    BF16 for the outlier columns, one FP32 accumulator per 128-row block)."""
     w, g, x, idx, kappa, lay, wb, ref = _full_pack(spec, tau, True, m=m)
     y = sp.spectra_gemm_small(lay, x)
     torch.cuda.synchronize()
@@ -383,8 +384,10 @@ def test_decoder_layer_4b_tensor_cores(spec, m, tau):
 
 @pytest.mark.parametrize("m", [8, 16, 32])
 def test_tensor_cores_unit_vectors_exact(m):
-    """x row r = e_{j_r}: every product is exact on the tensor cores, so row r of y
-    is column j_r of the dequantised matrix (plus its BF16 outlier column) bit for bit."""
+    """x row r = e_{j_r}: one nonzero product per output.  The tensor cores take
+    the bulk weights s * (c - z) as FP16 operands (one rounding to nearest
+    even), so row r of y is column j_r of the dequantised matrix rounded to
+    FP16, bit for bit, and an outlier column's BF16 weight exactly."""
     spec = wl.MatrixSpec("single", 200, 1024, 16)
     w, g, x, idx, kappa, lay, wb, ref = _full_pack(spec, 6.0, True)
     what = oracle.dequant(ref.can)
@@ -399,7 +402,8 @@ def test_tensor_cores_unit_vectors_exact(m):
         e[r, j] = 1.0
     y = sp.spectra_gemm_small(lay, e).cpu().numpy().astype(np.float64)
     for r, j in enumerate(cols):
-        expect = what[:, j] + (wvals[:, j] if j in ref.idx else 0.0)
+        bulk = what[:, j].astype(np.float16).astype(np.float64)
+        expect = bulk + (wvals[:, j] if j in ref.idx else 0.0)
         assert np.array_equal(y[r], expect), (r, j)
 
 
@@ -490,3 +494,42 @@ def test_tensor_cores_dependent_chain_reads_previous_output():
         cur = nxt
     assert torch.equal(bufs[-1], cur)
     sp.spectra_device_status()
+
+
+@pytest.mark.parametrize("m", [8, 16, 32])
+def test_tensor_cores_fp16_range_is_reported(m):
+    """The tensor-core path takes the bulk weights and x as FP16 operands.  An
+    x value beyond FP16's range, or a group whose scale times its largest
+    code offset overflows FP16, yields non-finite outputs; the launch reports
+    them through spectra_device_status as SPECTRA_ERR_RANGE instead of
+    returning them silently.  In-range inputs raise nothing."""
+    spec = wl.MatrixSpec("single", 256, 512, 4)
+    w, g, x = draw(spec, m=m)
+    lay = sp.pack_layer(w, g, np.inf)  # no outlier columns: every column is bulk
+    sp.spectra_device_status()
+    sp.spectra_gemm_small(lay, x)
+    torch.cuda.synchronize()
+    sp.spectra_device_status()  # in range: clear
+    xb = x.clone()
+    xb[0, 7] = 1.0e6  # beyond FP16 (BF16 holds it)
+    sp.spectra_gemm_small(lay, xb)
+    torch.cuda.synchronize()
+    with pytest.raises(sp.SpectraError) as e:
+        sp.spectra_device_status()
+    assert e.value.status == _lib.ERR_RANGE
+    # a group of row 3 spanning about [0, 80000]: FP16 scale 5332, zero point 0,
+    # so its largest weight decodes to 15 * 5332 = 79980 > 65504
+    wr = w.clone()
+    wr[3, 64:96] = wr[3, 64:96].abs()
+    wr[3, 64] = 80000.0
+    lay_r = sp.pack_layer(wr, g, np.inf)
+    sp.spectra_gemm_small(lay_r, x)
+    torch.cuda.synchronize()
+    with pytest.raises(sp.SpectraError) as e:
+        sp.spectra_device_status()
+    assert e.value.status == _lib.ERR_RANGE
+    # the CUDA-core path (m < 8) computes the same layer in FP32, unflagged
+    y1 = sp.spectra_gemm_small(lay_r, x[:1])
+    torch.cuda.synchronize()
+    sp.spectra_device_status()
+    assert torch.isfinite(y1).all()
