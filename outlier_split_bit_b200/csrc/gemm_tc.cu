@@ -26,23 +26,25 @@ namespace {
 //    with their exact BF16 weights.  The set's threads also stage x as the B
 //    operand: FP16 for the bulk (BF16 x converted, exact in FP16's normal
 //    range), BF16 for the outlier columns.
-//  * one MMA warp whose elected lane issues every tcgen05.mma of the CTA
+//  * one MMA warp per set, whose elected lane issues the set's tcgen05.mma
 //    (kind::f16, M = 128, N = MB, K = 16; A from TMEM, B from shared memory)
-//    into the block's FP32 accumulator in TMEM, so the scales need no FP32
-//    epilogue per group: the whole row sum stays in the tensor core until the
-//    block ends.  Consecutive MMAs rotate over NCH accumulators (independent
-//    dependency chains, so the tensor pipe overlaps them), summed in a fixed
-//    order when the block is read back.
+//    into the set's FP32 accumulator for the block in TMEM, so the scales
+//    need no FP32 epilogue per group: the row sums stay in the tensor core
+//    until the block ends.  The sets' accumulators are independent MMA
+//    dependency chains (so the tensor pipe overlaps them, and no issuer waits
+//    for another set), and a set's consecutive MMAs may rotate over NCH
+//    accumulators; all are summed in a fixed order when the block is read.
 //
 // Groups travel in chunks of H: the warps of a set store H groups' A operands
 // into one of the set's Q = 2 TMEM slots and arrive once on full[slot]; the
 // MMA lane waits, issues 2H MMAs and commits to done[slot].  A slot (and the
 // x image of the unit two units back) is rewritten only after done[] of the
 // chunk that last used it, so the MMAs that read them have completed.  At a
-// block end the MMA lane commits to dready[block & 1]; set 0 reads the
-// accumulator back (deferred until it has built the next block's first chunk,
-// so the MMA pipe stays fed) and arrives on dfree[block & 1], which the MMA
-// lane awaits before the block two later overwrites that accumulator.
+// block end each MMA lane commits to its set's dready[block & 1]; set 0 reads
+// every set's accumulator back (deferred until it has built the next block's
+// first chunk, so the MMA pipe stays fed) and arrives on the sets'
+// dfree[block & 1], which each MMA lane awaits before the block two later
+// overwrites its accumulator.
 //
 // Accuracy: each weight carries one FP16 rounding (relative 2^-11) and FP32
 // accumulation, well inside |y - y_ref| <= 2e-3 * sum|w_hat x| + 1e-5; with x
@@ -62,20 +64,20 @@ struct TcCfg {
     static constexpr int Q = 2;                    // chunk slots per set
     static constexpr int NCH = NCH_;               // accumulator chains per block
     static constexpr int CW = 4 * SETS;            // compute warps
-    static constexpr int WARPS = CW + 1;           // + the MMA warp
+    static constexpr int WARPS = CW + SETS;        // + one MMA warp per set
     static constexpr int ACOLS = H * 16;           // TMEM columns of one chunk's A operands
     static constexpr int DCOL = SETS * Q * ACOLS;  // A slots below, accumulators from here
     static constexpr int XBYTES = 256 * MB * 2;    // x image of one unit (256 columns)
     static constexpr int KSTEP = MB * 32;          // bytes of one 16-column K step of x
     static_assert(DCOL % 32 == 0, "accumulator alignment");
-    static_assert(DCOL + 2 * NCH * MB <= kTcTmemCols, "TMEM budget");
+    static_assert(DCOL + SETS * 2 * NCH * MB <= kTcTmemCols, "TMEM budget");
     static_assert(H >= 1 && H <= 8 && NCH >= 1 && NCH <= 4, "chunk shape");
 };
 
-// 16 rows: three sets; 32 rows: two sets.  Chunks of four groups, four
-// accumulator chains.
-using TcCfg16 = TcCfg<16, 3, 4, 4>;
-using TcCfg32 = TcCfg<32, 2, 4, 4>;
+// 16 rows: three sets, one accumulator each; 32 rows: two sets, two
+// accumulators each.  Chunks of four groups.
+using TcCfg16 = TcCfg<16, 3, 4, 1>;
+using TcCfg32 = TcCfg<32, 2, 4, 2>;
 
 struct TcArgs {
     Prob p;
@@ -347,10 +349,10 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
     uint64_t *bars = reinterpret_cast<uint64_t *>(ring_base + (size_t)C::CW * D * kStageBytes);
     uint64_t *full = bars + C::CW * D;        // [SETS][Q]
     uint64_t *done = full + C::SETS * C::Q;   // [SETS][Q]
-    uint64_t *dready = done + C::SETS * C::Q; // [2]
-    uint64_t *dfree = dready + 2;             // [2]
-    uint64_t *fin = dfree + 2;                // [1]
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(fin + 1);
+    uint64_t *dready = done + C::SETS * C::Q; // [SETS][2]
+    uint64_t *dfree = dready + C::SETS * 2;   // [SETS][2]
+    uint64_t *fin = dfree + C::SETS * 2;      // [SETS]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(fin + C::SETS);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     // this CTA's share of the units of every block it visits: a contiguous
@@ -361,9 +363,14 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
     const int ob0 = max(u0, a.S) - a.S;
     const int nunits = u1 - u0;
     const int bstride = (int)(gridDim.x / a.cl);
-    // MMAs of one block (the same for every block this CTA visits): two per group
-    int nmma = 0;
-    for (int lu = 0; lu < nunits; ++lu) nmma += 2 * tc_groups(a, tc_unit(a, sg0, nsg, ob0, lu));
+    // MMAs of one block per set (the same for every block this CTA visits):
+    // two per group
+    int nmma[C::SETS];
+#pragma unroll
+    for (int j = 0; j < C::SETS; ++j) {
+        nmma[j] = 0;
+        for (int lu = j; lu < nunits; lu += C::SETS) nmma[j] += 2 * tc_groups(a, tc_unit(a, sg0, nsg, ob0, lu));
+    }
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -376,11 +383,11 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
             mbar_init(smem_u32(&full[b]), 4u);  // one arrival per compute warp of the set
             mbar_init(smem_u32(&done[b]), 1u);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < C::SETS * 2; ++b) {
             mbar_init(smem_u32(&dready[b]), 1u);
             mbar_init(smem_u32(&dfree[b]), 4u);  // one arrival per warp of set 0
         }
-        mbar_init(smem_u32(&fin[0]), 1u);
+        for (int j = 0; j < C::SETS; ++j) mbar_init(smem_u32(&fin[j]), 1u);
         *abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -424,28 +431,30 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
         // Set 0 reads each block's accumulator back and stores its rows (or,
         // in a cluster, leaves them for the rank-ordered reduction).
         auto read_back = [&](int b, int blk) {
-            tc_wait(smem_u32(&dready[b & 1]), (uint32_t)(b >> 1) & 1u, abort);
-            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            const uint32_t td = tl + (uint32_t)(C::DCOL + (b & 1) * C::NCH * MB);
             float acc[MB];
-            if (nmma > 0) {  // CTA-uniform; a CTA without units adds zeros
-                tmem_ld_d<MB>(td, acc);
-            } else {
 #pragma unroll
-                for (int m = 0; m < MB; ++m) acc[m] = 0.f;
-            }
+            for (int m = 0; m < MB; ++m) acc[m] = 0.f;
 #pragma unroll
-            for (int c = 1; c < C::NCH; ++c) {
-                if (c < nmma) {  // CTA-uniform: chain c was written in this block
-                    float t2[MB];
-                    tmem_ld_d<MB>(td + (uint32_t)(c * MB), t2);
+            for (int js = 0; js < C::SETS; ++js) {
+                tc_wait(smem_u32(&dready[js * 2 + (b & 1)]), (uint32_t)(b >> 1) & 1u, abort);
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                const uint32_t td = tl + (uint32_t)(C::DCOL + ((js * 2 + (b & 1)) * C::NCH) * MB);
 #pragma unroll
-                    for (int m = 0; m < MB; ++m) acc[m] += t2[m];
+                for (int c = 0; c < C::NCH; ++c) {
+                    if (c < nmma[js]) {  // CTA-uniform: this accumulator was written in the block
+                        float t2[MB];
+                        tmem_ld_d<MB>(td + (uint32_t)(c * MB), t2);
+#pragma unroll
+                        for (int m = 0; m < MB; ++m) acc[m] += t2[m];
+                    }
                 }
             }
             asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&dfree[b & 1]));
+            if (lane == 0) {
+#pragma unroll
+                for (int js = 0; js < C::SETS; ++js) mbar_arrive(smem_u32(&dfree[js * 2 + (b & 1)]));
+            }
             const int t = 4 * blk + r;
             if (a.cl > 1) {
 #pragma unroll
@@ -531,59 +540,55 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
         if (pend >= 0) read_back(pend, pend_blk);
         ring_drain(ring);
     } else if (lane == 0) {
-        // ------------------------------------------------ MMA issuer (one lane)
-        int cj[C::SETS], xj[C::SETS];  // chunks and units of each set so far
-#pragma unroll
-        for (int j = 0; j < C::SETS; ++j) cj[j] = xj[j] = 0;
-        int b = 0;
+        // ------------------------------------------------ MMA issuer of set j (one lane)
+        const int j = warp - C::CW;
+        int cj = 0, xj = 0, b = 0;  // chunks, units and blocks of this set so far
+        const uint32_t x0 = smem_u32(ximg + (size_t)(j * 2) * C::XBYTES);
         for (int blk = blockIdx.x / a.cl; blk < args.nblk; blk += bstride, ++b) {
-            // the accumulator two blocks back has been read
-            if (b >= 2) tc_wait(smem_u32(&dfree[b & 1]), (uint32_t)((b - 2) >> 1) & 1u, abort);
+            // this set's accumulator two blocks back has been read
+            if (b >= 2) tc_wait(smem_u32(&dfree[j * 2 + (b & 1)]), (uint32_t)((b - 2) >> 1) & 1u, abort);
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            int mi = 0;  // MMAs of this block so far
-            for (int lu = 0; lu < nunits; ++lu) {
-                const int j = lu % C::SETS;
+            const uint32_t td0 = tmem + (uint32_t)(C::DCOL + ((j * 2 + (b & 1)) * C::NCH) * MB);
+            int mi = 0;  // this set's MMAs of the block so far
+            for (int lu = j; lu < nunits; lu += C::SETS, ++xj) {
                 const int u = tc_unit(a, sg0, nsg, ob0, lu);
                 const int ngr = tc_groups(a, u);
                 const uint32_t idesc = f16_idesc<MB>(u >= a.S);
-                const uint32_t xs0 = smem_u32(ximg + (size_t)(j * 2 + (xj[j] & 1)) * C::XBYTES);
-                for (int g0 = 0; g0 < ngr; g0 += C::H) {
-                    const int q = cj[j] & 1;
+                const uint32_t xs0 = x0 + (uint32_t)((xj & 1) * C::XBYTES);
+                for (int g0 = 0; g0 < ngr; g0 += C::H, ++cj) {
+                    const int q = cj & 1;
                     const int nh = min(C::H, ngr - g0);
-                    const bool ok = tc_wait(smem_u32(&full[j * C::Q + q]), (uint32_t)(cj[j] >> 1) & 1u, abort);
+                    const bool ok = tc_wait(smem_u32(&full[j * C::Q + q]), (uint32_t)(cj >> 1) & 1u, abort);
                     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
                     if (ok) {
-                        const uint32_t td0 = tmem + (uint32_t)(C::DCOL + (b & 1) * C::NCH * MB);
+                        const uint32_t ta0 = tmem + (uint32_t)((j * C::Q + q) * C::ACOLS);
                         for (int h = 0; h < nh; ++h) {
-                            const uint32_t ta = tmem + (uint32_t)((j * C::Q + q) * C::ACOLS + h * 16);
-                            const uint32_t xs = xs0 + (uint32_t)(2 * (g0 + h) * C::KSTEP);
 #pragma unroll
                             for (int k = 0; k < 2; ++k) {
-                                const uint64_t bdesc = umma_desc(xs + (uint32_t)(k * C::KSTEP), 128u, 256u);
+                                const uint32_t xs = xs0 + (uint32_t)((2 * (g0 + h) + k) * C::KSTEP);
+                                const uint64_t bdesc = umma_desc(xs, 128u, 256u);
                                 const uint32_t td = td0 + (uint32_t)((mi % C::NCH) * MB);
-                                // the first product of a chain in this block overwrites it
+                                // the first product into an accumulator in this block overwrites it
                                 const uint32_t accum = mi >= C::NCH ? 1u : 0u;
                                 ++mi;
                                 asm volatile(
                                     "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %3, 0;\n\t"
                                     "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p;\n\t}" ::"r"(td),
-                                    "r"(ta + 8u * k), "l"(bdesc), "r"(accum), "r"(idesc)
+                                    "r"(ta0 + (uint32_t)(h * 16 + 8 * k)), "l"(bdesc), "r"(accum), "r"(idesc)
                                     : "memory");
                             }
                         }
                     }
                     // one commit per chunk: done[] fires when all its MMAs completed
                     mma_commit(smem_u32(&done[j * C::Q + q]));
-                    ++cj[j];
                 }
-                ++xj[j];
             }
-            // the block's accumulator is complete once every MMA so far has completed
-            mma_commit(smem_u32(&dready[b & 1]));
+            // the set's accumulator is complete once every MMA so far has completed
+            mma_commit(smem_u32(&dready[j * 2 + (b & 1)]));
         }
         // every MMA this lane issued has completed before TMEM is released
-        mma_commit(smem_u32(&fin[0]));
-        tc_wait(smem_u32(&fin[0]), 0u, abort);
+        mma_commit(smem_u32(&fin[j]));
+        tc_wait(smem_u32(&fin[j]), 0u, abort);
     }
     __syncwarp();
 
@@ -626,7 +631,7 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
 template <typename C>
 size_t tc_smem_bytes(int depth) {
     return (size_t)C::SETS * 2 * C::XBYTES + (size_t)C::CW * depth * kStageBytes +
-           (size_t)(C::CW * depth + 2 * C::SETS * C::Q + 5) * 8 + 16;
+           (size_t)(C::CW * depth + 2 * C::SETS * C::Q + 5 * C::SETS) * 8 + 16;
 }
 
 template <typename C>

@@ -775,7 +775,7 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1) gemv_chain_kernel(const
     __shared__ int s_abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Stage<1> st = carve<1>(smem, args.sm, kPersistWarps);
-    if (threadIdx.x == 0) s_abort = 0;
+    if (threadIdx.x == 1) s_abort = 0;
     Ring ring;
     ring_init(ring, st.ring + (size_t)warp * args.sm.depth * kStageBytes,
               st.bar + warp * args.sm.depth, args.sm.depth, lane);
@@ -789,12 +789,22 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1) gemv_chain_kernel(const
         chain_next(args, warp, ic);
     }
     __syncthreads();
+    // the counter is polled and advanced by a thread that issues no weight
+    // copies (lane 1 of warp 0), so its fences wait for nothing but its own
+    // accesses
+    constexpr int kSignal = 1;
     int rbuf = 0;
     for (int p = 0; p < args.count; ++p) {
         const Prob &a = args.probs[p];
+        const bool mine = (int)blockIdx.x < a.items;
+        // the outlier column indices are part of the packed layer: load them
+        // before the wait
+        const XRange xr = x_range(a, 0, 1, 1);
+        XIdx xi;
+        if (mine) load_x_idx(a, xr, 1, xi);
         // every CTA has finished problem p - 1 (its y may be this x)
         if (p > 0) {
-            if (threadIdx.x == 0) {
+            if (threadIdx.x == kSignal) {
                 if (!s_abort && !counter_wait(args.done, (unsigned int)p * gridDim.x)) {
                     s_abort = 1;
                     atomicOr(&g_device_error, 1u);
@@ -803,10 +813,7 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1) gemv_chain_kernel(const
             }
             __syncthreads();
         }
-        if ((int)blockIdx.x < a.items) {
-            const XRange xr = x_range(a, 0, 1, 1);
-            XIdx xi;
-            load_x_idx(a, xr, 1, xi);
+        if (mine) {
             stage_x<1>(a, st, xr, xi);
             __syncthreads();
             for (int item = blockIdx.x; item < a.items; item += gridDim.x) {
@@ -843,7 +850,7 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1) gemv_chain_kernel(const
         }
         // this CTA's rows of problem p are stored: count it done
         __syncthreads();
-        if (threadIdx.x == 0) {
+        if (threadIdx.x == kSignal) {
             __threadfence();
             red_release_gpu_add(args.done, 1u);
         }

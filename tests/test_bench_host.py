@@ -82,7 +82,8 @@ def test_summary_is_last_and_short():
     sweep = [{"matrix": s.name, "m": m, "frac": 0.123} for s in wl.LAYER_4B for m in wl.BATCH_SWEEP]
     extra = {
         "decode_stream_tau6": {"us_per_step": 197.31, "frac": 0.6212},
-        "decode_stream_dependent_chain": {"us_per_step": 1148.22, "frac": 0.2712, "us_per_launch": 5.858},
+        "decode_stream_dependent_chain": {"us_per_step": 548.22, "frac": 0.6212, "us_per_launch": 548.22},
+        "decode_stream_dependent_launches": {"us_per_step": 1148.22, "frac": 0.2712, "us_per_launch": 5.858},
         "per_matrix_1p5b": per, "batch_sweep_4b": sweep,
         "lm_head_131072x3072": [{"frac_t_columns": f, "frac": 0.801} for f in wl.LM_HEAD_FRACTIONS],
         "lm_head_batch_131072x3072": [{"m": m, "frac": 0.371} for m in (1, 16, 32)],
@@ -98,5 +99,6 @@ def test_summary_is_last_and_short():
     assert len(text) < 1400, len(text)
     assert set(s["ge8MB_m1_frac"]) >= {"1p5b_gate", "4b_gate", "4b_up", "4b_down", "lm_head_t0.1"}
     assert s["tc_frac"]["4b_gate_m16"] == 0.123 and s["tc_frac"]["lm_head_m32"] == 0.371
-    assert s["chain"]["us_per_launch"] == 5.858 and s["stream_tau6"]["frac"] == 0.621
+    assert s["chain"]["frac"] == 0.621 and s["chain_196_launches"]["us"] == 1148.22
+    assert s["stream_tau6"]["frac"] == 0.621
     assert s["cpu"]["matvec_gbs"] == [0.1396, 12.3456]
