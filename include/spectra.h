@@ -335,10 +335,10 @@ SPECTRA_API spectra_status spectra_gemv_batched(const spectra_layer *layers,
  * tolerance and output type as spectra_gemv; arrays as spectra_gemv_batched,
  * 1 <= count <= SPECTRA_MAX_BATCH.  No y[i] may overlap another y[j] or an
  * x[j] with j <= i.
- *   workspace  device, >= spectra_gemv_chain_workspace_size() bytes, 16-byte
- *              aligned; the call zeroes its counter on `stream` first
- *              (cudaMemsetAsync), so consecutive calls may share it when
- *              they run in stream order.
+ *   workspace  device, >= spectra_gemv_chain_workspace_size(layers, count)
+ *              bytes, 16-byte aligned: the launch's completion counter,
+ *              which the call zeroes on `stream` first (cudaMemsetAsync).
+ *              Consecutive calls may share it when they run in stream order.
  * Every wait on the counter is bounded (one second of %globaltimer time); a
  * wait that gives up raises the flag that spectra_device_status reports as
  * SPECTRA_ERR_INTERNAL and the launch's outputs are invalid.  The CTAs wait
@@ -347,7 +347,9 @@ SPECTRA_API spectra_status spectra_gemv_batched(const spectra_layer *layers,
  * give up as above.  Asynchronous, allocates nothing.
  * Errors: INVALID_ARG, SHAPE, ALIGN, BUFFER_TOO_SMALL, UNSUPPORTED, CUDA.
  */
-SPECTRA_API size_t spectra_gemv_chain_workspace_size(void);
+/* Workspace bytes of spectra_gemv_chain over these layers; 0 for invalid
+ * arguments. */
+SPECTRA_API size_t spectra_gemv_chain_workspace_size(const spectra_layer *layers, int32_t count);
 SPECTRA_API spectra_status spectra_gemv_chain(const spectra_layer *layers,
                                               const uint16_t *const *x, void *const *y,
                                               int32_t count, spectra_dtype y_dtype,

@@ -298,13 +298,18 @@ def spectra_gemv_chain(layers=None, xs=None, ys=None, *, views: BatchViews | Non
                        workspace: torch.Tensor | None = None, stream=None) -> BatchViews:
     """Dependent batch-1 matvecs ys[i] = W_i xs[i], i in order, in one launch;
     xs[i] may be an earlier ys[j].  `workspace` (device, >=
-    spectra_gemv_chain_workspace_size() bytes) holds the launch's counter."""
+    spectra_gemv_chain_workspace_size(layers, count) bytes) holds the launch's
+    counters and partial sums; one is allocated and kept with the views when
+    none is given."""
     v = views if views is not None else BatchViews(layers, xs, ys)
     if workspace is None:
         workspace = getattr(v, "_chain_ws", None)
     if workspace is None:
         dev = v._keep[2][0].device
-        workspace = torch.empty(_L.spectra_gemv_chain_workspace_size(), dtype=torch.uint8, device=dev)
+        nbytes = _L.spectra_gemv_chain_workspace_size(v.layers, v.count)
+        if nbytes == 0:
+            raise SpectraError(_lib.ERR_INVALID_ARG, "spectra_gemv_chain_workspace_size")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
         v._chain_ws = workspace
     _check(_L.spectra_gemv_chain(v.layers, v.xs, v.ys, v.count, v.y_dtype, workspace.data_ptr(),
                                  workspace.numel() * workspace.element_size(), _stream(stream)),

@@ -76,7 +76,7 @@ SIGNATURES = {
     "spectra_gemv": (ctypes.c_int, [LP, P, P, ctypes.c_int, P]),
     "spectra_gemm_small": (ctypes.c_int, [LP, P, i32, P, ctypes.c_int, P]),
     "spectra_gemv_batched": (ctypes.c_int, [LP, P, P, i32, ctypes.c_int, P]),
-    "spectra_gemv_chain_workspace_size": (sz, []),
+    "spectra_gemv_chain_workspace_size": (sz, [LP, i32]),
     "spectra_gemv_chain": (ctypes.c_int, [LP, P, P, i32, ctypes.c_int, P, sz, P]),
     "spectra_device_status": (ctypes.c_int, [P]),
     "spectra_selftest_wait": (ctypes.c_int, [i32, P]),

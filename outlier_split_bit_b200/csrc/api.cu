@@ -333,7 +333,12 @@ spectra_status spectra_gemv_batched(const spectra_layer *layers, const uint16_t 
     return launch_gemv_batched(layers, x, y, count, (int)y_dtype, (cudaStream_t)stream, dev);
 }
 
-size_t spectra_gemv_chain_workspace_size(void) { return 256; }
+size_t spectra_gemv_chain_workspace_size(const spectra_layer *layers, int32_t count) {
+    if (!layers || count < 1 || count > SPECTRA_MAX_BATCH) return 0;
+    for (int32_t i = 0; i < count; ++i)
+        if (check_shape(layers[i].n, layers[i].k) != SPECTRA_OK) return 0;
+    return gemv_chain_workspace_bytes();
+}
 
 spectra_status spectra_gemv_chain(const spectra_layer *layers, const uint16_t *const *x,
                                   void *const *y, int32_t count, spectra_dtype y_dtype,
@@ -341,7 +346,7 @@ spectra_status spectra_gemv_chain(const spectra_layer *layers, const uint16_t *c
     if (!layers || !x || !y || !workspace) return SPECTRA_ERR_INVALID_ARG;
     if (count < 1 || count > SPECTRA_MAX_BATCH) return SPECTRA_ERR_SHAPE;
     if (y_dtype != SPECTRA_F32 && y_dtype != SPECTRA_BF16) return SPECTRA_ERR_INVALID_ARG;
-    if (workspace_bytes < spectra_gemv_chain_workspace_size()) return SPECTRA_ERR_BUFFER_TOO_SMALL;
+    if (workspace_bytes < 16) return SPECTRA_ERR_BUFFER_TOO_SMALL;
     if (!aligned16(workspace)) return SPECTRA_ERR_ALIGN;
     for (int32_t i = 0; i < count; ++i) {
         spectra_status st = check_layer(&layers[i]);
@@ -354,8 +359,8 @@ spectra_status spectra_gemv_chain(const spectra_layer *layers, const uint16_t *c
     DeviceInfo dev;
     spectra_status st = current_device(&dev);
     if (st != SPECTRA_OK) return st;
-    return launch_gemv_chain(layers, x, y, count, (int)y_dtype,
-                             static_cast<unsigned int *>(workspace), (cudaStream_t)stream, dev);
+    return launch_gemv_chain(layers, x, y, count, (int)y_dtype, workspace, workspace_bytes,
+                             (cudaStream_t)stream, dev);
 }
 
 spectra_status spectra_embed(const spectra_layer *table, const int32_t *ids, int32_t m, void *out,

@@ -57,6 +57,7 @@ namespace {
 constexpr int kClusterWarps = 8;               // warps per CTA of the cluster kernel
 constexpr int kPersistWarps = 16;              // warps per CTA of the persistent kernel
 constexpr int kMaxCtas = 320;                  // persistent grid bound (2 x SMs of a B200 + margin)
+constexpr size_t kChainWorkspace = 16;         // the chain kernel's completion counter (+ padding)
 
 // Launch-wide shared-memory geometry.
 struct Smem {
@@ -700,17 +701,21 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1)
 //
 // A sequence of batch-1 matvecs where problem i may read what problems
 // before it wrote (x of one layer = y of the last): one launch of one 16-warp
-// CTA per SM, all resident at once.  Every problem is spread over all CTAs (CTA c takes
-// its items c, c + ncta, ...), and before a CTA reads x of problem i it waits
-// until every CTA has counted problem i - 1 as done on a global counter
-// (release / acquire at GPU scope).  The weight rings keep prefetching across
-// problems while a CTA waits, so the weight stream overlaps the barrier.
+// CTA per SM, all resident at once.  Every problem is spread over all CTAs
+// (CTA c takes its items c, c + ncta, ...), and before a CTA reads x of
+// problem i it waits until every CTA has counted problem i - 1 as done on a
+// global counter (release / acquire at GPU scope).  The weight rings keep
+// prefetching across problems while a CTA waits, so the weight stream
+// overlaps the wait.  An item is tpc tiles x ppc slices (tpc x ppc = 16
+// warps); a tile's units are cut into contiguous slices, so the busiest warp
+// of a small problem holds as few units as the problem allows (a lone warp
+// decodes a unit in about a microsecond).
 
 struct ChainArgs {
     Smem sm;
     int count;                // problems
     unsigned int *done;       // completion counter (zeroed before the launch)
-    Prob probs[kMaxBatch];    // each with its own item shape (tpc x ppc = 16 warps)
+    Prob probs[kMaxBatch];    // each with its own item shape (ppc x tpc = 16 warps)
 };
 static_assert(sizeof(ChainArgs) <= 32760, "kernel parameter space");
 
@@ -730,18 +735,45 @@ __device__ __forceinline__ bool counter_wait(const unsigned int *ctr, unsigned i
     if (ld_acquire_gpu(ctr) >= target) return true;
     const uint64_t t0 = global_ns();
     for (uint32_t i = 0; i < kWaitRounds; ++i) {
-        __nanosleep(128);
+        __nanosleep(64);
         if (ld_acquire_gpu(ctr) >= target) return true;
         if (global_ns() - t0 > kWaitNs) return false;
     }
     return false;
 }
 
-// One warp's position in the chain's unit sequence: problem, item, tile,
-// slice and local unit.
+// Slice s of P of a tile as a contiguous range of its unit list
+// (super-groups, then outlier batches): with P >= U every slice has at most
+// one unit.
+__device__ __forceinline__ Slice slice_contig(const Prob &a, int s, int P) {
+    const int u0 = split_at(a.U, s, P), u1 = split_at(a.U, s + 1, P);
+    Slice r;
+    r.sg0 = u0;
+    r.nsg = max(0, min(u1, a.S) - u0);
+    r.ob0 = max(u0, a.S) - a.S;
+    r.nob = u1 - u0 - r.nsg;
+    return r;
+}
+
+// The tile and slice of warp `warp` in item `item` of a problem.
+struct ChainWork {
+    int t, tl, sl;
+    Slice slc;
+};
+
+__device__ __forceinline__ ChainWork chain_work(const Prob &a, int item, int warp) {
+    ChainWork w;
+    w.tl = warp / a.ppc;
+    w.sl = warp - w.tl * a.ppc;
+    w.t = item * a.tpc + w.tl;
+    w.slc = slice_contig(a, w.sl, a.ppc);
+    return w;
+}
+
+// One warp's position in the chain's unit sequence.
 struct ChainCursor {
-    int p, item, t, u;
-    Slice sl;
+    int p, item, u;
+    ChainWork w;
 };
 
 // Move the cursor to the first unit at or after (c.p, c.item) that this warp
@@ -750,12 +782,9 @@ __device__ __forceinline__ void chain_load(const ChainArgs &args, int warp, Chai
     while (c.p < args.count) {
         const Prob &a = args.probs[c.p];
         if (c.item < a.items) {
-            c.t = c.item * a.tpc + (warp >> a.lgp);
-            if (c.t < a.T) {
-                c.sl = slice_of_pow2(a, warp & (a.ppc - 1), a.lgp);
-                c.u = 0;
-                if (c.sl.nsg + c.sl.nob > 0) return;
-            }
+            c.w = chain_work(a, c.item, warp);
+            c.u = 0;
+            if (c.w.t < a.T && c.w.slc.nsg + c.w.slc.nob > 0) return;
             c.item += gridDim.x;
         } else {
             ++c.p;
@@ -765,7 +794,7 @@ __device__ __forceinline__ void chain_load(const ChainArgs &args, int warp, Chai
 }
 
 __device__ __forceinline__ void chain_next(const ChainArgs &args, int warp, ChainCursor &c) {
-    if (++c.u < c.sl.nsg + c.sl.nob) return;
+    if (++c.u < c.w.slc.nsg + c.w.slc.nob) return;
     c.item += gridDim.x;
     chain_load(args, warp, c);
 }
@@ -785,13 +814,13 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1) gemv_chain_kernel(const
     ic.item = blockIdx.x;
     chain_load(args, warp, ic);
     for (int d = 0; d < ring.D && ic.p < args.count; ++d) {
-        ring_issue(ring, args.probs[ic.p], ic.t, unit_id(args.probs[ic.p], ic.sl, ic.u), lane);
+        const Prob &ap = args.probs[ic.p];
+        ring_issue(ring, ap, ic.w.t, unit_id(ap, ic.w.slc, ic.u), lane);
         chain_next(args, warp, ic);
     }
     __syncthreads();
     // the counter is polled and advanced by a thread that issues no weight
-    // copies (lane 1 of warp 0), so its fences wait for nothing but its own
-    // accesses
+    // copies (lane 1 of warp 0)
     constexpr int kSignal = 1;
     int rbuf = 0;
     for (int p = 0; p < args.count; ++p) {
@@ -802,14 +831,13 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1) gemv_chain_kernel(const
         const XRange xr = x_range(a, 0, 1, 1);
         XIdx xi;
         if (mine) load_x_idx(a, xr, 1, xi);
-        // every CTA has finished problem p - 1 (its y may be this x)
+        // every CTA has finished problem p - 1 (its y may be this x); the
+        // acquire, then the CTA barrier, order the x loads after it
         if (p > 0) {
-            if (threadIdx.x == kSignal) {
-                if (!s_abort && !counter_wait(args.done, (unsigned int)p * gridDim.x)) {
-                    s_abort = 1;
-                    atomicOr(&g_device_error, 1u);
-                }
-                __threadfence();
+            if (threadIdx.x == kSignal && !s_abort &&
+                !counter_wait(args.done, (unsigned int)p * gridDim.x)) {
+                s_abort = 1;
+                atomicOr(&g_device_error, 1u);
             }
             __syncthreads();
         }
@@ -817,43 +845,39 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1) gemv_chain_kernel(const
             stage_x<1>(a, st, xr, xi);
             __syncthreads();
             for (int item = blockIdx.x; item < a.items; item += gridDim.x) {
-                const int tl = warp >> a.lgp, sl = warp & (a.ppc - 1);
-                const int t = item * a.tpc + tl;
-                const bool active = t < a.T;
-                const Slice slc = slice_of_pow2(a, sl, a.lgp);
-                const int nunits = active ? slc.nsg + slc.nob : 0;
+                const ChainWork cw = chain_work(a, item, warp);
+                const bool active = cw.t < a.T;
+                const int nunits = active ? cw.slc.nsg + cw.slc.nob : 0;
                 float yacc = 0.f;
                 for (int u = 0; u < nunits; ++u) {
                     const uint8_t *stage = ring_acquire(ring, lane);
-                    if (stage) compute_unit<1>(a, stage, lane, st, xr, unit_id(a, slc, u), &yacc);
+                    if (stage) compute_unit<1>(a, stage, lane, st, xr, unit_id(a, cw.slc, u), &yacc);
                     ring_release(ring);
                     if (ic.p < args.count) {
-                        ring_issue(ring, args.probs[ic.p], ic.t, unit_id(args.probs[ic.p], ic.sl, ic.u), lane);
+                        const Prob &ap = args.probs[ic.p];
+                        ring_issue(ring, ap, ic.w.t, unit_id(ap, ic.w.slc, ic.u), lane);
                         chain_next(args, warp, ic);
                     }
                 }
-                if (a.ppc == 1) {
-                    if (active) store_y(a, t, lane, 0, yacc);
-                } else {
+                float tot = yacc;
+                if (a.ppc > 1) {
                     // the ppc warps of one tile meet on their own barrier (ids 1..tpc)
                     float *red = st.red + (size_t)rbuf * kPersistWarps * 32;
                     red[warp * 32 + lane] = yacc;
-                    named_sync(1 + tl, 32 * a.ppc);
-                    if (active && sl == 0) {
-                        float tot = 0.f;
-                        for (int s2 = 0; s2 < a.ppc; ++s2) tot += red[(tl * a.ppc + s2) * 32 + lane];
-                        store_y(a, t, lane, 0, tot);
+                    named_sync(1 + cw.tl, 32 * a.ppc);
+                    if (cw.sl == 0) {
+                        tot = 0.f;
+                        for (int s2 = 0; s2 < a.ppc; ++s2) tot += red[(cw.tl * a.ppc + s2) * 32 + lane];
                     }
                     rbuf ^= 1;
                 }
+                if (cw.sl == 0 && active) store_y(a, cw.t, lane, 0, tot);
             }
         }
-        // this CTA's rows of problem p are stored: count it done
+        // this CTA's rows of problem p are stored: count it done (a release,
+        // after the CTA barrier, covers every warp's stores)
         __syncthreads();
-        if (threadIdx.x == kSignal) {
-            __threadfence();
-            red_release_gpu_add(args.done, 1u);
-        }
+        if (threadIdx.x == kSignal) red_release_gpu_add(args.done, 1u);
     }
     ring_drain(ring);
 }
@@ -1115,37 +1139,34 @@ spectra_status run_persistent(PersistArgs &args, int count, const DeviceInfo &de
     return e == cudaSuccess ? SPECTRA_OK : SPECTRA_ERR_CUDA;
 }
 
-// Chain kernel: per problem the item shape that spreads it over the most
-// CTAs with the smallest largest share: tpc tiles x ppc slices per item
-// (tpc x ppc = 16), items dealt round robin over `ncta` CTAs.
+// Chain kernel: per problem the item shape (tpc tiles x ppc slices, tpc x
+// ppc = 16) whose busiest warp holds the fewest units, items dealt round
+// robin over `ncta` CTAs.
 void chain_shape(const Geometry &g, int ncta, int *ppc, int *tpc) {
-    const int OB = (int)cdiv(g.O8, kOB);
-    double best = 1e300;
+    const int U = g.S + (int)cdiv(g.O8, kOB);
+    double best_cost = 1e300;
     for (int p = 1; p <= kPersistWarps; p *= 2) {
         const int tp = kPersistWarps / p;
         const int64_t items = cdiv(g.T, tp);
-        const double per_item = (double)tp * ((double)cdiv(g.S, p) * kSgBytes +
-                                              (double)cdiv(OB, p) * kOB * kOctBytes);
-        // rounds of items on the busiest CTA, each one the slowest slice
-        const double cost = (double)cdiv(items, ncta) * per_item / tp + (p > 1 ? 64.0 * p : 0.0);
-        if (cost < best - 1e-9) {
-            best = cost;
+        const double cost = (double)cdiv(items, ncta) * (double)cdiv(U, p) + (p > 1 ? 0.02 * p : 0.0);
+        if (cost < best_cost - 1e-9) {
+            best_cost = cost;
             *ppc = p;
             *tpc = tp;
         }
     }
 }
 
-spectra_status run_chain(ChainArgs &args, int count, unsigned int *done, const DeviceInfo &dev,
+spectra_status run_chain(ChainArgs &args, int count, void *ws, size_t ws_bytes, const DeviceInfo &dev,
                          cudaStream_t s) {
     const int ncta = dev.sm_count;
+    if (ws_bytes < kChainWorkspace) return SPECTRA_ERR_BUFFER_TOO_SMALL;
     Smem sm = {1, 0, 0, 0};
     for (int i = 0; i < count; ++i) {
         Prob &a = args.probs[i];
         const Geometry g = Geometry::of(a.n, a.k, a.n_o);
         chain_shape(g, ncta, &a.ppc, &a.tpc);
         a.lgp = 0;
-        while ((1 << a.lgp) < a.ppc) ++a.lgp;
         a.items = (int)cdiv(a.T, a.tpc);
         sm.xg = max(sm.xg, 8 * a.S);
         sm.xo = max(sm.xo, 8 * kOB * (a.U - a.S));
@@ -1155,7 +1176,7 @@ spectra_status run_chain(ChainArgs &args, int count, unsigned int *done, const D
     if (sm.depth == 0) return SPECTRA_ERR_SHAPE;
     args.sm = sm;
     args.count = count;
-    args.done = done;
+    args.done = static_cast<unsigned int *>(ws);
     const size_t smem = stage_bytes(1, kPersistWarps, sm);
     // the kernel also has a static shared word: raise the dynamic limit to
     // what this launch needs (the device maximum would leave no room for it)
@@ -1170,7 +1191,7 @@ spectra_status run_chain(ChainArgs &args, int count, unsigned int *done, const D
         return SPECTRA_ERR_CUDA;
     if (per_sm < 1) return SPECTRA_ERR_SHAPE;
     // the counter starts at zero in every launch
-    if (cudaMemsetAsync(done, 0, sizeof(unsigned int), s) != cudaSuccess) return SPECTRA_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, sizeof(unsigned int), s) != cudaSuccess) return SPECTRA_ERR_CUDA;
     gemv_chain_kernel<<<(unsigned)ncta, kPersistWarps * 32, smem, s>>>(args);
     return cudaGetLastError() == cudaSuccess ? SPECTRA_OK : SPECTRA_ERR_CUDA;
 }
@@ -1303,7 +1324,7 @@ spectra_status launch_gemv_batched(const spectra_layer *layers, const uint16_t *
 }
 
 spectra_status launch_gemv_chain(const spectra_layer *layers, const uint16_t *const *xs,
-                                 void *const *ys, int count, int ytype, unsigned int *done,
+                                 void *const *ys, int count, int ytype, void *ws, size_t ws_bytes,
                                  cudaStream_t s, const DeviceInfo &dev) {
     static std::mutex mu;
     static ChainArgs args;  // large: kept off the stack, guarded by the mutex
@@ -1312,8 +1333,10 @@ spectra_status launch_gemv_chain(const spectra_layer *layers, const uint16_t *co
         const Geometry g = Geometry::of(layers[i].n, bulk_cols(layers[i]), layers[i].n_outliers);
         fill_prob(args.probs[i], layers[i], g, xs[i], 1, ys[i], ytype);
     }
-    return run_chain(args, count, done, dev, s);
+    return run_chain(args, count, ws, ws_bytes, dev, s);
 }
+
+size_t gemv_chain_workspace_bytes() { return kChainWorkspace; }
 
 spectra_status launch_wait_selftest(int kind, cudaStream_t s) {
     if (kind == 0)

@@ -97,12 +97,13 @@ spectra_status launch_gemv_batched(const spectra_layer *layers, const uint16_t *
                                    void *const *ys, int count, int ytype, cudaStream_t s,
                                    const DeviceInfo &dev);
 
-// A dependent sequence of batch-1 matvecs in one launch
-// (count <= kMaxBatch): problem i reads x only after problems 0..i-1 have
-// stored y.  `done` is a device counter the call zeroes before the launch.
+// A dependent sequence of batch-1 matvecs in one launch (count <= kMaxBatch):
+// problem i reads x only after problems 0..i-1 have stored y.  `ws` holds the
+// launch's completion counter (zeroed by the call).
 spectra_status launch_gemv_chain(const spectra_layer *layers, const uint16_t *const *xs,
-                                 void *const *ys, int count, int ytype, unsigned int *done,
+                                 void *const *ys, int count, int ytype, void *ws, size_t ws_bytes,
                                  cudaStream_t s, const DeviceInfo &dev);
+size_t gemv_chain_workspace_bytes();
 
 // ---- tensor-core matmul (gemm_tc.cu) ----
 // y[m][n] for 8 <= m <= 32 batch rows on the tensor cores.

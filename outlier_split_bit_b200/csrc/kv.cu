@@ -13,19 +13,20 @@
 // slot, nibble g.
 //
 // Decode attention is split over the context ("split-K"): CTA (h, c) takes
-// the KV head h and the 128 positions of chunk c.
-//   1. thread t decodes K of position 128c + t -- (c - z) * s, exact in FP32
-//      -- against the FP32 query rows of the head's query group, staged in
-//      shared memory: one score per query head (FP32 accumulation);
+// the KV head h and the 128 positions of chunk c, with 512 threads.
+//   1. four threads per position decode K -- (c - z) * s, exact in FP32 --
+//      word q of every group (channels 32g + 8q .. +7), dot them with the FP32
+//      query rows of the head's query group staged in shared memory, and add
+//      their four partial scores with two shuffles (FP32 accumulation);
 //   2. per query head, the chunk's maximum m and sum l of exp(s - m);
-//   3. warp w takes positions 32w .. 32w + 31, lane l channels l, l + 32, ...:
-//      acc += exp(s - m) * v (FP32), reduced over the warps in fixed order.
-//      Each thread loads its position's V record, scales and zero word at
-//      the start (the loads overlap the K pass) and parks them in shared
-//      memory, so this pass reads no global memory; the buffer is reused for
-//      the cross-warp reduction.
+//   3. warp w takes positions 8w .. 8w + 7, lane l channels l, l + 32, ...:
+//      acc += exp(s - m) * v (FP32), reduced over the 16 warps in fixed order.
+//      Each position's V record, scales and zero word are loaded during the K
+//      pass (each of the four threads one word of every group) and parked in
+//      shared memory, so this pass reads no global memory.
 // The partials (m, l, acc[D]) of every chunk go to the workspace and a second
-// kernel merges them per query head:
+// kernel, launched as a programmatic dependent of the first (its launch
+// overlaps the chunks), merges them per query head and slice of 32 channels:
 //   out = sum_c exp(m_c - M) acc_c / sum_c exp(m_c - M) l_c,  M = max_c m_c.
 // Every order is fixed, so results repeat bit for bit.
 #include <cuda_bf16.h>
@@ -102,182 +103,218 @@ struct AttnArgs {
     float *out;     // [Hq][D]
 };
 
-template <int NG>
-__global__ void __launch_bounds__(kChunk) attn_partial_kernel(const AttnArgs a) {
+constexpr int kQuarter = 4;                        // threads per position in the K pass
+constexpr int kAttnThreads = kChunk * kQuarter;    // 512
+constexpr int kAttnWarps = kAttnThreads / 32;      // 16
+constexpr int kStatWarps = kChunk / 32;            // warps over the chunk's positions (stats)
+
+// Dynamic shared memory of the chunk kernel: query rows, scores, then a pool
+// holding first the chunk's V records and then the cross-warp partial sums.
+__host__ __device__ constexpr size_t attn_pool_bytes(int NG, int grp) {
+    const size_t vstage = (size_t)kChunk * (NG * 16 + NG * 2 + 4);
+    const size_t red = (size_t)kAttnWarps * grp * 32 * NG * 4;
+    return vstage > red ? vstage : red;
+}
+__host__ __device__ constexpr size_t attn_smem_bytes(int NG, int grp) {
+    return (size_t)kMaxGroup * 32 * NG * 4 + (size_t)kMaxGroup * kChunk * 4 + attn_pool_bytes(NG, grp);
+}
+
+__device__ __forceinline__ void attn_pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void attn_pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// GRP: the query-group size bucket (2, 4 or 8) the registers are sized for;
+// the loops run to the actual group size a.grp <= GRP.
+template <int NG, int GRP>
+__global__ void __launch_bounds__(kAttnThreads) attn_partial_kernel(const AttnArgs a) {
     constexpr int D = 32 * NG;
-    constexpr int kWarps = kChunk / 32;
-    // V of the chunk (phase 3), later the cross-warp partial sums
-    constexpr int kVStage = kChunk * (NG * 16 + NG * 2 + 4);
-    constexpr int kRed = kWarps * kMaxGroup * D * 4;
-    constexpr int kPool = kVStage > kRed ? kVStage : kRed;
-    __shared__ __align__(16) float qs[kMaxGroup][D];
-    __shared__ float sc[kMaxGroup][kChunk];
-    __shared__ __align__(16) unsigned char pool[kPool];
-    __shared__ float wmax[kWarps][kMaxGroup], wsum[kWarps][kMaxGroup];
+    extern __shared__ __align__(16) unsigned char dsm[];
+    float(*qs)[D] = reinterpret_cast<float(*)[D]>(dsm);                                      // [kMaxGroup][D]
+    float(*sc)[kChunk] = reinterpret_cast<float(*)[kChunk]>(dsm + kMaxGroup * D * 4);          // [kMaxGroup][kChunk]
+    unsigned char *pool = dsm + kMaxGroup * D * 4 + kMaxGroup * kChunk * 4;
+    uint32_t *vrec_s = reinterpret_cast<uint32_t *>(pool);                                   // [kChunk][NG][4]
+    uint16_t *vsc_s = reinterpret_cast<uint16_t *>(pool + kChunk * NG * 16);                 // [kChunk][NG]
+    uint32_t *vz_s = reinterpret_cast<uint32_t *>(pool + kChunk * (NG * 16 + NG * 2));       // [kChunk]
+    float *red = reinterpret_cast<float *>(pool);                                            // [kAttnWarps][grp][D]
+    __shared__ float wmax[kStatWarps][kMaxGroup], wsum[kStatWarps][kMaxGroup];
     __shared__ float cm[kMaxGroup], cl[kMaxGroup];
-    uint4 *vrec_s = reinterpret_cast<uint4 *>(pool);                                 // [kChunk][NG]
-    uint16_t *vsc_s = reinterpret_cast<uint16_t *>(pool + kChunk * NG * 16);         // [kChunk][NG]
-    uint32_t *vz_s = reinterpret_cast<uint32_t *>(pool + kChunk * (NG * 16 + NG * 2));  // [kChunk]
-    float(*red)[kMaxGroup][D] = reinterpret_cast<float(*)[kMaxGroup][D]>(pool);     // [kWarps]
     const int h = blockIdx.y, c = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int pos = tid >> 2, qd = tid & 3;  // position in the chunk, word of each group
     const int grp = a.grp;
-    const int tok = c * kChunk + tid;
-    // this position's V, loaded now, stored to shared memory after the K pass
-    uint4 vr[NG];
+    const int tok = c * kChunk + pos;
+    attn_pdl_launch_dependents();
+    attn_pdl_wait();  // the cache and the query may come from the previous kernel
+    // this position's V word qd of every group (and, thread 0 of the four,
+    // the scales and zero word), parked in shared memory after the K pass
+    uint32_t vw[NG];
     uint16_t vsr[NG];
     uint32_t vzr = 0;
-    if (tok < a.T) {
-        const size_t slot = (size_t)h * a.cap + tok;
+    const size_t slot = (size_t)h * a.cap + tok;
+    const bool valid = tok < a.T;
+    const uint32_t *vc32 = reinterpret_cast<const uint32_t *>(a.vc);
+    const uint32_t *kc32 = reinterpret_cast<const uint32_t *>(a.kc);
+    // K as well: every load of the position goes out before the first wait
+    uint32_t kw[NG];
+    uint16_t ksr[NG];
+    uint32_t kzr = 0;
 #pragma unroll
-        for (int g = 0; g < NG; ++g) {
-            vr[g] = a.vc[slot * NG + g];
-            vsr[g] = a.vs[slot * NG + g];
-        }
-        vzr = a.vz[slot];
-    } else {
-#pragma unroll
-        for (int g = 0; g < NG; ++g) {
-            vr[g] = make_uint4(0u, 0u, 0u, 0u);
-            vsr[g] = 0;
-        }
+    for (int g = 0; g < NG; ++g) {
+        kw[g] = valid ? kc32[(slot * NG + g) * 4 + qd] : 0u;
+        ksr[g] = valid ? a.ks[slot * NG + g] : (uint16_t)0;
+        vw[g] = valid ? vc32[(slot * NG + g) * 4 + qd] : 0u;
+        vsr[g] = (valid && qd == 0) ? a.vs[slot * NG + g] : (uint16_t)0;
     }
+    if (valid) kzr = a.kz[slot];
+    if (valid && qd == 0) vzr = a.vz[slot];
     // query rows of the group, FP32: every load issued before the first store
-    // (a load-store loop would wait out one round trip per element)
-    constexpr int kQPer = kMaxGroup * D / kChunk;
+    constexpr int kQPer = (kMaxGroup * D + kAttnThreads - 1) / kAttnThreads;
     uint32_t qraw[kQPer];
     const uint16_t *qh = a.q + (size_t)h * grp * D;  // the group's rows are contiguous
 #pragma unroll
     for (int u = 0; u < kQPer; ++u) {
-        const int i = tid + u * kChunk;
+        const int i = tid + u * kAttnThreads;
         qraw[u] = i < grp * D ? (uint32_t)qh[i] : 0u;
     }
 #pragma unroll
     for (int u = 0; u < kQPer; ++u) {
-        const int i = tid + u * kChunk;
+        const int i = tid + u * kAttnThreads;
         if (i < grp * D) qs[i / D][i % D] = __uint_as_float(qraw[u] << 16);
     }
     __syncthreads();
 
-    // 1. scores
-    float s[kMaxGroup];
+    // 1. scores: word qd of every group, then the four partial sums of a position
+    float s[GRP];
 #pragma unroll
-    for (int gi = 0; gi < kMaxGroup; ++gi) s[gi] = 0.f;
-    if (tok < a.T) {
-        const size_t slot = (size_t)h * a.cap + tok;
-        const uint32_t zw = a.kz[slot];
+    for (int gi = 0; gi < GRP; ++gi) s[gi] = 0.f;
+    if (valid) {
+        const uint32_t zw = kzr;
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
-            const uint4 rec = a.kc[slot * NG + g];
-            const float sg = __half2float(__ushort_as_half(a.ks[slot * NG + g]));
+            const uint32_t word = kw[g];
+            const float sg = __half2float(__ushort_as_half(ksr[g]));
             const float nzs = -(float)((zw >> (4 * g)) & 0xFu) * sg;  // -z * s, exact
-            const uint32_t wv[4] = {rec.x, rec.y, rec.z, rec.w};
 #pragma unroll
-            for (int w = 0; w < 4; ++w)
+            for (int j4 = 0; j4 < 2; ++j4) {
+                // channels 32g + 8qd + 4*j4 .. +3: (c - z) * s = fma(c, s, -z * s),
+                // exact; c as a float by the 2^23 mantissa trick
+                float kv[4];
 #pragma unroll
-                for (int j4 = 0; j4 < 2; ++j4) {
-                    // channels 32g + 8w + 4*j4 .. +3: (c - z) * s = fma(c, s, -z * s),
-                    // exact; c as a float by the 2^23 mantissa trick
-                    float kv[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const uint32_t code = (wv[w] >> (4 * (4 * j4 + u))) & 0xFu;
-                        kv[u] = fmaf(__uint_as_float(0x4B000000u | code) - 8388608.f, sg, nzs);
-                    }
-                    const int d4 = (32 * g + 8 * w + 4 * j4) / 4;
-#pragma unroll
-                    for (int gi = 0; gi < kMaxGroup; ++gi)
-                        if (gi < grp) {
-                            const float4 qv = reinterpret_cast<const float4 *>(qs[gi])[d4];
-                            s[gi] = fmaf(kv[0], qv.x, s[gi]);
-                            s[gi] = fmaf(kv[1], qv.y, s[gi]);
-                            s[gi] = fmaf(kv[2], qv.z, s[gi]);
-                            s[gi] = fmaf(kv[3], qv.w, s[gi]);
-                        }
+                for (int u = 0; u < 4; ++u) {
+                    const uint32_t code = (word >> (4 * (4 * j4 + u))) & 0xFu;
+                    kv[u] = fmaf(__uint_as_float(0x4B000000u | code) - 8388608.f, sg, nzs);
                 }
+                const int d4 = (32 * g + 8 * qd + 4 * j4) / 4;
+#pragma unroll
+                for (int gi = 0; gi < GRP; ++gi)
+                    if (gi < grp) {
+                        const float4 qv = reinterpret_cast<const float4 *>(qs[gi])[d4];
+                        s[gi] = fmaf(kv[0], qv.x, s[gi]);
+                        s[gi] = fmaf(kv[1], qv.y, s[gi]);
+                        s[gi] = fmaf(kv[2], qv.z, s[gi]);
+                        s[gi] = fmaf(kv[3], qv.w, s[gi]);
+                    }
+            }
         }
     }
 #pragma unroll
-    for (int gi = 0; gi < kMaxGroup; ++gi)
-        if (gi < grp) sc[gi][tid] = tok < a.T ? s[gi] * a.scale : -INFINITY;
+    for (int gi = 0; gi < GRP; ++gi) {
+        if (gi < grp) {
+            // (q0 + q1) + (q2 + q3): the same order on all four threads
+            s[gi] += __shfl_xor_sync(0xffffffffu, s[gi], 1);
+            s[gi] += __shfl_xor_sync(0xffffffffu, s[gi], 2);
+        }
+    }
+    if (qd == 0) {
+#pragma unroll
+        for (int gi = 0; gi < GRP; ++gi)
+            if (gi < grp) sc[gi][pos] = valid ? s[gi] * a.scale : -INFINITY;
+    }
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
-        vrec_s[tid * NG + g] = vr[g];
-        vsc_s[tid * NG + g] = vsr[g];
+        vrec_s[(pos * NG + g) * 4 + qd] = vw[g];
+        if (qd == 0) vsc_s[pos * NG + g] = vsr[g];
     }
-    vz_s[tid] = vzr;
+    if (qd == 0) vz_s[pos] = vzr;
+    __syncthreads();
 
-    // 2. chunk maximum and sum per query head (warp shuffles, then the warps in order)
+    // 2. chunk maximum and sum per query head: the first 4 warps, a position
+    //    per thread (warp shuffles, then the warps in order)
+    if (warp < kStatWarps) {
 #pragma unroll
-    for (int gi = 0; gi < kMaxGroup; ++gi) {
-        if (gi >= grp) break;
-        float m = sc[gi][tid];
+        for (int gi = 0; gi < kMaxGroup; ++gi) {
+            if (gi >= grp) break;
+            float m = sc[gi][tid];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (lane == 0) wmax[warp][gi] = m;
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if (lane == 0) wmax[warp][gi] = m;
+        }
     }
     __syncthreads();
     if (tid < grp) {
         float m = wmax[0][tid];
-        for (int w = 1; w < kWarps; ++w) m = fmaxf(m, wmax[w][tid]);
+        for (int w = 1; w < kStatWarps; ++w) m = fmaxf(m, wmax[w][tid]);
         cm[tid] = m;
     }
     __syncthreads();
+    if (warp < kStatWarps) {
+        const int t2 = c * kChunk + tid;
 #pragma unroll
-    for (int gi = 0; gi < kMaxGroup; ++gi) {
-        if (gi >= grp) break;
-        const float p = tok < a.T ? expf(sc[gi][tid] - cm[gi]) : 0.f;
-        sc[gi][tid] = p;
-        float l = p;
+        for (int gi = 0; gi < kMaxGroup; ++gi) {
+            if (gi >= grp) break;
+            const float p = t2 < a.T ? expf(sc[gi][tid] - cm[gi]) : 0.f;
+            sc[gi][tid] = p;
+            float l = p;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-        if (lane == 0) wsum[warp][gi] = l;
+            for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+            if (lane == 0) wsum[warp][gi] = l;
+        }
     }
     __syncthreads();
     if (tid < grp) {
         float l = 0.f;
-        for (int w = 0; w < kWarps; ++w) l += wsum[w][tid];
+        for (int w = 0; w < kStatWarps; ++w) l += wsum[w][tid];
         cl[tid] = l;
     }
 
-    // 3. weighted sum of V: warp w, positions 32w .. 32w + 31; lane l, channels l + 32g
-    float acc[kMaxGroup][NG];
+    // 3. weighted sum of V: warp w, positions 8w .. 8w + 7; lane l, channels l + 32g
+    float acc[GRP][NG];
 #pragma unroll
-    for (int gi = 0; gi < kMaxGroup; ++gi)
+    for (int gi = 0; gi < GRP; ++gi)
 #pragma unroll
         for (int g = 0; g < NG; ++g) acc[gi][g] = 0.f;
     const int w8 = lane >> 3, sh = 4 * (lane & 7);
-    const int nvalid = min(32, a.T - (c * kChunk + 32 * warp));
-#pragma unroll 4
-    for (int i = 0; i < 32; ++i) {
+    const int nvalid = min(8, a.T - (c * kChunk + 8 * warp));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
         if (i >= nvalid) break;
-        const int tl = 32 * warp + i;
+        const int tl = 8 * warp + i;
         const uint32_t zw = vz_s[tl];
-        const uint32_t *vrec = reinterpret_cast<const uint32_t *>(vrec_s + tl * NG);
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
-            const uint32_t word = vrec[4 * g + w8];
+            const uint32_t word = vrec_s[(tl * NG + g) * 4 + w8];
             const float sg = __half2float(__ushort_as_half(vsc_s[tl * NG + g]));
             const int z = (int)((zw >> (4 * g)) & 0xFu);
             const float vval = (float)((int)((word >> sh) & 0xFu) - z) * sg;
 #pragma unroll
-            for (int gi = 0; gi < kMaxGroup; ++gi)
+            for (int gi = 0; gi < GRP; ++gi)
                 if (gi < grp) acc[gi][g] = fmaf(sc[gi][tl], vval, acc[gi][g]);
         }
     }
     // lane l holds channel 32g + 8*(l/8) + l%8 = 32g + l; the V stage is dead
     __syncthreads();
 #pragma unroll
-    for (int gi = 0; gi < kMaxGroup; ++gi)
+    for (int gi = 0; gi < GRP; ++gi)
         if (gi < grp)
 #pragma unroll
-            for (int g = 0; g < NG; ++g) red[warp][gi][32 * g + lane] = acc[gi][g];
+            for (int g = 0; g < NG; ++g) red[((size_t)warp * grp + gi) * D + 32 * g + lane] = acc[gi][g];
     __syncthreads();
-    for (int i = tid; i < grp * D; i += kChunk) {
+    for (int i = tid; i < grp * D; i += kAttnThreads) {
         const int gi = i / D, d = i - gi * D;
         float v = 0.f;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) v += red[w][gi][d];
+        for (int w = 0; w < kAttnWarps; ++w) v += red[((size_t)w * grp + gi) * D + d];
         const size_t qi = (size_t)(h * grp + gi) * a.nch + c;
         a.ws_acc[qi * D + d] = v;
         if (d == 0) {
@@ -287,13 +324,13 @@ __global__ void __launch_bounds__(kChunk) attn_partial_kernel(const AttnArgs a) 
     }
 }
 
-// Merge of the chunk partials, one CTA per query head.  M (the largest chunk
-// maximum) and L = sum_c exp(m_c - M) l_c come from fixed-order block
-// reductions; the partial sums are staged slice by slice in shared memory
-// with independent 16-byte loads (one round trip per slice), and thread d
-// then sums channel d over the slice's chunks in order.
+// Merge of the chunk partials, one CTA per query head and slice of 32
+// channels.  M (the largest chunk maximum) and L = sum_c exp(m_c - M) l_c
+// come from fixed-order block reductions; warp w adds channel lane of the
+// chunks c = w, w + 8, ... in order (coalesced 128-byte rows), and the eight
+// warps' sums are added in warp order.
 constexpr int kMergeThreads = 256;
-constexpr int kMergeFloats = 8192;  // one slice: 32 KB of partial sums
+constexpr int kMergeWarps = kMergeThreads / 32;
 
 __device__ float block_max(float v, float *red) {
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -318,50 +355,88 @@ __device__ float block_sum(float v, float *red) {
 }
 
 __global__ void __launch_bounds__(kMergeThreads) attn_combine_kernel(const AttnArgs a, int D) {
-    __shared__ __align__(16) float buf[kMergeFloats];
-    __shared__ float wt[kMergeFloats / 32];
-    __shared__ float red[kMergeThreads / 32];
-    const int i = blockIdx.x, tid = threadIdx.x;
+    __shared__ float red[kMergeWarps];
+    __shared__ float part[kMergeWarps][32];
+    attn_pdl_wait();  // the chunk kernel's partials are complete
+    const int i = blockIdx.x, d0 = 32 * blockIdx.y, tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
     const int nch = a.nch;
     const float *ml = a.ws_ml + (size_t)i * nch * 2;
-    float m = -INFINITY;
+    const float *acc = a.ws_acc + (size_t)i * nch * D + d0 + lane;
+    // the first eight chunks of this warp (c = warp, warp + 8, ...) are loaded
+    // together with the statistics, before the maximum is known
+    float mv[8], av[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const int c = warp + u * kMergeWarps;
+        mv[u] = c < nch ? ml[2 * c] : -INFINITY;
+        av[u] = c < nch ? acc[(size_t)c * D] : 0.f;
+    }
+    float m = -INFINITY, lraw[2] = {0.f, 0.f}, mraw[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int c = tid + u * kMergeThreads;
+        if (c < nch) {
+            mraw[u] = ml[2 * c];
+            lraw[u] = ml[2 * c + 1];
+        }
+    }
     for (int c = tid; c < nch; c += kMergeThreads) m = fmaxf(m, ml[2 * c]);
     const float M = block_max(m, red);
     float l = 0.f;
-    for (int c = tid; c < nch; c += kMergeThreads) l += expf(ml[2 * c] - M) * ml[2 * c + 1];
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+        if (tid + u * kMergeThreads < nch) l += expf(mraw[u] - M) * lraw[u];
+    for (int c = tid + 2 * kMergeThreads; c < nch; c += kMergeThreads) l += expf(ml[2 * c] - M) * ml[2 * c + 1];
     const float L = block_sum(l, red);
-    const int per = kMergeFloats / D;  // chunks per slice
     float o = 0.f;
-    for (int c0 = 0; c0 < nch; c0 += per) {
-        const int nc = min(per, nch - c0);
-        const float4 *src = reinterpret_cast<const float4 *>(a.ws_acc + ((size_t)i * nch + c0) * D);
-        float4 *dst = reinterpret_cast<float4 *>(buf);
-        const int n4 = nc * D / 4;
-        int j = tid;
-        for (; j + 7 * kMergeThreads < n4; j += 8 * kMergeThreads) {
-            float4 v[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = src[j + u * kMergeThreads];
+    for (int u = 0; u < 8; ++u)
+        if (warp + u * kMergeWarps < nch) o = fmaf(expf(mv[u] - M), av[u], o);
+    // further chunks, eight loads in flight at a time
+    for (int c0 = warp + 8 * kMergeWarps; c0 < nch; c0 += 8 * kMergeWarps) {
 #pragma unroll
-            for (int u = 0; u < 8; ++u) dst[j + u * kMergeThreads] = v[u];
+        for (int u = 0; u < 8; ++u) {
+            const int c = c0 + u * kMergeWarps;
+            mv[u] = c < nch ? ml[2 * c] : -INFINITY;
+            av[u] = c < nch ? acc[(size_t)c * D] : 0.f;
         }
-        for (; j < n4; j += kMergeThreads) dst[j] = src[j];
-        for (int c = tid; c < nc; c += kMergeThreads) wt[c] = expf(ml[2 * (c0 + c)] - M);
-        __syncthreads();
-        if (tid < D)
-            for (int c = 0; c < nc; ++c) o = fmaf(wt[c], buf[c * D + tid], o);
-        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (c0 + u * kMergeWarps < nch) o = fmaf(expf(mv[u] - M), av[u], o);
     }
-    if (tid < D) a.out[(size_t)i * D + tid] = o / L;
+    part[warp][lane] = o;
+    __syncthreads();
+    if (warp == 0) {
+        float t = 0.f;
+#pragma unroll
+        for (int w = 0; w < kMergeWarps; ++w) t += part[w][lane];
+        a.out[(size_t)i * D + d0 + lane] = t / L;
+    }
 }
 
-template <int NG>
+template <int NG, int GRP>
 cudaError_t launch_attn(const AttnArgs &args, cudaStream_t s) {
-    attn_partial_kernel<NG><<<dim3((unsigned)args.nch, (unsigned)args.Hkv), kChunk, 0, s>>>(args);
-    cudaError_t e = cudaGetLastError();
+    const size_t smem = attn_smem_bytes(NG, args.grp);
+    cudaError_t e = cudaFuncSetAttribute(attn_partial_kernel<NG, GRP>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    attn_combine_kernel<<<(unsigned)args.Hq, kMergeThreads, 0, s>>>(args, 32 * NG);
-    return cudaGetLastError();
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)args.nch, (unsigned)args.Hkv, 1);
+    cfg.blockDim = dim3(kAttnThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, attn_partial_kernel<NG, GRP>, args);
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3((unsigned)args.Hq, (unsigned)NG, 1);
+    cfg.blockDim = dim3(kMergeThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    return cudaLaunchKernelEx(&cfg, attn_combine_kernel, args, 32 * NG);
 }
 
 }  // namespace
@@ -406,16 +481,22 @@ spectra_status launch_attention(const spectra_kv &k, const spectra_kv &v, const 
     a.ws_ml = static_cast<float *>(ws);
     a.ws_acc = a.ws_ml + ml_floats(Hq, a.nch);
     a.out = out;
+    const int bucket = a.grp <= 2 ? 2 : (a.grp <= 4 ? 4 : 8);
     cudaError_t e;
-    switch (k.head_dim / 32) {
-        case 1: e = launch_attn<1>(a, s); break;
-        case 2: e = launch_attn<2>(a, s); break;
-        case 3: e = launch_attn<3>(a, s); break;
-        case 4: e = launch_attn<4>(a, s); break;
-        case 5: e = launch_attn<5>(a, s); break;
-        case 6: e = launch_attn<6>(a, s); break;
-        case 7: e = launch_attn<7>(a, s); break;
-        case 8: e = launch_attn<8>(a, s); break;
+    switch (k.head_dim / 32 * 16 + bucket) {
+#define SPECTRA_ATTN_CASE(NG)                                      \
+    case NG * 16 + 2: e = launch_attn<NG, 2>(a, s); break;         \
+    case NG * 16 + 4: e = launch_attn<NG, 4>(a, s); break;         \
+    case NG * 16 + 8: e = launch_attn<NG, 8>(a, s); break;
+        SPECTRA_ATTN_CASE(1)
+        SPECTRA_ATTN_CASE(2)
+        SPECTRA_ATTN_CASE(3)
+        SPECTRA_ATTN_CASE(4)
+        SPECTRA_ATTN_CASE(5)
+        SPECTRA_ATTN_CASE(6)
+        SPECTRA_ATTN_CASE(7)
+        SPECTRA_ATTN_CASE(8)
+#undef SPECTRA_ATTN_CASE
         default: return SPECTRA_ERR_SHAPE;
     }
     return e == cudaSuccess ? SPECTRA_OK : SPECTRA_ERR_CUDA;

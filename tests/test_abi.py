@@ -239,15 +239,20 @@ def test_selftest_wait_argument_checks(L):
 
 
 def test_chain_argument_checks(L):
-    ws = L.spectra_gemv_chain_workspace_size()
-    assert ws >= 4
     lay = _lib.Layer(64, 128, 0, FAKE, FAKE, FAKE, None, None, 0, None)
     layers = (_lib.Layer * 1)(lay)
+    # the workspace size rejects bad arguments before touching the device
+    assert L.spectra_gemv_chain_workspace_size(None, 1) == 0
+    assert L.spectra_gemv_chain_workspace_size(layers, 0) == 0
+    bad_shape = (_lib.Layer * 1)(_lib.Layer(64, 100, 0, FAKE, FAKE, FAKE, None, None, 0, None))
+    assert L.spectra_gemv_chain_workspace_size(bad_shape, 1) == 0
+    ws = 16
     xs = (ctypes.c_void_p * 1)(FAKE)
     ys = (ctypes.c_void_p * 1)(FAKE)
     # argument errors come back before any CUDA call
     assert L.spectra_gemv_chain(layers, xs, ys, 1, 0, None, ws, None) == _lib.ERR_INVALID_ARG
     assert L.spectra_gemv_chain(layers, xs, ys, 1, 0, FAKE, ws - 1, None) == _lib.ERR_BUFFER_TOO_SMALL
+    ws = 1 << 20
     assert L.spectra_gemv_chain(layers, xs, ys, 1, 0, FAKE + 4, ws, None) == _lib.ERR_ALIGN
     assert L.spectra_gemv_chain(layers, xs, ys, 0, 0, FAKE, ws, None) == _lib.ERR_SHAPE
     assert L.spectra_gemv_chain(layers, xs, ys, _lib.MAX_BATCH + 1, 0, FAKE, ws, None) == _lib.ERR_SHAPE
