@@ -95,6 +95,8 @@ def _declare(L):
     L.spectra_ref_gather_bulk.restype = None
     L.spectra_ref_pack_outliers.argtypes = [i32, i32, P, P, i32, P]
     L.spectra_ref_pack_outliers.restype = None
+    L.spectra_ref_row_table.argtypes = [i32, i32, P, P, P, P, i32, P, i32, P, P, P, P]
+    L.spectra_ref_row_table.restype = None
     L.spectra_ref_gemm_compact.argtypes = [i32, i32, i32, P, P, P, P, P, P, i32, P, i32, P, P]
     L.spectra_ref_gemm_compact.restype = None
     L.spectra_ref_embed_compact.argtypes = [i32, i32, i32, P, P, P, P, P, P, i32, P, i32, P]
@@ -284,6 +286,34 @@ def embed(can: Canonical, w_bits: np.ndarray, idx: np.ndarray, ids) -> np.ndarra
                                  _p(out) if tok.size else None)
     if st != OK:
         raise OracleError(st)
+    return out
+
+
+# ------------------------------------------------------------------ row table
+
+@dataclass
+class RowTable:
+    """A table that is only gathered, every row's pieces contiguous."""
+    codes: np.ndarray     # uint8 [n * G * 16]
+    scales: np.ndarray    # uint16 [n * G]
+    zeros: np.ndarray     # uint32 [n * S]
+    outliers: np.ndarray  # uint16 [n * n_o]
+
+
+def row_table(can: Canonical, w_bits: np.ndarray, idx: np.ndarray) -> RowTable:
+    """Row-table layout of canonical arrays over k bulk columns (can.codes is
+    [n, k]); w_bits is the BF16 matrix [n, kw] the outlier values come from."""
+    codes = _c(can.codes, np.uint8)
+    n, k = codes.shape
+    w = _c(w_bits, np.uint16)
+    ix = _c(idx, np.int32)
+    G, S = k // 32, -(-(k // 32) // 8)
+    out = RowTable(np.zeros(n * G * 16, np.uint8), np.zeros(n * G, np.uint16),
+                   np.zeros(n * S, np.uint32), np.zeros(max(1, n * ix.size), np.uint16))
+    lib().spectra_ref_row_table(n, k, _p(codes), _p(_c(can.scales, np.uint16)), _p(_c(can.zeros, np.uint8)),
+                                _p(w), w.shape[1], _p(ix) if ix.size else None, ix.size, _p(out.codes),
+                                _p(out.scales), _p(out.zeros), _p(out.outliers))
+    out.outliers = out.outliers[: n * ix.size]
     return out
 
 

@@ -490,6 +490,41 @@ void spectra_ref_gather_bulk(const uint16_t *w, int32_t n, int32_t k, const int3
             w_b[i * k_bulk + p] = bulk_idx[p] < 0 ? 0 : w[i * k + bulk_idx[p]];
 }
 
+/*
+ * Row table: the layout of a table that is only gathered (an untied
+ * embedding).  Same canonical arrays as spectra_ref_pack_layout (codes,
+ * scales, zeros over k bulk columns; w is the BF16 matrix with kw columns per
+ * row); every row's pieces are contiguous:
+ *   rcodes   : byte (i*G + g)*16 + 4w + j/2 holds, in its low (j even) or high
+ *              (j odd) nibble, the code of bulk column 32g + 8w + j of row i;
+ *   rscales  : element i*G + g is the FP16 scale of group g of row i;
+ *   rzeros   : word i*S + g/8 holds in nibble g%8 the zero point of group g;
+ *   routl    : element i*n_o + o is W[i][idx[o]] (BF16 bits).
+ * G = k/32, S = ceil(G/8).  No padding rows.
+ */
+void spectra_ref_row_table(int32_t n, int32_t k, const uint8_t *codes, const uint16_t *scales,
+                           const uint8_t *zeros, const uint16_t *w, int32_t kw, const int32_t *idx,
+                           int32_t n_o, uint8_t *rcodes, uint16_t *rscales, uint32_t *rzeros,
+                           uint16_t *routl)
+{
+    const int64_t G = k / 32, S = cdiv(G, 8);
+    memset(rcodes, 0, (size_t)(n * G * 16));
+    memset(rzeros, 0, (size_t)(n * S) * 4);
+    for (int64_t i = 0; i < n; ++i) {
+        for (int64_t kk = 0; kk < k; ++kk) {
+            int64_t g = kk / 32, in = kk % 32, word = in / 8, j = in % 8;
+            uint8_t c = codes[i * k + kk] & 0xF;
+            rcodes[(i * G + g) * 16 + word * 4 + j / 2] |= (uint8_t)((j % 2) ? (c << 4) : c);
+        }
+        for (int64_t g = 0; g < G; ++g) {
+            rscales[i * G + g] = scales[i * G + g];
+            rzeros[i * S + g / 8] |= (uint32_t)(zeros[i * G + g] & 0xF) << (4 * (g % 8));
+        }
+        for (int64_t o = 0; o < n_o; ++o)
+            routl[i * n_o + o] = w[i * kw + idx[o]];
+    }
+}
+
 /* The outlier block alone, in the RT32 order of spectra_ref_pack_layout. */
 void spectra_ref_pack_outliers(int32_t n, int32_t k, const uint16_t *w, const int32_t *idx,
                                int32_t n_o, uint16_t *poutl)

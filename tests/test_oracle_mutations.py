@@ -62,6 +62,14 @@ MUTATIONS = {
     "attention_key_zero_index": ("double kv = ((double)kc[slot * D + d] - (double)kz[slot * G + d / 32]) * S;",
                                  "double kv = ((double)kc[slot * D + d] - (double)kz[slot * G + d % G]) * S;"),
     "attention_scale_dropped": ("sc[t] = scale * acc;", "sc[t] = acc;"),
+    "row_table_codes_transposed": ("rcodes[(i * G + g) * 16 + word * 4 + j / 2]",
+                                   "rcodes[(g * n + i) * 16 + word * 4 + j / 2]"),
+    "row_table_scales_transposed": ("rscales[i * G + g] = scales[i * G + g];",
+                                    "rscales[g * n + i] = scales[i * G + g];"),
+    "row_table_outlier_slot_reversed": ("routl[i * n_o + o] = w[i * kw + idx[o]];",
+                                        "routl[i * n_o + o] = w[i * kw + idx[n_o - 1 - o]];"),
+    "row_table_outlier_row_stride": ("routl[i * n_o + o] = w[i * kw + idx[o]];",
+                                     "routl[i * n_o + o] = w[i * k + idx[o]];"),
     "embed_zero_point_sign": ("dst[col] = ((double)codes[row * k + col] - (double)zeros[grp]) * S;",
                               "dst[col] = ((double)codes[row * k + col] + (double)zeros[grp]) * S;"),
 }
@@ -93,6 +101,8 @@ PIN_FUNCS = [
     pins.test_attention_exact_grid_is_textbook,
     pins.test_attention_one_token_and_zero_query,
     pins.test_kv_pack_golden_offsets,
+    pins.test_row_table_golden_offsets,
+    pins.test_row_table_rows_are_the_packed_rows,
 ]
 _PARAMS = {
     "test_quantizer_exact_grid": [{"S": 2.0 ** -7, "z": 5}],

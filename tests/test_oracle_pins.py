@@ -799,3 +799,63 @@ def test_attention_tolerance_covers_its_budget(ref):
                 p = np.exp(s2 - s2.max()); p /= p.sum()
                 o2 = p @ V[:, 0, d] + sign * 2e-3 * (p @ np.abs(V[:, 0, d]))
                 assert abs(o2 - out[i, d]) <= tol[i, d]
+
+
+# ----------------------------------------------------------------- row table
+
+def test_row_table_golden_offsets(ref, golden_dir):
+    """Each hand-derived offset of the row table holds the one planted value."""
+    lines = [l.split("#")[0].split() for l in open(os.path.join(golden_dir, "row_table_offsets.txt"))]
+    lines = [l for l in lines if l]
+    assert len(lines) == 14
+    for n, k, n_o, kind, row, col, off, nib in lines:
+        n, k, n_o, row, col, off = int(n), int(k), int(n_o), int(row), int(col), int(off)
+        G = k // 32
+        can = ref.Canonical(np.zeros((n, k), np.uint8), np.zeros((n, G), np.uint16), np.zeros((n, G), np.uint8))
+        w = np.zeros((n, k + 7), np.uint16)  # a wider BF16 matrix: the outlier values come by its stride
+        idx = np.arange(n_o, dtype=np.int32) * 3 + 1
+        if kind == "code":
+            can.codes[row, col] = 0xA
+        elif kind == "scale":
+            can.scales[row, col] = 0x1234
+        elif kind == "zero":
+            can.zeros[row, col] = 0x9
+        else:
+            w[row, idx[col]] = 0x4321
+        t = ref.row_table(can, w, idx)
+        if kind == "code":
+            assert np.flatnonzero(t.codes).tolist() == [off]
+            assert t.codes[off] == (0x0A if nib == "low" else 0xA0)
+        elif kind == "scale":
+            assert np.flatnonzero(t.scales).tolist() == [off] and t.scales[off] == 0x1234
+        elif kind == "zero":
+            assert np.flatnonzero(t.zeros).tolist() == [off]
+            assert t.zeros[off] == 0x9 << (4 * int(nib))
+        else:
+            assert np.flatnonzero(t.outliers).tolist() == [off] and t.outliers[off] == 0x4321
+
+
+def test_row_table_rows_are_the_packed_rows(ref):
+    """A row of the row table holds the same code records, scales, zero words
+    and outlier values as that row's lane of the RT32 layout (a permutation,
+    nothing rounded)."""
+    rng = np.random.default_rng(8)
+    n, k, n_o = 70, 320, 13
+    # BF16 bits of N(0, 0.02) values (the high half of their FP32 bits)
+    w = (rng.standard_normal((n, k)).astype(np.float32) * 0.02).view(np.uint32) >> 16
+    w = w.astype(np.uint16)
+    idx = np.sort(rng.choice(k, n_o, replace=False)).astype(np.int32)
+    can = ref.quantize(w, idx)
+    p = ref.pack_layout(can, w, idx)
+    t = ref.row_table(can, w, idx)
+    G, S, O8 = k // 32, -(-(k // 32) // 8), -(-n_o // 8)
+    for i in range(n):
+        tt, r = divmod(i, 32)
+        for g in range(G):
+            a = ((tt * G + g) * 32 + r) * 16
+            assert np.array_equal(t.codes[(i * G + g) * 16:(i * G + g + 1) * 16], p.codes[a:a + 16])
+            assert t.scales[i * G + g] == p.scales[((tt * S + g // 8) * 32 + r) * 8 + g % 8]
+        for s_ in range(S):
+            assert t.zeros[i * S + s_] == p.zeros[(tt * S + s_) * 32 + r]
+        for o in range(n_o):
+            assert t.outliers[i * n_o + o] == p.outliers[((tt * O8 + o // 8) * 32 + r) * 8 + o % 8]
