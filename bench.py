@@ -430,7 +430,24 @@ def extras(device, stream, peak_gbs, tau):
                          "gbs_single_flushed": round(b / us * 1e-3, 1),
                          "frac_single_flushed": round(b / us * 1e-3 / peak_gbs, 3)})
         out["embed_rows_131072x3072_bf16"] = rows
-        del w, lay
+        # the same table converted to a row table (every row contiguous): a
+        # gathered row reads only its own bytes
+        table = sp.spectra_row_table_from_layer(lay, stream=stream)
+        stream.synchronize()
+        rows = []
+        for m in (1, 64, 4096):
+            ids = torch.from_numpy(np.random.default_rng(m).integers(0, spec.n, m).astype(np.int32)).to(device)
+            o = torch.empty((m, spec.k), dtype=torch.bfloat16, device=device)
+            us, p10, p90 = time_single(
+                lambda: sp.spectra_embed_rows(table, ids, o, stream=stream), stream, 30, flush)
+            us_r = time_rotating([lambda: sp.spectra_embed_rows(table, ids, o, stream=stream)], stream, 200)
+            b = embed_bytes(spec.k, lay.n_outliers, m)
+            rows.append({"m": m, "n_outliers": lay.n_outliers, "us_single_flushed": round(us, 2),
+                         "us_back_to_back": round(us_r, 2), "bytes": b,
+                         "gbs_single_flushed": round(b / us * 1e-3, 1),
+                         "frac_single_flushed": round(b / us * 1e-3 / peak_gbs, 3)})
+        out["embed_rows_row_table_131072x3072_bf16"] = rows
+        del w, lay, table
         out["kv_attention_decode_8192"] = kv_rows(device, stream, peak_gbs, flush)
         out["single_512x512"] = single_512_rows(device, stream, peak_gbs, flush)
     return out
@@ -985,6 +1002,9 @@ def summary_of(line, extra, cpu):
     em = extra.get("embed_rows_131072x3072_bf16")
     if em:
         out["embed_4096_frac"] = em[-1]["frac_single_flushed"]
+    er = extra.get("embed_rows_row_table_131072x3072_bf16")
+    if er:
+        out["embed_4096_row_table_frac"] = er[-1]["frac_single_flushed"]
     if cpu:
         out["cpu"] = {"cores": cpu["cores"], "matvec_gbs": [cpu["matvec_gbs_1thread"], cpu["matvec_gbs_all_cores"]],
                       "pack_mw_s": [cpu["pack_mweights_per_s_1thread"], cpu["pack_mweights_per_s_all_cores"]]}
@@ -1154,14 +1174,21 @@ def run_embed(args):
     v = lay.view()
     stream = torch.cuda.Stream(device=device)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
-    fn = lambda: sp.spectra_embed(lay, ids, out, view=v, stream=stream)  # noqa: E731
+    if args.row_table:
+        table = sp.spectra_row_table_from_layer(lay, stream=stream)
+        stream.synchronize()
+        fn = lambda: sp.spectra_embed_rows(table, ids, out, stream=stream)  # noqa: E731
+    else:
+        fn = lambda: sp.spectra_embed(lay, ids, out, view=v, stream=stream)  # noqa: E731
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             fn()
         us, p10, p90 = time_single(fn, stream, args.steps, flush)
     b = embed_bytes(spec.k, lay.n_outliers, args.m)
+    sp.spectra_device_status(stream=stream)
     print(json.dumps({"case": "embed", "n": spec.n, "k": spec.k, "m": args.m, "tau": args.tau,
-                      "compact": args.compact, "n_outliers": lay.n_outliers, "us": round(us, 2),
+                      "compact": args.compact, "row_table": args.row_table,
+                      "n_outliers": lay.n_outliers, "us": round(us, 2),
                       "us_p10": round(p10, 2), "us_p90": round(p90, 2), "bytes": b,
                       "gbs": round(b / us * 1e-3, 1), "frac": round(b / us * 1e-3 / peak, 4)}),
           flush=True)
@@ -1202,6 +1229,8 @@ def main():
     ap.add_argument("--k", type=int, default=wl.LM_HEAD_K)
     ap.add_argument("--nt", type=int, default=0, help="Student-t columns of the single matrix")
     ap.add_argument("--m", type=int, default=1)
+    ap.add_argument("--row-table", action="store_true",
+                    help="--case embed: gather from the table converted to a row table")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

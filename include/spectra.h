@@ -386,6 +386,42 @@ SPECTRA_API spectra_status spectra_embed(const spectra_layer *table, const int32
                                          void *out, spectra_dtype out_dtype, void *stream);
 
 /*
+ * Row table: the layout for a table that is only gathered (an untied
+ * embedding).  The RT32 layout serves the matvec (a warp streams whole
+ * 32-row tiles) and puts a row's 16-byte records 512 bytes apart, so a
+ * gathered row moves whole DRAM lines for every record.  A row table keeps
+ * every row's pieces contiguous, G = k_bulk/32, S = ceil(G/8):
+ *   codes     : record (i*G + g)*16 bytes, the 32 codes of group g of row i
+ *               (word w, nibble j = bulk column 32g + 8w + j, as in RT32);
+ *   scales    : FP16 bits, element i*G + g;
+ *   zeros     : u32 word i*S + g/8, nibble g%8;
+ *   outlier_w : BF16 bits, element i*n_outliers + o = W[i][outlier_idx[o]];
+ *   outlier_idx and bulk_idx as in the layer.
+ * A row-table view is a spectra_layer whose four data buffers hold this
+ * layout (no padding rows).  Pass it only to spectra_embed_rows.
+ *
+ * spectra_row_table_sizes: bytes of each buffer for converting `layer`
+ * (n_pad = n; bulk_idx_bytes is 0 for a masked bulk).  Host only.
+ * spectra_row_table_from_layer: writes the row table of packed layer
+ * `layer` (RT32) into caller-owned device buffers codes (16-byte aligned),
+ * scales, zeros (4-byte aligned) and outlier_w (NULL when there are no
+ * outlier columns), a pure permutation of the layer's bytes, and fills
+ * *table_out with a view that shares the layer's outlier_idx and bulk_idx.
+ * Asynchronous, allocates nothing.
+ * spectra_embed_rows: spectra_embed over a row-table view: same output, bit
+ * for bit, and the same handling of bad ids; a requested row reads its
+ * contiguous pieces (k_bulk/2 + k_bulk/16 + 4S + 2*n_outliers bytes).
+ * Errors: INVALID_ARG, SHAPE, ALIGN, UNSUPPORTED, CUDA.
+ */
+SPECTRA_API spectra_status spectra_row_table_sizes(const spectra_layer *layer, spectra_sizes *out);
+SPECTRA_API spectra_status spectra_row_table_from_layer(const spectra_layer *layer, uint8_t *codes,
+                                                        uint16_t *scales, uint32_t *zeros,
+                                                        uint16_t *outlier_w, spectra_layer *table_out,
+                                                        void *stream);
+SPECTRA_API spectra_status spectra_embed_rows(const spectra_layer *table, const int32_t *ids, int32_t m,
+                                              void *out, spectra_dtype out_dtype, void *stream);
+
+/*
  * Health of the kernels on the current device.  The matvec kernels' waits
  * for the asynchronous weight copies are bounded: a wait that gives up
  * raises a per-device flag instead of hanging, and the outputs of that

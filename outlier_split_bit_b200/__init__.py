@@ -268,6 +268,59 @@ def spectra_embed(table: PackedLayer, ids: torch.Tensor, out: torch.Tensor | Non
     return out
 
 
+@dataclass
+class RowTable:
+    """Row-table buffers of a packed table (every row's pieces contiguous,
+    for gathers only) and the view over them; the index lists are the
+    layer's own."""
+    layer: PackedLayer
+    codes: torch.Tensor
+    scales: torch.Tensor
+    zeros: torch.Tensor
+    outlier_w: torch.Tensor
+    _view: Layer
+
+    def view(self) -> Layer:
+        return self._view
+
+    @property
+    def n(self) -> int:
+        return self.layer.n
+
+    @property
+    def k(self) -> int:
+        return self.layer.k
+
+
+def spectra_row_table_from_layer(layer: PackedLayer, *, stream=None) -> RowTable:
+    """Convert a packed layer (RT32) into a row table (new device buffers)."""
+    v = layer.view()
+    sz = Sizes()
+    _check(_L.spectra_row_table_sizes(ctypes.byref(v), ctypes.byref(sz)), "spectra_row_table_sizes")
+    dev = layer.codes.device
+    codes = _alloc(sz.codes_bytes, torch.uint8, dev)
+    scales = _alloc(sz.scales_bytes, torch.int16, dev)
+    zeros = _alloc(sz.zeros_bytes, torch.int32, dev)
+    outw = _alloc(max(2, sz.outlier_w_bytes), torch.int16, dev)
+    out = Layer()
+    _check(_L.spectra_row_table_from_layer(ctypes.byref(v), _ptr(codes), _ptr(scales), _ptr(zeros),
+                                           _ptr(outw) if layer.n_outliers else None, ctypes.byref(out),
+                                           _stream(stream)), "spectra_row_table_from_layer")
+    return RowTable(layer, codes, scales, zeros, outw, out)
+
+
+def spectra_embed_rows(table: RowTable, ids: torch.Tensor, out: torch.Tensor | None = None, *,
+                       out_dtype=torch.bfloat16, stream=None) -> torch.Tensor:
+    """spectra_embed over a row table: rows ids (int32 [m]) dequantised, out [m, k]."""
+    m = int(ids.numel())
+    if out is None:
+        out = torch.empty((m, table.k), dtype=out_dtype, device=ids.device)
+    _check(_L.spectra_embed_rows(ctypes.byref(table.view()), _ptr(ids) if m else None, m,
+                                 _ptr(out) if m else None, _DT[out.dtype], _stream(stream)),
+           "spectra_embed_rows")
+    return out
+
+
 class BatchViews:
     """Host arrays of layer views and device pointers for spectra_gemv_batched,
     built once and reused (e.g. for graph capture)."""

@@ -81,6 +81,9 @@ SIGNATURES = {
     "spectra_device_status": (ctypes.c_int, [P]),
     "spectra_selftest_wait": (ctypes.c_int, [i32, P]),
     "spectra_embed": (ctypes.c_int, [LP, P, i32, P, ctypes.c_int, P]),
+    "spectra_row_table_sizes": (ctypes.c_int, [LP, ctypes.POINTER(Sizes)]),
+    "spectra_row_table_from_layer": (ctypes.c_int, [LP, P, P, P, P, LP, P]),
+    "spectra_embed_rows": (ctypes.c_int, [LP, P, i32, P, ctypes.c_int, P]),
     "spectra_pack_plan_noalloc": (ctypes.c_int, [P, P, i32, i32, f64, P, P, ctypes.POINTER(i32), P]),
     "spectra_crc32": (ctypes.c_uint32, [ctypes.c_uint32, P, sz]),
     "spectra_kv_sizes": (ctypes.c_int, [i32, i32, i32, ctypes.POINTER(sz), ctypes.POINTER(sz),

@@ -375,7 +375,74 @@ spectra_status spectra_embed(const spectra_layer *table, const int32_t *ids, int
     DeviceInfo dev;
     st = current_device(&dev);
     if (st != SPECTRA_OK) return st;
-    return launch_embed(*table, ids, m, out, (int)out_dtype, (cudaStream_t)stream, dev);
+    return launch_embed(*table, ids, m, out, (int)out_dtype, false, (cudaStream_t)stream, dev);
+}
+
+spectra_status spectra_row_table_sizes(const spectra_layer *layer, spectra_sizes *out) {
+    if (!out) return SPECTRA_ERR_INVALID_ARG;
+    spectra_status st = check_layer(layer);
+    if (st != SPECTRA_OK) return st;
+    const int32_t kb = bulk_cols(*layer);
+    const Geometry g = Geometry::of(layer->n, kb, layer->n_outliers);
+    out->n_pad = layer->n;
+    out->codes_bytes = (size_t)layer->n * g.G * 16;
+    out->scales_bytes = (size_t)layer->n * g.G * 2;
+    out->zeros_bytes = (size_t)layer->n * g.S * 4;
+    out->outlier_idx_bytes = (size_t)layer->n_outliers * 4;
+    out->outlier_w_bytes = (size_t)layer->n * layer->n_outliers * 2;
+    out->k_bulk = kb;
+    out->bulk_idx_bytes = layer->bulk_idx ? (size_t)kb * 4 : 0;
+    return SPECTRA_OK;
+}
+
+spectra_status spectra_row_table_from_layer(const spectra_layer *layer, uint8_t *codes, uint16_t *scales,
+                                            uint32_t *zeros, uint16_t *outlier_w, spectra_layer *table_out,
+                                            void *stream) {
+    spectra_status st = check_layer(layer);
+    if (st != SPECTRA_OK) return st;
+    if (!codes || !scales || !zeros || !table_out) return SPECTRA_ERR_INVALID_ARG;
+    if (layer->n_outliers > 0 && !outlier_w) return SPECTRA_ERR_INVALID_ARG;
+    if (!aligned16(codes) || ((uintptr_t)scales & 1u) || !aligned4(zeros) ||
+        (outlier_w && ((uintptr_t)outlier_w & 1u)))
+        return SPECTRA_ERR_ALIGN;
+    DeviceInfo dev;
+    st = current_device(&dev);
+    if (st != SPECTRA_OK) return st;
+    spectra_layer t = *layer;  // shape and the (shared) index lists
+    t.codes = codes;
+    t.scales = scales;
+    t.zeros = zeros;
+    t.outlier_w = layer->n_outliers > 0 ? outlier_w : nullptr;
+    st = launch_row_table(*layer, t, (cudaStream_t)stream, dev);
+    if (st == SPECTRA_OK) *table_out = t;
+    return st;
+}
+
+spectra_status spectra_embed_rows(const spectra_layer *table, const int32_t *ids, int32_t m, void *out,
+                                  spectra_dtype out_dtype, void *stream) {
+    if (!table) return SPECTRA_ERR_INVALID_ARG;
+    if (table->n < 1 || table->k < 32 || (table->k % 32) != 0) return SPECTRA_ERR_SHAPE;
+    if (table->n_outliers < 0 || table->n_outliers > table->k) return SPECTRA_ERR_INVALID_ARG;
+    if (!table->codes || !table->scales || !table->zeros) return SPECTRA_ERR_INVALID_ARG;
+    if (table->n_outliers > 0 && (!table->outlier_idx || !table->outlier_w)) return SPECTRA_ERR_INVALID_ARG;
+    if (!aligned16(table->codes) || ((uintptr_t)table->scales & 1u) || !aligned4(table->zeros) ||
+        (table->n_outliers > 0 && (((uintptr_t)table->outlier_w & 1u) || !aligned4(table->outlier_idx))))
+        return SPECTRA_ERR_ALIGN;
+    if (table->bulk_idx) {
+        if (table->k_bulk != compact_width(table->k, table->n_outliers)) return SPECTRA_ERR_INVALID_ARG;
+        if (!aligned16(table->bulk_idx)) return SPECTRA_ERR_ALIGN;
+    } else if (table->k_bulk != 0 && table->k_bulk != table->k) {
+        return SPECTRA_ERR_INVALID_ARG;
+    }
+    if (out_dtype != SPECTRA_F32 && out_dtype != SPECTRA_BF16) return SPECTRA_ERR_INVALID_ARG;
+    if (m < 0) return SPECTRA_ERR_SHAPE;
+    if (m == 0) return SPECTRA_OK;
+    if (!ids || !out) return SPECTRA_ERR_INVALID_ARG;
+    if (!aligned4(ids) || !aligned16(out)) return SPECTRA_ERR_ALIGN;
+    DeviceInfo dev;
+    spectra_status st = current_device(&dev);
+    if (st != SPECTRA_OK) return st;
+    return launch_embed(*table, ids, m, out, (int)out_dtype, true, (cudaStream_t)stream, dev);
 }
 
 static spectra_status check_kv(const spectra_kv *c) {

@@ -66,7 +66,9 @@ __device__ __forceinline__ void put(uint8_t *row, int col, float v) {
         reinterpret_cast<float *>(row)[col] = v;
 }
 
-template <bool kBF16>
+// kRows: the table is a row table (every row's code records, scales, zero
+// words and outlier values contiguous) instead of the RT32 layout.
+template <bool kBF16, bool kRows>
 __global__ void __launch_bounds__(kEmbedMaxThreads) embed_kernel(const EmbedArgs a) {
     extern __shared__ uint4 rowbuf[];  // one output row: k * (2 or 4) bytes
     uint8_t *row = reinterpret_cast<uint8_t *>(rowbuf);
@@ -84,10 +86,20 @@ __global__ void __launch_bounds__(kEmbedMaxThreads) embed_kernel(const EmbedArgs
         for (int g = threadIdx.x; g < a.G; g += blockDim.x) {
             float v[32];
             if (ok) {
-                const uint4 rec = a.codes[((size_t)t * a.G + g) * 32 + lane];
-                const size_t sg = ((size_t)t * a.S + (g >> 3)) * 32 + lane;
-                const float s = __half2float(__ushort_as_half(a.scales[sg * 8 + (g & 7)]));
-                const int z = (int)((a.zeros[sg] >> (4 * (g & 7))) & 0xFu);
+                uint4 rec;
+                float s;
+                int z;
+                if constexpr (kRows) {
+                    // row id's pieces are contiguous: a warp reads 512 bytes of records
+                    rec = a.codes[(size_t)id * a.G + g];
+                    s = __half2float(__ushort_as_half(a.scales[(size_t)id * a.G + g]));
+                    z = (int)((a.zeros[(size_t)id * a.S + (g >> 3)] >> (4 * (g & 7))) & 0xFu);
+                } else {
+                    rec = a.codes[((size_t)t * a.G + g) * 32 + lane];
+                    const size_t sg = ((size_t)t * a.S + (g >> 3)) * 32 + lane;
+                    s = __half2float(__ushort_as_half(a.scales[sg * 8 + (g & 7)]));
+                    z = (int)((a.zeros[sg] >> (4 * (g & 7))) & 0xFu);
+                }
                 const uint32_t wv[4] = {rec.x, rec.y, rec.z, rec.w};
 #pragma unroll
                 for (int w = 0; w < 4; ++w)
@@ -136,8 +148,26 @@ __global__ void __launch_bounds__(kEmbedMaxThreads) embed_kernel(const EmbedArgs
                 }
             }
         }
-        // 2. outlier columns, an octet per thread at a time
-        if (a.n_o > 0) {
+        // 2. outlier columns: in a row table the row's values are contiguous
+        //    (a thread per value, coalesced); in RT32 an octet per thread
+        if constexpr (kRows) {
+            if (a.n_o > 0) {
+                __syncthreads();
+                const uint16_t *ov = reinterpret_cast<const uint16_t *>(a.outw) + (size_t)(ok ? id : 0) * a.n_o;
+                for (int j = threadIdx.x; j < a.n_o; j += blockDim.x) {
+                    const int col = __ldg(a.oidx + j);
+                    if (col < 0 || col >= a.k) {
+                        atomicOr(&g_embed_error, 2u);
+                        continue;
+                    }
+                    const uint32_t b = ok ? (uint32_t)ov[j] : 0u;
+                    if constexpr (kBF16)
+                        reinterpret_cast<uint16_t *>(row)[col] = (uint16_t)b;
+                    else
+                        reinterpret_cast<uint32_t *>(row)[col] = b << 16;
+                }
+            }
+        } else if (a.n_o > 0) {
             __syncthreads();
             for (int o = threadIdx.x; o < a.O8; o += blockDim.x) {
                 const uint4 wv = ok ? a.outw[((size_t)t * a.O8 + o) * 32 + lane] : make_uint4(0, 0, 0, 0);
@@ -168,7 +198,7 @@ __global__ void __launch_bounds__(kEmbedMaxThreads) embed_kernel(const EmbedArgs
     }
 }
 
-template <bool kBF16>
+template <bool kBF16, bool kRows>
 cudaError_t launch(const EmbedArgs &args, unsigned grid, unsigned threads, size_t smem,
                    cudaStream_t s) {
     cudaLaunchConfig_t cfg = {};
@@ -181,28 +211,55 @@ cudaError_t launch(const EmbedArgs &args, unsigned grid, unsigned threads, size_
     attr.val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, embed_kernel<kBF16>, args);
+    return cudaLaunchKernelEx(&cfg, embed_kernel<kBF16, kRows>, args);
 }
 
 std::mutex g_embed_mu;
-bool g_embed_ready[2][64];
+bool g_embed_ready[4][64];
 
 // Raise the dynamic shared-memory limit of the kernel once per device.
-template <bool kBF16>
+template <bool kBF16, bool kRows>
 cudaError_t prepare(const DeviceInfo &dev) {
     std::lock_guard<std::mutex> lock(g_embed_mu);
     if (dev.device < 0 || dev.device >= 64) return cudaErrorInvalidDevice;
-    if (g_embed_ready[kBF16][dev.device]) return cudaSuccess;
+    bool &ready = g_embed_ready[(kBF16 ? 1 : 0) + (kRows ? 2 : 0)][dev.device];
+    if (ready) return cudaSuccess;
     const cudaError_t e = cudaFuncSetAttribute(
-        embed_kernel<kBF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dev.smem_optin);
-    if (e == cudaSuccess) g_embed_ready[kBF16][dev.device] = true;
+        embed_kernel<kBF16, kRows>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dev.smem_optin);
+    if (e == cudaSuccess) ready = true;
     return e;
+}
+
+// RT32 -> row table: a grid-stride loop over every code record, scale, zero
+// word and outlier value of the table, each copied to its row-table place
+// (a permutation: nothing is recomputed).
+__global__ void row_table_kernel(const uint4 *__restrict__ codes, const uint16_t *__restrict__ scales,
+                                 const uint32_t *__restrict__ zeros, const uint16_t *__restrict__ outw,
+                                 int n, int G, int S, int n_o, uint4 *__restrict__ rcodes,
+                                 uint16_t *__restrict__ rscales, uint32_t *__restrict__ rzeros,
+                                 uint16_t *__restrict__ routl) {
+    const int O8 = (n_o + 7) / 8;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    for (int64_t e = i0; e < (int64_t)n * G; e += stride) {
+        const int64_t i = e / G, g = e - i * G, t = i >> 5, r = i & 31;
+        rcodes[e] = codes[(t * G + g) * 32 + r];
+        rscales[e] = scales[((t * S + (g >> 3)) * 32 + r) * 8 + (g & 7)];
+    }
+    for (int64_t e = i0; e < (int64_t)n * S; e += stride) {
+        const int64_t i = e / S, sg = e - i * S, t = i >> 5, r = i & 31;
+        rzeros[e] = zeros[(t * S + sg) * 32 + r];
+    }
+    for (int64_t e = i0; e < (int64_t)n * n_o; e += stride) {
+        const int64_t i = e / n_o, o = e - i * n_o, t = i >> 5, r = i & 31;
+        routl[e] = outw[((t * O8 + (o >> 3)) * 32 + r) * 8 + (o & 7)];
+    }
 }
 
 }  // namespace
 
 spectra_status launch_embed(const spectra_layer &l, const int32_t *ids, int m, void *out,
-                            int out_type, cudaStream_t s, const DeviceInfo &dev) {
+                            int out_type, bool rows, cudaStream_t s, const DeviceInfo &dev) {
     const bool bf16 = out_type == SPECTRA_BF16;
     const size_t smem = (size_t)l.k * (bf16 ? 2 : 4);
     if (smem > dev.smem_optin) return SPECTRA_ERR_SHAPE;
@@ -231,11 +288,34 @@ spectra_status launch_embed(const spectra_layer &l, const int32_t *ids, int m, v
     if (threads > kEmbedMaxThreads) threads = kEmbedMaxThreads;
     const int64_t cap = (int64_t)dev.sm_count * kEmbedCtasPerSm;
     const unsigned grid = (unsigned)(m < cap ? m : cap);
-    cudaError_t e = bf16 ? prepare<true>(dev) : prepare<false>(dev);
-    if (e != cudaSuccess) return SPECTRA_ERR_CUDA;
-    e = bf16 ? launch<true>(a, grid, (unsigned)threads, smem, s)
-             : launch<false>(a, grid, (unsigned)threads, smem, s);
+    cudaError_t e;
+    if (rows) {
+        e = bf16 ? prepare<true, true>(dev) : prepare<false, true>(dev);
+        if (e != cudaSuccess) return SPECTRA_ERR_CUDA;
+        e = bf16 ? launch<true, true>(a, grid, (unsigned)threads, smem, s)
+                 : launch<false, true>(a, grid, (unsigned)threads, smem, s);
+    } else {
+        e = bf16 ? prepare<true, false>(dev) : prepare<false, false>(dev);
+        if (e != cudaSuccess) return SPECTRA_ERR_CUDA;
+        e = bf16 ? launch<true, false>(a, grid, (unsigned)threads, smem, s)
+                 : launch<false, false>(a, grid, (unsigned)threads, smem, s);
+    }
     return e == cudaSuccess ? SPECTRA_OK : SPECTRA_ERR_CUDA;
+}
+
+spectra_status launch_row_table(const spectra_layer &src, const spectra_layer &dst, cudaStream_t s,
+                                const DeviceInfo &dev) {
+    const Geometry g = Geometry::of(src.n, bulk_cols(src), src.n_outliers);
+    const int64_t work = (int64_t)src.n * g.G;
+    int64_t blocks = cdiv(work, 256);
+    const int64_t cap = (int64_t)dev.sm_count * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    row_table_kernel<<<(unsigned)blocks, 256, 0, s>>>(
+        reinterpret_cast<const uint4 *>(src.codes), src.scales, src.zeros, src.outlier_w, src.n, g.G, g.S,
+        src.n_outliers, reinterpret_cast<uint4 *>(const_cast<uint8_t *>(dst.codes)), const_cast<uint16_t *>(dst.scales),
+        const_cast<uint32_t *>(dst.zeros), const_cast<uint16_t *>(dst.outlier_w));
+    return cudaGetLastError() == cudaSuccess ? SPECTRA_OK : SPECTRA_ERR_CUDA;
 }
 
 spectra_status embed_device_error(unsigned int *bits, cudaStream_t s) {

@@ -114,8 +114,12 @@ spectra_status tc_device_error(unsigned int *bits, cudaStream_t s);
 
 // ---- embedding-row gather (embed.cu) ----
 // Rows ids[0..m) of a packed table, dequantised (1 <= m).
+// `rows`: the view's buffers hold the row-table layout instead of RT32.
 spectra_status launch_embed(const spectra_layer &l, const int32_t *ids, int m, void *out,
-                            int out_type, cudaStream_t s, const DeviceInfo &dev);
+                            int out_type, bool rows, cudaStream_t s, const DeviceInfo &dev);
+// RT32 layer `src` -> the row-table buffers named by `dst`.
+spectra_status launch_row_table(const spectra_layer &src, const spectra_layer &dst, cudaStream_t s,
+                                const DeviceInfo &dev);
 // Reads (and clears) the gather's flag: bit 0 a token id outside the table,
 // bit 1 an outlier index outside [0, k).
 spectra_status embed_device_error(unsigned int *bits, cudaStream_t s);

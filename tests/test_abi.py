@@ -260,3 +260,23 @@ def test_chain_argument_checks(L):
     bad = (_lib.Layer * 1)(_lib.Layer(64, 100, 0, FAKE, FAKE, FAKE, None, None, 0, None))
     assert L.spectra_gemv_chain(bad, xs, ys, 1, 0, FAKE, ws, None) == _lib.ERR_SHAPE
 
+
+def test_row_table_argument_checks(L):
+    lay = _lib.Layer(64, 128, 0, FAKE, FAKE, FAKE, None, None, 0, None)
+    sz = _lib.Sizes()
+    assert L.spectra_row_table_sizes(ctypes.byref(lay), ctypes.byref(sz)) == _lib.OK
+    assert sz.codes_bytes == 64 * 4 * 16 and sz.scales_bytes == 64 * 4 * 2 and sz.zeros_bytes == 64 * 4
+    assert sz.outlier_w_bytes == 0 and sz.bulk_idx_bytes == 0
+    lay_o = _lib.Layer(64, 128, 5, FAKE, FAKE, FAKE, FAKE, FAKE, 0, None)
+    assert L.spectra_row_table_sizes(ctypes.byref(lay_o), ctypes.byref(sz)) == _lib.OK
+    assert sz.outlier_w_bytes == 64 * 5 * 2 and sz.outlier_idx_bytes == 5 * 4
+    assert L.spectra_row_table_sizes(ctypes.byref(lay), None) == _lib.ERR_INVALID_ARG
+    out = _lib.Layer()
+    assert L.spectra_row_table_from_layer(ctypes.byref(lay), None, FAKE, FAKE, None, ctypes.byref(out),
+                                          None) == _lib.ERR_INVALID_ARG
+    assert L.spectra_row_table_from_layer(ctypes.byref(lay), FAKE + 4, FAKE, FAKE, None, ctypes.byref(out),
+                                          None) == _lib.ERR_ALIGN
+    assert L.spectra_embed_rows(None, FAKE, 1, FAKE, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.spectra_embed_rows(ctypes.byref(lay), FAKE, -1, FAKE, 0, None) == _lib.ERR_SHAPE
+    assert L.spectra_embed_rows(ctypes.byref(lay), FAKE, 0, FAKE, 0, None) == _lib.OK
+
