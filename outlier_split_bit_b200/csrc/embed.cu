@@ -154,17 +154,28 @@ __global__ void __launch_bounds__(kEmbedMaxThreads) embed_kernel(const EmbedArgs
             if (a.n_o > 0) {
                 __syncthreads();
                 const uint16_t *ov = reinterpret_cast<const uint16_t *>(a.outw) + (size_t)(ok ? id : 0) * a.n_o;
-                for (int j = threadIdx.x; j < a.n_o; j += blockDim.x) {
-                    const int col = __ldg(a.oidx + j);
-                    if (col < 0 || col >= a.k) {
-                        atomicOr(&g_embed_error, 2u);
-                        continue;
+                // eight columns per thread at a time: every load before the first store
+                for (int j0 = threadIdx.x; j0 < a.n_o; j0 += 8 * blockDim.x) {
+                    int col[8];
+                    uint32_t b[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int j = j0 + u * (int)blockDim.x;
+                        col[u] = j < a.n_o ? __ldg(a.oidx + j) : -2;
+                        b[u] = (ok && j < a.n_o) ? (uint32_t)ov[j] : 0u;
                     }
-                    const uint32_t b = ok ? (uint32_t)ov[j] : 0u;
-                    if constexpr (kBF16)
-                        reinterpret_cast<uint16_t *>(row)[col] = (uint16_t)b;
-                    else
-                        reinterpret_cast<uint32_t *>(row)[col] = b << 16;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        if (col[u] == -2) continue;  // past the last slot
+                        if (col[u] < 0 || col[u] >= a.k) {
+                            atomicOr(&g_embed_error, 2u);
+                            continue;
+                        }
+                        if constexpr (kBF16)
+                            reinterpret_cast<uint16_t *>(row)[col[u]] = (uint16_t)b[u];
+                        else
+                            reinterpret_cast<uint32_t *>(row)[col[u]] = b[u] << 16;
+                    }
                 }
             }
         } else if (a.n_o > 0) {
@@ -230,6 +241,126 @@ cudaError_t prepare(const DeviceInfo &dev) {
     return e;
 }
 
+// Row-table gather: a warp per requested row (grid stride over the rows by
+// all warps), no shared memory and no block barriers.  Lane l decodes groups
+// l, l + 32, ... (the row's records, scales and zero words are contiguous, so
+// a warp reads 512 contiguous bytes of records per round) and writes each
+// group's 32 values straight out: 64 (BF16) or 128 (FP32) contiguous bytes
+// per lane, or, for a compacted bulk, each value to its column.  After a
+// __syncwarp (which orders the warp's writes) the lanes write the outlier
+// columns' stored BF16 values over their columns.
+template <bool kBF16>
+__global__ void __launch_bounds__(256) embed_rows_warp_kernel(const EmbedArgs a) {
+    constexpr int kEsz = kBF16 ? 2 : 4;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int lane = threadIdx.x & 31;
+    const int warps = (int)(gridDim.x * blockDim.x) >> 5;
+    for (int r = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5); r < a.m; r += warps) {
+        const int id = a.ids[r];
+        const bool ok = id >= 0 && id < a.n;
+        if (!ok && lane == 0) atomicOr(&g_embed_error, 1u);
+        uint8_t *row = reinterpret_cast<uint8_t *>(a.out) + (size_t)r * a.k * kEsz;
+        // this lane's groups g = lane, lane + 32, ...: the pieces of four of
+        // them are loaded before the first is decoded
+        constexpr int kPre = 4;
+        for (int g0 = lane; g0 < a.G; g0 += 32 * kPre) {
+            uint4 recs[kPre];
+            uint16_t sbits[kPre];
+            uint32_t zwords[kPre];
+#pragma unroll
+            for (int q = 0; q < kPre; ++q) {
+                const int gq = g0 + 32 * q;
+                const bool in = ok && gq < a.G;
+                recs[q] = in ? a.codes[(size_t)id * a.G + gq] : make_uint4(0u, 0u, 0u, 0u);
+                sbits[q] = in ? a.scales[(size_t)id * a.G + gq] : (uint16_t)0;
+                zwords[q] = in ? a.zeros[(size_t)id * a.S + (gq >> 3)] : 0u;
+            }
+#pragma unroll
+            for (int q = 0; q < kPre; ++q) {
+                const int g = g0 + 32 * q;
+                if (g >= a.G) break;
+                float v[32];
+                {
+                    // zero for a bad id: its pieces were loaded as zeros
+                    const float s = __half2float(__ushort_as_half(sbits[q]));
+                    const int z = (int)((zwords[q] >> (4 * (g & 7))) & 0xFu);
+                    const uint32_t wv[4] = {recs[q].x, recs[q].y, recs[q].z, recs[q].w};
+#pragma unroll
+                    for (int w = 0; w < 4; ++w)
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            v[8 * w + j] = (float)((int)((wv[w] >> (4 * j)) & 0xFu) - z) * s;
+                }
+                if (a.bidx == nullptr) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(row + (size_t)32 * kEsz * g);
+                    if constexpr (kBF16) {
+#pragma unroll
+                        for (int qq = 0; qq < 4; ++qq) {
+                            uint32_t p[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(v[8 * qq + 2 * e]));
+                                const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(v[8 * qq + 2 * e + 1]));
+                                p[e] = lo | (hi << 16);
+                            }
+                            dst[qq] = make_uint4(p[0], p[1], p[2], p[3]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int qq = 0; qq < 8; ++qq)
+                            dst[qq] = make_uint4(__float_as_uint(v[4 * qq]), __float_as_uint(v[4 * qq + 1]),
+                                                 __float_as_uint(v[4 * qq + 2]), __float_as_uint(v[4 * qq + 3]));
+                    }
+                } else {
+                    const int4 *bc = reinterpret_cast<const int4 *>(a.bidx + 32 * g);
+#pragma unroll
+                    for (int qq = 0; qq < 8; ++qq) {
+                        const int4 c4 = __ldg(bc + qq);
+                        const int c[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            if (c[e] < 0) continue;  // padding column
+                            if (c[e] >= a.k) {
+                                atomicOr(&g_embed_error, 2u);
+                                continue;
+                            }
+                            put<kBF16>(row, c[e], v[4 * qq + e]);
+                        }
+                    }
+                }
+            }
+        }
+        if (a.n_o > 0) {
+            __syncwarp();  // the bulk's writes of this row come first
+            const uint16_t *ov = reinterpret_cast<const uint16_t *>(a.outw) + (size_t)(ok ? id : 0) * a.n_o;
+            // eight columns per lane at a time: every load before the first store
+            for (int j0 = lane; j0 < a.n_o; j0 += 8 * 32) {
+                int col[8];
+                uint32_t b[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int j = j0 + 32 * u;
+                    col[u] = j < a.n_o ? __ldg(a.oidx + j) : -2;
+                    b[u] = (ok && j < a.n_o) ? (uint32_t)ov[j] : 0u;
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    if (col[u] == -2) continue;  // past the last slot
+                    if (col[u] < 0 || col[u] >= a.k) {
+                        atomicOr(&g_embed_error, 2u);
+                        continue;
+                    }
+                    if constexpr (kBF16)
+                        reinterpret_cast<uint16_t *>(row)[col[u]] = (uint16_t)b[u];
+                    else
+                        reinterpret_cast<uint32_t *>(row)[col[u]] = b[u] << 16;
+                }
+            }
+        }
+    }
+}
+
 // RT32 -> row table: a grid-stride loop over every code record, scale, zero
 // word and outlier value of the table, each copied to its row-table place
 // (a permutation: nothing is recomputed).
@@ -289,7 +420,24 @@ spectra_status launch_embed(const spectra_layer &l, const int32_t *ids, int m, v
     const int64_t cap = (int64_t)dev.sm_count * kEmbedCtasPerSm;
     const unsigned grid = (unsigned)(m < cap ? m : cap);
     cudaError_t e;
-    if (rows) {
+    if (rows && m >= 4 * dev.sm_count) {
+        // many rows: a warp per row, 8 warps per CTA, up to 8 CTAs per SM
+        // (few rows go to a CTA per row, whose threads share a row's groups)
+        int64_t blocks = cdiv(m, 8);
+        const int64_t bcap = (int64_t)dev.sm_count * 8;
+        if (blocks > bcap) blocks = bcap;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)blocks, 1, 1);
+        cfg.blockDim = dim3(256, 1, 1);
+        cfg.stream = s;
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr.val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        e = bf16 ? cudaLaunchKernelEx(&cfg, embed_rows_warp_kernel<true>, a)
+                 : cudaLaunchKernelEx(&cfg, embed_rows_warp_kernel<false>, a);
+    } else if (rows) {
         e = bf16 ? prepare<true, true>(dev) : prepare<false, true>(dev);
         if (e != cudaSuccess) return SPECTRA_ERR_CUDA;
         e = bf16 ? launch<true, true>(a, grid, (unsigned)threads, smem, s)

@@ -89,19 +89,37 @@ def test_row_table_lm_head_full_size_sampled(frac):
     assert np.array_equal(_got_bits(out), _expected_bits(rows, torch.bfloat16))
 
 
+@pytest.mark.parametrize("compact", [False, True], ids=["masked", "compacted"])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_row_table_many_rows(compact, dtype):
+    """Enough ids for the warp-per-row gather (at least four rows per SM),
+    with repeats and the last row, bit for bit against the oracle."""
+    spec = wl.MatrixSpec("single", 3000, 1056, 16)
+    lay, wb, ref, rt = _oracle_table(spec, 3.0, compact)
+    table = sp.spectra_row_table_from_layer(lay)
+    ids = _ids(spec.n, 1500, seed=4)
+    out = sp.spectra_embed_rows(table, torch.from_numpy(ids).to(DEV), out_dtype=dtype)
+    torch.cuda.synchronize()
+    sp.spectra_device_status()
+    rows = oracle.embed_compact(ref, wb, ids) if compact else oracle.embed(ref.can, wb, ref.idx, ids)
+    assert np.array_equal(_got_bits(out), _expected_bits(rows, dtype))
+
+
 def test_row_table_bad_ids_give_zero_rows_and_status():
     spec = wl.MatrixSpec("single", 64, 256, 4)
     w, g, _ = draw(spec)
     lay = sp.pack_layer(w, g, 3.0)
     table = sp.spectra_row_table_from_layer(lay)
-    ids = torch.tensor([3, -1, 64, 10], dtype=torch.int32, device=DEV)
-    out = sp.spectra_embed_rows(table, ids, out_dtype=torch.float32)
-    torch.cuda.synchronize()
-    with pytest.raises(sp.SpectraError) as e:
-        sp.spectra_device_status()
-    assert e.value.status == _lib.ERR_INVALID_ARG
-    assert torch.count_nonzero(out[1]) == 0 and torch.count_nonzero(out[2]) == 0
-    ref = sp.spectra_embed(lay, ids[[0, 3]], out_dtype=torch.float32)
-    torch.cuda.synchronize()
-    sp.spectra_device_status()  # the layer gather of good ids raises nothing
-    assert torch.equal(out[[0, 3]], ref)
+    # few ids (a CTA per row) and many (a warp per row)
+    for reps in (1, 200):
+        ids = torch.tensor([3, -1, 64, 10] * reps, dtype=torch.int32, device=DEV)
+        out = sp.spectra_embed_rows(table, ids, out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        with pytest.raises(sp.SpectraError) as e:
+            sp.spectra_device_status()
+        assert e.value.status == _lib.ERR_INVALID_ARG
+        assert torch.count_nonzero(out[1]) == 0 and torch.count_nonzero(out[2]) == 0
+        ref = sp.spectra_embed(lay, ids[[0, 3]], out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        sp.spectra_device_status()  # the layer gather of good ids raises nothing
+        assert torch.equal(out[[0, 3]], ref)
