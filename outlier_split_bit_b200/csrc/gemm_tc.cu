@@ -7,6 +7,8 @@
 // the same product.  For a batch of 8 or more rows the product is a real
 // dense contraction, so the decoded operand goes to the tensor cores (8..16
 // rows run the 16-row variant; its surplus rows are computed and dropped).
+#include <atomic>
+
 #include "stream.cuh"
 
 namespace spectra {
@@ -356,8 +358,12 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     // this CTA's share of the units of every block it visits: a contiguous
-    // range of the block's unit list (super-groups, then outlier batches), so
-    // with cl <= U every rank of a cluster has at least one unit
+    // range of the block's unit list (super-groups, then outlier batches),
+    // the same number of units per rank (with cl <= U every rank has at
+    // least one).  Units are counted, not weighted by their groups: a
+    // super-group of eight groups and an outlier batch of two measured about
+    // the same cost per unit (the batch's gathered x is a chain of two
+    // dependent loads per column, behind a single chunk)
     const int u0 = split_at(a.U, cr, a.cl), u1 = split_at(a.U, cr + 1, a.cl);
     const int sg0 = u0, nsg = max(0, min(u1, a.S) - u0);
     const int ob0 = max(u0, a.S) - a.S;
@@ -458,7 +464,7 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
             const int t = 4 * blk + r;
             if (a.cl > 1) {
 #pragma unroll
-                for (int m = 0; m < MB; ++m) red[(32 * r + lane) * MB + m] = acc[m];
+                for (int m = 0; m < MB; ++m) red[m * 128 + 32 * r + lane] = acc[m];
             } else if (t < a.T) {
                 bool bad = false;
 #pragma unroll
@@ -592,30 +598,33 @@ __global__ void __launch_bounds__(C::WARPS * 32, 1) gemm_tc_kernel(const TcArgs 
     }
     __syncwarp();
 
-    // cluster split (one block per cluster): rank 0 adds the ranks' sums in rank order
+    // cluster split (one block per cluster): rank cr adds the ranks' sums of
+    // batch rows m = cr, cr + cl, ... in rank order and stores them
     if (a.cl > 1) {
         cg::cluster_group cluster = cg::this_cluster();
         cluster.sync();
         const int blk = blockIdx.x / a.cl;
-        if (cr == 0 && warp < 4) {
-            const int t = 4 * blk + warp;
-            float yv[MB];
+        const int t = 4 * blk + warp;
+        if (warp < 4 && t < a.T) {
+            const float *rp[8];
 #pragma unroll
-            for (int m = 0; m < MB; ++m) yv[m] = 0.f;
-            for (int rk = 0; rk < a.cl; ++rk) {
-                const float *rp = cluster.map_shared_rank(red, rk) + (32 * warp + lane) * MB;
+            for (int rk = 0; rk < 8; ++rk)
+                rp[rk] = cluster.map_shared_rank(red, rk < a.cl ? rk : 0) + 32 * warp + lane;
+            bool bad = false;
 #pragma unroll
-                for (int m = 0; m < MB; ++m) yv[m] += rp[m];
+            for (int m = 0; m < MB; ++m) {
+                if (m % a.cl != cr || m >= a.m) continue;  // CTA-uniform
+                float v[8];
+#pragma unroll
+                for (int rk = 0; rk < 8; ++rk) v[rk] = rp[rk][m * 128];
+                float yv = 0.f;
+#pragma unroll
+                for (int rk = 0; rk < 8; ++rk)
+                    if (rk < a.cl) yv += v[rk];
+                store_y(a, t, lane, m, yv);
+                bad |= !isfinite(yv);
             }
-            if (t < a.T) {
-                bool bad = false;
-#pragma unroll
-                for (int m = 0; m < MB; ++m) {
-                    store_y(a, t, lane, m, yv[m]);
-                    bad |= (m < a.m) && !isfinite(yv[m]);
-                }
-                if (bad && 32 * t + lane < a.n) atomicOr(&g_device_error, 2u);
-            }
+            if (bad && 32 * t + lane < a.n) atomicOr(&g_device_error, 2u);
         }
         cluster.sync();
     }
@@ -634,6 +643,34 @@ size_t tc_smem_bytes(int depth) {
            (size_t)(C::CW * depth + 2 * C::SETS * C::Q + 5 * C::SETS) * 8 + 16;
 }
 
+// Clusters of `cl` CTAs of gemm_tc_kernel<C> (with `smem` bytes each) the
+// device holds at once; cached per device and cluster size, 0 if unknown.
+template <typename C>
+int tc_max_clusters(int cl, size_t smem, const DeviceInfo &dev) {
+    static std::atomic<int> cache[64][9];
+    if (dev.device < 0 || dev.device >= 64 || cl < 1 || cl > 8) return 0;
+    int v = cache[dev.device][cl].load(std::memory_order_relaxed);
+    if (v > 0) return v - 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(cl * dev.sm_count), 1, 1);
+    cfg.blockDim = dim3(C::WARPS * 32, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = cl;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<C>, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return 0;
+    }
+    cache[dev.device][cl].store(n + 1, std::memory_order_relaxed);
+    return n;
+}
+
 template <typename C>
 spectra_status run_tc(const Prob &a0, const DeviceInfo &dev, cudaStream_t s) {
     static bool done[64];
@@ -642,27 +679,31 @@ spectra_status run_tc(const Prob &a0, const DeviceInfo &dev, cudaStream_t s) {
     const Geometry g = Geometry::of(a0.n, a0.k, a0.n_o);
     const int64_t nblk = cdiv(g.T, 4);
     const int units = units_of(g);
+    int depth = 2;  // two units in flight per warp
+    while (depth > 1 && tc_smem_bytes<C>(depth) > dev.smem_optin) --depth;
+    const size_t smem = tc_smem_bytes<C>(depth);
+    if (smem > dev.smem_optin) return SPECTRA_ERR_SHAPE;
+    cudaError_t e = prepare_kernel(gemm_tc_kernel<C>, done, dev);
+    if (e != cudaSuccess) return SPECTRA_ERR_CUDA;
     int cl = 1;
     int64_t grid = nblk;
     if (nblk >= dev.sm_count) {
         grid = dev.sm_count;  // persistent over the blocks
     } else {
-        // one block per cluster, the clusters filling the SMs once
+        // one block per cluster: the largest cluster size whose nblk
+        // clusters the device holds at once (a cluster lives inside one GPC,
+        // so sizes that do not divide a GPC's SMs leave some idle and would
+        // push clusters into a second wave)
         cl = (int)(dev.sm_count / nblk);
         if (cl > 8) cl = 8;
         if (cl > units) cl = units;
+        while (cl > 1 && tc_max_clusters<C>(cl, smem, dev) < nblk) --cl;
         if (cl < 1) cl = 1;
         grid = nblk * cl;
     }
     args.p.cl = cl;
     args.nblk = (int)nblk;
-    int depth = 2;  // two units in flight per warp
-    while (depth > 1 && tc_smem_bytes<C>(depth) > dev.smem_optin) --depth;
     args.depth = depth;
-    const size_t smem = tc_smem_bytes<C>(depth);
-    if (smem > dev.smem_optin) return SPECTRA_ERR_SHAPE;
-    cudaError_t e = prepare_kernel(gemm_tc_kernel<C>, done, dev);
-    if (e != cudaSuccess) return SPECTRA_ERR_CUDA;
     e = launch_kernel(gemm_tc_kernel<C>, args, (unsigned)grid, smem, C::WARPS, cl, s);
     return e == cudaSuccess ? SPECTRA_OK : SPECTRA_ERR_CUDA;
 }
