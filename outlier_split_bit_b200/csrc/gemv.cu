@@ -200,7 +200,7 @@ struct XFirst {
     uint32_t lo[8], hi[8];
 };
 
-template <int MB>
+template <int MB, bool kL2>
 __device__ __forceinline__ void stage_x_load(const Prob &a, const XRange &xr, const XIdx &xi,
                                              XFirst &f) {
     const int nth = blockDim.x;
@@ -212,10 +212,10 @@ __device__ __forceinline__ void stage_x_load(const Prob &a, const XRange &xr, co
             if (a.bidx == nullptr) {
                 const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)m * a.kx + 32 * g);
 #pragma unroll
-                for (int w = 0; w < 4; ++w) f.v0[w] = __ldcg(src + w);
+                for (int w = 0; w < 4; ++w) f.v0[w] = ld_x<kL2>(src + w);
             } else {
 #pragma unroll
-                for (int w = 0; w < 4; ++w) f.v0[w] = bulk_x8_gather(a, m, 32 * g + 8 * w);
+                for (int w = 0; w < 4; ++w) f.v0[w] = bulk_x8_gather<kL2>(a, m, 32 * g + 8 * w);
             }
         }
     }
@@ -224,18 +224,15 @@ __device__ __forceinline__ void stage_x_load(const Prob &a, const XRange &xr, co
         const int c = threadIdx.x + i * nth;
         const int m = c % MB;
         const bool mv = c < np * MB && m < a.m;
-        f.lo[i] = (mv && xi.i0[i] >= 0) ? __ldcg(a.x + (size_t)m * a.kx + xi.i0[i]) : 0u;
-        f.hi[i] = (mv && xi.i1[i] >= 0) ? __ldcg(a.x + (size_t)m * a.kx + xi.i1[i]) : 0u;
+        f.lo[i] = (mv && xi.i0[i] >= 0) ? ld_x<kL2>(a.x + (size_t)m * a.kx + xi.i0[i]) : 0u;
+        f.hi[i] = (mv && xi.i1[i] >= 0) ? ld_x<kL2>(a.x + (size_t)m * a.kx + xi.i1[i]) : 0u;
     }
 }
 
-// (x is read with ld.global.cg: it may have been written by other CTAs of
-// the same launch -- the chain kernel -- so it must not come from a stale L1
-// line; read once per CTA, it gains nothing from L1 anyway.)
 // Stage x for a unit range: bulk groups as BF16 pairs in the decoder's order
 // with their FP32 sums X_g (column order), and the BF16 pairs of the outlier
 // slots, gathered through the index list; the first round comes from `f`.
-template <int MB>
+template <int MB, bool kL2>
 __device__ void stage_x_store(const Prob &a, const Stage<MB> &st, const XRange &xr,
                               const XFirst &f) {
     const int nth = blockDim.x;
@@ -254,10 +251,10 @@ __device__ void stage_x_store(const Prob &a, const Stage<MB> &st, const XRange &
             } else if (a.bidx == nullptr) {
                 const uint4 *src = reinterpret_cast<const uint4 *>(a.x + (size_t)m * a.kx + 32 * g);
 #pragma unroll
-                for (int w = 0; w < 4; ++w) v[w] = __ldcg(src + w);
+                for (int w = 0; w < 4; ++w) v[w] = ld_x<kL2>(src + w);
             } else {
 #pragma unroll
-                for (int w = 0; w < 4; ++w) v[w] = bulk_x8_gather(a, m, 32 * g + 8 * w);
+                for (int w = 0; w < 4; ++w) v[w] = bulk_x8_gather<kL2>(a, m, 32 * g + 8 * w);
             }
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
@@ -299,20 +296,20 @@ __device__ void stage_x_store(const Prob &a, const Stage<MB> &st, const XRange &
             if (c < np * MB) {
                 const int m = c % MB;
                 const bool mv = m < a.m;
-                const uint32_t l = (i0[i] >= 0 && mv) ? __ldcg(a.x + (size_t)m * a.kx + i0[i]) : 0u;
-                const uint32_t h = (i1[i] >= 0 && mv) ? __ldcg(a.x + (size_t)m * a.kx + i1[i]) : 0u;
+                const uint32_t l = (i0[i] >= 0 && mv) ? ld_x<kL2>(a.x + (size_t)m * a.kx + i0[i]) : 0u;
+                const uint32_t h = (i1[i] >= 0 && mv) ? ld_x<kL2>(a.x + (size_t)m * a.kx + i1[i]) : 0u;
                 st.xo[c] = l | (h << 16);
             }
         }
     }
 }
 
-template <int MB>
+template <int MB, bool kL2>
 __device__ __forceinline__ void stage_x(const Prob &a, const Stage<MB> &st, const XRange &xr,
                                         const XIdx &xi) {
     XFirst f;
-    stage_x_load<MB>(a, xr, xi, f);
-    stage_x_store<MB>(a, st, xr, f);
+    stage_x_load<MB, kL2>(a, xr, xi, f);
+    stage_x_store<MB, kL2>(a, st, xr, f);
 }
 
 // ---------------------------------------------------------------- units
@@ -483,9 +480,9 @@ __global__ void __launch_bounds__(kClusterWarps * 32, MB == 1 ? 2 : 1)
     load_x_idx(a, xr, MB, xi);
     pdl_wait();
     XFirst xf;
-    stage_x_load<MB>(a, xr, xi, xf);
+    stage_x_load<MB, false>(a, xr, xi, xf);
     for (; next < nunits && next < ring.D; ++next) ring_issue(ring, a, t, unit_id(a, slc, next), lane);
-    stage_x_store<MB>(a, st, xr, xf);
+    stage_x_store<MB, false>(a, st, xr, xf);
     __syncthreads();
 
     float yacc[MB];
@@ -629,12 +626,12 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1)
     pdl_wait();
     if (it0 < it1) {
         XFirst xf;
-        stage_x_load<MB>(args.probs[p], xr, xi, xf);
+        stage_x_load<MB, false>(args.probs[p], xr, xi, xf);
         for (; d < ring.D && ic.item < it1; ++d) {
             cursor_issue(args, ring, ic, lane);
             cursor_next(args, it1, warp, ic);
         }
-        stage_x_store<MB>(args.probs[p], st, xr, xf);
+        stage_x_store<MB, false>(args.probs[p], st, xr, xf);
         __syncthreads();
         cur_p = p;
     }
@@ -649,7 +646,7 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1)
             xr = x_range(a, 0, 1, 1);
             XIdx xi;
             load_x_idx(a, xr, MB, xi);
-            stage_x<MB>(a, st, xr, xi);
+            stage_x<MB, false>(a, st, xr, xi);
             __syncthreads();
             cur_p = p;
         }
@@ -842,7 +839,7 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1) gemv_chain_kernel(const
             __syncthreads();
         }
         if (mine) {
-            stage_x<1>(a, st, xr, xi);
+            stage_x<1, true>(a, st, xr, xi);
             __syncthreads();
             for (int item = blockIdx.x; item < a.items; item += gridDim.x) {
                 const ChainWork cw = chain_work(a, item, warp);

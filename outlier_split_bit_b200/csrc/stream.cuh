@@ -152,9 +152,21 @@ __device__ __forceinline__ uint32_t code_pair(uint32_t w) {
     return ((w >> (4 * sh)) & 0x000F000Fu) | 0x43004300u;
 }
 
+// A load of x.  kL2 = false: through L1 (ld.global.nc), for kernels in which
+// no CTA writes x (an earlier launch's output is ordered by the programmatic
+// dependency wait).  kL2 = true: at L2 (ld.global.cg), for the chain kernel,
+// where x may be the output of an earlier matvec of the same launch, so a
+// line cached in L1 before that write would be stale.
+template <bool kL2, typename T>
+__device__ __forceinline__ T ld_x(const T *p) {
+    if constexpr (kL2) return __ldcg(p);
+    else return __ldg(p);
+}
+
 // x of 8 consecutive columns c0..c0+7 of a compacted bulk for batch row m,
 // as 4 BF16 pairs in column order: gathered through the bulk column list,
 // padding (and any entry outside [0, kx)) read as +0.  c0 is a multiple of 8.
+template <bool kL2 = false>
 __device__ __forceinline__ uint4 bulk_x8_gather(const Prob &a, int m, int c0) {
     const uint16_t *xr = a.x + (size_t)m * a.kx;
     const int4 b0 = __ldg(reinterpret_cast<const int4 *>(a.bidx + c0));
@@ -162,7 +174,7 @@ __device__ __forceinline__ uint4 bulk_x8_gather(const Prob &a, int m, int c0) {
     const int c[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
     uint32_t h[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) h[e] = ((unsigned)c[e] < (unsigned)a.kx) ? (uint32_t)__ldcg(xr + c[e]) : 0u;
+    for (int e = 0; e < 8; ++e) h[e] = ((unsigned)c[e] < (unsigned)a.kx) ? (uint32_t)ld_x<kL2>(xr + c[e]) : 0u;
     return make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16),
                       h[6] | (h[7] << 16));
 }
