@@ -9,10 +9,13 @@ matvec per matrix with its own BF16 activation vector (196 matvecs, 1.31 G
 weights, 0.76 GB of packed bulk plus the BF16 outlier columns).  The
 activations of the synthetic stream are independent inputs, so the step is
 ONE spectra_gemv_batched launch that streams all 196 matrices in order
-(captured in a CUDA graph and replayed).  The same stream as a dependent
-chain -- 196 spectra_gemv launches where each may consume the previous
-output (programmatic dependent launch) -- is timed too and reported under
-"rows".  The packed weights exceed the 126 MB L2, so every step streams them
+(captured in a CUDA graph and replayed).  The same stream with dependencies
+is timed too and reported under "rows": as a chain where each matvec may
+consume the previous output, once as 196 spectra_gemv launches
+(programmatic dependent launch) and once as one spectra_gemv_chain launch;
+and in a decoder layer's stages (q, k, v read one input, so do gate and
+up: four stages per layer), once as 112 grouped launches and once as one
+spectra_gemv_chain launch with stages.  The packed weights exceed the 126 MB L2, so every step streams them
 from HBM.  The per-matrix and batch rows time back-to-back launches cycling
 over copies of the matrix that together exceed twice the L2 (each launch
 reads DRAM, launch latency overlaps as in a decode stream); the single-launch
@@ -29,9 +32,9 @@ replica of the stream: the problems are independent, there is no data-path
 collective, and the value is the bytes of all ranks over the slowest rank's
 time (weak scaling).
 
---impl reference times the CPU oracle (oracle/, IEEE double, one core) on a
-bounded sample of the same workload: whole 32-row tiles of each matrix,
-unpacked from the oracle's own packed layout and multiplied.
+--impl reference times the CPU oracle (oracle/, IEEE double) on every host
+core: a step is one pass over the seven matrices of layer 0, unpacked from
+the oracle's own packed layout and multiplied.
 """
 from __future__ import annotations
 
@@ -195,6 +198,16 @@ class Stream:
 
         self.batch = sp.BatchViews([it[1] for it in self.items], [it[2] for it in self.items],
                                    [it[3] for it in self.items])
+        # a decoder layer's dataflow: q, k and v read one input, gate and up
+        # read one input; o and down stand alone (four stages per layer)
+        stage_of = {"q": 0, "k": 0, "v": 0, "o": 1, "gate": 2, "up": 2, "down": 3}
+        self.stages = [4 * (i // len(wl.LAYER_1P5B)) + stage_of[it[0].name]
+                       for i, it in enumerate(self.items)]
+        self.stage_batches = []
+        for s in sorted(set(self.stages)):
+            sel = [it for it, st in zip(self.items, self.stages) if st == s]
+            self.stage_batches.append(sp.BatchViews([it[1] for it in sel], [it[2] for it in sel],
+                                                    [it[3] for it in sel]))
 
     def run(self, stream, mode):
         if mode == "batched":
@@ -204,6 +217,15 @@ class Stream:
             # one launch; every matrix waits for all earlier ones (dependent)
             self.sp.spectra_gemv_chain(views=self.batch, stream=stream)
             return 1
+        if mode == "stages_chain":
+            # one launch; every matrix waits for the earlier stages only
+            self.sp.spectra_gemv_chain(views=self.batch, stages=self.stages, stream=stream)
+            return 1
+        if mode == "stages_launches":
+            # one grouped launch per stage, in order (PDL)
+            for v in self.stage_batches:
+                self.sp.spectra_gemv_batched(views=v, stream=stream)
+            return len(self.stage_batches)
         # "launches": one spectra_gemv launch per matrix, in order (PDL)
         for spec, lay, x, y, view in self.items:
             self.sp.spectra_gemv(lay, x, y, view=view, stream=stream)
@@ -843,13 +865,15 @@ def run_ours(args):
     # and as 196 spectra_gemv launches in a graph (programmatic dependent launch)
     extra = {}
     for mode, key in (("chain", "decode_stream_dependent_chain"),
-                      ("launches", "decode_stream_dependent_launches")):
+                      ("launches", "decode_stream_dependent_launches"),
+                      ("stages_chain", "decode_stream_stages_chain"),
+                      ("stages_launches", "decode_stream_stages_launches")):
         chain_graph, chain_launches = st.capture(stream, mode)
         for _ in range(args.warmup):
             chain_graph.replay()
         stream.synchronize()
         barrier()
-        chain_steps = max(1, args.steps // 2) if mode == "launches" else args.steps
+        chain_steps = max(1, args.steps // 2) if mode.endswith("launches") else args.steps
         with torch.cuda.stream(stream):
             c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             c0.record(stream)
@@ -969,6 +993,11 @@ def summary_of(line, extra, cpu):
     cl = extra.get("decode_stream_dependent_launches")
     if cl:
         out["chain_196_launches"] = {"us": cl["us_per_step"], "frac": r(cl["frac"])}
+    for key, name in (("decode_stream_stages_chain", "stages_chain"),
+                      ("decode_stream_stages_launches", "stages_112_launches")):
+        sc = extra.get(key)
+        if sc:
+            out[name] = {"us": sc["us_per_step"], "frac": r(sc["frac"])}
     big = {}
     for row in extra.get("per_matrix_1p5b", []):
         if row["bytes"] >= 8_000_000:

@@ -357,6 +357,24 @@ SPECTRA_API spectra_status spectra_gemv_chain(const spectra_layer *layers,
                                               void *stream);
 
 /*
+ * spectra_gemv_chain with the matvecs grouped into stages, as a decoder
+ * layer's dataflow groups them (q, k and v read the same input; so do gate
+ * and up).  stage: HOST array [count], nondecreasing (the call reads it
+ * during the call only); matvec i reads x[i] only after every matvec of the
+ * stages before stage[i] has stored y, and the matvecs of one stage run with
+ * no wait between them.  So x[i] may be (or overlap) the output of any
+ * matvec of an earlier stage, never of its own stage, and no y[i] may
+ * overlap another y[j] or an x[j] of the same or an earlier stage.  With
+ * stage[i] = i it is spectra_gemv_chain.  Workspace, waits, limits and
+ * errors as spectra_gemv_chain; a decreasing stage array is INVALID_ARG.
+ */
+SPECTRA_API spectra_status spectra_gemv_chain_staged(const spectra_layer *layers,
+                                                     const uint16_t *const *x, void *const *y,
+                                                     int32_t count, spectra_dtype y_dtype,
+                                                     const int32_t *stage, void *workspace,
+                                                     size_t workspace_bytes, void *stream);
+
+/*
  * Embedding-row gather over a packed table (abstract: SpectraFusedEmbedding,
  * dequantisation of vocabulary embeddings on demand; highlight 5: vocabulary
  * tables stored in the 4-bit Group-32 format, rows gathered and dequantised

@@ -348,12 +348,15 @@ def spectra_gemv_batched(layers=None, xs=None, ys=None, *, views: BatchViews | N
 
 
 def spectra_gemv_chain(layers=None, xs=None, ys=None, *, views: BatchViews | None = None,
-                       workspace: torch.Tensor | None = None, stream=None) -> BatchViews:
+                       stages=None, workspace: torch.Tensor | None = None,
+                       stream=None) -> BatchViews:
     """Dependent batch-1 matvecs ys[i] = W_i xs[i], i in order, in one launch;
-    xs[i] may be an earlier ys[j].  `workspace` (device, >=
+    xs[i] may be an earlier ys[j].  With `stages` (a nondecreasing sequence of
+    ints, one per matvec) matvec i waits only for the matvecs of earlier
+    stages (spectra_gemv_chain_staged).  `workspace` (device, >=
     spectra_gemv_chain_workspace_size(layers, count) bytes) holds the launch's
-    counters and partial sums; one is allocated and kept with the views when
-    none is given."""
+    completion counter; one is allocated and kept with the views when none is
+    given."""
     v = views if views is not None else BatchViews(layers, xs, ys)
     if workspace is None:
         workspace = getattr(v, "_chain_ws", None)
@@ -364,9 +367,17 @@ def spectra_gemv_chain(layers=None, xs=None, ys=None, *, views: BatchViews | Non
             raise SpectraError(_lib.ERR_INVALID_ARG, "spectra_gemv_chain_workspace_size")
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
         v._chain_ws = workspace
-    _check(_L.spectra_gemv_chain(v.layers, v.xs, v.ys, v.count, v.y_dtype, workspace.data_ptr(),
-                                 workspace.numel() * workspace.element_size(), _stream(stream)),
-           "spectra_gemv_chain")
+    wsb = workspace.numel() * workspace.element_size()
+    if stages is None:
+        _check(_L.spectra_gemv_chain(v.layers, v.xs, v.ys, v.count, v.y_dtype, workspace.data_ptr(),
+                                     wsb, _stream(stream)), "spectra_gemv_chain")
+    else:
+        st = (ctypes.c_int32 * len(stages))(*[int(s) for s in stages])
+        if len(stages) != v.count:
+            raise SpectraError(_lib.ERR_INVALID_ARG, "spectra_gemv_chain_staged: one stage per matvec")
+        _check(_L.spectra_gemv_chain_staged(v.layers, v.xs, v.ys, v.count, v.y_dtype, st,
+                                            workspace.data_ptr(), wsb, _stream(stream)),
+               "spectra_gemv_chain_staged")
     return v
 
 

@@ -78,6 +78,7 @@ SIGNATURES = {
     "spectra_gemv_batched": (ctypes.c_int, [LP, P, P, i32, ctypes.c_int, P]),
     "spectra_gemv_chain_workspace_size": (sz, [LP, i32]),
     "spectra_gemv_chain": (ctypes.c_int, [LP, P, P, i32, ctypes.c_int, P, sz, P]),
+    "spectra_gemv_chain_staged": (ctypes.c_int, [LP, P, P, i32, ctypes.c_int, P, P, sz, P]),
     "spectra_device_status": (ctypes.c_int, [P]),
     "spectra_selftest_wait": (ctypes.c_int, [i32, P]),
     "spectra_embed": (ctypes.c_int, [LP, P, i32, P, ctypes.c_int, P]),

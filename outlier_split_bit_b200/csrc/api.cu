@@ -340,9 +340,11 @@ size_t spectra_gemv_chain_workspace_size(const spectra_layer *layers, int32_t co
     return gemv_chain_workspace_bytes();
 }
 
-spectra_status spectra_gemv_chain(const spectra_layer *layers, const uint16_t *const *x,
-                                  void *const *y, int32_t count, spectra_dtype y_dtype,
-                                  void *workspace, size_t workspace_bytes, void *stream) {
+namespace {
+// Arguments of the dependent-sequence entries (host-side checks only).
+spectra_status check_chain(const spectra_layer *layers, const uint16_t *const *x, void *const *y,
+                           int32_t count, spectra_dtype y_dtype, void *workspace,
+                           size_t workspace_bytes) {
     if (!layers || !x || !y || !workspace) return SPECTRA_ERR_INVALID_ARG;
     if (count < 1 || count > SPECTRA_MAX_BATCH) return SPECTRA_ERR_SHAPE;
     if (y_dtype != SPECTRA_F32 && y_dtype != SPECTRA_BF16) return SPECTRA_ERR_INVALID_ARG;
@@ -356,10 +358,35 @@ spectra_status spectra_gemv_chain(const spectra_layer *layers, const uint16_t *c
         if (y_dtype == SPECTRA_F32 ? !aligned4(y[i]) : ((uintptr_t)y[i] & 1u))
             return SPECTRA_ERR_ALIGN;
     }
-    DeviceInfo dev;
-    spectra_status st = current_device(&dev);
+    return SPECTRA_OK;
+}
+}  // namespace
+
+spectra_status spectra_gemv_chain(const spectra_layer *layers, const uint16_t *const *x,
+                                  void *const *y, int32_t count, spectra_dtype y_dtype,
+                                  void *workspace, size_t workspace_bytes, void *stream) {
+    spectra_status st = check_chain(layers, x, y, count, y_dtype, workspace, workspace_bytes);
     if (st != SPECTRA_OK) return st;
-    return launch_gemv_chain(layers, x, y, count, (int)y_dtype, workspace, workspace_bytes,
+    DeviceInfo dev;
+    st = current_device(&dev);
+    if (st != SPECTRA_OK) return st;
+    return launch_gemv_chain(layers, x, y, count, (int)y_dtype, nullptr, workspace, workspace_bytes,
+                             (cudaStream_t)stream, dev);
+}
+
+spectra_status spectra_gemv_chain_staged(const spectra_layer *layers, const uint16_t *const *x,
+                                         void *const *y, int32_t count, spectra_dtype y_dtype,
+                                         const int32_t *stage, void *workspace,
+                                         size_t workspace_bytes, void *stream) {
+    spectra_status st = check_chain(layers, x, y, count, y_dtype, workspace, workspace_bytes);
+    if (st != SPECTRA_OK) return st;
+    if (!stage) return SPECTRA_ERR_INVALID_ARG;
+    for (int32_t i = 1; i < count; ++i)
+        if (stage[i] < stage[i - 1]) return SPECTRA_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    st = current_device(&dev);
+    if (st != SPECTRA_OK) return st;
+    return launch_gemv_chain(layers, x, y, count, (int)y_dtype, stage, workspace, workspace_bytes,
                              (cudaStream_t)stream, dev);
 }
 

@@ -700,8 +700,10 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1)
 // before it wrote (x of one layer = y of the last): one launch of one 16-warp
 // CTA per SM, all resident at once.  Every problem is spread over all CTAs
 // (CTA c takes its items c, c + ncta, ...), and before a CTA reads x of
-// problem i it waits until every CTA has counted problem i - 1 as done on a
-// global counter (release / acquire at GPU scope).  The weight rings keep
+// problem i it waits until every CTA has counted the problems before i's
+// stage as done on a global counter (release / acquire at GPU scope); the
+// problems of one stage (q, k and v of a layer share their input) run
+// without a wait between them.  The weight rings keep
 // prefetching across problems while a CTA waits, so the weight stream
 // overlaps the wait.  An item is tpc tiles x ppc slices (tpc x ppc = 16
 // warps); a tile's units are cut into contiguous slices, so the busiest warp
@@ -712,6 +714,9 @@ struct ChainArgs {
     Smem sm;
     int count;                // problems
     unsigned int *done;       // completion counter (zeroed before the launch)
+    // problems that must be complete before problem p reads x: the index of
+    // the first problem of p's stage (p itself when every problem is a stage)
+    uint16_t need[kMaxBatch];
     Prob probs[kMaxBatch];    // each with its own item shape (ppc x tpc = 16 warps)
 };
 static_assert(sizeof(ChainArgs) <= 32760, "kernel parameter space");
@@ -820,6 +825,7 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1) gemv_chain_kernel(const
     // copies (lane 1 of warp 0)
     constexpr int kSignal = 1;
     int rbuf = 0;
+    int waited = 0;  // problems known complete
     for (int p = 0; p < args.count; ++p) {
         const Prob &a = args.probs[p];
         const bool mine = (int)blockIdx.x < a.items;
@@ -828,15 +834,18 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1) gemv_chain_kernel(const
         const XRange xr = x_range(a, 0, 1, 1);
         XIdx xi;
         if (mine) load_x_idx(a, xr, 1, xi);
-        // every CTA has finished problem p - 1 (its y may be this x); the
-        // acquire, then the CTA barrier, order the x loads after it
-        if (p > 0) {
+        // every CTA has finished the problems before p's stage (their y may
+        // be this x); the acquire, then the CTA barrier, order the x loads
+        // after it
+        const int need = args.need[p];
+        if (need > waited) {
             if (threadIdx.x == kSignal && !s_abort &&
-                !counter_wait(args.done, (unsigned int)p * gridDim.x)) {
+                !counter_wait(args.done, (unsigned int)need * gridDim.x)) {
                 s_abort = 1;
                 atomicOr(&g_device_error, 1u);
             }
             __syncthreads();
+            waited = need;
         }
         if (mine) {
             stage_x<1, true>(a, st, xr, xi);
@@ -1321,14 +1330,16 @@ spectra_status launch_gemv_batched(const spectra_layer *layers, const uint16_t *
 }
 
 spectra_status launch_gemv_chain(const spectra_layer *layers, const uint16_t *const *xs,
-                                 void *const *ys, int count, int ytype, void *ws, size_t ws_bytes,
-                                 cudaStream_t s, const DeviceInfo &dev) {
+                                 void *const *ys, int count, int ytype, const int32_t *stage,
+                                 void *ws, size_t ws_bytes, cudaStream_t s, const DeviceInfo &dev) {
     static std::mutex mu;
     static ChainArgs args;  // large: kept off the stack, guarded by the mutex
     std::lock_guard<std::mutex> lock(mu);
     for (int i = 0; i < count; ++i) {
         const Geometry g = Geometry::of(layers[i].n, bulk_cols(layers[i]), layers[i].n_outliers);
         fill_prob(args.probs[i], layers[i], g, xs[i], 1, ys[i], ytype);
+        // no stages: every problem waits for all earlier ones
+        args.need[i] = (uint16_t)((stage && i > 0 && stage[i] == stage[i - 1]) ? args.need[i - 1] : i);
     }
     return run_chain(args, count, ws, ws_bytes, dev, s);
 }

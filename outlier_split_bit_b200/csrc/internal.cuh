@@ -98,11 +98,12 @@ spectra_status launch_gemv_batched(const spectra_layer *layers, const uint16_t *
                                    const DeviceInfo &dev);
 
 // A dependent sequence of batch-1 matvecs in one launch (count <= kMaxBatch):
-// problem i reads x only after problems 0..i-1 have stored y.  `ws` holds the
-// launch's completion counter (zeroed by the call).
+// problem i reads x only after every problem of the earlier stages has stored
+// y (stage == nullptr: every problem is its own stage, so after 0..i-1).
+// `ws` holds the launch's completion counter (zeroed by the call).
 spectra_status launch_gemv_chain(const spectra_layer *layers, const uint16_t *const *xs,
-                                 void *const *ys, int count, int ytype, void *ws, size_t ws_bytes,
-                                 cudaStream_t s, const DeviceInfo &dev);
+                                 void *const *ys, int count, int ytype, const int32_t *stage,
+                                 void *ws, size_t ws_bytes, cudaStream_t s, const DeviceInfo &dev);
 size_t gemv_chain_workspace_bytes();
 
 // ---- tensor-core matmul (gemm_tc.cu) ----

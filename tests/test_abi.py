@@ -261,6 +261,23 @@ def test_chain_argument_checks(L):
     assert L.spectra_gemv_chain(bad, xs, ys, 1, 0, FAKE, ws, None) == _lib.ERR_SHAPE
 
 
+def test_staged_chain_argument_checks(L):
+    lay = _lib.Layer(64, 128, 0, FAKE, FAKE, FAKE, None, None, 0, None)
+    layers = (_lib.Layer * 3)(lay, lay, lay)
+    xs = (ctypes.c_void_p * 3)(FAKE, FAKE, FAKE)
+    ys = (ctypes.c_void_p * 3)(FAKE, FAKE, FAKE)
+    ws = 1 << 20
+    good = (ctypes.c_int32 * 3)(0, 0, 1)
+    # the same checks as spectra_gemv_chain, then the stage array: present
+    # and nondecreasing; all before any CUDA call
+    assert L.spectra_gemv_chain_staged(layers, xs, ys, 3, 0, good, None, ws, None) == _lib.ERR_INVALID_ARG
+    assert L.spectra_gemv_chain_staged(layers, xs, ys, 3, 0, good, FAKE, 15, None) == _lib.ERR_BUFFER_TOO_SMALL
+    assert L.spectra_gemv_chain_staged(layers, xs, ys, 0, 0, good, FAKE, ws, None) == _lib.ERR_SHAPE
+    assert L.spectra_gemv_chain_staged(layers, xs, ys, 3, 0, None, FAKE, ws, None) == _lib.ERR_INVALID_ARG
+    down = (ctypes.c_int32 * 3)(0, 1, 0)
+    assert L.spectra_gemv_chain_staged(layers, xs, ys, 3, 0, down, FAKE, ws, None) == _lib.ERR_INVALID_ARG
+
+
 def test_row_table_argument_checks(L):
     lay = _lib.Layer(64, 128, 0, FAKE, FAKE, FAKE, None, None, 0, None)
     sz = _lib.Sizes()

@@ -105,6 +105,74 @@ def test_chain_graph_capture_and_replay():
     sp.spectra_device_status()
 
 
+def _decoder_stages(tau, layers=2, seed=13):
+    """Two 1.5B-class decoder layers as the staged chain runs them: q, k, v
+    read one input (stage 0), o reads q's output (stage 1), gate and up read
+    o's output (stage 2), down reads gate's output (stage 3); the next layer's
+    q, k, v read down's output.  Outputs are BF16, every buffer distinct."""
+    specs = {s.name: s for s in wl.LAYER_1P5B}
+    x0 = wl.activations(specs["q"].k, 1, seed=7, device=DEV)[0]
+    mats, xs, ys, stage = [], [], [], []
+    cur = x0
+    for layer in range(layers):
+        def add(name, x, st):
+            spec = specs[name]
+            w, g, _ = draw(spec, seed=seed, layer=layer)
+            mats.append((spec, w, g, sp.pack_layer(w, g, tau)))
+            y = torch.full((spec.n,), float("nan"), dtype=torch.bfloat16, device=DEV)
+            xs.append(x)
+            ys.append(y)
+            stage.append(st)
+            return y
+        base = 4 * layer
+        yq = add("q", cur, base)
+        add("k", cur, base)
+        add("v", cur, base)
+        yo = add("o", yq, base + 1)
+        yg = add("gate", yo, base + 2)
+        add("up", yo, base + 2)
+        cur = add("down", yg, base + 3)
+    return mats, xs, ys, stage
+
+
+@pytest.mark.parametrize("tau", [3.0, 6.0])
+def test_staged_chain_against_oracle(tau):
+    """Each matvec reads the output of an earlier stage, never of its own;
+    every output against the oracle given the x it read."""
+    mats, xs, ys, stage = _decoder_stages(tau)
+    views = sp.spectra_gemv_chain([m[3] for m in mats], xs, ys, stages=stage)
+    torch.cuda.synchronize()
+    sp.spectra_device_status()
+    for (spec, w, g, lay), x_in, y in zip(mats, xs, ys):
+        assert torch.isfinite(y.float()).all(), spec.name
+        wb = wl.bits(w)
+        ref = oracle.pack(wb, np_gain(g), tau)
+        y_ref, bound = oracle.gemm(ref.can, wb, ref.idx, wl.bits(x_in))
+        check_gemv(y, y_ref[0], bound[0], bf16=True)
+    # a replay repeats every output bit for bit
+    first = [y.clone() for y in ys]
+    for y in ys:
+        y.fill_(float("nan"))
+    sp.spectra_gemv_chain(views=views, stages=stage)
+    torch.cuda.synchronize()
+    for a, b in zip(first, ys):
+        assert torch.equal(a, b)
+
+
+def test_staged_chain_with_one_matvec_per_stage_is_the_chain():
+    mats, xs, ys, _ = _decoder_stages(3.0, layers=1)
+    layers = [m[3] for m in mats]
+    sp.spectra_gemv_chain(layers, xs, ys)
+    torch.cuda.synchronize()
+    plain = [y.clone() for y in ys]
+    for y in ys:
+        y.fill_(float("nan"))
+    sp.spectra_gemv_chain(layers, xs, ys, stages=list(range(len(layers))))
+    torch.cuda.synchronize()
+    for a, b in zip(plain, ys):
+        assert torch.equal(a, b)
+
+
 def test_counter_wait_runs_out_and_reports_internal():
     sp.spectra_device_status()
     t0 = time.perf_counter()
