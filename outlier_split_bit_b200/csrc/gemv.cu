@@ -717,6 +717,9 @@ struct ChainArgs {
     // problems that must be complete before problem p reads x: the index of
     // the first problem of p's stage (p itself when every problem is a stage)
     uint16_t need[kMaxBatch];
+    // items of the earlier problems of p's stage: a stage's items are dealt
+    // over the CTAs as one list, so its problems run on different CTAs
+    int base[kMaxBatch];
     Prob probs[kMaxBatch];    // each with its own item shape (ppc x tpc = 16 warps)
 };
 static_assert(sizeof(ChainArgs) <= 32760, "kernel parameter space");
@@ -772,6 +775,14 @@ __device__ __forceinline__ ChainWork chain_work(const Prob &a, int item, int war
     return w;
 }
 
+// This CTA's first item of problem p (its later ones follow every gridDim.x):
+// item i of p is item base[p] + i of its stage's list, dealt round robin.
+__device__ __forceinline__ int chain_first(const ChainArgs &args, int p) {
+    const int n = (int)gridDim.x;
+    const int i0 = ((int)blockIdx.x - args.base[p]) % n;
+    return i0 < 0 ? i0 + n : i0;
+}
+
 // One warp's position in the chain's unit sequence.
 struct ChainCursor {
     int p, item, u;
@@ -790,7 +801,7 @@ __device__ __forceinline__ void chain_load(const ChainArgs &args, int warp, Chai
             c.item += gridDim.x;
         } else {
             ++c.p;
-            c.item = blockIdx.x;
+            if (c.p < args.count) c.item = chain_first(args, c.p);
         }
     }
 }
@@ -813,7 +824,7 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1) gemv_chain_kernel(const
     // weights are constant: the ring is filled before any wait
     ChainCursor ic;
     ic.p = 0;
-    ic.item = blockIdx.x;
+    ic.item = chain_first(args, 0);
     chain_load(args, warp, ic);
     for (int d = 0; d < ring.D && ic.p < args.count; ++d) {
         const Prob &ap = args.probs[ic.p];
@@ -828,7 +839,8 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1) gemv_chain_kernel(const
     int waited = 0;  // problems known complete
     for (int p = 0; p < args.count; ++p) {
         const Prob &a = args.probs[p];
-        const bool mine = (int)blockIdx.x < a.items;
+        const int first = chain_first(args, p);
+        const bool mine = first < a.items;
         // the outlier column indices are part of the packed layer: load them
         // before the wait
         const XRange xr = x_range(a, 0, 1, 1);
@@ -850,7 +862,7 @@ __global__ void __launch_bounds__(kPersistWarps * 32, 1) gemv_chain_kernel(const
         if (mine) {
             stage_x<1, true>(a, st, xr, xi);
             __syncthreads();
-            for (int item = blockIdx.x; item < a.items; item += gridDim.x) {
+            for (int item = first; item < a.items; item += gridDim.x) {
                 const ChainWork cw = chain_work(a, item, warp);
                 const bool active = cw.t < a.T;
                 const int nunits = active ? cw.slc.nsg + cw.slc.nob : 0;
@@ -1174,6 +1186,7 @@ spectra_status run_chain(ChainArgs &args, int count, void *ws, size_t ws_bytes, 
         chain_shape(g, ncta, &a.ppc, &a.tpc);
         a.lgp = 0;
         a.items = (int)cdiv(a.T, a.tpc);
+        args.base[i] = (i > 0 && args.need[i] == args.need[i - 1]) ? args.base[i - 1] + args.probs[i - 1].items : 0;
         sm.xg = max(sm.xg, 8 * a.S);
         sm.xo = max(sm.xo, 8 * kOB * (a.U - a.S));
     }
