@@ -312,7 +312,8 @@ SPECTRA_API spectra_status spectra_gemm_small(const spectra_layer *layer, const 
  * y[j].  This is the decode-step weight stream when the inputs of the
  * matrices are all available (e.g. q/k/v of one layer sharing x, or the
  * stream of a whole step whose activations are given); CTAs are issued in
- * problem order, so the weights are streamed in that order.  The host arrays
+ * problem order, so the weights are streamed in that order.  With count = 1
+ * it runs exactly as spectra_gemv.  The host arrays
  * are read during the call only.  Asynchronous, allocates nothing,
  * graph-capturable, programmatic dependent launch as spectra_gemv.
  * Errors: INVALID_ARG, SHAPE, ALIGN, UNSUPPORTED, CUDA.

@@ -1339,6 +1339,9 @@ spectra_status launch_gemv_batched(const spectra_layer *layers, const uint16_t *
         const Geometry g = Geometry::of(layers[i].n, bulk_cols(layers[i]), layers[i].n_outliers);
         fill_prob(args.probs[i], layers[i], g, xs[i], 1, ys[i], ytype);
     }
+    // one matrix: spectra_gemv's choice of kernel (the cluster kernel unless
+    // the matrix is large)
+    if (count == 1) return run_one<1>(args.probs[0], dev, s);
     return run_persistent<1>(args, count, dev, s);
 }
 

@@ -340,6 +340,21 @@ def test_batched_against_oracle(spec):
         check_gemv(y[r], y_ref[r], bound[r])
 
 
+@pytest.mark.parametrize("spec", [wl.LAYER_1P5B[0], wl.LAYER_1P5B[4]], ids=["q", "gate"])
+def test_batched_single_matrix_is_spectra_gemv(spec):
+    """A grouped launch of one matrix runs spectra_gemv's path: identical
+    bits, and within the tolerance of the oracle."""
+    w, g, x, idx, kappa, lay, wb, ref = _full_pack(spec, 3.0, True)
+    y1 = torch.full((spec.n,), float("nan"), device=DEV)
+    yb = torch.full((spec.n,), float("nan"), device=DEV)
+    sp.spectra_gemv(lay, x[0], y1)
+    sp.spectra_gemv_batched([lay], [x[0]], [yb])
+    torch.cuda.synchronize()
+    assert torch.equal(y1, yb)
+    y_ref, bound = oracle.gemm(ref.can, wb, ref.idx, wl.bits(x))
+    check_gemv(yb, y_ref[0], bound[0])
+
+
 def test_device_status_clear_after_all_launches():
     """No bounded wait in any matvec above gave up."""
     sp.spectra_device_status()
