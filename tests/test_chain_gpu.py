@@ -9,6 +9,9 @@ satisfy |y - y_ref| <= 2e-3 * sum|w_hat x| + 1e-5 against the oracle given
 the x it actually read (a BF16 output adds its own rounding), every stage
 must have read its predecessor's finished output, and the counter's bounded
 wait must give up (reported, no fault) when its target is never reached.
+spectra_gemv_chain_staged groups the matvecs as a decoder layer's dataflow
+does (q, k, v share an input; so do gate and up): a matvec reads the output
+of an earlier stage only.
 """
 import time
 
@@ -157,6 +160,25 @@ def test_staged_chain_against_oracle(tau):
     torch.cuda.synchronize()
     for a, b in zip(first, ys):
         assert torch.equal(a, b)
+
+
+def test_staged_chain_with_one_stage_is_independent_matvecs():
+    """One stage: no waits at all, the matvecs independent as in a grouped
+    launch; every output against the oracle."""
+    layers, xs, ys, refs = [], [], [], []
+    for spec in wl.LAYER_1P5B:
+        w, g, x = draw(spec, seed=9, layer=1)
+        layers.append(sp.pack_layer(w, g, 3.0))
+        xs.append(x[0])
+        ys.append(torch.full((spec.n,), float("nan"), device=DEV))
+        refs.append((wl.bits(w), np_gain(g), wl.bits(x)))
+    sp.spectra_gemv_chain(layers, xs, ys, stages=[0] * len(layers))
+    torch.cuda.synchronize()
+    sp.spectra_device_status()
+    for y, (wb, gn, xb) in zip(ys, refs):
+        ref = oracle.pack(wb, gn, 3.0)
+        y_ref, bound = oracle.gemm(ref.can, wb, ref.idx, xb)
+        check_gemv(y, y_ref[0], bound[0])
 
 
 def test_staged_chain_with_one_matvec_per_stage_is_the_chain():
