@@ -84,6 +84,9 @@ def test_summary_is_last_and_short():
         "decode_stream_tau6": {"us_per_step": 197.31, "frac": 0.6212},
         "decode_stream_dependent_chain": {"us_per_step": 548.22, "frac": 0.6212, "us_per_launch": 548.22},
         "decode_stream_dependent_launches": {"us_per_step": 1148.22, "frac": 0.2712, "us_per_launch": 5.858},
+        "decode_stream_stages_chain": {"us_per_step": 1250.24, "frac": 0.2479, "us_per_launch": 1250.24},
+        "decode_stream_stages_launches": {"us_per_step": 1106.35, "frac": 0.2801, "us_per_launch": 9.878},
+        "embed_rows_row_table_131072x3072_bf16": [{"frac_single_flushed": 0.224}],
         "per_matrix_1p5b": per, "batch_sweep_4b": sweep,
         "lm_head_131072x3072": [{"frac_t_columns": f, "frac": 0.801} for f in wl.LM_HEAD_FRACTIONS],
         "lm_head_batch_131072x3072": [{"m": m, "frac": 0.371} for m in (1, 16, 32)],
@@ -101,4 +104,5 @@ def test_summary_is_last_and_short():
     assert s["tc_frac"]["4b_gate_m16"] == 0.123 and s["tc_frac"]["lm_head_m32"] == 0.371
     assert s["chain"]["frac"] == 0.621 and s["chain_196_launches"]["us"] == 1148.22
     assert s["stream_tau6"]["frac"] == 0.621
+    assert s["stages_chain"]["us"] == 1250.24 and s["stages_112_launches"]["frac"] == 0.28
     assert s["cpu"]["matvec_gbs"] == [0.1396, 12.3456]
