@@ -165,6 +165,16 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- workload
 
+def decoder_stages(names):
+    """Stage of every matrix of a stack listed layer by layer in the order
+    q, k, v, o, gate, up, down: a decoder layer's dataflow, where q, k and v
+    read one input and gate and up read one input, o and down alone (four
+    stages per layer)."""
+    stage_of = {"q": 0, "k": 0, "v": 0, "o": 1, "gate": 2, "up": 2, "down": 3}
+    per = len(wl.LAYER_1P5B)
+    return [4 * (i // per) + stage_of[n] for i, n in enumerate(names)]
+
+
 class Stream:
     """The packed 28-layer weight stream with its activation and output buffers."""
 
@@ -198,11 +208,7 @@ class Stream:
 
         self.batch = sp.BatchViews([it[1] for it in self.items], [it[2] for it in self.items],
                                    [it[3] for it in self.items])
-        # a decoder layer's dataflow: q, k and v read one input, gate and up
-        # read one input; o and down stand alone (four stages per layer)
-        stage_of = {"q": 0, "k": 0, "v": 0, "o": 1, "gate": 2, "up": 2, "down": 3}
-        self.stages = [4 * (i // len(wl.LAYER_1P5B)) + stage_of[it[0].name]
-                       for i, it in enumerate(self.items)]
+        self.stages = decoder_stages([it[0].name for it in self.items])
         self.stage_batches = []
         for s in sorted(set(self.stages)):
             sel = [it for it, st in zip(self.items, self.stages) if st == s]

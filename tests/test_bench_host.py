@@ -106,3 +106,13 @@ def test_summary_is_last_and_short():
     assert s["stream_tau6"]["frac"] == 0.621
     assert s["stages_chain"]["us"] == 1250.24 and s["stages_112_launches"]["frac"] == 0.28
     assert s["cpu"]["matvec_gbs"] == [0.1396, 12.3456]
+
+
+def test_decoder_stages_group_shared_inputs():
+    names = [s.name for _ in range(3) for s in wl.LAYER_1P5B]
+    st = bench.decoder_stages(names)
+    # q, k, v | o | gate, up | down, four stages per layer, nondecreasing
+    assert st[:7] == [0, 0, 0, 1, 2, 2, 3]
+    assert st[7:14] == [4, 4, 4, 5, 6, 6, 7]
+    assert st == sorted(st) and len(set(st)) == 12
+
